@@ -1,0 +1,500 @@
+#!/usr/bin/env python
+"""Benchmark of the batch-1 MXFP4 MoE decode step on B200 (one JSON line on stdout).
+
+Workload (one "step"): the full decode step -- 42 distinct Ling-shaped MoE layers
+(hidden 2560, moe_intermediate 768, 512 routed experts top-8 with softmax
+renormalisation, one BF16 shared expert of 768, MXFP4 experts: ~67 GB of weights,
+so nothing stays in the 126 MB L2 between steps) followed by the 157,184 x 2,560
+FP8 LM head with argmax, at M = 1 (decode) and M = 4 (verify window).  Seeded
+synthetic weights and tokens; every timed step gets a fresh token row.
+
+value  = algorithmic HBM bytes of the step (weights the method must read + its
+         activation I/O, counted from the step's actual routing) / device time,
+         summed over ranks (replicas), in GB/s, at M = 1.
+e2e    = the same metric through the C-ABI graph launch with the token copied in
+         from pinned host memory and logits + argmax copied back, per step.
+roofline = the dominant kernel of the step, timed live by CUDA events recorded
+         around every launch inside a captured step.
+cpu_baseline = the CPU oracle timed on the host on a bounded sample.
+
+--impl reference times the CPU oracle (the reference arm) on the same metric.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "decode-step µs and achieved HBM GB/s at M=1/M=4 (fraction of ~8 TB/s)"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--layers", type=int, default=42)
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of CPU-oracle time for cpu_baseline")
+    ap.add_argument("--ref-layers", type=int, default=4, help="layers per reference-arm step")
+    ap.add_argument("--skip-m4", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------------------
+# algorithmic bytes
+# ---------------------------------------------------------------------------
+def layer_bytes(S, M, n_unique):
+    """Bytes one MoE layer must move: router + shared expert (BF16) + the distinct
+    routed experts' MXFP4 codes and scales, plus activation I/O (x in, residual in/out)."""
+    router = S.E * S.H * 2
+    shared = 3 * S.Is * S.H * 2
+    routed = n_unique * S.expert_bytes
+    io = M * S.H * (2 + 4 + 4)
+    return router + shared + routed + io
+
+
+def lm_bytes(V, H, M):
+    return V * H + V * 4 + M * V * 4 + M * H * 2 + M * 4
+
+
+def kernel_bytes(S, M, n_unique, V):
+    """Per-launch algorithmic bytes of each kernel of a layer (and the LM head)."""
+    return {
+        "k_dense": S.E * S.H * 2 + 2 * S.Is * S.H * 2 + M * S.H * (2 + 4) + M * (S.E * 4 + S.Is * 4),
+        "k_experts13": n_unique * 2 * S.I * (S.H // 2 + S.H // 32) + M * S.H * 2 + n_unique * M * S.I * 4,
+        "k_experts2": n_unique * S.H * (S.I // 2 + S.I // 32) + S.Is * S.H * 2 + n_unique * M * S.I * 4
+        + M * S.Is * 4 + M * S.H * 8,
+        "k_final_norm": M * S.H * (4 + 2),
+        "k_lm_gemv": lm_bytes(V, S.H, M),
+    }
+
+
+# ---------------------------------------------------------------------------
+# clocks sampler (nvidia-smi during the timed region)
+# ---------------------------------------------------------------------------
+class Clocks:
+    FIELDS = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuids):
+        self.uuids = set(u.lower() for u in uuids if u)
+        self.proc = None
+        self.lines = []
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.t:
+            self.t.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 10:
+                continue
+            if self.uuids and f[1].lower() not in self.uuids:
+                continue
+            try:
+                sm.append(float(f[2]))
+                mx.append(float(f[3]))
+            except ValueError:
+                continue
+            names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+            for nm, v in zip(names, f[6:10]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def run_ours(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from moe_decode_weight_router_b200 import (DecodeGraph, DecodeModel, build, decode_step,
+                                               decode_step_workspace_bytes, lm_head_fp8_quantize, synth)
+
+    build.build()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    S, V, L = synth.LING, synth.VOCAB, args.layers
+    seed = args.seed + 1000 * rank
+
+    # model: L distinct layers + LM head quantised online (once, outside the timed region)
+    layers = [synth.layer(S, seed, l, device=dev) for l in range(L)]
+    w_lm = synth.lm_head(V, S.H, seed, device=dev)
+    lm_q, lm_s = lm_head_fp8_quantize(w_lm)
+    torch.cuda.synchronize()
+    del w_lm
+    torch.cuda.empty_cache()
+    model = DecodeModel(layers=layers, lm_q=lm_q, lm_s=lm_s, top_k=S.k)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return t.item()
+
+    def sum_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.SUM)
+        return t.item()
+
+    K, W = args.steps, args.warmup
+    props = torch.cuda.get_device_properties(dev)
+    uuid = str(getattr(props, "uuid", "")) if hasattr(props, "uuid") else ""
+    if uuid and not uuid.startswith("GPU-"):
+        uuid = "GPU-" + uuid
+    uuids = [None] * world
+    if world > 1:
+        dist.all_gather_object(uuids, uuid)
+    else:
+        uuids = [uuid]
+
+    results = {}
+    for M in ([1] if args.skip_m4 else [1, 4]):
+        xs = [synth.tokens(M, S.H, seed, tid=100 + i, device=dev) for i in range(K + W)]
+        ws = torch.empty(decode_step_workspace_bytes(model, M), dtype=torch.uint8, device=dev)
+        # routing of every step's token (untimed) -> exact algorithmic bytes per step
+        step_bytes, uniq = [], []
+        for x in xs:
+            r = decode_step(model, x, trace=True, want_logits=False, ws=ws)
+            ids = r["ids_trace"].cpu().numpy()
+            nu = [len(np.unique(ids[l])) for l in range(L)]
+            uniq.append(nu)
+            step_bytes.append(sum(layer_bytes(S, M, n) for n in nu) + lm_bytes(V, S.H, M))
+        x_buf = xs[0].clone()
+        logits = torch.empty((M, V), dtype=torch.float32, device=dev)
+        am = torch.empty((M,), dtype=torch.int32, device=dev)
+        g = DecodeGraph(model, x_buf, logits, am, ws)
+        for i in range(W):
+            x_buf.copy_(xs[i])
+            g.launch()
+        torch.cuda.synchronize()
+        clk = Clocks(uuids) if rank == 0 else None
+        if clk:
+            clk.start()
+            time.sleep(0.3)
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(K):
+            x_buf.copy_(xs[W + i])
+            g.launch()
+        e1.record()
+        torch.cuda.synchronize()
+        barrier()
+        clocks = clk.stop() if clk else None
+        ms_total = max_over_ranks(e0.elapsed_time(e1))
+        bytes_rank = float(sum(step_bytes[W:W + K]))
+        bytes_all = sum_over_ranks(bytes_rank)
+        ms_step = ms_total / K
+        res = {
+            "ms_per_step": ms_step,
+            "us_per_step": 1000.0 * ms_step,
+            "gbps": bytes_all / (ms_total * 1e-3) / 1e9,
+            "bytes_per_step": bytes_rank / K,
+            "mean_unique_experts": float(np.mean([np.mean(u) for u in uniq[W:W + K]])),
+            "clocks": clocks,
+        }
+
+        # e2e through the C ABI: pinned host token in, logits + argmax out, per step
+        xh = [x.cpu().pin_memory() for x in xs]
+        lh = torch.empty((M, V), dtype=torch.float32).pin_memory()
+        ah = torch.empty((M,), dtype=torch.int32).pin_memory()
+        for i in range(W):
+            x_buf.copy_(xh[i], non_blocking=True)
+            g.launch()
+            lh.copy_(logits, non_blocking=True)
+            ah.copy_(am, non_blocking=True)
+        torch.cuda.synchronize()
+        barrier()
+        e0.record()
+        for i in range(K):
+            x_buf.copy_(xh[W + i], non_blocking=True)
+            g.launch()
+            lh.copy_(logits, non_blocking=True)
+            ah.copy_(am, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        barrier()
+        ms_e2e = max_over_ranks(e0.elapsed_time(e1))
+        res["e2e"] = {"value": bytes_all / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s", "us_per_step": 1000 * ms_e2e / K,
+                      "h2d_bytes_per_step": M * S.H * 2, "d2h_bytes_per_step": M * V * 4 + M * 4}
+        g.close()
+
+        # live per-kernel timing: events around every launch inside a captured step
+        if M == 1:
+            n_launch = 3 * L + 2
+            evs = [torch.cuda.Event(enable_timing=True) for _ in range(2 * n_launch)]
+            gk = DecodeGraph(model, x_buf, logits, am, ws, events=evs)
+            names = ["k_dense", "k_experts13", "k_experts2"] * L + ["k_final_norm", "k_lm_gemv"]
+            tot = {n: 0.0 for n in set(names)}
+            cnt = {n: 0 for n in set(names)}
+            kb = {n: 0.0 for n in set(names)}
+            reps = max(3, min(K, 10))
+            for i in range(reps):
+                x_buf.copy_(xs[W + (i % K)])
+                gk.launch()
+                torch.cuda.synchronize()
+                nu = uniq[W + (i % K)]
+                for j, n in enumerate(names):
+                    tot[n] += evs[2 * j].elapsed_time(evs[2 * j + 1])
+                    cnt[n] += 1
+                    lay = min(j // 3, L - 1)
+                    kb[n] += kernel_bytes(S, M, nu[lay], V)[n]
+            gk.close()
+            ker = {}
+            for n in tot:
+                avg_ms = tot[n] / cnt[n]
+                ker[n] = {"launches_per_step": cnt[n] // reps, "avg_us": 1000 * avg_ms,
+                          "share": tot[n] / sum(tot.values()), "gbps": (kb[n] / cnt[n]) / (avg_ms * 1e-3) / 1e9}
+            res["kernels"] = ker
+        results[M] = res
+
+    # CPU oracle baseline (rank 0, single GPU only): a bounded sample of the same step
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(model, S, V, args.cpu_budget)
+    return results, cpu
+
+
+def _threads():
+    n = os.environ.get("OMP_NUM_THREADS")
+    if n and n.isdigit():
+        return int(n)
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(model, S, V, budget_s):
+    """Oracle (as it stands) on the host over the same decode step at M = 1: the
+    chained layers in order until the time budget is spent (all of them when it
+    allows), then the LM head (all rows when the budget allows, else a slice);
+    GB/s over the algorithmic bytes actually covered."""
+    import numpy as np
+    import torch
+
+    import oracle
+    from moe_decode_weight_router_b200 import synth
+
+    oracle.lib()
+
+    def fetch_of(Ly):
+        def fetch(lst):
+            idx = torch.tensor(lst, dtype=torch.long, device=Ly["w13c"].device)
+            return {n: synth.bits(Ly[n].index_select(0, idx)) for n in ("w13c", "w13s", "w2c", "w2s")}
+        return fetch
+
+    x = synth.bits(synth.tokens(1, S.H, 7, tid=900))
+    t_all = 0.0
+    nb = 0
+    n_done = 0
+    for Ly in model.layers:
+        spec = [{"wr": synth.bits(Ly["wr"]), "experts": fetch_of(Ly),
+                 "shared": {"sw13": synth.bits(Ly["sw13"]), "sw2": synth.bits(Ly["sw2"])}}]
+        # host copies of this layer's router/shared weights happen outside the timed calls
+        t0 = time.perf_counter()
+        ids, w, _, _ = oracle.route(x, spec[0]["wr"], S.k)
+        t1 = time.perf_counter()
+        ex = spec[0]["experts"](sorted(set(ids.reshape(-1).tolist())))
+        t2 = time.perf_counter()
+        y = oracle.moe_layer(x, ids, w, _remap(ex, ids), spec[0]["shared"])
+        h = (np.vectorize(oracle.bf16_value)(x) if n_done == 0 else h) + y
+        x = oracle.rmsnorm_bf16(h)
+        t3 = time.perf_counter()
+        t_all += (t1 - t0) + (t3 - t2)
+        nb += layer_bytes(S, 1, len(np.unique(ids)))
+        n_done += 1
+        if t_all > budget_s:
+            break
+    vs = V if t_all < 0.8 * budget_s else 8192
+    q = synth.bits(model.lm_q[:vs])
+    sc = model.lm_s[:vs].cpu().numpy()
+    t0 = time.perf_counter()
+    oracle.lmhead_logits(x, q, sc)
+    t_all += time.perf_counter() - t0
+    nb += lm_bytes(vs, S.H, 1)
+    return {"value": nb / t_all / 1e9, "unit": "GB/s", "cores": _threads(), "kind": "oracle",
+            "sample": f"{n_done} of {len(model.layers)} chained Ling layers at M=1 + LM head rows [0,{vs}) of {V}; "
+                      f"{t_all:.2f} s of oracle time (host copies of the weights excluded)"}
+
+
+def _remap(ex, ids):
+    """Expert arrays fetched for sorted(set(ids)) re-indexed by expert id for the oracle."""
+    uniq = sorted(set(ids.reshape(-1).tolist()))
+    pos = {e: i for i, e in enumerate(uniq)}
+
+    def fetch(lst):
+        sel = [pos[e] for e in lst]
+        return {n: ex[n][sel] for n in ex}
+    return fetch
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the CPU oracle as it stands
+# ---------------------------------------------------------------------------
+def run_reference(args):
+    """The CPU oracle as it stands, on the same metric: each step is a bounded sample
+    of the decode step at M = 1 -- ``--ref-layers`` chained Ling layers (two distinct
+    layers alternated) and the LM head over 16,384 vocabulary rows."""
+    import numpy as np
+
+    import oracle
+    from moe_decode_weight_router_b200 import synth
+
+    S, V = synth.LING, synth.VOCAB
+    oracle.lib()
+    distinct = [{k: synth.bits(v) for k, v in synth.layer(S, args.seed, l, device="cpu").items()} for l in range(2)]
+    spec = [{"wr": Ly["wr"], "experts": Ly, "shared": {"sw13": Ly["sw13"], "sw2": Ly["sw2"]}}
+            for Ly in (distinct[i % 2] for i in range(args.ref_layers))]
+    vs = 16384
+    q = synth.bits(synth.e4m3_codes((vs, S.H), args.seed))
+    s = synth.row_scales(vs, args.seed).numpy()
+    xs = [synth.bits(synth.tokens(1, S.H, args.seed, tid=100 + i)) for i in range(args.steps + args.warmup)]
+    for i in range(args.warmup):
+        oracle.decode_step(xs[i], spec, q, s, S.k)
+    t0 = time.perf_counter()
+    nb = 0
+    for i in range(args.steps):
+        out = oracle.decode_step(xs[args.warmup + i], spec, q, s, S.k)
+        nb += sum(layer_bytes(S, 1, len(np.unique(ids))) for ids in out["ids"]) + lm_bytes(vs, S.H, 1)
+    dt = time.perf_counter() - t0
+    val = nb / dt / 1e9
+    sample = f"per step: {args.ref_layers} chained Ling layers at M=1 + LM head rows [0,{vs}) of {V}"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * dt / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "decode step sample (CPU oracle), M=1", "M": 1, "layers": args.ref_layers,
+                   "vocab_rows": vs},
+        "cpu_baseline": {"value": val, "unit": "GB/s", "cores": _threads(), "kind": "oracle", "sample": sample},
+        "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args)
+        return 0
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    if world > 1:
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    results, cpu = run_ours(args, rank, world, local_rank)
+    if rank == 0:
+        pk, src = peaks()
+        hbm = float(pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        r1 = results[1]
+        ker = r1.get("kernels", {})
+        dom = max(ker, key=lambda n: ker[n]["share"]) if ker else None
+        roof = None
+        if dom:
+            ach = ker[dom]["gbps"]
+            roof = {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+                    "traffic": None, "peak_source": f"{src} hbm_gbs (copy, burst)"}
+        line = {
+            "metric": METRIC, "value": r1["gbps"], "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": r1["ms_per_step"], "us_per_step": r1["us_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "mxfp4/fp8 weights x bf16 activations, f32 accumulate", "data": "synthetic",
+            "frac_of_8tbs": r1["gbps"] / world / NOMINAL_HBM_GBS, "frac_of_measured_hbm": r1["gbps"] / world / hbm,
+            "config": {"workload": f"decode step: {args.layers} MoE layers (H2560 I768 E512 top-8 + shared 768, "
+                                   "MXFP4) + FP8 LM head 157184x2560, M=1",
+                       "M": 1, "layers": args.layers, "hidden": 2560, "experts": 512, "top_k": 8, "vocab": 157184,
+                       "l2": "inputs larger than L2: ~67 GB of distinct layer weights streamed per step",
+                       "parallelism": "replicas" if world > 1 else "single GPU"},
+            "e2e": {k: v for k, v in r1["e2e"].items()},
+            "gpu_launches": (3 * args.layers + 2) * args.steps,
+            "clocks": r1["clocks"],
+            "roofline": roof,
+            "kernels": ker,
+            "cpu_baseline": cpu,
+        }
+        if 4 in results:
+            r4 = results[4]
+            line["m4"] = {"us_per_step": r4["us_per_step"], "gbps": r4["gbps"],
+                          "frac_of_8tbs": r4["gbps"] / world / NOMINAL_HBM_GBS,
+                          "frac_of_measured_hbm": r4["gbps"] / world / hbm,
+                          "mean_unique_experts": r4["mean_unique_experts"], "e2e": r4["e2e"], "clocks": r4["clocks"]}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,258 @@
+/*
+ * moe_decode.h -- C ABI of libmoe_decode.so: the batch-1 MXFP4 mixture-of-experts
+ * decode step on NVIDIA B200 (sm_100a).
+ *
+ * What is computed (sources):
+ *  - "知识卡片：NVIDIA DGX Spark 上提升 MoE 推理吞吐的三种方法" (DGX Spark MoE
+ *    knowledge card), section 事件概述或研究问题 ("overview"): decode at batch 1 is
+ *    bound by reading weights, the MoE and the LM head dominate; every MoE layer
+ *    routes a token to 8 of 512 routed experts plus 1 shared expert.
+ *  - same card, section 方法/产品要点 ("methods"), item 1: the routed experts are
+ *    MXFP4 with moe_intermediate_size = 768; item 2: the LM head (vocabulary GEMM
+ *    157,184 x 2,560, BF16 in the checkpoint) is quantised online to FP8 when the
+ *    head is built, halving its bytes; item 3: a 4-token verify window can fire up
+ *    to 32 distinct experts.
+ *  - "英伟达称不换芯片也能提速：DGX Spark靠软件优化多吐42.5%的token", section
+ *    不换卡，快在哪: the three optimisations and the 157,184 x 2,560 output layer.
+ *  Formats: OCP Microscaling (MX) v1.0 -- MXFP4 = FP4 E2M1 codes with one E8M0
+ *  scale 2^(e-127) per 32 consecutive elements; FP8 E4M3 (bias 7, max 448).
+ *
+ * Conventions for every entry point:
+ *  - All tensor arguments are DEVICE pointers (cudaMalloc'd or equivalent) unless
+ *    stated; the caller owns every buffer.  The library never allocates, frees or
+ *    synchronises; every call is asynchronous and ordered on `stream`.
+ *  - Arguments are validated on the host before anything is enqueued; a non-OK
+ *    status means nothing was launched.  No C++ exception crosses the ABI.
+ *  - Pointers must be 16-byte aligned (MOE_ERR_ALIGNMENT otherwise).
+ *  - Layouts are row-major, "[out][in]" for weights (the Linear convention).
+ *    BF16 tensors are raw uint16 bit patterns.  MXFP4 codes: two per byte along
+ *    the input dimension, element 2j in the LOW nibble of byte j; the scale byte
+ *    b of a row covers input elements [32b, 32b+32).  E2M1 bit 3 = sign, bits 2..1
+ *    exponent (bias 1), bit 0 mantissa.
+ *  - W13 stacks the gate projection (rows [0, I)) over the up projection (rows
+ *    [I, 2I)); SwiGLU a = silu(gate) * up, kept in fp32.
+ *  - Routing: l = x . Wr^T in fp32; the top_k largest logits (ties to the lower
+ *    expert index); weights = softmax over the selected logits (= the softmax
+ *    over all experts renormalised over the selected).
+ *  - Workspaces are caller-owned scratch of at least the *_workspace_bytes()
+ *    size; their contents on entry do not matter and are clobbered.
+ *  - A CUDA error while enqueuing returns MOE_ERR_CUDA; moe_last_cuda_error()
+ *    then gives the cudaError_t value (per calling thread).
+ *  - Thread safety: stateless apart from the caller's buffers and the per-thread
+ *    last-error value; concurrent calls on different workspaces are safe.
+ */
+#ifndef MOE_DECODE_H
+#define MOE_DECODE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Layout-compatible with cudaStream_t / CUstream; NULL = the legacy default stream. */
+typedef struct CUstream_st* moe_stream_t;
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,       /* NULL where a buffer is required, negative size, ... */
+  MOE_ERR_UNSUPPORTED_SHAPE = 2, /* a size outside the limits listed per entry point */
+  MOE_ERR_ALIGNMENT = 3,         /* a pointer not 16-byte aligned */
+  MOE_ERR_WORKSPACE = 4,         /* workspace NULL or smaller than required */
+  MOE_ERR_DTYPE = 5,             /* a model buffer tagged with the wrong format */
+  MOE_ERR_CUDA = 6,              /* the CUDA runtime refused a launch */
+  MOE_ERR_TIMEOUT = 7            /* a bounded device-side wait gave up */
+} moe_status_t;
+
+/* Human-readable name of a status value (static storage). */
+MOE_API const char* moe_status_string(int status);
+/* ABI version of this header: MOE_ABI_VERSION. */
+#define MOE_ABI_VERSION 1
+MOE_API int moe_abi_version(void);
+/* cudaError_t of the last MOE_ERR_CUDA returned on the calling thread (0 if none). */
+MOE_API int moe_last_cuda_error(void);
+/* Device-side status of the last call that used workspace `ws`: synchronises
+ * `stream`, then reads the status word every call clears on entry.  MOE_OK, or
+ * MOE_ERR_TIMEOUT when a bounded device wait gave up (the kernel returned early
+ * instead of hanging; its outputs are then incomplete).  Host-blocking: meant for
+ * checks and tests, not for the hot path. */
+MOE_API moe_status_t moe_workspace_status(const void* ws, moe_stream_t stream);
+
+/* ------------------------------------------------------------------------- */
+/* Router (knowledge card, overview: 8 of 512 routed experts per token)       */
+/* ------------------------------------------------------------------------- */
+
+/* Bytes of workspace moe_route needs for M tokens and E experts. */
+MOE_API size_t moe_route_workspace_bytes(int M, int E);
+
+/* Router logits, top-k selection and renormalised weights for M tokens.
+ *   x_bf16        [M][H]  bf16 activations
+ *   w_router_bf16 [E][H]  bf16 router weight
+ *   topk_ids      [M][top_k] int32 out: selected experts, descending logit,
+ *                 ties broken toward the lower index
+ *   topk_w        [M][top_k] fp32 out: softmax over the selected logits (sums to 1)
+ *   logits_opt    [M][E] fp32 out, or NULL
+ * Limits: 1 <= M <= 8; H % 64 == 0, 64 <= H <= 4096; E % 16 == 0, 16 <= E <= 1024;
+ *         1 <= top_k <= min(8, E). */
+MOE_API moe_status_t moe_route(const void* x_bf16, int M, int H, const void* w_router_bf16, int E,
+                       int top_k, int32_t* topk_ids, float* topk_w, float* logits_opt,
+                       void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* ------------------------------------------------------------------------- */
+/* Routed MXFP4 experts + BF16 shared expert (knowledge card, methods item 1)  */
+/* ------------------------------------------------------------------------- */
+
+/* Bytes of workspace moe_mxfp4_experts needs. */
+MOE_API size_t moe_experts_workspace_bytes(int M, int H, int I, int E, int top_k, int Is);
+
+/* One MoE layer for M tokens under a given routing:
+ *   y[t] = sum_j topk_w[t][j] * W2_e (silu(Wg_e x_t) * Wu_e x_t),  e = topk_ids[t][j]
+ *        + Ws2 (silu(Wsg x_t) * Wsu x_t)                  (when the shared expert is given)
+ *   x_bf16       [M][H] bf16
+ *   topk_ids     [M][top_k] int32 expert ids in [0, E)   (device)
+ *   topk_w       [M][top_k] fp32 weights                  (device)
+ *   w13_codes    [E][2I][H/2]  u8   MXFP4 codes of gate (rows < I) and up (rows >= I)
+ *   w13_scales   [E][2I][H/32] u8   E8M0
+ *   w2_codes     [E][H][I/2]   u8
+ *   w2_scales    [E][H][I/32]  u8
+ *   shared_w13_bf16 [2Is][H] bf16 (gate rows then up rows) and shared_w2_bf16 [H][Is]
+ *                 bf16, both NULL (with Is = 0) when the layer has no shared expert
+ *   y            [M][H] fp32 out (overwritten)
+ * Every distinct expert among the M*top_k selections is streamed from HBM once
+ * per call, whatever the number of tokens that chose it.  Activations stay BF16
+ * (the products are formed exactly and accumulated in fp32).
+ * Ids outside [0, E) contribute nothing (they are dropped on the device, never read
+ * out of bounds).  A token listing the same expert twice gives it both weights.
+ * Limits: 1 <= M <= 8 (decode / verify windows); H % 64 == 0, 64 <= H <= 4096;
+ *         I % 32 == 0, 32 <= I <= 1024; Is % 32 == 0, 0 <= Is <= 1024;
+ *         E % 16 == 0, 16 <= E <= 1024; 1 <= top_k <= min(8, E). */
+MOE_API moe_status_t moe_mxfp4_experts(const void* x_bf16, int M, int H, int I, int E, int top_k,
+                               const int32_t* topk_ids, const float* topk_w,
+                               const uint8_t* w13_codes, const uint8_t* w13_scales,
+                               const uint8_t* w2_codes, const uint8_t* w2_scales,
+                               const void* shared_w13_bf16, const void* shared_w2_bf16, int Is,
+                               float* y, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* ------------------------------------------------------------------------- */
+/* FP8 LM head (knowledge card, methods item 2; retelling, 不换卡，快在哪)        */
+/* ------------------------------------------------------------------------- */
+
+/* Online FP8 quantisation of a BF16 LM head, done once when the head is built:
+ *   amax_v = max_h |W[v][h]|;  s_v = amax_v / 448 (fp32 division; 1.0 if amax_v == 0)
+ *   w_e4m3[v][h] = e4m3 round-to-nearest-even of W[v][h] / s_v (fp32 division),
+ *                  saturating at +-448.
+ *   w_bf16 [V][H] bf16 in; w_e4m3 [V][H] u8 out; row_scale [V] fp32 out.
+ * Limits: 1 <= V; H % 16 == 0, 16 <= H <= 16384. */
+MOE_API moe_status_t lm_head_fp8_quantize(const void* w_bf16, int V, int H, uint8_t* w_e4m3,
+                                  float* row_scale, moe_stream_t stream);
+
+/* Bytes of workspace lm_head_fp8_gemv needs. */
+MOE_API size_t lm_head_workspace_bytes(int M, int V, int H);
+
+/* logits[t][v] = row_scale[v] * sum_h e4m3(w_e4m3[v][h]) * x[t][h]  (fp32 accumulation)
+ * argmax[t]    = the index of the largest logit of row t, lowest index on ties.
+ *   x_bf16 [M][H] bf16; logits [M][V] fp32 out (may be NULL: argmax only);
+ *   argmax [M] int32 out.
+ * Limits: 1 <= M <= 8; 1 <= V <= 2^26; H % 64 == 0, 64 <= H <= 2560. */
+MOE_API moe_status_t lm_head_fp8_gemv(const void* x_bf16, int M, int V, int H, const uint8_t* w_e4m3,
+                              const float* row_scale, float* logits, int32_t* argmax,
+                              void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* ------------------------------------------------------------------------- */
+/* Whole decode step: L MoE layers + FP8 LM head                              */
+/* ------------------------------------------------------------------------- */
+
+/* Format tags carried by every model buffer, checked by decode_step.  A buffer
+ * whose tag disagrees with its role is rejected (MOE_ERR_DTYPE) instead of being
+ * silently reinterpreted -- e.g. FP8 LM-head bytes read as BF16. */
+enum {
+  MOE_FMT_NONE = 0,
+  MOE_FMT_BF16 = 1,
+  MOE_FMT_MXFP4_CODES = 2,
+  MOE_FMT_E8M0_SCALES = 3,
+  MOE_FMT_E4M3 = 4,
+  MOE_FMT_F32 = 5
+};
+
+typedef struct {
+  const void* ptr; /* device pointer */
+  int fmt;         /* MOE_FMT_* */
+} moe_buf_t;
+
+typedef struct {
+  moe_buf_t router;      /* [E][H]   bf16 */
+  moe_buf_t w13_codes;   /* [E][2I][H/2]  MXFP4 codes */
+  moe_buf_t w13_scales;  /* [E][2I][H/32] E8M0 */
+  moe_buf_t w2_codes;    /* [E][H][I/2]   MXFP4 codes */
+  moe_buf_t w2_scales;   /* [E][H][I/32]  E8M0 */
+  moe_buf_t shared_w13;  /* [2Is][H] bf16, or ptr NULL when Is == 0 */
+  moe_buf_t shared_w2;   /* [H][Is]  bf16, or ptr NULL when Is == 0 */
+} moe_layer_t;
+
+typedef struct {
+  int n_layers;               /* L >= 1 */
+  int H, I, E, top_k, Is, V;  /* shapes shared by all layers (limits as above) */
+  float rms_eps;              /* RMSNorm epsilon of the layer-chaining stand-in (1e-6) */
+  const moe_layer_t* layers;  /* HOST array of n_layers entries */
+  moe_buf_t lm_head;          /* [V][H] e4m3 codes (from lm_head_fp8_quantize) */
+  moe_buf_t lm_scale;         /* [V] fp32 row scales */
+} moe_model_t;
+
+/* Optional debug trace of a decode step (device buffers, any may be NULL):
+ *   x  [L+1][M][H] bf16: each layer's input and the LM head's input
+ *   h  [L+1][M][H] fp32: the residual stream entering each layer, and the final one
+ *   ids [L][M][top_k] int32, w [L][M][top_k] fp32: each layer's routing
+ *   events: NULL or an array of n_events cudaEvent_t handles (host array, created by
+ *     the caller) recorded on the step's stream around every kernel: events[2i] before
+ *     and events[2i+1] after launch i, launches ordered (router+shared W13, routed W13,
+ *     W2+combine) per layer, then the final RMSNorm, then the LM head; 3L+2 launches.
+ *     Fewer events than 2(3L+2) record the first n_events/2 launches only. */
+typedef struct {
+  void* x;
+  float* h;
+  int32_t* ids;
+  float* w;
+  void** events;
+  int n_events;
+} moe_trace_t;
+
+MOE_API size_t decode_step_workspace_bytes(const moe_model_t* model, int M);
+
+/* One decode step for an M-token window (M = 1 decode, M = 4 verify window):
+ *   h_0 = fp32(x);  for l < L:  x_l = (l == 0 ? x : bf16(RMSNorm(h_l))),
+ *                               h_{l+1} = h_l + MoE_l(x_l)       (route + experts + shared)
+ *   x_L = bf16(RMSNorm(h_L));   logits = FP8 LM head(x_L);  argmax per row.
+ * RMSNorm has unit weight: h / sqrt(mean(h^2) + rms_eps).  It stands in for the
+ * attention blocks between MoE layers, which are not part of this library.
+ *   model  HOST pointer; its buffers are device pointers with format tags
+ *   x_bf16 [M][H] bf16; logits [M][V] fp32 out (may be NULL); argmax [M] int32 out
+ *   trace_opt HOST pointer or NULL.
+ * Limits: as moe_mxfp4_experts (1 <= M <= 8) and lm_head_fp8_gemv (H <= 2560). */
+MOE_API moe_status_t decode_step(const moe_model_t* model, const void* x_bf16, int M, float* logits,
+                         int32_t* argmax, const moe_trace_t* trace_opt, void* ws,
+                         size_t ws_bytes, moe_stream_t stream);
+
+/* A whole decode step captured once as a CUDA graph (about 3 launches per layer),
+ * replayed with a single launch.  The graph binds the given x, logits, argmax and
+ * workspace pointers: refill x in place between launches.  The handle is a small
+ * host object owned by the caller (decode_step_graph_destroy); no device memory is
+ * allocated.  The model's buffers must stay valid while the handle lives. */
+typedef struct moe_graph_s* moe_graph_t;
+MOE_API moe_status_t decode_step_graph_create(const moe_model_t* model, const void* x_bf16, int M, float* logits,
+                                      int32_t* argmax, const moe_trace_t* trace_opt, void* ws,
+                                      size_t ws_bytes, moe_graph_t* out);
+MOE_API moe_status_t decode_step_graph_launch(moe_graph_t graph, moe_stream_t stream);
+MOE_API void decode_step_graph_destroy(moe_graph_t graph);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_DECODE_H */

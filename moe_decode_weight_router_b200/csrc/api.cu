@@ -1,0 +1,634 @@
+// api.cu -- the C ABI of libmoe_decode.so (declared in include/moe_decode.h).
+//
+// Host side only: argument validation (before anything is enqueued), workspace
+// carving, launch configuration (one block per SM for the streamed kernels,
+// shared-memory stage counts from the device's opt-in limit) and the per-layer
+// launch sequence of the decode step.
+#include <cuda_runtime.h>
+
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/moe_decode.h"
+#include "decode_kernels.cuh"
+#include "lmhead_kernels.cuh"
+
+using namespace moe;
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+moe_status_t cuda_fail(cudaError_t e) {
+  g_last_cuda_error = static_cast<int>(e);
+  return MOE_ERR_CUDA;
+}
+
+#define MOE_CUDA(call)                          \
+  do {                                          \
+    cudaError_t e_ = (call);                    \
+    if (e_ != cudaSuccess) return cuda_fail(e_); \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+size_t up256(size_t b) { return (b + 255) / 256 * 256; }
+
+struct DevInfo {
+  int sms = 0;
+  int smem_optin = 0;
+};
+
+// Per-device launch facts and one-time kernel attributes (opt-in shared memory).
+moe_status_t dev_info(DevInfo* out) {
+  static std::mutex mu;
+  static DevInfo cache[64];
+  static bool ready[64] = {};
+  int dev = 0;
+  MOE_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return MOE_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!ready[dev]) {
+    DevInfo d;
+    MOE_CUDA(cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev));
+    MOE_CUDA(cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev));
+    const int lim = d.smem_optin;
+    MOE_CUDA(cudaFuncSetAttribute(k_dense, cudaFuncAttributeMaxDynamicSharedMemorySize, lim));
+    MOE_CUDA(cudaFuncSetAttribute(k_experts13<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim));
+    MOE_CUDA(cudaFuncSetAttribute(k_experts13<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim));
+    MOE_CUDA(cudaFuncSetAttribute(k_experts13<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim));
+    MOE_CUDA(cudaFuncSetAttribute(k_experts13<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim));
+    MOE_CUDA(cudaFuncSetAttribute(k_experts2<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim));
+    MOE_CUDA(cudaFuncSetAttribute(k_experts2<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim));
+    MOE_CUDA(cudaFuncSetAttribute(k_experts2<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim));
+    MOE_CUDA(cudaFuncSetAttribute(k_experts2<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim));
+    MOE_CUDA(cudaFuncSetAttribute(k_lm_gemv, cudaFuncAttributeMaxDynamicSharedMemorySize, lim));
+    cache[dev] = d;
+    ready[dev] = true;
+  }
+  *out = cache[dev];
+  return MOE_OK;
+}
+
+// ---- shape checks -----------------------------------------------------------
+bool ok_M(int M) { return M >= 1 && M <= MAX_M; }
+bool ok_H(int H) { return H >= 64 && H <= 4096 && H % 64 == 0; }
+bool ok_I(int I) { return I >= 32 && I <= 1024 && I % 32 == 0; }
+bool ok_Is(int Is) { return Is >= 0 && Is <= 1024 && Is % 32 == 0; }
+bool ok_E(int E) { return E >= 16 && E <= 1024 && E % 16 == 0; }
+bool ok_k(int k, int E) { return k >= 1 && k <= 8 && k <= E; }
+bool ok_H_lm(int H) { return H >= 64 && H <= 2560 && H % 64 == 0; }
+
+// ---- workspace layouts ------------------------------------------------------
+constexpr size_t CTRL_BYTES = 256;  // status (int @0), counters (@4, @8), argmax keys (@64)
+
+struct Ctrl {
+  int* status;
+  unsigned* route_counter;
+  unsigned* lm_counter;
+  unsigned long long* keys;
+};
+Ctrl ctrl_of(void* ws) {
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  return Ctrl{reinterpret_cast<int*>(b), reinterpret_cast<unsigned*>(b + 4), reinterpret_cast<unsigned*>(b + 8),
+              reinterpret_cast<unsigned long long*>(b + 64)};
+}
+
+size_t slots_of(int M, int E, int k) { return static_cast<size_t>(M * k < E ? M * k : E); }
+
+struct ExpertsWs {
+  float* a_shared;
+  float* a_routed;
+  size_t bytes;
+};
+ExpertsWs experts_ws(void* ws, int M, int H, int I, int E, int k, int Is) {
+  (void)H;
+  size_t off = CTRL_BYTES;
+  ExpertsWs w{};
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  w.a_shared = reinterpret_cast<float*>(b + off);
+  off += up256((size_t)M * Is * 4);
+  w.a_routed = reinterpret_cast<float*>(b + off);
+  off += up256(slots_of(M, E, k) * M * I * 4);
+  w.bytes = off;
+  return w;
+}
+
+struct StepWs {
+  float* logits;
+  int32_t* ids;
+  float* w;
+  __nv_bfloat16* x_cur;
+  float* h;
+  float* a_shared;
+  float* a_routed;
+  __nv_bfloat16* x_final;
+  size_t bytes;
+};
+StepWs step_ws(void* ws, int M, int H, int I, int E, int k, int Is) {
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  size_t off = CTRL_BYTES;
+  StepWs s{};
+  s.logits = reinterpret_cast<float*>(b + off);
+  off += up256((size_t)M * E * 4);
+  s.ids = reinterpret_cast<int32_t*>(b + off);
+  off += up256((size_t)M * k * 4);
+  s.w = reinterpret_cast<float*>(b + off);
+  off += up256((size_t)M * k * 4);
+  s.x_cur = reinterpret_cast<__nv_bfloat16*>(b + off);
+  off += up256((size_t)M * H * 2);
+  s.h = reinterpret_cast<float*>(b + off);
+  off += up256((size_t)M * H * 4);
+  s.a_shared = reinterpret_cast<float*>(b + off);
+  off += up256((size_t)M * Is * 4);
+  s.a_routed = reinterpret_cast<float*>(b + off);
+  off += up256(slots_of(M, E, k) * M * I * 4);
+  s.x_final = reinterpret_cast<__nv_bfloat16*>(b + off);
+  off += up256((size_t)M * H * 2);
+  s.bytes = off;
+  return s;
+}
+
+// ---- launchers ----------------------------------------------------------------
+moe_status_t launch_dense(const DenseParams& p, cudaStream_t st) {
+  const int grid = p.n_rtiles + p.n_stiles;
+  if (grid == 0) return MOE_OK;
+  k_dense<<<grid, DENSE_THREADS, dense_smem_bytes(p.H), st>>>(p);
+  MOE_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
+
+// Stage count of a streamed kernel: as many as fit, at most MAX_STAGES, and a
+// multiple of the consumer-warp count.  Consumer warp w takes items w, w+NC, ...
+// and item i uses stage i % S, so with S % NC == 0 the warp waiting on a stage's
+// next phase is the warp that consumed its previous phase -- the mbarrier parity
+// it waits on can never alias a phase that has not completed yet.
+int stages_for(const DevInfo& d, size_t fixed, size_t stage) {
+  if ((size_t)d.smem_optin <= fixed) return 0;
+  size_t s = ((size_t)d.smem_optin - fixed) / stage;
+  if (s > (size_t)MAX_STAGES) s = MAX_STAGES;
+  return (int)(s / N_CONSUMERS * N_CONSUMERS);
+}
+
+moe_status_t launch_e13(E13Params p, const DevInfo& d, cudaStream_t st) {
+  const size_t fixed = e13_fixed_bytes(p.H), stage = e13_stage_bytes(p.H);
+  p.stages = stages_for(d, fixed, stage);
+  if (p.stages < N_CONSUMERS) return MOE_ERR_UNSUPPORTED_SHAPE;
+  const size_t smem = fixed + (size_t)p.stages * stage;
+  const int grid = d.sms;
+  switch ((p.M + 1) / 2) {
+    case 1: k_experts13<1><<<grid, EXPERT_THREADS, smem, st>>>(p); break;
+    case 2: k_experts13<2><<<grid, EXPERT_THREADS, smem, st>>>(p); break;
+    case 3: k_experts13<3><<<grid, EXPERT_THREADS, smem, st>>>(p); break;
+    default: k_experts13<4><<<grid, EXPERT_THREADS, smem, st>>>(p); break;
+  }
+  MOE_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
+
+moe_status_t launch_e2(E2Params p, const DevInfo& d, cudaStream_t st) {
+  const size_t fixed = e2_fixed_bytes(p.M, p.I, p.Is), stage = e2_stage_bytes(p.I, p.Is);
+  p.stages = stages_for(d, fixed, stage);
+  if (p.stages < N_CONSUMERS) return MOE_ERR_UNSUPPORTED_SHAPE;
+  const size_t smem = fixed + (size_t)p.stages * stage;
+  // Each block's contiguous item range must touch at most E2_MAX_LOCAL_SLOTS experts.
+  const long long htiles = p.H / 16;
+  const long long nch = p.Is > 0 ? (p.Is + SHARED_CHUNK - 1) / SHARED_CHUNK : 0;
+  const long long Tmax = (long long)slots_of(p.M, p.E, p.top_k) * htiles + htiles * nch;
+  long long grid = d.sms;
+  while ((Tmax + grid - 1) / grid > (E2_MAX_LOCAL_SLOTS - 1) * htiles + 1) grid *= 2;
+  switch ((p.M + 1) / 2) {
+    case 1: k_experts2<1><<<(int)grid, EXPERT_THREADS, smem, st>>>(p); break;
+    case 2: k_experts2<2><<<(int)grid, EXPERT_THREADS, smem, st>>>(p); break;
+    case 3: k_experts2<3><<<(int)grid, EXPERT_THREADS, smem, st>>>(p); break;
+    default: k_experts2<4><<<(int)grid, EXPERT_THREADS, smem, st>>>(p); break;
+  }
+  MOE_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
+
+moe_status_t launch_lm(LMParams p, const DevInfo& d, cudaStream_t st) {
+  const size_t fixed = lm_fixed_bytes(p.H), stage = lm_stage_bytes(p.H);
+  p.stages = stages_for(d, fixed, stage);
+  if (p.stages < N_CONSUMERS) return MOE_ERR_UNSUPPORTED_SHAPE;
+  const size_t smem = fixed + (size_t)p.stages * stage;
+  const long long T = (p.V + 15) / 16;
+  const int grid = (int)(T < d.sms ? T : d.sms);
+  k_lm_gemv<<<grid, EXPERT_THREADS, smem, st>>>(p);
+  MOE_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
+
+// Records events[2i] / events[2i+1] around launch i when the caller asked for them.
+struct EventHook {
+  cudaEvent_t* ev = nullptr;
+  int n = 0;
+  int i = 0;
+  moe_status_t before(cudaStream_t st) {
+    if (ev && 2 * i + 1 < n) MOE_CUDA(cudaEventRecord(ev[2 * i], st));
+    return MOE_OK;
+  }
+  moe_status_t after(cudaStream_t st) {
+    if (ev && 2 * i + 1 < n) MOE_CUDA(cudaEventRecord(ev[2 * i + 1], st));
+    ++i;
+    return MOE_OK;
+  }
+};
+
+// ---- validation helpers ---------------------------------------------------------
+#define REQ(cond, code) \
+  do {                  \
+    if (!(cond)) return (code); \
+  } while (0)
+
+moe_status_t check_ptrs_aligned(std::initializer_list<const void*> ps) {
+  for (const void* p : ps)
+    if (p && !aligned16(p)) return MOE_ERR_ALIGNMENT;
+  return MOE_OK;
+}
+
+moe_status_t check_layer_buf(const moe_buf_t& b, int fmt, bool required) {
+  if (!b.ptr) return required ? MOE_ERR_INVALID_ARG : MOE_OK;
+  if (b.fmt != fmt) return MOE_ERR_DTYPE;
+  if (!aligned16(b.ptr)) return MOE_ERR_ALIGNMENT;
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(int status) {
+  switch (status) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED_SHAPE: return "MOE_ERR_UNSUPPORTED_SHAPE";
+    case MOE_ERR_ALIGNMENT: return "MOE_ERR_ALIGNMENT";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+    case MOE_ERR_DTYPE: return "MOE_ERR_DTYPE";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT";
+    default: return "MOE_ERR_UNKNOWN";
+  }
+}
+
+int moe_abi_version(void) { return MOE_ABI_VERSION; }
+int moe_last_cuda_error(void) { return g_last_cuda_error; }
+
+moe_status_t moe_workspace_status(const void* ws, moe_stream_t stream) {
+  REQ(ws, MOE_ERR_INVALID_ARG);
+  MOE_CUDA(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)));
+  int st = 0;
+  MOE_CUDA(cudaMemcpy(&st, ws, sizeof st, cudaMemcpyDeviceToHost));
+  return st == 0 ? MOE_OK : (moe_status_t)st;
+}
+
+size_t moe_route_workspace_bytes(int M, int E) {
+  if (!ok_M(M) || !ok_E(E)) return 0;
+  return CTRL_BYTES + up256((size_t)M * E * 4);
+}
+
+moe_status_t moe_route(const void* x_bf16, int M, int H, const void* w_router_bf16, int E, int top_k,
+                       int32_t* topk_ids, float* topk_w, float* logits_opt, void* ws, size_t ws_bytes,
+                       moe_stream_t stream) {
+  REQ(x_bf16 && w_router_bf16 && topk_ids && topk_w, MOE_ERR_INVALID_ARG);
+  REQ(ok_M(M) && ok_H(H) && ok_E(E) && ok_k(top_k, E), MOE_ERR_UNSUPPORTED_SHAPE);
+  moe_status_t s = check_ptrs_aligned({x_bf16, w_router_bf16, topk_ids, topk_w, logits_opt, ws});
+  if (s != MOE_OK) return s;
+  REQ(ws && ws_bytes >= moe_route_workspace_bytes(M, E), MOE_ERR_WORKSPACE);
+  DevInfo d;
+  if ((s = dev_info(&d)) != MOE_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  Ctrl c = ctrl_of(ws);
+  MOE_CUDA(cudaMemsetAsync(ws, 0, CTRL_BYTES, st));
+  DenseParams p{};
+  p.x = static_cast<const __nv_bfloat16*>(x_bf16);
+  p.mode = 0;
+  p.M = M;
+  p.H = H;
+  p.wr = static_cast<const __nv_bfloat16*>(w_router_bf16);
+  p.E = E;
+  p.top_k = top_k;
+  p.n_rtiles = E / 16;
+  p.logits_ws = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + CTRL_BYTES);
+  p.logits_out = logits_opt;
+  p.ids = topk_ids;
+  p.w = topk_w;
+  p.counter = c.route_counter;
+  return launch_dense(p, st);
+}
+
+size_t moe_experts_workspace_bytes(int M, int H, int I, int E, int top_k, int Is) {
+  if (!ok_M(M) || !ok_H(H) || !ok_I(I) || !ok_E(E) || !ok_k(top_k, E) || !ok_Is(Is)) return 0;
+  return experts_ws(nullptr, M, H, I, E, top_k, Is).bytes;
+}
+
+moe_status_t moe_mxfp4_experts(const void* x_bf16, int M, int H, int I, int E, int top_k,
+                               const int32_t* topk_ids, const float* topk_w, const uint8_t* w13_codes,
+                               const uint8_t* w13_scales, const uint8_t* w2_codes, const uint8_t* w2_scales,
+                               const void* shared_w13_bf16, const void* shared_w2_bf16, int Is, float* y,
+                               void* ws, size_t ws_bytes, moe_stream_t stream) {
+  REQ(x_bf16 && topk_ids && topk_w && w13_codes && w13_scales && w2_codes && w2_scales && y, MOE_ERR_INVALID_ARG);
+  REQ(ok_M(M) && ok_H(H) && ok_I(I) && ok_E(E) && ok_k(top_k, E) && ok_Is(Is), MOE_ERR_UNSUPPORTED_SHAPE);
+  REQ((Is == 0) == (shared_w13_bf16 == nullptr) && (Is == 0) == (shared_w2_bf16 == nullptr), MOE_ERR_INVALID_ARG);
+  moe_status_t s = check_ptrs_aligned({x_bf16, topk_ids, topk_w, w13_codes, w13_scales, w2_codes, w2_scales,
+                                       shared_w13_bf16, shared_w2_bf16, y, ws});
+  if (s != MOE_OK) return s;
+  const size_t need = moe_experts_workspace_bytes(M, H, I, E, top_k, Is);
+  REQ(ws && ws_bytes >= need, MOE_ERR_WORKSPACE);
+  DevInfo d;
+  if ((s = dev_info(&d)) != MOE_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  Ctrl c = ctrl_of(ws);
+  ExpertsWs w = experts_ws(ws, M, H, I, E, top_k, Is);
+  MOE_CUDA(cudaMemsetAsync(ws, 0, CTRL_BYTES, st));
+  MOE_CUDA(cudaMemsetAsync(y, 0, (size_t)M * H * sizeof(float), st));
+  if (Is > 0) {
+    DenseParams p{};
+    p.x = static_cast<const __nv_bfloat16*>(x_bf16);
+    p.mode = 0;
+    p.M = M;
+    p.H = H;
+    p.E = E;
+    p.top_k = top_k;
+    p.n_rtiles = 0;
+    p.sw13 = static_cast<const __nv_bfloat16*>(shared_w13_bf16);
+    p.Is = Is;
+    p.n_stiles = Is / 8;
+    p.a_shared = w.a_shared;
+    p.counter = c.route_counter;
+    if ((s = launch_dense(p, st)) != MOE_OK) return s;
+  }
+  E13Params a{};
+  a.x = static_cast<const __nv_bfloat16*>(x_bf16);
+  a.M = M;
+  a.H = H;
+  a.I = I;
+  a.E = E;
+  a.top_k = top_k;
+  a.ids = topk_ids;
+  a.w = topk_w;
+  a.w13c = w13_codes;
+  a.w13s = w13_scales;
+  a.a_routed = w.a_routed;
+  a.status = c.status;
+  if ((s = launch_e13(a, d, st)) != MOE_OK) return s;
+  E2Params b{};
+  b.M = M;
+  b.H = H;
+  b.I = I;
+  b.E = E;
+  b.top_k = top_k;
+  b.Is = Is;
+  b.ids = topk_ids;
+  b.w = topk_w;
+  b.w2c = w2_codes;
+  b.w2s = w2_scales;
+  b.sw2 = static_cast<const __nv_bfloat16*>(shared_w2_bf16);
+  b.a_routed = w.a_routed;
+  b.a_shared = w.a_shared;
+  b.out = y;
+  b.status = c.status;
+  return launch_e2(b, d, st);
+}
+
+moe_status_t lm_head_fp8_quantize(const void* w_bf16, int V, int H, uint8_t* w_e4m3, float* row_scale,
+                                  moe_stream_t stream) {
+  REQ(w_bf16 && w_e4m3 && row_scale, MOE_ERR_INVALID_ARG);
+  REQ(V >= 1 && H >= 16 && H <= 16384 && H % 16 == 0, MOE_ERR_UNSUPPORTED_SHAPE);
+  moe_status_t s = check_ptrs_aligned({w_bf16, w_e4m3, row_scale});
+  if (s != MOE_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const long long blocks = ((long long)V + 7) / 8;
+  k_lm_quantize<<<(unsigned)blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(w_bf16), V, H, w_e4m3,
+                                                   row_scale);
+  MOE_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
+
+size_t lm_head_workspace_bytes(int M, int V, int H) {
+  if (!ok_M(M) || V < 1 || !ok_H_lm(H)) return 0;
+  return CTRL_BYTES;
+}
+
+moe_status_t lm_head_fp8_gemv(const void* x_bf16, int M, int V, int H, const uint8_t* w_e4m3,
+                              const float* row_scale, float* logits, int32_t* argmax, void* ws, size_t ws_bytes,
+                              moe_stream_t stream) {
+  REQ(x_bf16 && w_e4m3 && row_scale && argmax, MOE_ERR_INVALID_ARG);
+  REQ(ok_M(M) && V >= 1 && V <= (1 << 26) && ok_H_lm(H), MOE_ERR_UNSUPPORTED_SHAPE);
+  moe_status_t s = check_ptrs_aligned({x_bf16, w_e4m3, row_scale, logits, argmax, ws});
+  if (s != MOE_OK) return s;
+  REQ(ws && ws_bytes >= lm_head_workspace_bytes(M, V, H), MOE_ERR_WORKSPACE);
+  DevInfo d;
+  if ((s = dev_info(&d)) != MOE_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  Ctrl c = ctrl_of(ws);
+  MOE_CUDA(cudaMemsetAsync(ws, 0, CTRL_BYTES, st));
+  LMParams p{};
+  p.x = static_cast<const __nv_bfloat16*>(x_bf16);
+  p.M = M;
+  p.V = V;
+  p.H = H;
+  p.w = w_e4m3;
+  p.rs = row_scale;
+  p.logits = logits;
+  p.argmax = argmax;
+  p.keys = c.keys;
+  p.counter = c.lm_counter;
+  p.status = c.status;
+  return launch_lm(p, d, st);
+}
+
+static moe_status_t check_model(const moe_model_t* m) {
+  REQ(m && m->layers, MOE_ERR_INVALID_ARG);
+  REQ(m->n_layers >= 1 && m->n_layers <= 4096, MOE_ERR_UNSUPPORTED_SHAPE);
+  REQ(ok_H_lm(m->H) && ok_I(m->I) && ok_E(m->E) && ok_k(m->top_k, m->E) && ok_Is(m->Is), MOE_ERR_UNSUPPORTED_SHAPE);
+  REQ(m->V >= 1 && m->V <= (1 << 26), MOE_ERR_UNSUPPORTED_SHAPE);
+  REQ(m->rms_eps >= 0.0f, MOE_ERR_INVALID_ARG);
+  moe_status_t s;
+  for (int l = 0; l < m->n_layers; ++l) {
+    const moe_layer_t& L = m->layers[l];
+    if ((s = check_layer_buf(L.router, MOE_FMT_BF16, true)) != MOE_OK) return s;
+    if ((s = check_layer_buf(L.w13_codes, MOE_FMT_MXFP4_CODES, true)) != MOE_OK) return s;
+    if ((s = check_layer_buf(L.w13_scales, MOE_FMT_E8M0_SCALES, true)) != MOE_OK) return s;
+    if ((s = check_layer_buf(L.w2_codes, MOE_FMT_MXFP4_CODES, true)) != MOE_OK) return s;
+    if ((s = check_layer_buf(L.w2_scales, MOE_FMT_E8M0_SCALES, true)) != MOE_OK) return s;
+    if ((s = check_layer_buf(L.shared_w13, MOE_FMT_BF16, m->Is > 0)) != MOE_OK) return s;
+    if ((s = check_layer_buf(L.shared_w2, MOE_FMT_BF16, m->Is > 0)) != MOE_OK) return s;
+  }
+  if ((s = check_layer_buf(m->lm_head, MOE_FMT_E4M3, true)) != MOE_OK) return s;
+  if ((s = check_layer_buf(m->lm_scale, MOE_FMT_F32, true)) != MOE_OK) return s;
+  return MOE_OK;
+}
+
+size_t decode_step_workspace_bytes(const moe_model_t* model, int M) {
+  if (check_model(model) != MOE_OK || !ok_M(M)) return 0;
+  return step_ws(nullptr, M, model->H, model->I, model->E, model->top_k, model->Is).bytes;
+}
+
+moe_status_t decode_step(const moe_model_t* model, const void* x_bf16, int M, float* logits, int32_t* argmax,
+                         const moe_trace_t* trace_opt, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  moe_status_t s = check_model(model);
+  if (s != MOE_OK) return s;
+  REQ(x_bf16 && argmax, MOE_ERR_INVALID_ARG);
+  REQ(ok_M(M), MOE_ERR_UNSUPPORTED_SHAPE);
+  moe_trace_t tr{};
+  if (trace_opt) tr = *trace_opt;
+  if ((s = check_ptrs_aligned({x_bf16, logits, argmax, ws, tr.x, tr.h, tr.ids, tr.w})) != MOE_OK) return s;
+  const int H = model->H, I = model->I, E = model->E, k = model->top_k, Is = model->Is, L = model->n_layers;
+  REQ(ws && ws_bytes >= decode_step_workspace_bytes(model, M), MOE_ERR_WORKSPACE);
+  DevInfo d;
+  if ((s = dev_info(&d)) != MOE_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  Ctrl c = ctrl_of(ws);
+  StepWs w = step_ws(ws, M, H, I, E, k, Is);
+  MOE_CUDA(cudaMemsetAsync(ws, 0, CTRL_BYTES, st));
+  const __nv_bfloat16* x_in = static_cast<const __nv_bfloat16*>(x_bf16);
+  __nv_bfloat16* xt = static_cast<__nv_bfloat16*>(tr.x);
+  EventHook hook;
+  hook.ev = reinterpret_cast<cudaEvent_t*>(tr.events);
+  hook.n = tr.events ? tr.n_events : 0;
+  for (int l = 0; l < L; ++l) {
+    const moe_layer_t& Ly = model->layers[l];
+    const size_t mh = (size_t)M * H, mk = (size_t)M * k;
+    DenseParams p{};
+    p.x = x_in;
+    p.h = w.h;
+    p.mode = l == 0 ? 0 : 1;
+    p.eps = model->rms_eps;
+    p.x_out = w.x_cur;
+    p.x_trace = xt ? xt + l * mh : nullptr;
+    p.h_trace = tr.h ? tr.h + l * mh : nullptr;
+    p.M = M;
+    p.H = H;
+    p.wr = static_cast<const __nv_bfloat16*>(Ly.router.ptr);
+    p.E = E;
+    p.top_k = k;
+    p.n_rtiles = E / 16;
+    p.logits_ws = w.logits;
+    p.ids = w.ids;
+    p.w = w.w;
+    p.ids_trace = tr.ids ? tr.ids + l * mk : nullptr;
+    p.w_trace = tr.w ? tr.w + l * mk : nullptr;
+    p.counter = c.route_counter;
+    p.sw13 = static_cast<const __nv_bfloat16*>(Ly.shared_w13.ptr);
+    p.Is = Is;
+    p.n_stiles = Is / 8;
+    p.a_shared = w.a_shared;
+    if ((s = hook.before(st)) != MOE_OK || (s = launch_dense(p, st)) != MOE_OK || (s = hook.after(st)) != MOE_OK)
+      return s;
+    E13Params a{};
+    a.x = l == 0 ? x_in : w.x_cur;
+    a.M = M;
+    a.H = H;
+    a.I = I;
+    a.E = E;
+    a.top_k = k;
+    a.ids = w.ids;
+    a.w = w.w;
+    a.w13c = static_cast<const uint8_t*>(Ly.w13_codes.ptr);
+    a.w13s = static_cast<const uint8_t*>(Ly.w13_scales.ptr);
+    a.a_routed = w.a_routed;
+    a.status = c.status;
+    if ((s = hook.before(st)) != MOE_OK || (s = launch_e13(a, d, st)) != MOE_OK || (s = hook.after(st)) != MOE_OK)
+      return s;
+    E2Params b{};
+    b.M = M;
+    b.H = H;
+    b.I = I;
+    b.E = E;
+    b.top_k = k;
+    b.Is = Is;
+    b.ids = w.ids;
+    b.w = w.w;
+    b.w2c = static_cast<const uint8_t*>(Ly.w2_codes.ptr);
+    b.w2s = static_cast<const uint8_t*>(Ly.w2_scales.ptr);
+    b.sw2 = static_cast<const __nv_bfloat16*>(Ly.shared_w2.ptr);
+    b.a_routed = w.a_routed;
+    b.a_shared = w.a_shared;
+    b.out = w.h;
+    b.status = c.status;
+    if ((s = hook.before(st)) != MOE_OK || (s = launch_e2(b, d, st)) != MOE_OK || (s = hook.after(st)) != MOE_OK)
+      return s;
+  }
+  if ((s = hook.before(st)) != MOE_OK) return s;
+  k_final_norm<<<1, 256, 0, st>>>(w.h, M, H, model->rms_eps, w.x_final, xt ? xt + (size_t)L * M * H : nullptr,
+                                  tr.h ? tr.h + (size_t)L * M * H : nullptr);
+  MOE_CUDA(cudaGetLastError());
+  if ((s = hook.after(st)) != MOE_OK) return s;
+  LMParams q{};
+  q.x = w.x_final;
+  q.M = M;
+  q.V = model->V;
+  q.H = H;
+  q.w = static_cast<const uint8_t*>(model->lm_head.ptr);
+  q.rs = static_cast<const float*>(model->lm_scale.ptr);
+  q.logits = logits;
+  q.argmax = argmax;
+  q.keys = c.keys;
+  q.counter = c.lm_counter;
+  q.status = c.status;
+  if ((s = hook.before(st)) != MOE_OK || (s = launch_lm(q, d, st)) != MOE_OK) return s;
+  return hook.after(st);
+}
+
+// ---- graph capture of a whole step -------------------------------------------
+struct moe_graph_s {
+  cudaGraph_t graph;
+  cudaGraphExec_t exec;
+};
+
+moe_status_t decode_step_graph_create(const moe_model_t* model, const void* x_bf16, int M, float* logits,
+                                      int32_t* argmax, const moe_trace_t* trace_opt, void* ws, size_t ws_bytes,
+                                      moe_graph_t* out) {
+  REQ(out, MOE_ERR_INVALID_ARG);
+  *out = nullptr;
+  DevInfo d;
+  moe_status_t s = dev_info(&d);  // kernel attributes are set before capture begins
+  if (s != MOE_OK) return s;
+  cudaStream_t cs;
+  MOE_CUDA(cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking));
+  cudaError_t e = cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal);
+  if (e != cudaSuccess) {
+    cudaStreamDestroy(cs);
+    return cuda_fail(e);
+  }
+  s = decode_step(model, x_bf16, M, logits, argmax, trace_opt, ws, ws_bytes, reinterpret_cast<moe_stream_t>(cs));
+  cudaGraph_t g = nullptr;
+  e = cudaStreamEndCapture(cs, &g);
+  cudaStreamDestroy(cs);
+  if (s != MOE_OK) {
+    if (g) cudaGraphDestroy(g);
+    return s;
+  }
+  if (e != cudaSuccess) return cuda_fail(e);
+  cudaGraphExec_t ex;
+  e = cudaGraphInstantiate(&ex, g, 0);
+  if (e != cudaSuccess) {
+    cudaGraphDestroy(g);
+    return cuda_fail(e);
+  }
+  moe_graph_s* h = new (std::nothrow) moe_graph_s{g, ex};
+  if (!h) {
+    cudaGraphExecDestroy(ex);
+    cudaGraphDestroy(g);
+    return MOE_ERR_INVALID_ARG;
+  }
+  *out = h;
+  return MOE_OK;
+}
+
+moe_status_t decode_step_graph_launch(moe_graph_t g, moe_stream_t stream) {
+  REQ(g, MOE_ERR_INVALID_ARG);
+  MOE_CUDA(cudaGraphLaunch(g->exec, reinterpret_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+void decode_step_graph_destroy(moe_graph_t g) {
+  if (!g) return;
+  cudaGraphExecDestroy(g->exec);
+  cudaGraphDestroy(g->graph);
+  delete g;
+}
+
+}  // extern "C"

@@ -1,0 +1,222 @@
+// lmhead_kernels.cuh -- FP8 (e4m3) LM head: online quantisation and the GEMV + argmax.
+//
+// Source: DGX Spark MoE knowledge card (知识卡片：NVIDIA DGX Spark 上提升 MoE 推理吞吐的
+// 三种方法), section 方法/产品要点 item 2: the 157,184 x 2,560 vocabulary projection is
+// stored BF16 in the checkpoint and quantised to FP8 when the head is constructed,
+// which halves the bytes every generated token has to read.
+//
+// Quantisation (once): one fp32 scale per output row, s = amax/448, codes =
+// e4m3 RNE-saturating of w/s (IEEE fp32 divisions, hardware cvt).
+// GEMV: rows stream HBM -> shared memory through bulk copies; e4m3 codes widen to
+// f16 exactly (hardware cvt), the warp tensor-core product accumulates in fp32,
+// the row scale and the activation's power-of-two range shift are applied in
+// the epilogue.  The argmax is folded in: per-thread best -> warp -> block ->
+// one 64-bit atomicMax per token (value key << 32 | ~index, so equal values keep
+// the lowest index) -> the last block converts the keys to indices.
+#pragma once
+
+#include "decode_kernels.cuh"
+
+namespace moe {
+
+// ---------------------------------------------------------------------------
+// k_lm_quantize: one warp per row
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k_lm_quantize(const __nv_bfloat16* __restrict__ w, int V, int H,
+                                                     uint8_t* __restrict__ q, float* __restrict__ rs) {
+  const int lane = threadIdx.x & 31;
+  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (row >= V) return;
+  const __nv_bfloat16* wr = w + row * H;
+  float amax = 0.0f;
+  for (int c = lane; c < H / 8; c += 32) {
+    const uint4 v = *reinterpret_cast<const uint4*>(wr + 8 * c);
+    const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      amax = fmaxf(amax, fabsf(__low2float(b[j])));
+      amax = fmaxf(amax, fabsf(__high2float(b[j])));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const float s = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 448.0f);
+  if (lane == 0) rs[row] = s;
+  uint8_t* qr = q + row * H;
+  for (int c = lane; c < H / 8; c += 32) {
+    const uint4 v = *reinterpret_cast<const uint4*>(wr + 8 * c);
+    const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&v);
+    uint32_t lo = 0, hi = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t pr = f32x2_to_e4m3x2(__fdiv_rn(__low2float(b[j]), s), __fdiv_rn(__high2float(b[j]), s));
+      if (j < 2)
+        lo |= pr << (16 * j);
+      else
+        hi |= pr << (16 * (j - 2));
+    }
+    *reinterpret_cast<uint2*>(qr + 8 * c) = make_uint2(lo, hi);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// k_lm_gemv: 16-row tiles, producer warp + 4 consumer warps
+// ---------------------------------------------------------------------------
+struct LMParams {
+  const __nv_bfloat16* x;  // [M][H]
+  int M, V, H;
+  const uint8_t* w;        // [V][H] e4m3
+  const float* rs;         // [V]
+  float* logits;           // [M][V] or null
+  int32_t* argmax;         // [M]
+  unsigned long long* keys;  // [MAX_M], zero on entry
+  unsigned* counter;         // zero on entry
+  int* status;
+  int stages;
+};
+
+__host__ __device__ inline size_t lm_stage_bytes(int H) {
+  size_t b = 16 * (size_t)padded_stride(H);
+  return (b + 127) / 128 * 128;
+}
+__host__ __device__ inline size_t lm_fixed_bytes(int H) { return 128 + 8 * (size_t)padded_stride(2u * H); }
+
+__device__ __forceinline__ unsigned long long argmax_key(float v, int idx) {
+  return ((unsigned long long)float_key(v) << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)idx);
+}
+
+__global__ void __launch_bounds__(EXPERT_THREADS, 1) k_lm_gemv(LMParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ float s_inv[MAX_M];
+  __shared__ unsigned long long s_best[N_CONSUMERS][MAX_M];
+  __shared__ int s_last;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int M = p.M, V = p.V, H = p.H, S = p.stages;
+  const uint32_t xss = padded_stride(2u * H);
+  const uint32_t ls = padded_stride(H);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+  uint64_t* empty = full + MAX_STAGES;
+  uint8_t* xs = smem + 128;
+  uint8_t* stages = smem + lm_fixed_bytes(H);
+  const size_t sbytes = lm_stage_bytes(H);
+
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const long long T = (V + 15) / 16;
+  const long long start = T * blockIdx.x / gridDim.x;
+  const long long end = T * (blockIdx.x + 1) / gridDim.x;
+  const int nloc = (int)(end - start);
+
+  if (warp == N_CONSUMERS) {
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_first();
+      for (int i = 0; i < nloc; ++i) {
+        const int s = i % S;
+        if (i >= S && !mbar_wait(&empty[s], ((i / S) - 1) & 1, p.status)) break;
+        const long long v0 = (start + i) * 16;
+        const int nrows = (int)min(16LL, (long long)V - v0);
+        uint8_t* st = stages + s * sbytes;
+        mbar_arrive_expect_tx(&full[s], (uint32_t)nrows * H);
+        for (int rr = 0; rr < nrows; ++rr)
+          bulk_g2s(st + rr * ls, p.w + (size_t)(v0 + rr) * H, H, &full[s], pol);
+      }
+      for (int i = (nloc > S ? nloc - S : 0); i < nloc; ++i) mbar_wait(&full[i % S], (i / S) & 1, p.status);
+    }
+    return;
+  }
+
+  stage_x_f16(p.x, M, H, xs, xss, s_inv);
+  unsigned long long bestA = 0ull, bestB = 0ull;  // tokens 2t and 2t+1
+  const int ta = 2 * t, tb = 2 * t + 1;
+  for (int i = warp; i < nloc; i += N_CONSUMERS) {
+    const int s = i % S;
+    if (!mbar_wait(&full[s], (i / S) & 1, p.status)) return;
+    const long long v0 = (start + i) * 16;
+    const uint8_t* st = stages + s * sbytes;
+    float c[4] = {0.f, 0.f, 0.f, 0.f};
+    const bool xact = g < M;
+    for (int j = 0; j < H / 64; ++j) {
+      const uint4 A0 = lds128(st + g * ls + 64 * j + 16 * t);
+      const uint4 A1 = lds128(st + (8 + g) * ls + 64 * j + 16 * t);
+      const uint4 zero = make_uint4(0, 0, 0, 0);
+      const uint4 X0 = xact ? lds128(xs + g * xss + 2 * (64 * j + 16 * t)) : zero;
+      const uint4 X1 = xact ? lds128(xs + g * xss + 2 * (64 * j + 16 * t) + 16) : zero;
+      uint32_t P[8], Q[8];
+      e4m3x4_to_f16x2(A0.x, P[0], P[1]);
+      e4m3x4_to_f16x2(A0.y, P[2], P[3]);
+      e4m3x4_to_f16x2(A0.z, P[4], P[5]);
+      e4m3x4_to_f16x2(A0.w, P[6], P[7]);
+      e4m3x4_to_f16x2(A1.x, Q[0], Q[1]);
+      e4m3x4_to_f16x2(A1.y, Q[2], Q[3]);
+      e4m3x4_to_f16x2(A1.z, Q[4], Q[5]);
+      e4m3x4_to_f16x2(A1.w, Q[6], Q[7]);
+      const uint32_t X[8] = {X0.x, X0.y, X0.z, X0.w, X1.x, X1.y, X1.z, X1.w};
+#pragma unroll
+      for (int s4 = 0; s4 < 4; ++s4) mma_f16(c, P[2 * s4], Q[2 * s4], P[2 * s4 + 1], Q[2 * s4 + 1], X[2 * s4], X[2 * s4 + 1]);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+    const long long va = v0 + g, vb = v0 + g + 8;
+    const float rsa = va < V ? __ldg(p.rs + va) : 0.0f;
+    const float rsb = vb < V ? __ldg(p.rs + vb) : 0.0f;
+    if (ta < M) {
+      const float la = c[0] * rsa * s_inv[ta], lb = c[2] * rsb * s_inv[ta];
+      if (va < V) {
+        if (p.logits) p.logits[(size_t)ta * V + va] = la;
+        bestA = max(bestA, argmax_key(la, (int)va));
+      }
+      if (vb < V) {
+        if (p.logits) p.logits[(size_t)ta * V + vb] = lb;
+        bestA = max(bestA, argmax_key(lb, (int)vb));
+      }
+    }
+    if (tb < M) {
+      const float la = c[1] * rsa * s_inv[tb], lb = c[3] * rsb * s_inv[tb];
+      if (va < V) {
+        if (p.logits) p.logits[(size_t)tb * V + va] = la;
+        bestB = max(bestB, argmax_key(la, (int)va));
+      }
+      if (vb < V) {
+        if (p.logits) p.logits[(size_t)tb * V + vb] = lb;
+        bestB = max(bestB, argmax_key(lb, (int)vb));
+      }
+    }
+  }
+  // lanes with the same t hold the same tokens: reduce over g
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    bestA = max(bestA, __shfl_xor_sync(0xffffffffu, bestA, o));
+    bestB = max(bestB, __shfl_xor_sync(0xffffffffu, bestB, o));
+  }
+  if (g == 0) {
+    s_best[warp][ta] = bestA;
+    s_best[warp][tb] = bestB;
+  }
+  named_barrier(1, 32 * N_CONSUMERS);
+  if (warp == 0 && lane < M) {
+    unsigned long long b = 0ull;
+    for (int w = 0; w < N_CONSUMERS; ++w) b = max(b, s_best[w][lane]);
+    if (b) atomicMax(p.keys + lane, b);
+  }
+  __threadfence();
+  named_barrier(1, 32 * N_CONSUMERS);
+  if (tid == 0) s_last = (atomicAdd(p.counter, 1u) == gridDim.x - 1);
+  named_barrier(1, 32 * N_CONSUMERS);
+  if (s_last) {
+    __threadfence();
+    if (tid < M) {
+      const unsigned long long k = atomicExch(p.keys + tid, 0ull);
+      p.argmax[tid] = (int32_t)(0xFFFFFFFFu - (uint32_t)(k & 0xFFFFFFFFull));
+    }
+    if (tid == 0) *p.counter = 0u;
+  }
+}
+
+}  // namespace moe

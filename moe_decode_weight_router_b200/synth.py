@@ -110,3 +110,17 @@ def bits(t: torch.Tensor):
     if t.dtype == torch.bfloat16:
         return t.view(torch.int16).numpy().view("uint16")
     return t.numpy()
+
+
+def e4m3_codes(shape, seed: int, tid: int = 6_001, device="cpu") -> torch.Tensor:
+    """Uniform E4M3 code bytes with the two NaN codes (0x7F, 0xFF) redrawn as 0x00
+    -- for exercising the FP8 GEMV on its own, independent of any quantiser."""
+    c = uniform_bytes(shape, seed, tid, device)
+    return torch.where((c & 0x7F) == 0x7F, torch.zeros_like(c), c)
+
+
+def row_scales(V: int, seed: int, tid: int = 6_002, device="cpu") -> torch.Tensor:
+    """Positive fp32 row scales, log-uniform in [2^-14, 2^-8]."""
+    g = _gen(seed, tid, device)
+    u = torch.rand((V,), generator=g, device=device, dtype=torch.float32)
+    return torch.exp2(-14.0 + 6.0 * u)

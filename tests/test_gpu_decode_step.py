@@ -1,0 +1,127 @@
+"""GPU parity of the whole decode step (L chained MoE layers + FP8 LM head).
+
+Teacher-forced: each checked layer is recomputed by the oracle from the GPU's own
+bf16 input of that layer (from the step's trace), so a near-tie routing flip in
+one layer cannot make every later layer diverge; the residual update
+h_{l+1} - h_l is compared with the oracle's layer output, the RMSNorm hand-off
+x_{l+1} = bf16(RMSNorm(h_{l+1})) is checked against the oracle's, and the LM head
+against the oracle on the GPU's final x."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from moe_decode_weight_router_b200 import DecodeGraph, DecodeModel, decode_step, decode_step_workspace_bytes, synth
+from tests._bruteforce import bf16_to_f64
+from tests._gpu import MARGIN_FLAG, assert_rows_close, need_gpu, rel_l2_rows
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    need_gpu()
+
+
+def _model(shape, n_layers, V, seed):
+    layers = [synth.layer(shape, seed, l, device="cuda") for l in range(n_layers)]
+    q = synth.e4m3_codes((V, shape.H), seed, device="cuda")
+    s = synth.row_scales(V, seed, device="cuda")
+    return DecodeModel(layers=layers, lm_q=q, lm_s=s, top_k=shape.k)
+
+
+def _fetch(L):
+    def fetch(lst):
+        idx = torch.tensor(lst, dtype=torch.long, device="cuda")
+        return {n: synth.bits(L[n].index_select(0, idx)) for n in ("w13c", "w13s", "w2c", "w2s")}
+    return fetch
+
+
+def _check_step(model, shape, x, res, layers_to_check):
+    xt = res["x_trace"]
+    ht = res["h_trace"].cpu().numpy()
+    ids_t = res["ids_trace"].cpu().numpy()
+    L = len(model.layers)
+    M = x.shape[0]
+    np.testing.assert_array_equal(synth.bits(xt[0]), synth.bits(x))
+    np.testing.assert_array_equal(ht[0], bf16_to_f64(synth.bits(x)).astype(np.float32))
+    for l in layers_to_check:
+        Ly = model.layers[l]
+        xl = synth.bits(xt[l])
+        o_ids, o_w, _, margin = oracle.route(xl, synth.bits(Ly["wr"]), shape.k)
+        ids_use = o_ids.copy()
+        for t in range(M):
+            if margin[t] >= MARGIN_FLAG:
+                assert list(ids_t[l, t]) == list(o_ids[t]), (l, t)
+            else:
+                ids_use[t] = ids_t[l, t]  # flagged near-tie: follow the GPU's choice
+        w_use = oracle.softmax_weights_at(oracle.route(xl, synth.bits(Ly["wr"]), shape.k)[2], ids_use)
+        y_ref = oracle.moe_layer(xl, ids_use, w_use, _fetch(Ly),
+                                 {"sw13": synth.bits(Ly["sw13"]), "sw2": synth.bits(Ly["sw2"])})
+        dh = ht[l + 1].astype(np.float64) - ht[l].astype(np.float64)
+        # the residual update is compared against the layer output; the fp32 residual sum
+        # itself rounds at |h| * 2^-24, far below the tolerance
+        assert_rows_close(dh, y_ref, what=f"layer {l} output")
+        # hand-off: x_{l+1} = bf16(RMSNorm(h_{l+1})) within one bf16 step of the oracle's
+        x_next = oracle.rmsnorm_bf16(ht[l + 1].astype(np.float64))
+        got = bf16_to_f64(synth.bits(xt[l + 1]))
+        ref = bf16_to_f64(x_next)
+        assert np.all(np.abs(got - ref) <= np.abs(ref) * 2.0 ** -7 + 1e-30)
+    # LM head on the GPU's final input
+    logits_ref, am_ref, gap = oracle.lmhead_logits(synth.bits(xt[L]), synth.bits(model.lm_q), model.lm_s.cpu().numpy())
+    assert_rows_close(res["logits"].cpu().numpy(), logits_ref, what="logits")
+    am = res["argmax"].cpu().numpy()
+    for t in range(M):
+        if gap[t] >= MARGIN_FLAG * max(1.0, abs(logits_ref[t, am_ref[t]])):
+            assert am[t] == am_ref[t]
+
+
+@pytest.mark.parametrize("M", [1, 4, 8])
+def test_tiny_chain_all_layers(M):
+    S = synth.TINY
+    model = _model(S, 4, 1000, 21 + M)
+    x = synth.tokens(M, S.H, 21, device="cuda")
+    res = decode_step(model, x, trace=True)
+    torch.cuda.synchronize()
+    _check_step(model, S, x, res, range(4))
+
+
+def test_tiny_chain_free_running_matches_oracle_chain():
+    S = synth.TINY
+    model = _model(S, 3, 1000, 31)
+    x = synth.tokens(2, S.H, 31, device="cuda")
+    res = decode_step(model, x, trace=True)
+    torch.cuda.synchronize()
+    spec = [{"wr": synth.bits(L["wr"]), "experts": _fetch(L),
+             "shared": {"sw13": synth.bits(L["sw13"]), "sw2": synth.bits(L["sw2"])}} for L in model.layers]
+    out = oracle.decode_step(synth.bits(x), spec, synth.bits(model.lm_q), model.lm_s.cpu().numpy(), S.k)
+    if all(np.all(m >= MARGIN_FLAG) for m in out["margin"]):
+        assert_rows_close(res["h_trace"][-1].cpu().numpy(), out["h"], what="free-running h_L")
+        assert_rows_close(res["logits"].cpu().numpy(), out["logits"], what="free-running logits")
+
+
+@pytest.mark.parametrize("M", [1, 4])
+def test_ling_42_layers_sampled(M):
+    """Full size: 42 distinct Ling-shaped layers (~67 GB MXFP4) and the 157,184 x 2,560
+    FP8 LM head, in the same launch configuration the benchmark times; layers
+    0, 1, 20 and 41 and the LM head are recomputed by the oracle."""
+    S = synth.LING
+    model = _model(S, synth.N_LAYERS, synth.VOCAB, 41 + M)
+    x = synth.tokens(M, S.H, 41 + M, device="cuda")
+    res = decode_step(model, x, trace=True)
+    torch.cuda.synchronize()
+    _check_step(model, S, x, res, [0, 1, 20, 41])
+    # the captured graph replays the same step bit for bit (same kernels, same order)
+    ws = torch.empty(decode_step_workspace_bytes(model, M), dtype=torch.uint8, device="cuda")
+    logits = torch.empty((M, synth.VOCAB), dtype=torch.float32, device="cuda")
+    am = torch.empty((M,), dtype=torch.int32, device="cuda")
+    g = DecodeGraph(model, x, logits, am, ws)
+    g.launch()
+    g.launch()
+    torch.cuda.synchronize()
+    g.close()
+    r = rel_l2_rows(logits.cpu().numpy(), res["logits"].cpu().numpy())
+    assert np.all(r < 1e-4)
+    assert np.array_equal(am.cpu().numpy(), res["argmax"].cpu().numpy())
+    del model
+    torch.cuda.empty_cache()
