@@ -203,6 +203,10 @@ def decode_step_workspace_bytes(model: DecodeModel, M: int) -> int:
 def _event_array(events):
     if not events:
         return None, 0
+    for e in events:
+        if not e.cuda_event:  # torch creates the CUDA event lazily, on its first record
+            e.record()
+    torch.cuda.current_stream().synchronize()
     arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
     return arr, len(events)
 
@@ -249,12 +253,18 @@ def decode_step(model: DecodeModel, x: torch.Tensor, *, want_logits: bool = True
 class DecodeGraph:
     """decode_step captured once as a CUDA graph bound to fixed x / logits / argmax buffers."""
 
-    def __init__(self, model: DecodeModel, x: torch.Tensor, logits, argmax, ws, events=None):
+    def __init__(self, model: DecodeModel, x: torch.Tensor, logits, argmax, ws, events=None, trace=None):
+        """``trace``: optional dict with x_trace/h_trace/ids_trace/w_trace device tensors
+        (shapes as decode_step(trace=True) returns) that every replay fills."""
         self.model, self.x, self.logits, self.argmax, self.ws = model, x, logits, argmax, ws
         self._m = model.cstruct()
         self._evs, nev = _event_array(events)
-        self.events = events
-        tr = _abi.Trace(None, None, None, None, self._evs, nev) if self._evs is not None else None
+        self.events, self.trace = events, trace
+        tr = None
+        if trace is not None or self._evs is not None:
+            t = trace or {}
+            tr = _abi.Trace(*(t[n].data_ptr() if n in t else None for n in ("x_trace", "h_trace", "ids_trace",
+                                                                              "w_trace")), self._evs, nev)
         h = ctypes.c_void_p()
         _check("decode_step_graph_create", _lib().decode_step_graph_create(
             ctypes.byref(self._m), _ptr(x), x.shape[0], _ptr(logits), _ptr(argmax),

@@ -37,7 +37,20 @@ size_t up256(size_t b) { return (b + 255) / 256 * 256; }
 struct DevInfo {
   int sms = 0;
   int smem_optin = 0;
+  // largest dynamic shared memory per kernel family: the opt-in limit minus the
+  // kernel's own static shared memory
+  int dyn_dense = 0, dyn_e13 = 0, dyn_e2 = 0, dyn_lm = 0;
 };
+
+template <class K>
+cudaError_t allow_dyn_smem(K kernel, int optin, int* dyn) {
+  cudaFuncAttributes a;
+  cudaError_t e = cudaFuncGetAttributes(&a, kernel);
+  if (e != cudaSuccess) return e;
+  const int lim = optin - static_cast<int>(a.sharedSizeBytes);
+  *dyn = (*dyn == 0 || lim < *dyn) ? lim : *dyn;
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
+}
 
 // Per-device launch facts and one-time kernel attributes (opt-in shared memory).
 moe_status_t dev_info(DevInfo* out) {
@@ -53,16 +66,16 @@ moe_status_t dev_info(DevInfo* out) {
     MOE_CUDA(cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev));
     MOE_CUDA(cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev));
     const int lim = d.smem_optin;
-    MOE_CUDA(cudaFuncSetAttribute(k_dense, cudaFuncAttributeMaxDynamicSharedMemorySize, lim));
-    MOE_CUDA(cudaFuncSetAttribute(k_experts13<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim));
-    MOE_CUDA(cudaFuncSetAttribute(k_experts13<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim));
-    MOE_CUDA(cudaFuncSetAttribute(k_experts13<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim));
-    MOE_CUDA(cudaFuncSetAttribute(k_experts13<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim));
-    MOE_CUDA(cudaFuncSetAttribute(k_experts2<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim));
-    MOE_CUDA(cudaFuncSetAttribute(k_experts2<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim));
-    MOE_CUDA(cudaFuncSetAttribute(k_experts2<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim));
-    MOE_CUDA(cudaFuncSetAttribute(k_experts2<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim));
-    MOE_CUDA(cudaFuncSetAttribute(k_lm_gemv, cudaFuncAttributeMaxDynamicSharedMemorySize, lim));
+    MOE_CUDA(allow_dyn_smem(k_dense, lim, &d.dyn_dense));
+    MOE_CUDA(allow_dyn_smem(k_experts13<1>, lim, &d.dyn_e13));
+    MOE_CUDA(allow_dyn_smem(k_experts13<2>, lim, &d.dyn_e13));
+    MOE_CUDA(allow_dyn_smem(k_experts13<3>, lim, &d.dyn_e13));
+    MOE_CUDA(allow_dyn_smem(k_experts13<4>, lim, &d.dyn_e13));
+    MOE_CUDA(allow_dyn_smem(k_experts2<1>, lim, &d.dyn_e2));
+    MOE_CUDA(allow_dyn_smem(k_experts2<2>, lim, &d.dyn_e2));
+    MOE_CUDA(allow_dyn_smem(k_experts2<3>, lim, &d.dyn_e2));
+    MOE_CUDA(allow_dyn_smem(k_experts2<4>, lim, &d.dyn_e2));
+    MOE_CUDA(allow_dyn_smem(k_lm_gemv, lim, &d.dyn_lm));
     cache[dev] = d;
     ready[dev] = true;
   }
@@ -163,16 +176,16 @@ moe_status_t launch_dense(const DenseParams& p, cudaStream_t st) {
 // and item i uses stage i % S, so with S % NC == 0 the warp waiting on a stage's
 // next phase is the warp that consumed its previous phase -- the mbarrier parity
 // it waits on can never alias a phase that has not completed yet.
-int stages_for(const DevInfo& d, size_t fixed, size_t stage) {
-  if ((size_t)d.smem_optin <= fixed) return 0;
-  size_t s = ((size_t)d.smem_optin - fixed) / stage;
+int stages_for(int dyn_limit, size_t fixed, size_t stage) {
+  if ((size_t)dyn_limit <= fixed) return 0;
+  size_t s = ((size_t)dyn_limit - fixed) / stage;
   if (s > (size_t)MAX_STAGES) s = MAX_STAGES;
   return (int)(s / N_CONSUMERS * N_CONSUMERS);
 }
 
 moe_status_t launch_e13(E13Params p, const DevInfo& d, cudaStream_t st) {
   const size_t fixed = e13_fixed_bytes(p.H), stage = e13_stage_bytes(p.H);
-  p.stages = stages_for(d, fixed, stage);
+  p.stages = stages_for(d.dyn_e13, fixed, stage);
   if (p.stages < N_CONSUMERS) return MOE_ERR_UNSUPPORTED_SHAPE;
   const size_t smem = fixed + (size_t)p.stages * stage;
   const int grid = d.sms;
@@ -188,7 +201,7 @@ moe_status_t launch_e13(E13Params p, const DevInfo& d, cudaStream_t st) {
 
 moe_status_t launch_e2(E2Params p, const DevInfo& d, cudaStream_t st) {
   const size_t fixed = e2_fixed_bytes(p.M, p.I, p.Is), stage = e2_stage_bytes(p.I, p.Is);
-  p.stages = stages_for(d, fixed, stage);
+  p.stages = stages_for(d.dyn_e2, fixed, stage);
   if (p.stages < N_CONSUMERS) return MOE_ERR_UNSUPPORTED_SHAPE;
   const size_t smem = fixed + (size_t)p.stages * stage;
   // Each block's contiguous item range must touch at most E2_MAX_LOCAL_SLOTS experts.
@@ -209,7 +222,7 @@ moe_status_t launch_e2(E2Params p, const DevInfo& d, cudaStream_t st) {
 
 moe_status_t launch_lm(LMParams p, const DevInfo& d, cudaStream_t st) {
   const size_t fixed = lm_fixed_bytes(p.H), stage = lm_stage_bytes(p.H);
-  p.stages = stages_for(d, fixed, stage);
+  p.stages = stages_for(d.dyn_lm, fixed, stage);
   if (p.stages < N_CONSUMERS) return MOE_ERR_UNSUPPORTED_SHAPE;
   const size_t smem = fixed + (size_t)p.stages * stage;
   const long long T = (p.V + 15) / 16;
@@ -224,12 +237,15 @@ struct EventHook {
   cudaEvent_t* ev = nullptr;
   int n = 0;
   int i = 0;
+  // External records: under stream capture they become event-record graph nodes
+  // (a plain record would only mark a capture dependency); outside capture they are
+  // ordinary records.
   moe_status_t before(cudaStream_t st) {
-    if (ev && 2 * i + 1 < n) MOE_CUDA(cudaEventRecord(ev[2 * i], st));
+    if (ev && 2 * i + 1 < n) MOE_CUDA(cudaEventRecordWithFlags(ev[2 * i], st, cudaEventRecordExternal));
     return MOE_OK;
   }
   moe_status_t after(cudaStream_t st) {
-    if (ev && 2 * i + 1 < n) MOE_CUDA(cudaEventRecord(ev[2 * i + 1], st));
+    if (ev && 2 * i + 1 < n) MOE_CUDA(cudaEventRecordWithFlags(ev[2 * i + 1], st, cudaEventRecordExternal));
     ++i;
     return MOE_OK;
   }

@@ -111,17 +111,22 @@ def test_ling_42_layers_sampled(M):
     res = decode_step(model, x, trace=True)
     torch.cuda.synchronize()
     _check_step(model, S, x, res, [0, 1, 20, 41])
-    # the captured graph replays the same step bit for bit (same kernels, same order)
+    # the captured graph (one launch per step) is checked against the oracle the same way,
+    # through the trace it fills; two runs need not agree bit for bit with each other
+    # (fp32 atomic accumulation order), each must agree with the oracle
     ws = torch.empty(decode_step_workspace_bytes(model, M), dtype=torch.uint8, device="cuda")
-    logits = torch.empty((M, synth.VOCAB), dtype=torch.float32, device="cuda")
-    am = torch.empty((M,), dtype=torch.int32, device="cuda")
-    g = DecodeGraph(model, x, logits, am, ws)
+    res_g = {"logits": torch.empty((M, synth.VOCAB), dtype=torch.float32, device="cuda"),
+             "argmax": torch.empty((M,), dtype=torch.int32, device="cuda")}
+    L = len(model.layers)
+    res_g["x_trace"] = torch.empty((L + 1, M, S.H), dtype=torch.bfloat16, device="cuda")
+    res_g["h_trace"] = torch.empty((L + 1, M, S.H), dtype=torch.float32, device="cuda")
+    res_g["ids_trace"] = torch.empty((L, M, S.k), dtype=torch.int32, device="cuda")
+    res_g["w_trace"] = torch.empty((L, M, S.k), dtype=torch.float32, device="cuda")
+    g = DecodeGraph(model, x, res_g["logits"], res_g["argmax"], ws, trace=res_g)
     g.launch()
     g.launch()
     torch.cuda.synchronize()
     g.close()
-    r = rel_l2_rows(logits.cpu().numpy(), res["logits"].cpu().numpy())
-    assert np.all(r < 1e-4)
-    assert np.array_equal(am.cpu().numpy(), res["argmax"].cpu().numpy())
+    _check_step(model, S, x, res_g, [0, 41])
     del model
     torch.cuda.empty_cache()
