@@ -165,6 +165,26 @@ MOE_API moe_status_t lm_head_fp8_gemv(const void* x_bf16, int M, int V, int H, c
                               const float* row_scale, float* logits, int32_t* argmax,
                               void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* Allocation-free variant of lm_head_fp8_gemv (no counterpart on the pages; it
+ * exists for integration).  Some callers cannot hand this library any scratch
+ * memory: an operator slot that passes only input and output tensors and has no
+ * workspace argument, a runtime whose device memory is fixed at start-up and may
+ * not grow, or code that must not call cudaMalloc because it synchronises the
+ * device.  This entry point takes inputs and outputs only and allocates nothing;
+ * the 256-byte control block the GEMV needs (argmax keys of up to 8 tokens, a
+ * completion counter, the status word) is a static device array inside the library,
+ * one per device that loads it, held until the process exits.
+ *   Arguments, layouts, results and errors: as lm_head_fp8_gemv.  M above 8 (the
+ *   keys the static block holds) returns MOE_ERR_UNSUPPORTED_SHAPE.
+ *   The first call on a device looks up the array's device address (a one-time,
+ *   host-side set-up): make that first call before any stream capture.
+ *   Every call shares the one array and clears it on entry, so calls whose GPU
+ *   work overlaps (other streams, other host threads, the same device) race and
+ *   corrupt each other's argmax; serialise them. */
+MOE_API moe_status_t lm_head_fp8_gemv_noalloc(const void* x_bf16, int M, int V, int H,
+                                              const uint8_t* w_e4m3, const float* row_scale,
+                                              float* logits, int32_t* argmax, moe_stream_t stream);
+
 /* ------------------------------------------------------------------------- */
 /* Whole decode step: L MoE layers + FP8 LM head                              */
 /* ------------------------------------------------------------------------- */

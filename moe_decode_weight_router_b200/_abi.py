@@ -51,6 +51,7 @@ SIGNATURES = {
     "lm_head_fp8_quantize": (I, [P, I, I, P, P, P]),
     "lm_head_workspace_bytes": (Z, [I, I, I]),
     "lm_head_fp8_gemv": (I, [P, I, I, I, P, P, P, P, P, Z, P]),
+    "lm_head_fp8_gemv_noalloc": (I, [P, I, I, I, P, P, P, P, P]),
     "decode_step_workspace_bytes": (Z, [ctypes.POINTER(Model), I]),
     "decode_step": (I, [ctypes.POINTER(Model), P, I, P, P, ctypes.POINTER(Trace), P, Z, P]),
     "decode_step_graph_create": (I, [ctypes.POINTER(Model), P, I, P, P, ctypes.POINTER(Trace), P, Z,

@@ -159,6 +159,23 @@ def lm_head_fp8_gemv(x, q, s, *, want_logits: bool = True, ws=None, out=None, st
     return logits, am
 
 
+def lm_head_fp8_gemv_noalloc(x, q, s, *, want_logits: bool = True, out=None, stream=None):
+    """As lm_head_fp8_gemv, through the entry point that takes no workspace (the
+    library's static per-device control block; calls must not overlap)."""
+    _dev_bf16(x, "x")
+    M, H = x.shape
+    V = q.shape[0]
+    dev = x.device
+    if out is None:
+        logits = torch.empty((M, V), dtype=torch.float32, device=dev) if want_logits else None
+        am = torch.empty((M,), dtype=torch.int32, device=dev)
+    else:
+        logits, am = out
+    _check("lm_head_fp8_gemv_noalloc", _lib().lm_head_fp8_gemv_noalloc(
+        _ptr(x), M, V, H, _ptr(q), _ptr(s), _ptr(logits), _ptr(am), _stream(stream)))
+    return logits, am
+
+
 # ---------------------------------------------------------------------------
 # Whole decode step
 # ---------------------------------------------------------------------------

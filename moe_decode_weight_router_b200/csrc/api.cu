@@ -648,3 +648,62 @@ void decode_step_graph_destroy(moe_graph_t g) {
 }
 
 }  // extern "C"
+
+// ---- allocation-free LM head ---------------------------------------------------
+// The control block lm_head_fp8_gemv keeps in the caller's workspace (status word,
+// completion counter, argmax keys of up to MAX_M tokens) lives here instead: one
+// 256-byte copy per device that loads the library, kept until the process exits.
+static __device__ __align__(256) unsigned char g_lm_noalloc_scratch[CTRL_BYTES];
+
+namespace {
+// Device address of g_lm_noalloc_scratch on the current device.  The name is only a
+// host-side stand-in for the array, so the address is looked up once per device
+// (with that device current) and cached.
+moe_status_t lm_noalloc_scratch(void** out) {
+  static std::mutex mu;
+  static void* addr[64];
+  static bool ready[64] = {};
+  int dev = 0;
+  MOE_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return MOE_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!ready[dev]) {
+    void* p = nullptr;
+    MOE_CUDA(cudaGetSymbolAddress(&p, g_lm_noalloc_scratch));
+    addr[dev] = p;
+    ready[dev] = true;
+  }
+  *out = addr[dev];
+  return MOE_OK;
+}
+}  // namespace
+
+extern "C" moe_status_t lm_head_fp8_gemv_noalloc(const void* x_bf16, int M, int V, int H, const uint8_t* w_e4m3,
+                                                 const float* row_scale, float* logits, int32_t* argmax,
+                                                 moe_stream_t stream) {
+  REQ(x_bf16 && w_e4m3 && row_scale && argmax, MOE_ERR_INVALID_ARG);
+  // the static control block holds argmax keys for at most MAX_M (8) tokens
+  REQ(ok_M(M) && V >= 1 && V <= (1 << 26) && ok_H_lm(H), MOE_ERR_UNSUPPORTED_SHAPE);
+  moe_status_t s = check_ptrs_aligned({x_bf16, w_e4m3, row_scale, logits, argmax});
+  if (s != MOE_OK) return s;
+  DevInfo d;
+  if ((s = dev_info(&d)) != MOE_OK) return s;
+  void* scratch = nullptr;
+  if ((s = lm_noalloc_scratch(&scratch)) != MOE_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  Ctrl c = ctrl_of(scratch);
+  MOE_CUDA(cudaMemsetAsync(scratch, 0, CTRL_BYTES, st));  // counters and keys start at zero
+  LMParams p{};
+  p.x = static_cast<const __nv_bfloat16*>(x_bf16);
+  p.M = M;
+  p.V = V;
+  p.H = H;
+  p.w = w_e4m3;
+  p.rs = row_scale;
+  p.logits = logits;
+  p.argmax = argmax;
+  p.keys = c.keys;
+  p.counter = c.lm_counter;
+  p.status = c.status;
+  return launch_lm(p, d, st);
+}
