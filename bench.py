@@ -51,6 +51,7 @@ def parse_args():
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of CPU-oracle time for cpu_baseline")
     ap.add_argument("--ref-layers", type=int, default=4, help="layers per reference-arm step")
     ap.add_argument("--skip-m4", action="store_true")
+    ap.add_argument("--per-layer", action="store_true", help="force the three-kernels-per-layer path")
     return ap.parse_args()
 
 
@@ -162,7 +163,8 @@ def run_ours(args, rank, world, local_rank):
     import torch.distributed as dist
 
     from moe_decode_weight_router_b200 import (DecodeGraph, DecodeModel, build, decode_step,
-                                               decode_step_workspace_bytes, lm_head_fp8_quantize, synth)
+                                               decode_step_launch_names, decode_step_workspace_bytes,
+                                               lm_head_fp8_quantize, synth)
 
     build.build()
     torch.cuda.set_device(local_rank)
@@ -177,7 +179,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     del w_lm
     torch.cuda.empty_cache()
-    model = DecodeModel(layers=layers, lm_q=lm_q, lm_s=lm_s, top_k=S.k)
+    model = DecodeModel(layers=layers, lm_q=lm_q, lm_s=lm_s, top_k=S.k, step_path=1 if args.per_layer else 0)
 
     def barrier():
         if world > 1:
@@ -248,6 +250,7 @@ def run_ours(args, rank, world, local_rank):
         bytes_all = sum_over_ranks(bytes_rank)
         ms_step = ms_total / K
         res = {
+            "launches_per_step": len(decode_step_launch_names(model, M)),
             "ms_per_step": ms_step,
             "us_per_step": 1000.0 * ms_step,
             "gbps": bytes_all / (ms_total * 1e-3) / 1e9,
@@ -283,10 +286,9 @@ def run_ours(args, rank, world, local_rank):
 
         # live per-kernel timing: events around every launch inside a captured step
         if M == 1:
-            n_launch = 3 * L + 2
-            evs = [torch.cuda.Event(enable_timing=True) for _ in range(2 * n_launch)]
+            names = decode_step_launch_names(model, M)
+            evs = [torch.cuda.Event(enable_timing=True) for _ in range(2 * len(names))]
             gk = DecodeGraph(model, x_buf, logits, am, ws, events=evs)
-            names = ["k_dense", "k_experts13", "k_experts2"] * L + ["k_final_norm", "k_lm_gemv"]
             tot = {n: 0.0 for n in set(names)}
             cnt = {n: 0 for n in set(names)}
             kb = {n: 0.0 for n in set(names)}
@@ -299,14 +301,18 @@ def run_ours(args, rank, world, local_rank):
                 for j, n in enumerate(names):
                     tot[n] += evs[2 * j].elapsed_time(evs[2 * j + 1])
                     cnt[n] += 1
-                    lay = min(j // 3, L - 1)
-                    kb[n] += kernel_bytes(S, M, nu[lay], V)[n]
+                    if n == "k_step":
+                        kb[n] += sum(layer_bytes(S, M, u) for u in nu)
+                    else:
+                        lay = min(j // 3, L - 1)
+                        kb[n] += kernel_bytes(S, M, nu[lay], V)[n]
             gk.close()
             ker = {}
             for n in tot:
                 avg_ms = tot[n] / cnt[n]
                 ker[n] = {"launches_per_step": cnt[n] // reps, "avg_us": 1000 * avg_ms,
-                          "share": tot[n] / sum(tot.values()), "gbps": (kb[n] / cnt[n]) / (avg_ms * 1e-3) / 1e9}
+                          "share": tot[n] / sum(tot.values()), "gbps": (kb[n] / cnt[n]) / (avg_ms * 1e-3) / 1e9,
+                          "bytes_per_launch": kb[n] / cnt[n]}
             res["kernels"] = ker
         results[M] = res
 
@@ -477,7 +483,7 @@ def main():
                        "l2": "inputs larger than L2: ~67 GB of distinct layer weights streamed per step",
                        "parallelism": "replicas" if world > 1 else "single GPU"},
             "e2e": {k: v for k, v in r1["e2e"].items()},
-            "gpu_launches": (3 * args.layers + 2) * args.steps,
+            "gpu_launches": r1["launches_per_step"] * args.steps,
             "clocks": r1["clocks"],
             "roofline": roof,
             "kernels": ker,

@@ -223,7 +223,15 @@ typedef struct {
   const moe_layer_t* layers;  /* HOST array of n_layers entries */
   moe_buf_t lm_head;          /* [V][H] e4m3 codes (from lm_head_fp8_quantize) */
   moe_buf_t lm_scale;         /* [V] fp32 row scales */
+  int step_path;              /* MOE_STEP_AUTO or MOE_STEP_PER_LAYER */
 } moe_model_t;
+
+/* How decode_step runs the layers.  AUTO: one persistent kernel for all layers
+ * (cooperative launch, one block per SM) followed by the LM-head kernel, when the
+ * model fits it (n_layers <= 64, H % 128 == 0); otherwise three kernels per layer.
+ * PER_LAYER: always three kernels per layer (router + shared W13, routed W13,
+ * W2 + combine), a final RMSNorm kernel and the LM head. */
+enum { MOE_STEP_AUTO = 0, MOE_STEP_PER_LAYER = 1 };
 
 /* Optional debug trace of a decode step (device buffers, any may be NULL):
  *   x  [L+1][M][H] bf16: each layer's input and the LM head's input
@@ -233,7 +241,11 @@ typedef struct {
  *     the caller) recorded on the step's stream around every kernel: events[2i] before
  *     and events[2i+1] after launch i, launches ordered (router+shared W13, routed W13,
  *     W2+combine) per layer, then the final RMSNorm, then the LM head; 3L+2 launches.
- *     Fewer events than 2(3L+2) record the first n_events/2 launches only. */
+ *     Fewer events than 2 x (launch count) record the first n_events/2 launches only
+ *     (decode_step_launch_names gives the launches).
+ *   timeline: NULL or [2*L*16 + 4*4096] uint64 %globaltimer stamps (ns), for profiling
+ *     the persistent path: [2][L][16] phase boundaries of blocks 0 and G-1, then block 0's
+ *     first 4096 weight items as (issued, data ready, done, wait started). */
 typedef struct {
   void* x;
   float* h;
@@ -241,9 +253,16 @@ typedef struct {
   float* w;
   void** events;
   int n_events;
+  unsigned long long* timeline;
 } moe_trace_t;
 
 MOE_API size_t decode_step_workspace_bytes(const moe_model_t* model, int M);
+
+/* The kernels one decode_step call launches, in order (the order of the trace's
+ * event pairs): writes up to max_names static name strings into names (may be NULL)
+ * and returns the count, or -1 for an invalid model / M.  Needs the CUDA device
+ * (the choice of path depends on it). */
+MOE_API int decode_step_launch_names(const moe_model_t* model, int M, const char** names, int max_names);
 
 /* One decode step for an M-token window (M = 1 decode, M = 4 verify window):
  *   h_0 = fp32(x);  for l < L:  x_l = (l == 0 ? x : bf16(RMSNorm(h_l))),

@@ -31,11 +31,14 @@ class Layer(ctypes.Structure):
 class Model(ctypes.Structure):
     _fields_ = [("n_layers", I), ("H", I), ("I", I), ("E", I), ("top_k", I), ("Is", I), ("V", I),
                 ("rms_eps", ctypes.c_float), ("layers", ctypes.POINTER(Layer)), ("lm_head", Buf),
-                ("lm_scale", Buf)]
+                ("lm_scale", Buf), ("step_path", I)]
+
+STEP_AUTO, STEP_PER_LAYER = 0, 1
 
 
 class Trace(ctypes.Structure):
-    _fields_ = [("x", P), ("h", P), ("ids", P), ("w", P), ("events", ctypes.POINTER(P)), ("n_events", I)]
+    _fields_ = [("x", P), ("h", P), ("ids", P), ("w", P), ("events", ctypes.POINTER(P)), ("n_events", I),
+                ("timeline", P)]
 
 
 # name -> (restype, argtypes); every symbol the header declares
@@ -53,6 +56,7 @@ SIGNATURES = {
     "lm_head_fp8_gemv": (I, [P, I, I, I, P, P, P, P, P, Z, P]),
     "lm_head_fp8_gemv_noalloc": (I, [P, I, I, I, P, P, P, P, P]),
     "decode_step_workspace_bytes": (Z, [ctypes.POINTER(Model), I]),
+    "decode_step_launch_names": (I, [ctypes.POINTER(Model), I, ctypes.POINTER(ctypes.c_char_p), I]),
     "decode_step": (I, [ctypes.POINTER(Model), P, I, P, P, ctypes.POINTER(Trace), P, Z, P]),
     "decode_step_graph_create": (I, [ctypes.POINTER(Model), P, I, P, P, ctypes.POINTER(Trace), P, Z,
                                      ctypes.POINTER(P)]),

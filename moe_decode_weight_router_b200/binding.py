@@ -188,6 +188,7 @@ class DecodeModel:
     top_k: int
     rms_eps: float = 1e-6
     lm_fmt: int = _abi.FMT_E4M3
+    step_path: int = _abi.STEP_AUTO
     _keep: list = field(default_factory=list, repr=False)
 
     def cstruct(self) -> _abi.Model:
@@ -207,9 +208,21 @@ class DecodeModel:
                 arr[i].shared_w2 = _abi.Buf(L["sw2"].data_ptr(), _abi.FMT_BF16)
         m = _abi.Model(len(self.layers), H, I, E, self.top_k, Is, self.lm_q.shape[0], self.rms_eps,
                        ctypes.cast(arr, ctypes.POINTER(_abi.Layer)),
-                       _abi.Buf(self.lm_q.data_ptr(), self.lm_fmt), _abi.Buf(self.lm_s.data_ptr(), _abi.FMT_F32))
+                       _abi.Buf(self.lm_q.data_ptr(), self.lm_fmt), _abi.Buf(self.lm_s.data_ptr(), _abi.FMT_F32),
+                       self.step_path)
         self._keep = [arr, m]
         return m
+
+
+def decode_step_launch_names(model: DecodeModel, M: int) -> list:
+    """Names of the kernels one decode_step launches, in launch order."""
+    m = model.cstruct()
+    n = _lib().decode_step_launch_names(ctypes.byref(m), M, None, 0)
+    if n < 0:
+        raise MoeError("decode_step_launch_names", 1)
+    arr = (ctypes.c_char_p * n)()
+    _lib().decode_step_launch_names(ctypes.byref(m), M, arr, n)
+    return [a.decode() for a in arr]
 
 
 def decode_step_workspace_bytes(model: DecodeModel, M: int) -> int:
@@ -229,7 +242,7 @@ def _event_array(events):
 
 
 def decode_step(model: DecodeModel, x: torch.Tensor, *, want_logits: bool = True, trace: bool = False, ws=None,
-                out=None, stream=None, events=None):
+                out=None, stream=None, events=None, timeline=None):
     """One decode step.  Returns dict(logits, argmax[, trace tensors]).
 
     ``events``: optional list of torch.cuda.Event(enable_timing=True), recorded in
@@ -258,6 +271,10 @@ def decode_step(model: DecodeModel, x: torch.Tensor, *, want_logits: bool = True
                         res["w_trace"].data_ptr(), evs, nev)
     elif evs is not None:
         tr = _abi.Trace(None, None, None, None, evs, nev)
+    if timeline is not None:
+        if tr is None:
+            tr = _abi.Trace(None, None, None, None, None, 0)
+        tr.timeline = timeline.data_ptr()
     if ws is None:
         ws = _ws(_lib().decode_step_workspace_bytes(ctypes.byref(m), M), dev)
     _check("decode_step", _lib().decode_step(ctypes.byref(m), _ptr(x), M, _ptr(logits), _ptr(am),

@@ -13,6 +13,7 @@
 #include "../../include/moe_decode.h"
 #include "decode_kernels.cuh"
 #include "lmhead_kernels.cuh"
+#include "step_kernel.cuh"
 
 using namespace moe;
 
@@ -39,7 +40,8 @@ struct DevInfo {
   int smem_optin = 0;
   // largest dynamic shared memory per kernel family: the opt-in limit minus the
   // kernel's own static shared memory
-  int dyn_dense = 0, dyn_e13 = 0, dyn_e2 = 0, dyn_lm = 0;
+  int dyn_dense = 0, dyn_e13 = 0, dyn_e2 = 0, dyn_lm = 0, dyn_step = 0;
+  int coop = 0;
 };
 
 template <class K>
@@ -67,15 +69,11 @@ moe_status_t dev_info(DevInfo* out) {
     MOE_CUDA(cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev));
     const int lim = d.smem_optin;
     MOE_CUDA(allow_dyn_smem(k_dense, lim, &d.dyn_dense));
-    MOE_CUDA(allow_dyn_smem(k_experts13<1>, lim, &d.dyn_e13));
-    MOE_CUDA(allow_dyn_smem(k_experts13<2>, lim, &d.dyn_e13));
-    MOE_CUDA(allow_dyn_smem(k_experts13<3>, lim, &d.dyn_e13));
-    MOE_CUDA(allow_dyn_smem(k_experts13<4>, lim, &d.dyn_e13));
-    MOE_CUDA(allow_dyn_smem(k_experts2<1>, lim, &d.dyn_e2));
-    MOE_CUDA(allow_dyn_smem(k_experts2<2>, lim, &d.dyn_e2));
-    MOE_CUDA(allow_dyn_smem(k_experts2<3>, lim, &d.dyn_e2));
-    MOE_CUDA(allow_dyn_smem(k_experts2<4>, lim, &d.dyn_e2));
+    MOE_CUDA(allow_dyn_smem(k_experts13, lim, &d.dyn_e13));
+    MOE_CUDA(allow_dyn_smem(k_experts2, lim, &d.dyn_e2));
     MOE_CUDA(allow_dyn_smem(k_lm_gemv, lim, &d.dyn_lm));
+    MOE_CUDA(allow_dyn_smem(k_step, lim, &d.dyn_step));
+    MOE_CUDA(cudaDeviceGetAttribute(&d.coop, cudaDevAttrCooperativeLaunch, dev));
     cache[dev] = d;
     ready[dev] = true;
   }
@@ -128,6 +126,8 @@ ExpertsWs experts_ws(void* ws, int M, int H, int I, int E, int k, int Is) {
 }
 
 struct StepWs {
+  unsigned* ctr;
+  size_t ctrl_bytes;  // control block + per-layer counters, cleared every step
   float* logits;
   int32_t* ids;
   float* w;
@@ -138,10 +138,13 @@ struct StepWs {
   __nv_bfloat16* x_final;
   size_t bytes;
 };
-StepWs step_ws(void* ws, int M, int H, int I, int E, int k, int Is) {
+StepWs step_ws(void* ws, int L, int M, int H, int I, int E, int k, int Is) {
   uint8_t* b = static_cast<uint8_t*>(ws);
   size_t off = CTRL_BYTES;
   StepWs s{};
+  s.ctr = reinterpret_cast<unsigned*>(b + off);
+  off += up256((size_t)L * CTR_PER_LAYER * sizeof(unsigned));
+  s.ctrl_bytes = off;
   s.logits = reinterpret_cast<float*>(b + off);
   off += up256((size_t)M * E * 4);
   s.ids = reinterpret_cast<int32_t*>(b + off);
@@ -155,7 +158,7 @@ StepWs step_ws(void* ws, int M, int H, int I, int E, int k, int Is) {
   s.a_shared = reinterpret_cast<float*>(b + off);
   off += up256((size_t)M * Is * 4);
   s.a_routed = reinterpret_cast<float*>(b + off);
-  off += up256(slots_of(M, E, k) * M * I * 4);
+  off += up256((size_t)MAX_SLOTS * M * I * 4);
   s.x_final = reinterpret_cast<__nv_bfloat16*>(b + off);
   off += up256((size_t)M * H * 2);
   s.bytes = off;
@@ -189,12 +192,7 @@ moe_status_t launch_e13(E13Params p, const DevInfo& d, cudaStream_t st) {
   if (p.stages < N_CONSUMERS) return MOE_ERR_UNSUPPORTED_SHAPE;
   const size_t smem = fixed + (size_t)p.stages * stage;
   const int grid = d.sms;
-  switch ((p.M + 1) / 2) {
-    case 1: k_experts13<1><<<grid, EXPERT_THREADS, smem, st>>>(p); break;
-    case 2: k_experts13<2><<<grid, EXPERT_THREADS, smem, st>>>(p); break;
-    case 3: k_experts13<3><<<grid, EXPERT_THREADS, smem, st>>>(p); break;
-    default: k_experts13<4><<<grid, EXPERT_THREADS, smem, st>>>(p); break;
-  }
+  k_experts13<<<grid, EXPERT_THREADS, smem, st>>>(p);
   MOE_CUDA(cudaGetLastError());
   return MOE_OK;
 }
@@ -210,12 +208,7 @@ moe_status_t launch_e2(E2Params p, const DevInfo& d, cudaStream_t st) {
   const long long Tmax = (long long)slots_of(p.M, p.E, p.top_k) * htiles + htiles * nch;
   long long grid = d.sms;
   while ((Tmax + grid - 1) / grid > (E2_MAX_LOCAL_SLOTS - 1) * htiles + 1) grid *= 2;
-  switch ((p.M + 1) / 2) {
-    case 1: k_experts2<1><<<(int)grid, EXPERT_THREADS, smem, st>>>(p); break;
-    case 2: k_experts2<2><<<(int)grid, EXPERT_THREADS, smem, st>>>(p); break;
-    case 3: k_experts2<3><<<(int)grid, EXPERT_THREADS, smem, st>>>(p); break;
-    default: k_experts2<4><<<(int)grid, EXPERT_THREADS, smem, st>>>(p); break;
-  }
+  k_experts2<<<(int)grid, EXPERT_THREADS, smem, st>>>(p);
   MOE_CUDA(cudaGetLastError());
   return MOE_OK;
 }
@@ -229,6 +222,34 @@ moe_status_t launch_lm(LMParams p, const DevInfo& d, cudaStream_t st) {
   const int grid = (int)(T < d.sms ? T : d.sms);
   k_lm_gemv<<<grid, EXPERT_THREADS, smem, st>>>(p);
   MOE_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
+
+// The whole-step persistent kernel serves the model when it fits: at most
+// STEP_MAX_LAYERS layers, H a multiple of 128 (router/shared tiles split into four
+// 32-column-aligned quarters), cooperative launch available, and a shared-memory ring
+// of at least N_CONSUMERS stages next to the activation region.
+bool use_persistent(const moe_model_t& m, int M, const DevInfo& d, int* stages) {
+  if (m.step_path == MOE_STEP_PER_LAYER) return false;
+  if (m.n_layers > STEP_MAX_LAYERS || m.H % 128 != 0 || !d.coop) return false;
+  const size_t fixed = STEP_FIXED + step_act_bytes(M, m.H, m.I, m.Is);
+  *stages = stages_for(d.dyn_step, fixed, step_stage_bytes(m.H, m.I, m.Is));
+  return *stages >= N_CONSUMERS;
+}
+
+moe_status_t launch_step(const StepParams& sp, const DevInfo& d, cudaStream_t st) {
+  const size_t smem = STEP_FIXED + (size_t)sp.stages * step_stage_bytes(sp.H, sp.I, sp.Is) + sp.act_bytes;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(d.sms);
+  cfg.blockDim = dim3(STEP_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;  // all blocks co-resident: the grid-wide waits need it
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  MOE_CUDA(cudaLaunchKernelEx(&cfg, k_step, sp));
   return MOE_OK;
 }
 
@@ -477,9 +498,33 @@ static moe_status_t check_model(const moe_model_t* m) {
   return MOE_OK;
 }
 
+int decode_step_launch_names(const moe_model_t* model, int M, const char** names, int max_names) {
+  if (check_model(model) != MOE_OK || !ok_M(M)) return -1;
+  DevInfo d;
+  if (dev_info(&d) != MOE_OK) return -1;
+  int n = 0;
+  auto put = [&](const char* nm) {
+    if (names && n < max_names) names[n] = nm;
+    ++n;
+  };
+  int stages = 0;
+  if (use_persistent(*model, M, d, &stages)) {
+    put("k_step");
+  } else {
+    for (int l = 0; l < model->n_layers; ++l) {
+      put("k_dense");
+      put("k_experts13");
+      put("k_experts2");
+    }
+    put("k_final_norm");
+  }
+  put("k_lm_gemv");
+  return n;
+}
+
 size_t decode_step_workspace_bytes(const moe_model_t* model, int M) {
   if (check_model(model) != MOE_OK || !ok_M(M)) return 0;
-  return step_ws(nullptr, M, model->H, model->I, model->E, model->top_k, model->Is).bytes;
+  return step_ws(nullptr, model->n_layers, M, model->H, model->I, model->E, model->top_k, model->Is).bytes;
 }
 
 moe_status_t decode_step(const moe_model_t* model, const void* x_bf16, int M, float* logits, int32_t* argmax,
@@ -490,20 +535,59 @@ moe_status_t decode_step(const moe_model_t* model, const void* x_bf16, int M, fl
   REQ(ok_M(M), MOE_ERR_UNSUPPORTED_SHAPE);
   moe_trace_t tr{};
   if (trace_opt) tr = *trace_opt;
-  if ((s = check_ptrs_aligned({x_bf16, logits, argmax, ws, tr.x, tr.h, tr.ids, tr.w})) != MOE_OK) return s;
+  if ((s = check_ptrs_aligned({x_bf16, logits, argmax, ws, tr.x, tr.h, tr.ids, tr.w, tr.timeline})) != MOE_OK) return s;
   const int H = model->H, I = model->I, E = model->E, k = model->top_k, Is = model->Is, L = model->n_layers;
   REQ(ws && ws_bytes >= decode_step_workspace_bytes(model, M), MOE_ERR_WORKSPACE);
   DevInfo d;
   if ((s = dev_info(&d)) != MOE_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   Ctrl c = ctrl_of(ws);
-  StepWs w = step_ws(ws, M, H, I, E, k, Is);
-  MOE_CUDA(cudaMemsetAsync(ws, 0, CTRL_BYTES, st));
+  StepWs w = step_ws(ws, L, M, H, I, E, k, Is);
+  MOE_CUDA(cudaMemsetAsync(ws, 0, w.ctrl_bytes, st));
   const __nv_bfloat16* x_in = static_cast<const __nv_bfloat16*>(x_bf16);
   __nv_bfloat16* xt = static_cast<__nv_bfloat16*>(tr.x);
   EventHook hook;
   hook.ev = reinterpret_cast<cudaEvent_t*>(tr.events);
   hook.n = tr.events ? tr.n_events : 0;
+  int step_stages = 0;
+  if (use_persistent(*model, M, d, &step_stages)) {
+    StepParams sp{};
+    sp.L = L;
+    sp.M = M;
+    sp.H = H;
+    sp.I = I;
+    sp.E = E;
+    sp.k = k;
+    sp.Is = Is;
+    sp.eps = model->rms_eps;
+    sp.stages = step_stages;
+    sp.act_bytes = step_act_bytes(M, H, I, Is);
+    sp.x_in = x_in;
+    sp.h = w.h;
+    sp.x_final = w.x_final;
+    sp.logits = w.logits;
+    sp.a_shared = w.a_shared;
+    sp.a_routed = w.a_routed;
+    sp.ctr = w.ctr;
+    sp.status = c.status;
+    sp.x_trace = xt;
+    sp.h_trace = tr.h;
+    sp.ids_trace = tr.ids;
+    sp.w_trace = tr.w;
+    sp.timeline = tr.timeline;
+    for (int l = 0; l < L; ++l) {
+      const moe_layer_t& Ly = model->layers[l];
+      sp.layer[l] = LayerPtrs{static_cast<const __nv_bfloat16*>(Ly.router.ptr),
+                              static_cast<const uint8_t*>(Ly.w13_codes.ptr),
+                              static_cast<const uint8_t*>(Ly.w13_scales.ptr),
+                              static_cast<const uint8_t*>(Ly.w2_codes.ptr),
+                              static_cast<const uint8_t*>(Ly.w2_scales.ptr),
+                              static_cast<const __nv_bfloat16*>(Ly.shared_w13.ptr),
+                              static_cast<const __nv_bfloat16*>(Ly.shared_w2.ptr)};
+    }
+    if ((s = hook.before(st)) != MOE_OK || (s = launch_step(sp, d, st)) != MOE_OK || (s = hook.after(st)) != MOE_OK)
+      return s;
+  } else {
   for (int l = 0; l < L; ++l) {
     const moe_layer_t& Ly = model->layers[l];
     const size_t mh = (size_t)M * H, mk = (size_t)M * k;
@@ -572,6 +656,7 @@ moe_status_t decode_step(const moe_model_t* model, const void* x_bf16, int M, fl
                                   tr.h ? tr.h + (size_t)L * M * H : nullptr);
   MOE_CUDA(cudaGetLastError());
   if ((s = hook.after(st)) != MOE_OK) return s;
+  }
   LMParams q{};
   q.x = w.x_final;
   q.M = M;

@@ -145,9 +145,12 @@ __device__ __forceinline__ void rms_rows(const float* h, int M, int H, float eps
   const int nw = blockDim.x >> 5;
   for (int t = warp; t < M; t += nw) {
     float ss = 0.0f;
-    for (int i = lane; i < H; i += 32) {
-      const float v = h[(size_t)t * H + i];
-      ss = fmaf(v, v, ss);
+    for (int c = lane; c < H / 4; c += 32) {
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(h + (size_t)t * H) + c);
+      ss = fmaf(v.x, v.x, ss);
+      ss = fmaf(v.y, v.y, ss);
+      ss = fmaf(v.z, v.z, ss);
+      ss = fmaf(v.w, v.w, ss);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
@@ -348,7 +351,12 @@ __device__ __forceinline__ void stage_x_f16(const __nv_bfloat16* x, int M, int H
   for (int tok = warp; tok < MAX_M; tok += N_CONSUMERS) {
     float amax = 0.0f;
     if (tok < M)
-      for (int i = lane; i < H; i += 32) amax = fmaxf(amax, fabsf(__bfloat162float(x[(size_t)tok * H + i])));
+      for (int c = lane; c < H / 8; c += 32) {
+        const uint4 v = *reinterpret_cast<const uint4*>(x + (size_t)tok * H + 8 * c);
+        const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) amax = fmaxf(amax, fmaxf(fabsf(__low2float(b[j])), fabsf(__high2float(b[j]))));
+      }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     if (lane == 0) {
@@ -358,80 +366,132 @@ __device__ __forceinline__ void stage_x_f16(const __nv_bfloat16* x, int M, int H
     }
   }
   named_barrier(1, 32 * N_CONSUMERS);
-  for (int i = tid; i < MAX_M * (H / 2); i += 32 * N_CONSUMERS) {
-    const int tok = i / (H / 2), c = i % (H / 2);
-    __half2 v = __floats2half2_rn(0.0f, 0.0f);
+  for (int i = tid; i < MAX_M * (H / 8); i += 32 * N_CONSUMERS) {
+    const int tok = i / (H / 8), c = i % (H / 8);
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
     if (tok < M) {
+      v = *reinterpret_cast<const uint4*>(x + (size_t)tok * H + 8 * c);
       const float sc = exp2i(s_shift[tok]);
-      const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(x + (size_t)tok * H + 2 * c);
-      v = __floats2half2_rn(__low2float(b) * sc, __high2float(b) * sc);
+      uint32_t* w = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&w[j]);
+        const __half2 hh = __floats2half2_rn(__low2float(b) * sc, __high2float(b) * sc);
+        w[j] = *reinterpret_cast<const uint32_t*>(&hh);
+      }
     }
-    *reinterpret_cast<__half2*>(xs + tok * xss + 4 * c) = v;
+    *reinterpret_cast<uint4*>(xs + tok * xss + 16 * c) = v;
   }
   named_barrier(1, 32 * N_CONSUMERS);
 }
 
-// The warp's 16 x K MXFP4 tile against NP passes of (2 tokens x 4 scale blocks):
-// thread (g, t) owns scale block 4q+t of rows g and g+8 (16 codes bytes each);
-// column n of pass p is (block n%4, token n/4 + 2p) -- the B operand is zero
-// outside its block, so every MMA column sums exactly one scale block and the
-// E8M0 factor is applied in fp32 afterwards.
-//   codes_g/codes_g8: row g / row g+8 codes in shared memory; sc_g/sc_g8: their scale bytes
-//   xb: f16 activation rows (stride xss bytes) holding the B operand (block-aligned)
-//   acc[p][0/1]: row g / g+8 partial sums for token t/2 + 2p (blocks 2(t&1), 2(t&1)+1)
-template <int NP>
+// Largest E8M0 scale byte of a row, for rows g and g+8 (the 4 lanes of a lane
+// group split the row's bytes and combine with two shuffles).
+__device__ __forceinline__ void row_scale_max(const uint8_t* sc_g, const uint8_t* sc_g8, int nb, uint32_t& mg,
+                                              uint32_t& mg8) {
+  const int t = threadIdx.x & 3;
+  uint32_t a = 0u, b = 0u;
+  for (int i = t; i < nb; i += 4) {
+    a = max(a, (uint32_t)sc_g[i]);
+    b = max(b, (uint32_t)sc_g8[i]);
+  }
+  a = max(a, __shfl_xor_sync(0xffffffffu, a, 1));
+  b = max(b, __shfl_xor_sync(0xffffffffu, b, 1));
+  a = max(a, __shfl_xor_sync(0xffffffffu, a, 2));
+  b = max(b, __shfl_xor_sync(0xffffffffu, b, 2));
+  mg = a;
+  mg8 = b;
+}
+
+// f16x2 of 2^d in both halves, d = e - ref <= 0: normal for d >= -14, subnormal
+// down to 2^-24, 0 below.  Exact wherever it is not 0.
+__device__ __forceinline__ uint32_t pow2_f16x2(int d) {
+  uint32_t b = d >= -14 ? (uint32_t)(d + 15) << 10 : (d >= -24 ? 1u << (d + 24) : 0u);
+  return b | (b << 16);
+}
+
+__device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// The warp's 16 x K MXFP4 tile (rows g and g+8 of each lane group) against up to 8
+// token columns.  Thread (g, t) owns scale block 4q+t of both rows: its 32 codes per
+// row widen to f16 with the hardware e2m1x2 conversion and are multiplied by
+// 2^(e - e_ref) with e_ref the row's largest scale -- an exact power-of-two
+// rescaling (blocks more than 2^23 below the row maximum flush to zero: an error
+// below 2^-20 of the row's largest block).  Every MMA column is then one token and
+// the fp32 accumulators run over the whole row; 2^(e_ref - 127) is applied at the
+// end.  c[]: c0 (row g, token 2t), c1 (row g, token 2t+1), c2 (row g+8, token 2t),
+// c3 (row g+8, token 2t+1).  Tokens >= M read zeros.
+//   codes_g/codes_g8: row g / row g+8 codes in shared memory; sc_g/sc_g8: their scales
+//   xb: f16 activation rows (stride xss bytes), token n at xb + n*xss
+// Latency: the next group's codes and scales are loaded while this group computes;
+// each group issues its 32 conversions back to back, then 8 MMAs into 4 accumulators.
 __device__ __forceinline__ void mxfp4_tile_dot(const uint8_t* codes_g, const uint8_t* codes_g8,
                                                const uint8_t* sc_g, const uint8_t* sc_g8, int nb,
-                                               const uint8_t* xb, uint32_t xss, int M, float (&acc)[NP][2]) {
+                                               const uint8_t* xb, uint32_t xss, int M, float (&c)[4]) {
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const int nq = (nb + 3) / 4;
+  const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+  uint32_t ref_g, ref_g8;
+  row_scale_max(sc_g, sc_g8, nb, ref_g, ref_g8);
+  const bool xact = g < M;
+  const uint8_t* xrow = xb + g * xss;
+  float acc[4][4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) acc[u][0] = acc[u][1] = acc[u][2] = acc[u][3] = 0.0f;
+  uint4 nA0, nA1;
+  uint32_t ns0, ns1;
+  {
+    const bool v = t < nb;
+    nA0 = v ? lds128(codes_g + 16 * t) : zero;
+    nA1 = v ? lds128(codes_g8 + 16 * t) : zero;
+    ns0 = v ? sc_g[t] : 0u;
+    ns1 = v ? sc_g8[t] : 0u;
+  }
   for (int q = 0; q < nq; ++q) {
+    const uint4 A0 = nA0, A1 = nA1;
+    const uint32_t e0 = ns0, e1 = ns1;
     const int beta = 4 * q + t;
-    const bool valid = beta < nb;
-    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
-    const uint4 A0 = valid ? lds128(codes_g + 16 * beta) : zero;
-    const uint4 A1 = valid ? lds128(codes_g8 + 16 * beta) : zero;
-    const int sb = 4 * q + 2 * (t & 1);
-    const float s00 = sb < nb ? e8m0_to_f32(sc_g[sb]) : 0.0f;
-    const float s01 = sb + 1 < nb ? e8m0_to_f32(sc_g[sb + 1]) : 0.0f;
-    const float s10 = sb < nb ? e8m0_to_f32(sc_g8[sb]) : 0.0f;
-    const float s11 = sb + 1 < nb ? e8m0_to_f32(sc_g8[sb + 1]) : 0.0f;
-    uint32_t X[NP][16];
-#pragma unroll
-    for (int p = 0; p < NP; ++p) {
-      const int tok = g / 4 + 2 * p;
-      const bool active = ((g & 3) == t) && tok < M && valid;
-#pragma unroll
-      for (int ii = 0; ii < 4; ++ii) {
-        const uint4 v = active ? lds128(xb + tok * xss + 64 * beta + 16 * ii) : zero;
-        X[p][4 * ii + 0] = v.x;
-        X[p][4 * ii + 1] = v.y;
-        X[p][4 * ii + 2] = v.z;
-        X[p][4 * ii + 3] = v.w;
-      }
+    if (q + 1 < nq) {
+      const int b2 = beta + 4;
+      const bool v = b2 < nb;
+      nA0 = v ? lds128(codes_g + 16 * b2) : zero;
+      nA1 = v ? lds128(codes_g8 + 16 * b2) : zero;
+      ns0 = v ? sc_g[b2] : 0u;
+      ns1 = v ? sc_g8[b2] : 0u;
     }
-    float c[NP][4];
+    const bool valid = beta < nb;
+    uint4 X[4];
 #pragma unroll
-    for (int p = 0; p < NP; ++p) c[p][0] = c[p][1] = c[p][2] = c[p][3] = 0.0f;
+    for (int wd = 0; wd < 4; ++wd) X[wd] = (xact && valid) ? lds128(xrow + 64 * beta + 16 * wd) : zero;
+    const uint32_t f0 = pow2_f16x2((int)e0 - (int)ref_g), f1 = pow2_f16x2((int)e1 - (int)ref_g8);
+    uint32_t h[16], k[16];
     const uint32_t a0w[4] = {A0.x, A0.y, A0.z, A0.w};
     const uint32_t a1w[4] = {A1.x, A1.y, A1.z, A1.w};
 #pragma unroll
     for (int wd = 0; wd < 4; ++wd) {
-      uint32_t h0, h1, h2, h3, k0, k1, k2, k3;
-      e2m1x8_to_f16x2(a0w[wd], h0, h1, h2, h3);
-      e2m1x8_to_f16x2(a1w[wd], k0, k1, k2, k3);
-#pragma unroll
-      for (int p = 0; p < NP; ++p) {
-        mma_f16(c[p], h0, k0, h1, k1, X[p][4 * wd + 0], X[p][4 * wd + 1]);
-        mma_f16(c[p], h2, k2, h3, k3, X[p][4 * wd + 2], X[p][4 * wd + 3]);
-      }
+      e2m1x8_to_f16x2(a0w[wd], h[4 * wd], h[4 * wd + 1], h[4 * wd + 2], h[4 * wd + 3]);
+      e2m1x8_to_f16x2(a1w[wd], k[4 * wd], k[4 * wd + 1], k[4 * wd + 2], k[4 * wd + 3]);
     }
 #pragma unroll
-    for (int p = 0; p < NP; ++p) {
-      acc[p][0] = fmaf(c[p][0], s00, fmaf(c[p][1], s01, acc[p][0]));
-      acc[p][1] = fmaf(c[p][2], s10, fmaf(c[p][3], s11, acc[p][1]));
+    for (int j = 0; j < 16; ++j) {
+      h[j] = hmul2_u32(h[j], f0);
+      k[j] = hmul2_u32(k[j], f1);
+    }
+#pragma unroll
+    for (int wd = 0; wd < 4; ++wd) {
+      mma_f16(acc[wd], h[4 * wd], k[4 * wd], h[4 * wd + 1], k[4 * wd + 1], X[wd].x, X[wd].y);
+      mma_f16(acc[wd], h[4 * wd + 2], k[4 * wd + 2], h[4 * wd + 3], k[4 * wd + 3], X[wd].z, X[wd].w);
     }
   }
+  const float r0 = e8m0_to_f32(ref_g), r1 = e8m0_to_f32(ref_g8);
+  c[0] = ((acc[0][0] + acc[1][0]) + (acc[2][0] + acc[3][0])) * r0;
+  c[1] = ((acc[0][1] + acc[1][1]) + (acc[2][1] + acc[3][1])) * r0;
+  c[2] = ((acc[0][2] + acc[1][2]) + (acc[2][2] + acc[3][2])) * r1;
+  c[3] = ((acc[0][3] + acc[1][3]) + (acc[2][3] + acc[3][3])) * r1;
 }
 
 // ---------------------------------------------------------------------------
@@ -452,12 +512,11 @@ struct E13Params {
 constexpr int EXPERT_THREADS = 32 * (N_CONSUMERS + 1);
 
 __host__ __device__ inline size_t e13_stage_bytes(int H) {
-  size_t b = 16 * (size_t)padded_stride(H / 2) + 16 * (size_t)(H / 32);
+  size_t b = 16 * (size_t)(H / 2) + 16 * (size_t)(H / 32);  // contiguous rows: 4 bulk copies per item
   return (b + 127) / 128 * 128;
 }
 __host__ __device__ inline size_t e13_fixed_bytes(int H) { return 128 + 8 * (size_t)padded_stride(2u * H); }
 
-template <int NP>
 __global__ void __launch_bounds__(EXPERT_THREADS, 1) k_experts13(E13Params p) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ Plan P;
@@ -466,7 +525,7 @@ __global__ void __launch_bounds__(EXPERT_THREADS, 1) k_experts13(E13Params p) {
   const int g = lane >> 2, t = lane & 3;
   const int M = p.M, H = p.H, I = p.I, S = p.stages;
   const uint32_t xss = padded_stride(2u * H);
-  const uint32_t cs = padded_stride(H / 2);
+  const uint32_t cs = H / 2;
   const int nb = H / 32;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);
   uint64_t* empty = full + MAX_STAGES;
@@ -502,10 +561,8 @@ __global__ void __launch_bounds__(EXPERT_THREADS, 1) k_experts13(E13Params p) {
         const size_t e2I = (size_t)P.ids[u] * 2 * I;
         uint8_t* st = stages + s * sbytes;
         mbar_arrive_expect_tx(&full[s], 16 * rowb + 2 * scb);
-        for (int rr = 0; rr < 8; ++rr) {
-          bulk_g2s(st + rr * cs, p.w13c + (e2I + r0 + rr) * rowb, rowb, &full[s], pol);
-          bulk_g2s(st + (8 + rr) * cs, p.w13c + (e2I + I + r0 + rr) * rowb, rowb, &full[s], pol);
-        }
+        bulk_g2s(st, p.w13c + (e2I + r0) * rowb, 8 * rowb, &full[s], pol);
+        bulk_g2s(st + 8 * cs, p.w13c + (e2I + I + r0) * rowb, 8 * rowb, &full[s], pol);
         bulk_g2s(st + 16 * cs, p.w13s + (e2I + r0) * (H / 32), scb, &full[s], pol);
         bulk_g2s(st + 16 * cs + scb, p.w13s + (e2I + I + r0) * (H / 32), scb, &full[s], pol);
       }
@@ -522,22 +579,16 @@ __global__ void __launch_bounds__(EXPERT_THREADS, 1) k_experts13(E13Params p) {
     const long long item = start + i;
     const int u = (int)(item / ntile), r0 = 8 * (int)(item % ntile);
     const uint8_t* st = stages + s * sbytes;
-    float acc[NP][2];
-#pragma unroll
-    for (int q = 0; q < NP; ++q) acc[q][0] = acc[q][1] = 0.0f;
-    mxfp4_tile_dot<NP>(st + g * cs, st + (8 + g) * cs, st + 16 * cs + g * (H / 32),
-                       st + 16 * cs + (8 + g) * (H / 32), nb, xs, xss, M, acc);
+    float c[4];
+    mxfp4_tile_dot(st + g * cs, st + (8 + g) * cs, st + 16 * cs + g * (H / 32), st + 16 * cs + (8 + g) * (H / 32),
+                   nb, xs, xss, M, c);
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
 #pragma unroll
-    for (int q = 0; q < NP; ++q) {
-      acc[q][0] += __shfl_xor_sync(0xffffffffu, acc[q][0], 1);
-      acc[q][1] += __shfl_xor_sync(0xffffffffu, acc[q][1], 1);
-      const int tok = t / 2 + 2 * q;
-      if ((t & 1) == 0 && tok < M) {
-        const float gate = acc[q][0] * s_inv[tok], up = acc[q][1] * s_inv[tok];
-        p.a_routed[((size_t)u * M + tok) * I + r0 + g] = silu_f32(gate) * up;
-      }
+    for (int e = 0; e < 2; ++e) {
+      const int tok = 2 * t + e;  // rows g (gate) and g+8 (up) of intermediate index r0 + g
+      if (tok < M)
+        p.a_routed[((size_t)u * M + tok) * I + r0 + g] = silu_f32(c[e] * s_inv[tok]) * (c[2 + e] * s_inv[tok]);
     }
   }
 }
@@ -563,7 +614,7 @@ constexpr int E2_MAX_LOCAL_SLOTS = 3;
 constexpr int SHARED_CHUNK = 256;
 
 __host__ __device__ inline size_t e2_stage_bytes(int I, int Is) {
-  size_t r = 16 * (size_t)padded_stride(I / 2) + 16 * (size_t)(I / 32);
+  size_t r = 16 * (size_t)(I / 2) + 16 * (size_t)(I / 32);
   size_t s = Is > 0 ? 16 * (size_t)padded_stride(2 * SHARED_CHUNK) : 0;
   size_t b = r > s ? r : s;
   return (b + 127) / 128 * 128;
@@ -576,7 +627,6 @@ __host__ __device__ inline size_t e2_fixed_bytes(int M, int I, int Is) {
   return (b + 127) / 128 * 128;
 }
 
-template <int NP>
 __global__ void __launch_bounds__(EXPERT_THREADS, 1) k_experts2(E2Params p) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ Plan P;
@@ -586,7 +636,7 @@ __global__ void __launch_bounds__(EXPERT_THREADS, 1) k_experts2(E2Params p) {
   const int M = p.M, H = p.H, I = p.I, Is = p.Is, S = p.stages;
   const uint32_t ass = padded_stride(2u * I);
   const uint32_t sss = Is > 0 ? padded_stride(2u * Is) : 0u;
-  const uint32_t cs = padded_stride(I / 2);
+  const uint32_t cs = I / 2;
   const uint32_t css = padded_stride(2 * SHARED_CHUNK);
   const int nb = I / 32;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);
@@ -629,8 +679,7 @@ __global__ void __launch_bounds__(EXPERT_THREADS, 1) k_experts2(E2Params p) {
           const size_t eH = (size_t)P.ids[u] * H;
           const uint32_t rowb = I / 2, scb = 16 * (I / 32);
           mbar_arrive_expect_tx(&full[s], 16 * rowb + scb);
-          for (int rr = 0; rr < 16; ++rr)
-            bulk_g2s(st + rr * cs, p.w2c + (eH + h0 + rr) * rowb, rowb, &full[s], pol);
+          bulk_g2s(st, p.w2c + (eH + h0) * rowb, 16 * rowb, &full[s], pol);
           bulk_g2s(st + 16 * cs, p.w2s + (eH + h0) * (I / 32), scb, &full[s], pol);
         } else {
           const long long si = item - Tr;
@@ -693,24 +742,20 @@ __global__ void __launch_bounds__(EXPERT_THREADS, 1) k_experts2(E2Params p) {
     if (item < Tr) {
       const int u = (int)(item / htiles), h0 = 16 * (int)(item % htiles);
       const int uu = u - u_lo;
-      float acc[NP][2];
-#pragma unroll
-      for (int q = 0; q < NP; ++q) acc[q][0] = acc[q][1] = 0.0f;
-      mxfp4_tile_dot<NP>(st + g * cs, st + (8 + g) * cs, st + 16 * cs + g * (I / 32),
-                         st + 16 * cs + (8 + g) * (I / 32), nb, af + (size_t)uu * MAX_M * ass, ass, M, acc);
+      float c[4];
+      mxfp4_tile_dot(st + g * cs, st + (8 + g) * cs, st + 16 * cs + g * (I / 32), st + 16 * cs + (8 + g) * (I / 32),
+                     nb, af + (size_t)uu * MAX_M * ass, ass, M, c);
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
 #pragma unroll
-      for (int q = 0; q < NP; ++q) {
-        acc[q][0] += __shfl_xor_sync(0xffffffffu, acc[q][0], 1);
-        acc[q][1] += __shfl_xor_sync(0xffffffffu, acc[q][1], 1);
-        const int tok = t / 2 + 2 * q;
-        if ((t & 1) == 0 && tok < M) {
+      for (int e = 0; e < 2; ++e) {
+        const int tok = 2 * t + e;
+        if (tok < M) {
           const float wt = P.w[u][tok];
           if (wt != 0.0f) {
             const float f = wt * s_pscale[uu][tok];
-            atomicAdd(p.out + (size_t)tok * H + h0 + g, acc[q][0] * f);
-            atomicAdd(p.out + (size_t)tok * H + h0 + g + 8, acc[q][1] * f);
+            atomicAdd(p.out + (size_t)tok * H + h0 + g, c[e] * f);
+            atomicAdd(p.out + (size_t)tok * H + h0 + g + 8, c[2 + e] * f);
           }
         }
       }

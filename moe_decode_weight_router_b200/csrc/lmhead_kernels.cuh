@@ -76,7 +76,7 @@ struct LMParams {
 };
 
 __host__ __device__ inline size_t lm_stage_bytes(int H) {
-  size_t b = 16 * (size_t)padded_stride(H);
+  size_t b = 16 * (size_t)H;  // 16 contiguous rows: one bulk copy per tile
   return (b + 127) / 128 * 128;
 }
 __host__ __device__ inline size_t lm_fixed_bytes(int H) { return 128 + 8 * (size_t)padded_stride(2u * H); }
@@ -94,7 +94,7 @@ __global__ void __launch_bounds__(EXPERT_THREADS, 1) k_lm_gemv(LMParams p) {
   const int g = lane >> 2, t = lane & 3;
   const int M = p.M, V = p.V, H = p.H, S = p.stages;
   const uint32_t xss = padded_stride(2u * H);
-  const uint32_t ls = padded_stride(H);
+  const uint32_t ls = H;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);
   uint64_t* empty = full + MAX_STAGES;
   uint8_t* xs = smem + 128;
@@ -124,8 +124,7 @@ __global__ void __launch_bounds__(EXPERT_THREADS, 1) k_lm_gemv(LMParams p) {
         const int nrows = (int)min(16LL, (long long)V - v0);
         uint8_t* st = stages + s * sbytes;
         mbar_arrive_expect_tx(&full[s], (uint32_t)nrows * H);
-        for (int rr = 0; rr < nrows; ++rr)
-          bulk_g2s(st + rr * ls, p.w + (size_t)(v0 + rr) * H, H, &full[s], pol);
+        bulk_g2s(st, p.w + (size_t)v0 * H, (uint32_t)nrows * H, &full[s], pol);
       }
       for (int i = (nloc > S ? nloc - S : 0); i < nloc; ++i) mbar_wait(&full[i % S], (i / S) & 1, p.status);
     }
@@ -141,7 +140,11 @@ __global__ void __launch_bounds__(EXPERT_THREADS, 1) k_lm_gemv(LMParams p) {
     const long long v0 = (start + i) * 16;
     const uint8_t* st = stages + s * sbytes;
     float c[4] = {0.f, 0.f, 0.f, 0.f};
+    float c4[4][4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) c4[u][0] = c4[u][1] = c4[u][2] = c4[u][3] = 0.0f;
     const bool xact = g < M;
+#pragma unroll 2
     for (int j = 0; j < H / 64; ++j) {
       const uint4 A0 = lds128(st + g * ls + 64 * j + 16 * t);
       const uint4 A1 = lds128(st + (8 + g) * ls + 64 * j + 16 * t);
@@ -159,8 +162,11 @@ __global__ void __launch_bounds__(EXPERT_THREADS, 1) k_lm_gemv(LMParams p) {
       e4m3x4_to_f16x2(A1.w, Q[6], Q[7]);
       const uint32_t X[8] = {X0.x, X0.y, X0.z, X0.w, X1.x, X1.y, X1.z, X1.w};
 #pragma unroll
-      for (int s4 = 0; s4 < 4; ++s4) mma_f16(c, P[2 * s4], Q[2 * s4], P[2 * s4 + 1], Q[2 * s4 + 1], X[2 * s4], X[2 * s4 + 1]);
+      for (int s4 = 0; s4 < 4; ++s4)
+        mma_f16(c4[s4], P[2 * s4], Q[2 * s4], P[2 * s4 + 1], Q[2 * s4 + 1], X[2 * s4], X[2 * s4 + 1]);
     }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) c[e] = (c4[0][e] + c4[1][e]) + (c4[2][e] + c4[3][e]);
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
     const long long va = v0 + g, vb = v0 + g + 8;

@@ -161,7 +161,7 @@ def test_decode_step_other_errors(lib):
     need3 = lib.decode_step_workspace_bytes(ctypes.byref(m3), 1)
     assert 0 < need3 < need
     m4, k4 = _model()
-    tr = _abi.Trace(A + 4, None, None, None, None, 0)
+    tr = _abi.Trace(A + 4, None, None, None, None, 0, None)
     assert lib.decode_step(ctypes.byref(m4), A, 1, A, A, ctypes.byref(tr), A, need, None) == 3
 
 

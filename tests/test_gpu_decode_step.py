@@ -11,7 +11,8 @@ import pytest
 import torch
 
 import oracle
-from moe_decode_weight_router_b200 import DecodeGraph, DecodeModel, decode_step, decode_step_workspace_bytes, synth
+from moe_decode_weight_router_b200 import (DecodeGraph, DecodeModel, decode_step, decode_step_launch_names,
+                                           decode_step_workspace_bytes, synth, workspace_status)
 from tests._bruteforce import bf16_to_f64
 from tests._gpu import MARGIN_FLAG, assert_rows_close, need_gpu, rel_l2_rows
 
@@ -23,11 +24,14 @@ def _gpu():
     need_gpu()
 
 
-def _model(shape, n_layers, V, seed):
+def _model(shape, n_layers, V, seed, path=0):
     layers = [synth.layer(shape, seed, l, device="cuda") for l in range(n_layers)]
     q = synth.e4m3_codes((V, shape.H), seed, device="cuda")
     s = synth.row_scales(V, seed, device="cuda")
-    return DecodeModel(layers=layers, lm_q=q, lm_s=s, top_k=shape.k)
+    return DecodeModel(layers=layers, lm_q=q, lm_s=s, top_k=shape.k, step_path=path)
+
+
+PATHS = {"persistent": 0, "per_layer": 1}
 
 
 def _fetch(L):
@@ -76,13 +80,18 @@ def _check_step(model, shape, x, res, layers_to_check):
             assert am[t] == am_ref[t]
 
 
+@pytest.mark.parametrize("path", list(PATHS))
 @pytest.mark.parametrize("M", [1, 4, 8])
-def test_tiny_chain_all_layers(M):
+def test_tiny_chain_all_layers(M, path):
     S = synth.TINY
-    model = _model(S, 4, 1000, 21 + M)
+    model = _model(S, 4, 1000, 21 + M, PATHS[path])
     x = synth.tokens(M, S.H, 21, device="cuda")
+    names = decode_step_launch_names(model, M)
+    assert names == (["k_step", "k_lm_gemv"] if path == "persistent" else
+                     ["k_dense", "k_experts13", "k_experts2"] * 4 + ["k_final_norm", "k_lm_gemv"])
     res = decode_step(model, x, trace=True)
     torch.cuda.synchronize()
+    assert workspace_status(res["ws"]) == 0
     _check_step(model, S, x, res, range(4))
 
 
@@ -100,16 +109,17 @@ def test_tiny_chain_free_running_matches_oracle_chain():
         assert_rows_close(res["logits"].cpu().numpy(), out["logits"], what="free-running logits")
 
 
-@pytest.mark.parametrize("M", [1, 4])
-def test_ling_42_layers_sampled(M):
+@pytest.mark.parametrize("M,path", [(1, "persistent"), (4, "persistent"), (1, "per_layer")])
+def test_ling_42_layers_sampled(M, path):
     """Full size: 42 distinct Ling-shaped layers (~67 GB MXFP4) and the 157,184 x 2,560
     FP8 LM head, in the same launch configuration the benchmark times; layers
     0, 1, 20 and 41 and the LM head are recomputed by the oracle."""
     S = synth.LING
-    model = _model(S, synth.N_LAYERS, synth.VOCAB, 41 + M)
+    model = _model(S, synth.N_LAYERS, synth.VOCAB, 41 + M, PATHS[path])
     x = synth.tokens(M, S.H, 41 + M, device="cuda")
     res = decode_step(model, x, trace=True)
     torch.cuda.synchronize()
+    assert workspace_status(res["ws"]) == 0
     _check_step(model, S, x, res, [0, 1, 20, 41])
     # the captured graph (one launch per step) is checked against the oracle the same way,
     # through the trace it fills; two runs need not agree bit for bit with each other
