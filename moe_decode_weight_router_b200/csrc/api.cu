@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -127,7 +128,9 @@ ExpertsWs experts_ws(void* ws, int M, int H, int I, int E, int k, int Is) {
 
 struct StepWs {
   unsigned* ctr;
-  size_t ctrl_bytes;  // control block + per-layer counters, cleared every step
+  unsigned long long* tlogits;  // persistent step: tagged router logits [M][E]
+  unsigned long long* tshared;  // persistent step: tagged shared activation [M][Is]
+  size_t ctrl_bytes;  // control block, per-layer counters and the tagged buffers, cleared every step
   float* logits;
   int32_t* ids;
   float* w;
@@ -144,6 +147,10 @@ StepWs step_ws(void* ws, int L, int M, int H, int I, int E, int k, int Is) {
   StepWs s{};
   s.ctr = reinterpret_cast<unsigned*>(b + off);
   off += up256((size_t)L * CTR_PER_LAYER * sizeof(unsigned));
+  s.tlogits = reinterpret_cast<unsigned long long*>(b + off);
+  off += up256((size_t)M * E * 8);
+  s.tshared = reinterpret_cast<unsigned long long*>(b + off);
+  off += up256((size_t)M * Is * 8);
   s.ctrl_bytes = off;
   s.logits = reinterpret_cast<float*>(b + off);
   off += up256((size_t)M * E * 4);
@@ -153,8 +160,8 @@ StepWs step_ws(void* ws, int L, int M, int H, int I, int E, int k, int Is) {
   off += up256((size_t)M * k * 4);
   s.x_cur = reinterpret_cast<__nv_bfloat16*>(b + off);
   off += up256((size_t)M * H * 2);
-  s.h = reinterpret_cast<float*>(b + off);
-  off += up256((size_t)M * H * 4);
+  s.h = reinterpret_cast<float*>(b + off);  // [2][M][H]: the persistent step alternates by layer
+  off += up256((size_t)2 * M * H * 4);
   s.a_shared = reinterpret_cast<float*>(b + off);
   off += up256((size_t)M * Is * 4);
   s.a_routed = reinterpret_cast<float*>(b + off);
@@ -227,18 +234,40 @@ moe_status_t launch_lm(LMParams p, const DevInfo& d, cudaStream_t st) {
 
 // The whole-step persistent kernel serves the model when it fits: at most
 // STEP_MAX_LAYERS layers, H a multiple of 128 (router/shared tiles split into four
-// 32-column-aligned quarters), cooperative launch available, and a shared-memory ring
-// of at least N_CONSUMERS stages next to the activation region.
-bool use_persistent(const moe_model_t& m, int M, const DevInfo& d, int* stages) {
+// 32-column-aligned quarters), cooperative launch available, and a shared-memory
+// ring next to the activation region that holds at least N_CONSUMERS of the
+// largest items (one per consumer warp in flight).
+bool use_persistent(const moe_model_t& m, int M, const DevInfo& d, uint32_t* ring_bytes) {
   if (m.step_path == MOE_STEP_PER_LAYER) return false;
   if (m.n_layers > STEP_MAX_LAYERS || m.H % 128 != 0 || !d.coop) return false;
   const size_t fixed = STEP_FIXED + step_act_bytes(M, m.H, m.I, m.Is);
-  *stages = stages_for(d.dyn_step, fixed, step_stage_bytes(m.H, m.I, m.Is));
-  return *stages >= N_CONSUMERS;
+  if ((size_t)d.dyn_step <= fixed) return false;
+  const size_t ring = ((size_t)d.dyn_step - fixed) / 128 * 128;
+  *ring_bytes = (uint32_t)ring;
+  // a block's contiguous routed-W2 range of n items (H/16 per expert) touches at most
+  // (n - 2) / (H/16) + 2 experts; their activations must fit the block's cache
+  const long long T = m.H / 16;
+  const long long n = ((long long)slots_of(M, m.E, m.top_k) * T + d.sms - 1) / d.sms;
+  const long long span = n <= 1 ? 1 : (n - 2) / T + 2;
+  if (span > CR_CACHE) return false;
+  return ring >= (size_t)N_CONSUMERS * step_max_item_bytes(m.H, m.I, m.Is);
+}
+
+// Bound on the bytes a block keeps in flight in the persistent step (MOE_STEP_INFLIGHT_KB
+// overrides; 0 = the whole ring).  Enough to keep HBM streaming, small enough that the
+// loads and polls of the dependency chain do not wait behind a queue of weight copies.
+uint32_t step_inflight_bytes() {
+  static const uint32_t v = [] {
+    const char* e = getenv("MOE_STEP_INFLIGHT_KB");
+    long kb = e ? strtol(e, nullptr, 10) : 0;
+    if (kb < 0) kb = 0;
+    return (uint32_t)kb * 1024u;
+  }();
+  return v;
 }
 
 moe_status_t launch_step(const StepParams& sp, const DevInfo& d, cudaStream_t st) {
-  const size_t smem = STEP_FIXED + (size_t)sp.stages * step_stage_bytes(sp.H, sp.I, sp.Is) + sp.act_bytes;
+  const size_t smem = STEP_FIXED + (size_t)sp.ring_bytes + sp.act_bytes;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(d.sms);
   cfg.blockDim = dim3(STEP_THREADS);
@@ -507,8 +536,8 @@ int decode_step_launch_names(const moe_model_t* model, int M, const char** names
     if (names && n < max_names) names[n] = nm;
     ++n;
   };
-  int stages = 0;
-  if (use_persistent(*model, M, d, &stages)) {
+  uint32_t ring_bytes = 0;
+  if (use_persistent(*model, M, d, &ring_bytes)) {
     put("k_step");
   } else {
     for (int l = 0; l < model->n_layers; ++l) {
@@ -549,8 +578,8 @@ moe_status_t decode_step(const moe_model_t* model, const void* x_bf16, int M, fl
   EventHook hook;
   hook.ev = reinterpret_cast<cudaEvent_t*>(tr.events);
   hook.n = tr.events ? tr.n_events : 0;
-  int step_stages = 0;
-  if (use_persistent(*model, M, d, &step_stages)) {
+  uint32_t ring_bytes = 0;
+  if (use_persistent(*model, M, d, &ring_bytes)) {
     StepParams sp{};
     sp.L = L;
     sp.M = M;
@@ -560,13 +589,14 @@ moe_status_t decode_step(const moe_model_t* model, const void* x_bf16, int M, fl
     sp.k = k;
     sp.Is = Is;
     sp.eps = model->rms_eps;
-    sp.stages = step_stages;
+    sp.ring_bytes = ring_bytes;
     sp.act_bytes = step_act_bytes(M, H, I, Is);
     sp.x_in = x_in;
     sp.h = w.h;
     sp.x_final = w.x_final;
-    sp.logits = w.logits;
-    sp.a_shared = w.a_shared;
+    sp.logits = w.tlogits;
+    sp.a_shared = w.tshared;
+    sp.inflight_bytes = step_inflight_bytes();
     sp.a_routed = w.a_routed;
     sp.ctr = w.ctr;
     sp.status = c.status;

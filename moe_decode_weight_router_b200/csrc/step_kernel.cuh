@@ -1,30 +1,36 @@
 // step_kernel.cuh -- the whole decode step (all MoE layers) as one persistent kernel.
 //
 // One block per SM for the whole step (cooperative launch: all blocks co-resident).
-// Warp 4 of each block is the producer: one thread walks this block's sequence of
-// weight tiles for every layer and moves them HBM -> shared memory with bulk copies
-// (TMA engine) into a ring of stages; it also issues L2 prefetches for tiles whose
-// identity is already known -- the next layer's router/shared-expert tiles and this
-// layer's shared-W2 tiles while the layer waits on its router, and a sliding window
-// of routed tiles once the routing is known -- so HBM keeps streaming across the
-// layer's dependency points.  Warps 0-3 consume the ring in order (item i -> warp
-// i % 4) and synchronise only where the data forces it:
+// The last warp of each block is the producer: it walks this block's sequence of weight
+// tiles for every layer and moves them HBM -> shared memory with bulk copies (TMA
+// engine) into a byte-addressed ring, each tile taking exactly its own bytes, so the
+// bytes in flight per SM stay high whatever the tile mix.  The tiles whose identity
+// does not depend on the routing (router rows, shared-expert rows) come first in
+// every layer, so the producer runs ahead across the layer boundary and the
+// routing-dependent tiles are the only ones that wait for the top-k.  Warps 0-7
+// consume the ring in order (item i -> warp i % 8) and synchronise only where the
+// data forces it:
 //   router tiles complete  -> every block takes the top-k itself (same code, same bits)
-//   expert u's W13 complete -> its W2 tiles may start (per-expert counter)
 //   shared W13 complete    -> the shared W2 tiles may start
+// (router logits and shared activations carry the layer number in the same 64-bit
+// word, so readers poll the data itself: no writer fence, no separate counter)
+//   expert u's W13 complete -> its W2 tiles may start (per-expert counter)
 //   residual h complete    -> the next layer's RMSNorm may start (grid-wide counter)
+// The residual is double-buffered by layer parity: layer l adds into h[l & 1], which
+// every block first initialises (its slice) from h[(l - 1) & 1] while it reads that
+// buffer for its RMSNorm, so no block's accumulation can reach a buffer another
+// block is still normalising.
 // Every wait is a bounded spin (abort flag + status word after WAIT_LIMIT_NS), so a
 // fault in one block ends the step with MOE_ERR_TIMEOUT instead of a hang.
 //
 // Per layer, in ring order, block c processes (every item one or a few contiguous
-// bulk copies -- the copy count, not the byte count, is what a bulk-copy engine
-// pays for):
-//   A: router items (4 experts' rows) and shared-W13 items (2 gate + 2 up rows),
-//      fixed assignment j = c, c+G, ...; weight rows are the MMA's N operand and
-//      the tokens its M operand, so one warp covers the full K of its 4 rows.
-//   B: routed W13 items (distinct expert, 8 gate + 8 up rows), a contiguous range.
-//   C: routed W2 items (distinct expert, 16 output rows), a contiguous range, then
-//      shared-W2 items (4 output rows), fixed assignment.
+// bulk copies):
+//   A:  router items (4 experts' rows) and shared-W13 items (2 gate + 2 up rows),
+//       fixed assignment j = c, c+G, ...; weight rows are the MMA's N operand and
+//       the tokens its M operand, so one warp covers the full K of its 4 rows.
+//   CS: shared-W2 items (4 output rows), fixed assignment.
+//   B:  routed W13 items (distinct expert, 8 gate + 8 up rows), a contiguous range.
+//   CR: routed W2 items (distinct expert, 16 output rows), a contiguous range.
 // Sources: DGX Spark MoE knowledge card (知识卡片：NVIDIA DGX Spark 上提升 MoE 推理吞吐的
 // 三种方法), 事件概述或研究问题 (batch-1 decode bound by weight reads; 8 of 512 experts
 // + 1 shared) and 方法/产品要点 items 1 and 3.
@@ -35,10 +41,14 @@
 namespace moe {
 
 constexpr int STEP_MAX_LAYERS = 64;
-constexpr int STEP_THREADS = 32 * (N_CONSUMERS + 1);
-constexpr int CTR_ROUTER = 0, CTR_SHARED = 1, CTR_H = 2, CTR_EXP = 4;
+constexpr int STEP_CONSUMERS = 8;  // consumer warps: two per SM sub-partition, to hide latency
+constexpr int STEP_THREADS = 32 * (STEP_CONSUMERS + 1);
+constexpr int CR_CACHE = 4;         // routed experts whose W2 activation a block keeps staged
+constexpr int STEP_SLOTS = 32;  // ring items in flight at most (one full/empty mbarrier pair each)
+constexpr int CTR_H = 2, CTR_HINIT = 3, CTR_EXP = 4;  // slots 0-1 unused
 constexpr int CTR_PER_LAYER = CTR_EXP + MAX_SLOTS;
-constexpr int STEP_PREFETCH_AHEAD = 8;  // routed items prefetched into L2 ahead of the ring
+constexpr size_t STEP_FIXED = 1024;  // full[32], empty[32], plan and h-init barriers
+constexpr int STAGE_REG_F4 = 4;      // residual float4s a consumer thread keeps in registers (M = 1 at H = 2560)
 
 struct LayerPtrs {
   const __nv_bfloat16* wr;
@@ -53,13 +63,14 @@ struct LayerPtrs {
 struct StepParams {
   int L, M, H, I, E, k, Is;
   float eps;
-  int stages;
+  uint32_t ring_bytes;
   uint32_t act_bytes;
+  uint32_t inflight_bytes;    // producer cap on copied-but-not-landed bytes (0: the ring)
   const __nv_bfloat16* x_in;  // [M][H]
-  float* h;                   // [M][H] residual stream
+  float* h;                   // [2][M][H] residual stream, buffer l & 1 is layer l's output
   __nv_bfloat16* x_final;     // [M][H] LM-head input
-  float* logits;              // [M][E]
-  float* a_shared;            // [M][Is]
+  unsigned long long* logits;    // [M][E] tagged: (l + 1) << 32 | fp32 bits, zero on entry
+  unsigned long long* a_shared;  // [M][Is] tagged like logits
   float* a_routed;            // [MAX_SLOTS][M][I]
   unsigned* ctr;              // [L][CTR_PER_LAYER], zero on entry
   int* status;
@@ -78,35 +89,68 @@ __device__ __forceinline__ void stamp(const StepParams& p, int l, int slot) {
   const bool first = blockIdx.x == 0, last = blockIdx.x == gridDim.x - 1;
   if (!first && !last) return;
   const int tid = threadIdx.x;
-  if (tid != 0 && tid != 32 * N_CONSUMERS) return;
+  if (tid != 0 && tid != 32 * STEP_CONSUMERS) return;
   p.timeline[((size_t)(last ? 1 : 0) * p.L + l) * 16 + slot] = globaltimer_ns();
 }
-// Profiling: block 0's first STEP_ITEM_LOG ring items -- (issued, data ready, done)
-// stamps after the [2][L][16] phase stamps.
+// Profiling: block 0's first STEP_ITEM_LOG ring items -- (issued, data ready, done,
+// consumer started waiting) stamps after the [2][L][16] phase stamps.
 constexpr int STEP_ITEM_LOG = 4096;
 __device__ __forceinline__ void item_stamp(const StepParams& p, long long i, int which) {
   if (!p.timeline || blockIdx.x != 0 || i >= STEP_ITEM_LOG || (threadIdx.x & 31) != 0) return;
   p.timeline[(size_t)2 * p.L * 16 + (size_t)i * 4 + which] = globaltimer_ns();
 }
 
-// Stage geometry shared by host and device: the largest item -- 4 bf16 rows of H
-// (router / shared W13), 16 MXFP4 rows of H + scales (routed W13), 16 MXFP4 rows of
-// I + scales (routed W2), 4 bf16 rows of Is (shared W2).
-__host__ __device__ inline size_t step_stage_bytes(int H, int I, int Is) {
-  size_t b = 8 * (size_t)H;
-  const size_t b13 = 8 * (size_t)H + (size_t)H / 2, b2 = 8 * (size_t)I + (size_t)I / 2, bs = 8 * (size_t)Is;
-  if (b13 > b) b = b13;
-  if (b2 > b) b = b2;
-  if (bs > b) b = bs;
-  return (b + 127) / 128 * 128;
+// ---------------------------------------------------------------------------
+// geometry shared by host and device
+// ---------------------------------------------------------------------------
+enum : int { IT_A = 0, IT_B = 1, IT_CR = 2, IT_CS = 3 };
+
+// Ring bytes of one item: 4 bf16 rows of H (router / shared W13), 16 MXFP4 rows of
+// H + their scales (routed W13), 16 MXFP4 rows of I + scales (routed W2), 4 bf16
+// rows of Is (shared W2); 128-byte granules.
+__host__ __device__ inline uint32_t step_item_bytes(int type, int H, int I, int Is) {
+  size_t b;
+  if (type == IT_A)
+    b = 8 * (size_t)H;
+  else if (type == IT_B)
+    b = 8 * (size_t)H + (size_t)H / 2;
+  else if (type == IT_CR)
+    b = 8 * (size_t)I + (size_t)I / 2;
+  else
+    b = 8 * (size_t)Is;
+  return (uint32_t)((b + 127) / 128 * 128);
+}
+__host__ __device__ inline uint32_t step_max_item_bytes(int H, int I, int Is) {
+  uint32_t b = step_item_bytes(IT_A, H, I, Is);
+  for (int t = IT_B; t <= IT_CS; ++t) {
+    const uint32_t x = step_item_bytes(t, H, I, Is);
+    if (x > b) b = x;
+  }
+  return b;
+}
+// Activation region: A/B phases hold the bf16 layer input xb16 [M][xss] at 0 and the
+// f16 copy xf16 [M][xss] after it; the shared-W2 phase adds the hi/lo bf16 halves of
+// the shared activation [2][M][sss], over xb16 when they fit there (xb16 is dead once
+// the router and shared-W13 items are done); the routed-W2 phase holds the f16
+// activations of the (at most CR_CACHE) experts of the block's range [CR_CACHE][M][ass] at 0.
+__host__ __device__ inline bool step_shared_over_xb16(int H, int Is) {
+  return 2u * (Is > 0 ? padded_stride(2u * Is) : 0u) <= padded_stride(2u * H);
 }
 __host__ __device__ inline uint32_t step_act_bytes(int M, int H, int I, int Is) {
-  const uint32_t xs = 2u * M * padded_stride(2u * H);  // bf16 rows (A phase) + f16 rows (B phase)
-  const uint32_t c = 2u * M * (Is > 0 ? padded_stride(2u * Is) : 0u) + (uint32_t)N_CONSUMERS * M * padded_stride(2u * I);
-  const uint32_t b = xs > c ? xs : c;
-  return (b + 127) / 128 * 128;
+  const uint32_t xss = padded_stride(2u * H), sss = Is > 0 ? padded_stride(2u * Is) : 0u;
+  uint32_t a = 2u * M * xss + (step_shared_over_xb16(H, Is) ? 0u : 2u * M * sss);
+  const uint32_t c = (uint32_t)CR_CACHE * M * padded_stride(2u * I);
+  if (c > a) a = c;
+  return (a + 127) / 128 * 128;
 }
-constexpr size_t STEP_FIXED = 256;  // mbarriers
+// Deterministic placement in the byte ring (producer and every consumer warp walk
+// the same item sequence and compute the same offsets): an item that would cross
+// the end starts over at 0.
+__device__ __forceinline__ uint32_t ring_take(uint32_t& pos, uint32_t n, uint32_t R) {
+  const uint32_t s = pos + n <= R ? pos : 0u;
+  pos = s + n;
+  return s;
+}
 
 // ---------------------------------------------------------------------------
 // small helpers
@@ -121,8 +165,14 @@ __device__ __forceinline__ int ld_volatile_i32(const int* p) {
   asm volatile("ld.volatile.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
-__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_tagged(unsigned long long* p, float v, uint32_t tag) {
+  const unsigned long long w = ((unsigned long long)tag << 32) | __float_as_uint(v);
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
 }
 __device__ __forceinline__ void signal_counter(unsigned* c) {
   __threadfence();
@@ -136,7 +186,7 @@ __device__ __noinline__ bool wait_counter(const unsigned* c, unsigned target, in
   if (ld_acquire_u32(c) >= target) return true;
   const unsigned long long t0 = globaltimer_ns();
   while (true) {
-    __nanosleep(40);
+    __nanosleep(32);
     if (ld_acquire_u32(c) >= target) return true;
     if (*abort_flag) return false;
     if (ld_volatile_i32(status) != 0 || globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
@@ -160,23 +210,59 @@ __device__ __forceinline__ bool ring_wait(uint64_t* bar, uint32_t parity, int* s
     }
   }
 }
+// Gives up the whole step: records the timeout once and raises the block's abort flag.
+__device__ __noinline__ void step_give_up(int* status, volatile int* abort_flag) {
+  atomicCAS(status, 0, DEV_ERR_TIMEOUT);
+  *abort_flag = 1;
+}
+// Tagged reads: n words (n <= 8, pointers in w[]) are loaded together and retried
+// until every tag equals `tag` (bounded; false after the limit or an abort).
+__device__ __forceinline__ bool await_tagged(const unsigned long long* const* w, int n, uint32_t tag, float* v,
+                                             int* status, volatile int* abort_flag) {
+  unsigned long long x[8];
+  unsigned long long t0 = 0;
+  while (true) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) x[j] = j < n ? ld_relaxed_u64(w[j]) : ((unsigned long long)tag << 32);
+    bool ok = true;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) ok = ok && (uint32_t)(x[j] >> 32) == tag;
+    if (ok) break;
+    if (*abort_flag) return false;
+    if (t0 == 0) t0 = globaltimer_ns();
+    if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
+      step_give_up(status, abort_flag);
+      return false;
+    }
+    __nanosleep(20);
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    if (j < n) v[j] = __uint_as_float((uint32_t)x[j]);
+  return true;
+}
+// Time-bounded wait for a copy to land, used only when the block is about to exit
+// (the abort flag is ignored: copies in flight must finish before shared memory goes).
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  const unsigned long long t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity))
+    if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) return;
+}
 
 // ---------------------------------------------------------------------------
-// the per-layer work list of one block
+// the per-layer work list of one block: A, CS, then (after the routing) B, CR
 // ---------------------------------------------------------------------------
-enum : int { IT_A = 0, IT_B = 1, IT_CR = 2, IT_CS = 3 };
-
 struct Item {
   int type;
-  int a, b;  // A: item j;  B: slot, r0;  CR: slot, h0;  CS: first row
+  int a, b;  // A: item j;  CS: first row;  B: slot, r0;  CR: slot, h0
 };
 
 struct Work {
   int nA;             // A items of this block
+  int nS;             // shared-W2 items of this block
   long long b0, nB;   // routed W13 range
   long long c0, nC;   // routed W2 range
-  int nS;             // shared-W2 items of this block
-  __device__ void init_A(const StepParams& p) {
+  __device__ void init_fixed(const StepParams& p) {
     const int c = blockIdx.x, G = gridDim.x;
     const int TA = p.E / 4 + p.Is / 2;
     nA = c < TA ? (TA - 1 - c) / G + 1 : 0;
@@ -194,15 +280,22 @@ struct Work {
     c0 = TC * c / G;
     nC = TC * (c + 1) / G - c0;
   }
-  __device__ Item at(const StepParams& p, int r) const {
+  __device__ Item at(const StepParams& p, long long r) const {
     Item it;
     if (r < nA) {
       it.type = IT_A;
-      it.a = blockIdx.x + r * gridDim.x;
+      it.a = blockIdx.x + (int)r * gridDim.x;
       it.b = 0;
       return it;
     }
     r -= nA;
+    if (r < nS) {
+      it.type = IT_CS;
+      it.a = 4 * (blockIdx.x + (int)r * gridDim.x);
+      it.b = 0;
+      return it;
+    }
+    r -= nS;
     if (r < nB) {
       const long long x = b0 + r;
       it.type = IT_B;
@@ -210,18 +303,11 @@ struct Work {
       it.b = 8 * (int)(x % (p.I / 8));
       return it;
     }
-    r -= (int)nB;
-    if (r < nC) {
-      const long long x = c0 + r;
-      it.type = IT_CR;
-      it.a = (int)(x / (p.H / 16));
-      it.b = 16 * (int)(x % (p.H / 16));
-      return it;
-    }
-    r -= (int)nC;
-    it.type = IT_CS;
-    it.a = 4 * (blockIdx.x + r * gridDim.x);
-    it.b = 0;
+    r -= nB;
+    const long long x = c0 + r;
+    it.type = IT_CR;
+    it.a = (int)(x / (p.H / 16));
+    it.b = 16 * (int)(x % (p.H / 16));
     return it;
   }
 };
@@ -231,88 +317,101 @@ struct Work {
 // ---------------------------------------------------------------------------
 struct Producer {
   const StepParams& p;
-  uint8_t* stages;
-  size_t sbytes;
+  uint8_t* ring;
+  uint32_t R;
   uint64_t* full;
   uint64_t* empty;
+  uint32_t* fs;  // [STEP_SLOTS] ring start / end of the items in flight (lane 0)
+  uint32_t* fe;
   uint64_t pol;
-  int S;
-  long long i;  // ring index
+  long long i;        // next ring item
+  long long oldest;   // oldest item whose release lane 0 has not seen yet
+  long long land;     // oldest item lane 0 has not seen land yet
+  uint32_t pos;       // ring placement cursor
+  uint32_t inflight;  // bytes copied but not seen landed (lane 0)
+  uint32_t cap;       // bound on inflight: enough to keep HBM busy, no more, so that
+                      // the latency-bound loads of the dependency chain do not queue
   volatile int* abort_flag;
   int lane;
 
-  // Run by all 32 lanes of the producer warp: lane 0 takes the stage and arms its
-  // barrier, then one lane per contiguous run issues its bulk copy.
+  // Run by all 32 lanes of the producer warp: lane 0 frees the item's bytes (waits
+  // for the release of the oldest items until neither their bytes nor their
+  // barrier slot are needed), waits until the bytes in flight leave room under the
+  // cap, and arms the barrier, then one lane per contiguous run issues its bulk
+  // copy.  Items in flight occupy one arc of the ring in allocation order, so the
+  // items the new one overlaps are always the oldest.
   __device__ bool issue(const LayerPtrs& Lp, const Plan& P, const Item& it) {
-    const int s = (int)(i % S);
+    const uint32_t n = step_item_bytes(it.type, p.H, p.I, p.Is);
+    const uint32_t s0 = ring_take(pos, n, R);
+    const int slot = (int)(i % STEP_SLOTS);
     int ok = 1;
-    if (lane == 0 && i >= S) ok = ring_wait(&empty[s], (uint32_t)(((i / S) - 1) & 1), p.status, abort_flag);
+    if (lane == 0) {
+      while (oldest < i) {
+        const int os = (int)(oldest % STEP_SLOTS);
+        const bool need = (i - oldest >= STEP_SLOTS) || (fs[os] < s0 + n && s0 < fe[os]);
+        if (!need) break;
+        if (!ring_wait(&empty[os], (uint32_t)((oldest / STEP_SLOTS) & 1), p.status, abort_flag)) {
+          ok = 0;
+          break;
+        }
+        ++oldest;
+      }
+      // released items have landed (their slots still hold their extents: slot i % 32
+      // is the only one rewritten below, and it belonged to item i - 32 < oldest)
+      for (; land < oldest; ++land) inflight -= fe[land % STEP_SLOTS] - fs[land % STEP_SLOTS];
+      while (ok && land < i && inflight + n > cap) {
+        const int ls = (int)(land % STEP_SLOTS);
+        if (!ring_wait(&full[ls], (uint32_t)((land / STEP_SLOTS) & 1), p.status, abort_flag)) {
+          ok = 0;
+          break;
+        }
+        inflight -= fe[ls] - fs[ls];
+        ++land;
+      }
+      fs[slot] = s0;
+      fe[slot] = s0 + n;
+      inflight += n;
+    }
     ok = __shfl_sync(0xffffffffu, ok, 0);
     if (!ok) return false;
-    uint8_t* st = stages + (size_t)s * sbytes;
+    uint8_t* st = ring + s0;
+    uint64_t* fb = &full[slot];
     const int H = p.H, I = p.I, Is = p.Is;
     item_stamp(p, i, 0);
     if (it.type == IT_A) {
       const int nr = p.E / 4;
-      if (lane == 0) mbar_arrive_expect_tx(&full[s], 4u * 2u * H);
+      if (lane == 0) mbar_arrive_expect_tx(fb, 4u * 2u * H);
       __syncwarp();
       if (it.a < nr) {
-        if (lane == 0) bulk_g2s(st, Lp.wr + (size_t)4 * it.a * H, 4u * 2u * H, &full[s], pol);
+        if (lane == 0) bulk_g2s(st, Lp.wr + (size_t)4 * it.a * H, 4u * 2u * H, fb, pol);
       } else {
         const int sh = it.a - nr;  // gate rows 2sh, 2sh+1 -> rows 0,1; up rows -> rows 2,3
-        if (lane == 0) bulk_g2s(st, Lp.sw13 + (size_t)2 * sh * H, 2u * 2u * H, &full[s], pol);
-        if (lane == 1) bulk_g2s(st + 4 * H, Lp.sw13 + (size_t)(Is + 2 * sh) * H, 2u * 2u * H, &full[s], pol);
+        if (lane == 0) bulk_g2s(st, Lp.sw13 + (size_t)2 * sh * H, 2u * 2u * H, fb, pol);
+        if (lane == 1) bulk_g2s(st + 4 * H, Lp.sw13 + (size_t)(Is + 2 * sh) * H, 2u * 2u * H, fb, pol);
       }
+    } else if (it.type == IT_CS) {
+      if (lane == 0) mbar_arrive_expect_tx(fb, 4u * 2u * Is);
+      __syncwarp();
+      if (lane == 0) bulk_g2s(st, Lp.sw2 + (size_t)it.a * Is, 4u * 2u * Is, fb, pol);
     } else if (it.type == IT_B) {
       const size_t e2I = (size_t)P.ids[it.a] * 2 * I;
       const uint32_t runb = 8u * (H / 2), scb = 8u * (H / 32);
-      if (lane == 0) mbar_arrive_expect_tx(&full[s], 2 * runb + 2 * scb);
+      if (lane == 0) mbar_arrive_expect_tx(fb, 2 * runb + 2 * scb);
       __syncwarp();
-      if (lane == 0) bulk_g2s(st, Lp.w13c + (e2I + it.b) * (H / 2), runb, &full[s], pol);
-      if (lane == 1) bulk_g2s(st + runb, Lp.w13c + (e2I + I + it.b) * (H / 2), runb, &full[s], pol);
-      if (lane == 2) bulk_g2s(st + 2 * runb, Lp.w13s + (e2I + it.b) * (H / 32), scb, &full[s], pol);
-      if (lane == 3) bulk_g2s(st + 2 * runb + scb, Lp.w13s + (e2I + I + it.b) * (H / 32), scb, &full[s], pol);
-    } else if (it.type == IT_CR) {
+      if (lane == 0) bulk_g2s(st, Lp.w13c + (e2I + it.b) * (H / 2), runb, fb, pol);
+      if (lane == 1) bulk_g2s(st + runb, Lp.w13c + (e2I + I + it.b) * (H / 2), runb, fb, pol);
+      if (lane == 2) bulk_g2s(st + 2 * runb, Lp.w13s + (e2I + it.b) * (H / 32), scb, fb, pol);
+      if (lane == 3) bulk_g2s(st + 2 * runb + scb, Lp.w13s + (e2I + I + it.b) * (H / 32), scb, fb, pol);
+    } else {
       const size_t eH = (size_t)P.ids[it.a] * H;
       const uint32_t runb = 16u * (I / 2), scb = 16u * (I / 32);
-      if (lane == 0) mbar_arrive_expect_tx(&full[s], runb + scb);
+      if (lane == 0) mbar_arrive_expect_tx(fb, runb + scb);
       __syncwarp();
-      if (lane == 0) bulk_g2s(st, Lp.w2c + (eH + it.b) * (I / 2), runb, &full[s], pol);
-      if (lane == 1) bulk_g2s(st + runb, Lp.w2s + (eH + it.b) * (I / 32), scb, &full[s], pol);
-    } else {
-      if (lane == 0) mbar_arrive_expect_tx(&full[s], 4u * 2u * Is);
-      __syncwarp();
-      if (lane == 0) bulk_g2s(st, Lp.sw2 + (size_t)it.a * Is, 4u * 2u * Is, &full[s], pol);
+      if (lane == 0) bulk_g2s(st, Lp.w2c + (eH + it.b) * (I / 2), runb, fb, pol);
+      if (lane == 1) bulk_g2s(st + runb, Lp.w2s + (eH + it.b) * (I / 32), scb, fb, pol);
     }
     ++i;
     return true;
-  }
-
-  // L2 prefetch of an item's bytes (same runs as issue()).
-  __device__ void prefetch(const LayerPtrs& Lp, const Plan* P, const Item& it) {
-    const int H = p.H, I = p.I, Is = p.Is;
-    if (it.type == IT_A) {
-      const int nr = p.E / 4;
-      if (it.a < nr) {
-        if (lane == 0) prefetch_l2(Lp.wr + (size_t)4 * it.a * H, 4u * 2u * H);
-      } else {
-        const int sh = it.a - nr;
-        if (lane == 0) prefetch_l2(Lp.sw13 + (size_t)2 * sh * H, 2u * 2u * H);
-        if (lane == 1) prefetch_l2(Lp.sw13 + (size_t)(Is + 2 * sh) * H, 2u * 2u * H);
-      }
-    } else if (it.type == IT_B) {
-      const size_t e2I = (size_t)P->ids[it.a] * 2 * I;
-      if (lane == 0) prefetch_l2(Lp.w13c + (e2I + it.b) * (H / 2), 8u * (H / 2));
-      if (lane == 1) prefetch_l2(Lp.w13c + (e2I + I + it.b) * (H / 2), 8u * (H / 2));
-      if (lane == 2) prefetch_l2(Lp.w13s + (e2I + it.b) * (H / 32), 8u * (H / 32));
-      if (lane == 3) prefetch_l2(Lp.w13s + (e2I + I + it.b) * (H / 32), 8u * (H / 32));
-    } else if (it.type == IT_CR) {
-      const size_t eH = (size_t)P->ids[it.a] * H;
-      if (lane == 0) prefetch_l2(Lp.w2c + (eH + it.b) * (I / 2), 16u * (I / 2));
-      if (lane == 1) prefetch_l2(Lp.w2s + (eH + it.b) * (I / 32), 16u * (I / 32));
-    } else {
-      if (lane == 0) prefetch_l2(Lp.sw2 + (size_t)it.a * Is, 4u * 2u * Is);
-    }
   }
 };
 
@@ -320,115 +419,174 @@ struct Producer {
 // consumer-side pieces
 // ---------------------------------------------------------------------------
 // Consumer-only barrier (the 4 consumer warps; the producer never joins).
-__device__ __forceinline__ void csync() { named_barrier(1, 32 * N_CONSUMERS); }
+__device__ __forceinline__ void csync() { named_barrier(1, 32 * STEP_CONSUMERS); }
 
 // The layer input in two forms: bf16 x_l (router / shared-expert operand) at
 // xb16 and f16 x_l scaled by a per-token power of two (MXFP4 operand) at xf16.
-// Layer 0 takes the input; later layers x = bf16(RMSNorm(h)).  One pass collects
-// the sum of squares and max |h| per token (deterministic reduction order, the same
-// in every block), the second writes both copies.  max_i bf16(|h_i| r) equals
-// bf16(max_i |h_i| r) because rounding is monotonic, so the shift is exact.
-__device__ void stage_layer_input(const StepParams& p, int l, uint8_t* xb16, uint8_t* xf16, uint32_t xss,
-                                  float* s_part, float* s_amx, float* s_r, int* s_sh, float* s_inv) {
+// Layer 0 takes the input; later layers x = bf16(RMSNorm(h)), h the previous
+// layer's residual buffer.  The same pass copies this block's slice of that
+// residual (or of fp32(input) at layer 0) into this layer's accumulation buffer.
+// The residual is read once when a thread's share fits in registers (STAGE_REG_F4
+// float4s), else twice.  Every block reduces in the same order (per thread over its
+// float4s, then the warp butterfly, then warps 0..3), so all blocks get the same
+// bits -- they take the top-k independently and must agree.  max_i bf16(|h_i| r)
+// equals bf16(max_i |h_i| r) because rounding is monotonic, so the shift is exact.
+__device__ __forceinline__ float4 load_residual4(const StepParams& p, int l, const float* hin, int q) {
+  if (l == 0) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p.x_in + 4 * (size_t)q);
+    const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
+    const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
+    return make_float4(__low2float(a), __high2float(a), __low2float(b), __high2float(b));
+  }
+  return __ldcg(reinterpret_cast<const float4*>(hin) + q);
+}
+__device__ __forceinline__ void write_layer_input4(uint8_t* xb16, uint8_t* xf16, uint32_t off, float4 v, float r,
+                                                   float sc) {
+  const __nv_bfloat162 a = __floats2bfloat162_rn(v.x * r, v.y * r);
+  const __nv_bfloat162 b = __floats2bfloat162_rn(v.z * r, v.w * r);
+  uint2 u;
+  u.x = *reinterpret_cast<const uint32_t*>(&a);
+  u.y = *reinterpret_cast<const uint32_t*>(&b);
+  *reinterpret_cast<uint2*>(xb16 + off) = u;
+  const __half2 ha = __floats2half2_rn(__low2float(a) * sc, __high2float(a) * sc);
+  const __half2 hb = __floats2half2_rn(__low2float(b) * sc, __high2float(b) * sc);
+  u.x = *reinterpret_cast<const uint32_t*>(&ha);
+  u.y = *reinterpret_cast<const uint32_t*>(&hb);
+  *reinterpret_cast<uint2*>(xf16 + off) = u;
+}
+__device__ __forceinline__ void accumulate4(float4 v, float& ss, float& am) {
+  ss = fmaf(v.x, v.x, ss);
+  ss = fmaf(v.y, v.y, ss);
+  ss = fmaf(v.z, v.z, ss);
+  ss = fmaf(v.w, v.w, ss);
+  am = fmaxf(am, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+}
+
+__device__ void stage_layer_input(const StepParams& p, int l, const float* hin, float* hout, uint8_t* xb16,
+                                  uint8_t* xf16, uint32_t xss, float* s_part, float* s_amx, float* s_r, int* s_sh,
+                                  float* s_inv) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int M = p.M, H = p.H, nt = 32 * N_CONSUMERS;
-  for (int tok = 0; tok < M; ++tok) {
-    float ss = 0.0f, am = 0.0f;
-    if (l == 0) {
-      for (int c = tid; c < H / 8; c += nt) {
-        const uint4 v = *reinterpret_cast<const uint4*>(p.x_in + (size_t)tok * H + 8 * c);
-        const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&v);
+  const int M = p.M, H = p.H, nt = 32 * STEP_CONSUMERS;
+  const int per = H / 4, Q = M * per;  // float4s per token / in total
+  const int q0 = (int)((long long)Q * blockIdx.x / gridDim.x), q1 = (int)((long long)Q * (blockIdx.x + 1) / gridDim.x);
+  float4* hout4 = reinterpret_cast<float4*>(hout);
+  const bool inreg = Q <= STAGE_REG_F4 * nt;
+  float4 v[STAGE_REG_F4];
+  int tq[STAGE_REG_F4], cq[STAGE_REG_F4];  // token and float4 column of q = tid + nt*j
+  if (inreg) {
+    {
+      int tok = tid / per, c = tid - tok * per;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) am = fmaxf(am, fmaxf(fabsf(__low2float(b[j])), fabsf(__high2float(b[j]))));
-      }
-    } else {
-      for (int c = tid; c < H / 4; c += nt) {
-        const float4 v = __ldcg(reinterpret_cast<const float4*>(p.h + (size_t)tok * H) + c);
-        ss = fmaf(v.x, v.x, ss);
-        ss = fmaf(v.y, v.y, ss);
-        ss = fmaf(v.z, v.z, ss);
-        ss = fmaf(v.w, v.w, ss);
-        am = fmaxf(am, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+      for (int j = 0; j < STAGE_REG_F4; ++j) {
+        tq[j] = tok;
+        cq[j] = c;
+        c += nt;
+        while (c >= per) {
+          c -= per;
+          ++tok;
+        }
       }
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      ss += __shfl_xor_sync(0xffffffffu, ss, o);
-      am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+    for (int j = 0; j < STAGE_REG_F4; ++j) {
+      const int q = tid + nt * j;
+      v[j] = q < Q ? load_residual4(p, l, hin, q) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    if (lane == 0) {
-      s_part[tok * N_CONSUMERS + warp] = ss;
-      s_amx[tok * N_CONSUMERS + warp] = am;
+#pragma unroll
+    for (int j = 0; j < STAGE_REG_F4; ++j) {
+      const int q = tid + nt * j;
+      if (q >= q0 && q < q1) hout4[q] = v[j];
+    }
+    for (int tok = 0; tok < M; ++tok) {
+      float ss = 0.0f, am = 0.0f;
+#pragma unroll
+      for (int j = 0; j < STAGE_REG_F4; ++j)
+        if (tq[j] == tok) accumulate4(v[j], ss, am);  // q >= Q: token M, never matched
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+      }
+      if (lane == 0) {
+        s_part[tok * STEP_CONSUMERS + warp] = ss;
+        s_amx[tok * STEP_CONSUMERS + warp] = am;
+      }
+    }
+  } else {
+    for (int tok = 0; tok < M; ++tok) {
+      float ss = 0.0f, am = 0.0f;
+      for (int c = tid; c < per; c += nt) {
+        const int q = tok * per + c;
+        const float4 w = load_residual4(p, l, hin, q);
+        if (q >= q0 && q < q1) hout4[q] = w;
+        accumulate4(w, ss, am);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+      }
+      if (lane == 0) {
+        s_part[tok * STEP_CONSUMERS + warp] = ss;
+        s_amx[tok * STEP_CONSUMERS + warp] = am;
+      }
     }
   }
   csync();
   if (tid < M) {
     float ss = 0.0f, am = 0.0f;
-    for (int w = 0; w < N_CONSUMERS; ++w) {
-      ss += s_part[tid * N_CONSUMERS + w];
-      am = fmaxf(am, s_amx[tid * N_CONSUMERS + w]);
+    for (int w = 0; w < STEP_CONSUMERS; ++w) {
+      ss += s_part[tid * STEP_CONSUMERS + w];
+      am = fmaxf(am, s_amx[tid * STEP_CONSUMERS + w]);
     }
     const float r = l == 0 ? 1.0f : 1.0f / sqrtf(ss / (float)H + p.eps);
     s_r[tid] = r;
-    const float amx = l == 0 ? am : __bfloat162float(__float2bfloat16_rn(am * r));
-    const int sh = f16_range_shift(amx);
+    const int sh = f16_range_shift(__bfloat162float(__float2bfloat16_rn(am * r)));
     s_sh[tid] = sh;
     s_inv[tid] = exp2i(-sh);
   }
   csync();
-  if (l == 0) {
-    for (int i = tid; i < M * (H / 8); i += nt) {
-      const int tok = i / (H / 8), c = i % (H / 8);
-      uint4 v = *reinterpret_cast<const uint4*>(p.x_in + (size_t)tok * H + 8 * c);
-      *reinterpret_cast<uint4*>(xb16 + tok * xss + 16 * c) = v;
-      const float sc = exp2i(s_sh[tok]);
-      uint32_t* w = reinterpret_cast<uint32_t*>(&v);
+  if (inreg) {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&w[j]);
-        const __half2 hh = __floats2half2_rn(__low2float(b) * sc, __high2float(b) * sc);
-        w[j] = *reinterpret_cast<const uint32_t*>(&hh);
-      }
-      *reinterpret_cast<uint4*>(xf16 + tok * xss + 16 * c) = v;
-    }
+    for (int j = 0; j < STAGE_REG_F4; ++j)
+      if (tq[j] < M)
+        write_layer_input4(xb16, xf16, tq[j] * xss + 8 * cq[j], v[j], s_r[tq[j]], exp2i(s_sh[tq[j]]));
   } else {
-    for (int i = tid; i < M * (H / 4); i += nt) {
-      const int tok = i / (H / 4), c = i % (H / 4);
-      const float4 v = __ldcg(reinterpret_cast<const float4*>(p.h + (size_t)tok * H) + c);
-      const float r = s_r[tok], sc = exp2i(s_sh[tok]);
-      const __nv_bfloat162 a = __floats2bfloat162_rn(v.x * r, v.y * r);
-      const __nv_bfloat162 b = __floats2bfloat162_rn(v.z * r, v.w * r);
-      uint2 u;
-      u.x = *reinterpret_cast<const uint32_t*>(&a);
-      u.y = *reinterpret_cast<const uint32_t*>(&b);
-      *reinterpret_cast<uint2*>(xb16 + tok * xss + 8 * c) = u;
-      const __half2 ha = __floats2half2_rn(__low2float(a) * sc, __high2float(a) * sc);
-      const __half2 hb = __floats2half2_rn(__low2float(b) * sc, __high2float(b) * sc);
-      u.x = *reinterpret_cast<const uint32_t*>(&ha);
-      u.y = *reinterpret_cast<const uint32_t*>(&hb);
-      *reinterpret_cast<uint2*>(xf16 + tok * xss + 8 * c) = u;
+    for (int q = tid; q < Q; q += nt) {
+      const int tok = q / per, c = q - tok * per;
+      write_layer_input4(xb16, xf16, tok * xss + 8 * c, load_residual4(p, l, hin, q), s_r[tok], exp2i(s_sh[tok]));
     }
   }
-  csync();
+  csync();  // also orders this block's slice stores before the h-init hand-off
 }
 
 // Top-k of every token from the complete router logits (same rule as k_dense:
-// largest logit, lowest index on ties), then the union plan.  The 4 consumer warps
-// each take a quarter of the experts and keep their own top-k (a global top-k
-// element is always in its quarter's top-k, ties included), then one warp per
-// token merges the 4k candidates.
+// largest logit, lowest index on ties), then the union plan.  The 8 consumer warps
+// each take an eighth of the experts and keep their own top-k (a global top-k
+// element is always in its part's top-k, ties included), then one warp per token
+// merges the 8k candidates.
 __device__ void step_topk(const StepParams& p, int l, Plan& P, int32_t* s_ids, float* s_wts, uint32_t* s_ck,
-                          int32_t* s_ci) {
+                          int32_t* s_ci, volatile int* s_abort_ptr) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int E = p.E, k = p.k, M = p.M;
-  const int per = (E + N_CONSUMERS - 1) / N_CONSUMERS;  // experts per warp (<= 256)
+  const int per = (E + STEP_CONSUMERS - 1) / STEP_CONSUMERS;  // experts per warp (<= 256)
   const int e0 = warp * per;
   for (int tok = 0; tok < M; ++tok) {
     uint32_t key[8];
+    {
+      const unsigned long long* w[8];
+      int n = 0;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int off = lane + 32 * i, e = e0 + off;
-      key[i] = (off < per && e < E) ? float_key(__ldcg(p.logits + tok * E + e)) : 0u;
+      for (int i = 0; i < 8; ++i) {
+        const int off = lane + 32 * i, e = e0 + off;
+        w[i] = p.logits + tok * E + e;
+        if (off < per && e < E) n = i + 1;  // valid columns are a prefix
+      }
+      float lv[8];
+      if (!await_tagged(w, n, (uint32_t)l + 1u, lv, p.status, s_abort_ptr))
+        n = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) key[i] = i < n ? float_key(lv[i]) : 0u;
     }
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
@@ -447,30 +605,39 @@ __device__ void step_topk(const StepParams& p, int l, Plan& P, int32_t* s_ids, f
         for (int i = 0; i < 8; ++i)
           if (e0 + lane + 32 * i == mi) key[i] = 0u;
         if (lane == 0) {
-          s_ck[(tok * N_CONSUMERS + warp) * 8 + j] = mk;
-          s_ci[(tok * N_CONSUMERS + warp) * 8 + j] = mk ? mi : 0x7fffffff;
+          s_ck[(tok * STEP_CONSUMERS + warp) * 8 + j] = mk;
+          s_ci[(tok * STEP_CONSUMERS + warp) * 8 + j] = mk ? mi : 0x7fffffff;
         }
       }
     }
   }
   csync();
-  for (int tok = warp; tok < M; tok += N_CONSUMERS) {
-    const int nc = N_CONSUMERS * k;  // <= 32 candidates, one per lane
-    uint32_t ck = 0u;
-    int ci = 0x7fffffff;
-    if (lane < nc) {
-      ck = s_ck[(tok * N_CONSUMERS + lane / k) * 8 + lane % k];
-      ci = s_ci[(tok * N_CONSUMERS + lane / k) * 8 + lane % k];
+  for (int tok = warp; tok < M; tok += STEP_CONSUMERS) {
+    const int nc = STEP_CONSUMERS * k;  // <= 64 candidates, two per lane
+    uint32_t ck[2] = {0u, 0u};
+    int ci[2] = {0x7fffffff, 0x7fffffff};
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int c = lane + 32 * r;
+      if (c < nc) {
+        ck[r] = s_ck[(tok * STEP_CONSUMERS + c / k) * 8 + c % k];
+        ci[r] = s_ci[(tok * STEP_CONSUMERS + c / k) * 8 + c % k];
+      }
     }
     int sel_id = 0;
     uint32_t sel_key = 0u;
     for (int j = 0; j < k; ++j) {
-      const uint32_t mk = __reduce_max_sync(0xffffffffu, ck);
-      const int mi = (int)__reduce_min_sync(0xffffffffu, (unsigned)(ck == mk ? ci : 0x7fffffff));
-      if (ck == mk && ci == mi) {
-        ck = 0u;
-        ci = 0x7fffffff;
-      }
+      const int b = (ck[1] > ck[0] || (ck[1] == ck[0] && ci[1] < ci[0])) ? 1 : 0;
+      const uint32_t bk = b ? ck[1] : ck[0];
+      const int bi = b ? ci[1] : ci[0];
+      const uint32_t mk = __reduce_max_sync(0xffffffffu, bk);
+      const int mi = (int)__reduce_min_sync(0xffffffffu, (unsigned)(bk == mk ? bi : 0x7fffffff));
+#pragma unroll
+      for (int r = 0; r < 2; ++r)
+        if (ck[r] == mk && ci[r] == mi) {
+          ck[r] = 0u;
+          ci[r] = 0x7fffffff;
+        }
       if (lane == j) {
         sel_id = mi;
         sel_key = mk;
@@ -540,182 +707,233 @@ __device__ __forceinline__ void rows4_dot(const uint8_t* wrows, uint32_t wstride
 __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant__ StepParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ Plan P;
-  __shared__ float s_part[MAX_M * N_CONSUMERS];
+  __shared__ float s_part[MAX_M * STEP_CONSUMERS];
   __shared__ float s_r[MAX_M];
   __shared__ float s_inv[MAX_M];
-  __shared__ float s_pscale[N_CONSUMERS][MAX_M];
+  __shared__ float s_pscale[CR_CACHE][MAX_M];
   __shared__ int32_t s_ids[MAX_SLOTS];
   __shared__ float s_wts[MAX_SLOTS];
-  __shared__ float s_amx[MAX_M * N_CONSUMERS];
+  __shared__ float s_amx[MAX_M * STEP_CONSUMERS];
   __shared__ int s_sh[MAX_M];
-  __shared__ uint32_t s_ck[MAX_M * N_CONSUMERS * 8];
-  __shared__ int32_t s_ci[MAX_M * N_CONSUMERS * 8];
+  __shared__ uint32_t s_ck[MAX_M * STEP_CONSUMERS * 8];
+  __shared__ int32_t s_ci[MAX_M * STEP_CONSUMERS * 8];
+  __shared__ uint32_t s_fs[STEP_SLOTS], s_fe[STEP_SLOTS];
   __shared__ volatile int s_abort;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
-  const int M = p.M, H = p.H, I = p.I, Is = p.Is, L = p.L, S = p.stages;
+  const int M = p.M, H = p.H, I = p.I, Is = p.Is, L = p.L;
+  const uint32_t R = p.ring_bytes;
   const unsigned G = gridDim.x;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);
-  uint64_t* empty = full + MAX_STAGES;
-  uint64_t* plan_bar = empty + MAX_STAGES;
-  uint8_t* stages = smem + STEP_FIXED;
-  const size_t sbytes = step_stage_bytes(H, I, Is);
-  uint8_t* act = stages + (size_t)S * sbytes;
+  uint64_t* empty = full + STEP_SLOTS;
+  uint64_t* plan_bar = empty + STEP_SLOTS;  // consumers -> producer: this layer's plan is built
+  uint64_t* hinit_bar = plan_bar + 1;       // consumers -> producer: this block's h slice is copied
+  uint8_t* ring = smem + STEP_FIXED;
+  uint8_t* act = ring + R;
   const uint32_t xss = padded_stride(2u * H);
   const uint32_t sss = Is > 0 ? padded_stride(2u * Is) : 0u;
   const uint32_t ass = padded_stride(2u * I);
-  uint8_t* xb16 = act;                                 // A/B phases: bf16 x rows [M][xss]
-  uint8_t* xf16 = act + (size_t)M * xss;               //             f16 x rows  [M][xss]
-  uint8_t* shi = act;                                  // C phase: shared a, bf16 hi  [M][sss]
-  uint8_t* slo = act + (size_t)M * sss;                //                    bf16 lo  [M][sss]
-  uint8_t* afw = act + 2 * (size_t)M * sss;            //          routed a per warp [4][M][ass]
+  uint8_t* xb16 = act;                    // A phase: bf16 x rows [M][xss]
+  uint8_t* xf16 = act + (size_t)M * xss;  // B phase: f16 x rows  [M][xss]
+  uint8_t* shi = step_shared_over_xb16(H, Is) ? act : act + 2 * (size_t)M * xss;  // CS: shared a, bf16 hi
+  uint8_t* slo = shi + (size_t)M * sss;                                            //     bf16 lo
+  uint8_t* afc = act;                     // CR phase: routed a of the block's experts [CR_CACHE][M][ass]
+  const uint32_t bytesA = step_item_bytes(IT_A, H, I, Is), bytesS = step_item_bytes(IT_CS, H, I, Is);
+  const uint32_t bytesB = step_item_bytes(IT_B, H, I, Is), bytesC = step_item_bytes(IT_CR, H, I, Is);
 
   if (tid == 0) {
-    for (int s = 0; s < S; ++s) {
+    for (int s = 0; s < STEP_SLOTS; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
     mbar_init(plan_bar, 1);
+    mbar_init(hinit_bar, 1);
     fence_mbar_init();
     s_abort = 0;
   }
   __syncthreads();
 
   // ---------------- producer ----------------
-  if (warp == N_CONSUMERS) {
-    Producer pr{p, stages, sbytes, full, empty, policy_evict_first(), S, 0, &s_abort, lane};
+  if (warp == STEP_CONSUMERS) {
+    Producer pr{p,  ring, R,  full, empty, s_fs, s_fe, policy_evict_first(), 0, 0, 0, 0u, 0u,
+                p.inflight_bytes ? p.inflight_bytes : R, &s_abort, lane};
     bool ok = true;
     for (int l = 0; l < L && ok; ++l) {
       const LayerPtrs& Lp = p.layer[l];
       Work W;
-      W.init_A(p);
-      for (int r = 0; r < W.nA && ok; ++r) ok = pr.issue(Lp, P, W.at(p, r));
+      W.init_fixed(p);
+      for (int r = 0; r < W.nA + W.nS && ok; ++r) ok = pr.issue(Lp, P, W.at(p, r));
       if (!ok) break;
       stamp(p, l, 12);
-      // routing-independent items: this layer's shared W2, the next layer's router/shared W13
-      for (int r = 0; r < W.nS; ++r) pr.prefetch(Lp, nullptr, W.at(p, W.nA + r));
-      if (l + 1 < L)
-        for (int r = 0; r < W.nA; ++r) pr.prefetch(p.layer[l + 1], nullptr, W.at(p, r));
       int got = 1;
+      // the consumers' slice copy of h (ordered before their arrive by a block
+      // barrier) is published here, off their critical path: fence, then count
+      if (lane == 0) {
+        got = ring_wait(hinit_bar, (uint32_t)(l & 1), p.status, &s_abort);
+        if (got) signal_counter(p.ctr + (size_t)l * CTR_PER_LAYER + CTR_HINIT);
+      }
+      if (!__shfl_sync(0xffffffffu, got, 0)) break;
       if (lane == 0) got = ring_wait(plan_bar, (uint32_t)(l & 1), p.status, &s_abort);
       if (!__shfl_sync(0xffffffffu, got, 0)) break;
       stamp(p, l, 13);
       W.init_routed(p, P.n_unique);
-      const int nR = (int)(W.nB + W.nC);
-      for (int r = 0; r < nR && r < STEP_PREFETCH_AHEAD; ++r) pr.prefetch(Lp, &P, W.at(p, W.nA + r));
-      for (int r = 0; r < nR && ok; ++r) {
-        if (r + STEP_PREFETCH_AHEAD < nR) pr.prefetch(Lp, &P, W.at(p, W.nA + r + STEP_PREFETCH_AHEAD));
-        ok = pr.issue(Lp, P, W.at(p, W.nA + r));
-      }
+      const long long nR = W.nB + W.nC;
+      for (long long r = 0; r < nR && ok; ++r) ok = pr.issue(Lp, P, W.at(p, W.nA + W.nS + r));
       stamp(p, l, 14);
-      for (int r = 0; r < W.nS && ok; ++r) ok = pr.issue(Lp, P, W.at(p, W.nA + nR + r));
-      stamp(p, l, 15);
     }
-    // drain: the last use of every stage has landed before the block may exit
-    if (lane == 0 && !s_abort)
-      for (long long j = (pr.i > S ? pr.i - S : 0); j < pr.i; ++j)
-        ring_wait(&full[j % S], (uint32_t)((j / S) & 1), p.status, &s_abort);
+    // every copy issued lands before the block may exit
+    if (lane == 0)
+      for (long long j = (pr.i > STEP_SLOTS ? pr.i - STEP_SLOTS : 0); j < pr.i; ++j)
+        drain_wait(&full[j % STEP_SLOTS], (uint32_t)((j / STEP_SLOTS) & 1));
     return;
   }
 
   // ---------------- consumers ----------------
   unsigned* ctr = p.ctr;
-  long long i = 0;  // ring index
+  long long i = 0;   // ring item
+  uint32_t pos = 0;  // ring placement cursor (same walk as the producer's)
   for (int l = 0; l < L; ++l) {
     unsigned* lc = ctr + (size_t)l * CTR_PER_LAYER;
+    float* hout = p.h + (size_t)(l & 1) * M * H;
+    const float* hin = p.h + (size_t)((l + 1) & 1) * M * H;  // layer l-1's buffer
     stamp(p, l, 0);
     if (l > 0) {
       if (tid == 0) wait_counter(ctr + (size_t)(l - 1) * CTR_PER_LAYER + CTR_H, G, p.status, &s_abort);
       csync();
     }
     stamp(p, l, 1);
-    stage_layer_input(p, l, xb16, xf16, xss, s_part, s_amx, s_r, s_sh, s_inv);
+    stage_layer_input(p, l, hin, hout, xb16, xf16, xss, s_part, s_amx, s_r, s_sh, s_inv);
+    if (tid == 0) mbar_arrive(hinit_bar);
     stamp(p, l, 2);
-    if (blockIdx.x == 0) {
-      for (int e = tid; e < M * H; e += 32 * N_CONSUMERS) {
+    if (blockIdx.x == 0 && (p.x_trace || p.h_trace)) {
+      for (int e = tid; e < M * H; e += 32 * STEP_CONSUMERS) {
         const int tok = e / H, c = e % H;
         const __nv_bfloat16 xv = *reinterpret_cast<const __nv_bfloat16*>(xb16 + tok * xss + 2 * c);
-        float hv;
-        if (l == 0) {
-          hv = __bfloat162float(xv);
-          p.h[e] = hv;
-        } else {
-          hv = __ldcg(p.h + e);
-        }
+        const float hv = l == 0 ? __bfloat162float(p.x_in[e]) : __ldcg(hin + e);
         if (p.x_trace) p.x_trace[(size_t)l * M * H + e] = xv;
         if (p.h_trace) p.h_trace[(size_t)l * M * H + e] = hv;
-      }
-      if (l == 0) {
-        csync();
-        if (tid == 0) signal_counter(ctr + 3);  // h initialised
       }
     }
 
     // ---- A: router items (4 experts) and shared-W13 items (2 gate + 2 up rows) ----
     Work W;
-    W.init_A(p);
+    W.init_fixed(p);
     const int nr = p.E / 4;
-    for (int r = 0; r < W.nA; ++r) {
-      const long long ii = i + r;
-      if ((int)(ii % N_CONSUMERS) != warp) continue;
-      const int s = (int)(ii % S);
+    for (int r = 0; r < W.nA; ++r, ++i) {
+      const uint32_t s0 = ring_take(pos, bytesA, R);
+      if ((int)(i % STEP_CONSUMERS) != warp) continue;
+      const int slot = (int)(i % STEP_SLOTS);
       const Item it = W.at(p, r);
       const bool router = it.a < nr;
       float c[4] = {0.f, 0.f, 0.f, 0.f};
-      item_stamp(p, ii, 3);
-      if (ring_wait(&full[s], (uint32_t)((ii / S) & 1), p.status, &s_abort)) {
-        item_stamp(p, ii, 1);
+      item_stamp(p, i, 3);
+      if (ring_wait(&full[slot], (uint32_t)((i / STEP_SLOTS) & 1), p.status, &s_abort)) {
+        item_stamp(p, i, 1);
         // shared items: columns (0,1,2,3) = (gate 2s, up 2s, gate 2s+1, up 2s+1) from
         // smem rows (0, 2, 1, 3), so a thread's two columns are a (gate, up) pair
         const int wrow = g < 4 ? (router ? g : ((g & 1) ? 2 : 0) + (g >> 1)) : -1;
-        rows4_dot(stages + (size_t)s * sbytes, 2u * H, wrow, g < M ? xb16 + g * xss : nullptr, nullptr, H, c);
+        rows4_dot(ring + s0, 2u * H, wrow, g < M ? xb16 + g * xss : nullptr, nullptr, H, c);
       }
       __syncwarp();
-      item_stamp(p, ii, 2);
-      if (lane == 0) mbar_arrive(&empty[s]);
+      item_stamp(p, i, 2);
+      if (lane == 0) mbar_arrive(&empty[slot]);
       if (t < 2 && g < M) {
+        const uint32_t tag = (uint32_t)l + 1u;
         if (router) {
-          p.logits[g * p.E + 4 * it.a + 2 * t] = c[0];
-          p.logits[g * p.E + 4 * it.a + 2 * t + 1] = c[1];
+          st_tagged(p.logits + g * p.E + 4 * it.a + 2 * t, c[0], tag);
+          st_tagged(p.logits + g * p.E + 4 * it.a + 2 * t + 1, c[1], tag);
         } else {
-          p.a_shared[g * Is + 2 * (it.a - nr) + t] = silu_f32(c[0]) * c[1];
+          st_tagged(p.a_shared + g * Is + 2 * (it.a - nr) + t, silu_f32(c[0]) * c[1], tag);
         }
       }
-      __syncwarp();
-      if (lane == 0) signal_counter(lc + (router ? CTR_ROUTER : CTR_SHARED));
     }
-    i += W.nA;
     stamp(p, l, 3);
 
-    // ---- top-k and plan (every block, identical) ----
-    if (tid == 0) wait_counter(lc + CTR_ROUTER, (unsigned)(p.E / 4), p.status, &s_abort);
-    csync();
+    // ---- top-k and plan (every block, identical; polls the tagged logits) ----
     stamp(p, l, 4);
-    step_topk(p, l, P, s_ids, s_wts, s_ck, s_ci);
+    step_topk(p, l, P, s_ids, s_wts, s_ck, s_ci, &s_abort);
     if (tid == 0) mbar_arrive(plan_bar);
     stamp(p, l, 5);
-    W.init_routed(p, P.n_unique);
+
+    // ---- CS: shared W2 (activation as bf16 hi + lo), accumulated into h ----
+    if (W.nS > 0) {
+      for (int e = tid; e < M * (Is / 8); e += 32 * STEP_CONSUMERS) {
+        const int tok = e / (Is / 8), c8 = e % (Is / 8);
+        const unsigned long long* w[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) w[j] = p.a_shared + (size_t)tok * Is + 8 * c8 + j;
+        float a8[8];
+        if (!await_tagged(w, 8, (uint32_t)l + 1u, a8, p.status, &s_abort)) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) a8[j] = 0.0f;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const __nv_bfloat16 hi = __float2bfloat16_rn(a8[j]);
+          const __nv_bfloat16 lo = __float2bfloat16_rn(a8[j] - __bfloat162float(hi));
+          *reinterpret_cast<__nv_bfloat16*>(shi + tok * sss + 2 * (8 * c8 + j)) = hi;
+          *reinterpret_cast<__nv_bfloat16*>(slo + tok * sss + 2 * (8 * c8 + j)) = lo;
+        }
+      }
+    }
+    if (tid == 0) wait_counter(lc + CTR_HINIT, G, p.status, &s_abort);  // every slice of h initialised
+    csync();
     stamp(p, l, 6);
+    for (int r = 0; r < W.nS; ++r, ++i) {
+      const uint32_t s0 = ring_take(pos, bytesS, R);
+      if ((int)(i % STEP_CONSUMERS) != warp) continue;
+      const int slot = (int)(i % STEP_SLOTS);
+      const Item it = W.at(p, W.nA + r);
+      // 4 output rows (N) against the activation rows m = 2*token + {hi, lo} (M)
+      float c[4] = {0.f, 0.f, 0.f, 0.f};
+      item_stamp(p, i, 3);
+      if (ring_wait(&full[slot], (uint32_t)((i / STEP_SLOTS) & 1), p.status, &s_abort)) {
+        item_stamp(p, i, 1);
+        const uint8_t* src = (g & 1) ? slo : shi;
+        const int t0 = g >> 1, t1 = 4 + (g >> 1);
+        rows4_dot(ring + s0, 2u * Is, g < 4 ? g : -1, t0 < M ? src + t0 * sss : nullptr,
+                  t1 < M ? src + t1 * sss : nullptr, Is, c);
+      }
+      __syncwarp();
+      item_stamp(p, i, 2);
+      if (lane == 0) mbar_arrive(&empty[slot]);
+      // hi + lo: rows m = 2tok (lane group g even) and 2tok + 1 (g odd)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) c[e] += __shfl_xor_sync(0xffffffffu, c[e], 4);
+      if ((g & 1) == 0 && t < 2) {
+        const int t0 = g >> 1, t1 = 4 + (g >> 1);
+        if (t0 < M) {
+          atomicAdd(hout + (size_t)t0 * H + it.a + 2 * t, c[0]);
+          atomicAdd(hout + (size_t)t0 * H + it.a + 2 * t + 1, c[1]);
+        }
+        if (t1 < M) {
+          atomicAdd(hout + (size_t)t1 * H + it.a + 2 * t, c[2]);
+          atomicAdd(hout + (size_t)t1 * H + it.a + 2 * t + 1, c[3]);
+        }
+      }
+    }
+    stamp(p, l, 7);
 
     // ---- B: routed W13 + SwiGLU ----
-    for (int r = 0; r < W.nB; ++r) {
-      const long long ii = i + r;
-      if ((int)(ii % N_CONSUMERS) != warp) continue;
-      const int s = (int)(ii % S);
-      const Item it = W.at(p, W.nA + r);
+    W.init_routed(p, P.n_unique);
+    for (long long r = 0; r < W.nB; ++r, ++i) {
+      const uint32_t s0 = ring_take(pos, bytesB, R);
+      if ((int)(i % STEP_CONSUMERS) != warp) continue;
+      const int slot = (int)(i % STEP_SLOTS);
+      const Item it = W.at(p, W.nA + W.nS + r);
       float c[4] = {0.f, 0.f, 0.f, 0.f};
-      item_stamp(p, ii, 3);
-      if (ring_wait(&full[s], (uint32_t)((ii / S) & 1), p.status, &s_abort)) {
-        item_stamp(p, ii, 1);
-        const uint8_t* st = stages + (size_t)s * sbytes;
+      item_stamp(p, i, 3);
+      if (ring_wait(&full[slot], (uint32_t)((i / STEP_SLOTS) & 1), p.status, &s_abort)) {
+        item_stamp(p, i, 1);
+        const uint8_t* st = ring + s0;
         const uint8_t* sc = st + 8 * H;  // 16 scale rows of H/32 after the 16 code rows of H/2
         mxfp4_tile_dot(st + g * (H / 2), st + (8 + g) * (H / 2), sc + g * (H / 32), sc + (8 + g) * (H / 32), H / 32,
                        xf16, xss, M, c);
       }
       __syncwarp();
-      item_stamp(p, ii, 2);
-      if (lane == 0) mbar_arrive(&empty[s]);
+      item_stamp(p, i, 2);
+      if (lane == 0) mbar_arrive(&empty[slot]);
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int tok = 2 * t + e;  // rows g (gate) and g+8 (up) of intermediate index it.b + g
@@ -725,134 +943,87 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
       __syncwarp();
       if (lane == 0) signal_counter(lc + CTR_EXP + it.a);
     }
-    i += W.nB;
-    stamp(p, l, 7);
-    csync();  // the activation region is free for the C phase
     stamp(p, l, 8);
-
-    // ---- C: routed W2 (weighted) + shared W2, accumulated into h ----
-    if (W.nS > 0) {
-      if (tid == 0) wait_counter(lc + CTR_SHARED, (unsigned)(Is / 2), p.status, &s_abort);
-      csync();
-      for (int e = tid; e < M * (Is / 4); e += 32 * N_CONSUMERS) {
-        const int tok = e / (Is / 4), c4 = e % (Is / 4);
-        const float4 v = __ldcg(reinterpret_cast<const float4*>(p.a_shared + (size_t)tok * Is) + c4);
-        const float a4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const __nv_bfloat16 hi = __float2bfloat16_rn(a4[j]);
-          const __nv_bfloat16 lo = __float2bfloat16_rn(a4[j] - __bfloat162float(hi));
-          *reinterpret_cast<__nv_bfloat16*>(shi + tok * sss + 2 * (4 * c4 + j)) = hi;
-          *reinterpret_cast<__nv_bfloat16*>(slo + tok * sss + 2 * (4 * c4 + j)) = lo;
-        }
-      }
-      csync();
-    }
-    if (l == 0) {
-      if (tid == 0) wait_counter(ctr + 3, 1u, p.status, &s_abort);  // h initialised by block 0
-      csync();
-    }
+    csync();  // xf16 and the shared halves are dead: the routed-W2 activation copies take the region
     stamp(p, l, 9);
-    int cached_slot = -1;
-    uint8_t* my_af = afw + (size_t)warp * M * ass;
-    const int nC = (int)W.nC;
-    for (int r = 0; r < nC + W.nS; ++r) {
-      const long long ii = i + r;
-      if ((int)(ii % N_CONSUMERS) != warp) continue;
-      const int s = (int)(ii % S);
-      const Item it = W.at(p, W.nA + (int)W.nB + r);
-      const uint8_t* st = stages + (size_t)s * sbytes;
-      if (it.type == IT_CR) {
-        const int u = it.a;
-        if (u != cached_slot) {
-          if (lane == 0) wait_counter(lc + CTR_EXP + u, (unsigned)(I / 8), p.status, &s_abort);
-          __syncwarp();
-          for (int tok = 0; tok < M; ++tok) {
-            const bool live = P.w[u][tok] != 0.0f;
-            const float4* src = reinterpret_cast<const float4*>(p.a_routed + ((size_t)u * M + tok) * I);
-            float4 v[8];  // I <= 1024: at most 8 float4 per lane
-            float amax = 0.0f;
-#pragma unroll
-            for (int jj = 0; jj < 8; ++jj) {
-              const int c4 = lane + 32 * jj;
-              v[jj] = (live && c4 < I / 4) ? __ldcg(src + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
-              amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v[jj].x), fabsf(v[jj].y)), fmaxf(fabsf(v[jj].z), fabsf(v[jj].w))));
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-            const int sh = f16_range_shift(amax);
-            const float scl = exp2i(sh);
-#pragma unroll
-            for (int jj = 0; jj < 8; ++jj) {
-              const int c4 = lane + 32 * jj;
-              if (c4 < I / 4) {
-                const __half2 h0 = __floats2half2_rn(v[jj].x * scl, v[jj].y * scl);
-                const __half2 h1 = __floats2half2_rn(v[jj].z * scl, v[jj].w * scl);
-                uint2 u2;
-                u2.x = *reinterpret_cast<const uint32_t*>(&h0);
-                u2.y = *reinterpret_cast<const uint32_t*>(&h1);
-                *reinterpret_cast<uint2*>(my_af + tok * ass + 8 * c4) = u2;
-              }
-            }
-            if (lane == 0) s_pscale[warp][tok] = live ? exp2i(-sh) : 0.0f;
-          }
-          __syncwarp();
-          cached_slot = u;
-        }
-        float c[4] = {0.f, 0.f, 0.f, 0.f};
-        item_stamp(p, ii, 3);
-      if (ring_wait(&full[s], (uint32_t)((ii / S) & 1), p.status, &s_abort)) {
-          item_stamp(p, ii, 1);
-          const uint8_t* sc = st + 8 * I;  // 16 scale rows of I/32 after the 16 code rows of I/2
-          mxfp4_tile_dot(st + g * (I / 2), st + (8 + g) * (I / 2), sc + g * (I / 32), sc + (8 + g) * (I / 32), I / 32,
-                         my_af, ass, M, c);
-        }
+
+    // ---- CR: routed W2 (weighted), accumulated into h ----
+    // The block's contiguous range touches experts u_first..u_last (at most CR_CACHE,
+    // checked by the host).  Warp w stages expert u_first + w's activation once its
+    // W13 items are complete everywhere: f16 with its own power-of-two shift.
+    const long long baseC = W.nA + W.nS + W.nB;
+    const int u_first = W.nC > 0 ? W.at(p, baseC).a : 0;
+    if (W.nC > 0) {
+      const int u_last = W.at(p, baseC + W.nC - 1).a;
+      const int u = u_first + warp;
+      if (warp < CR_CACHE && u <= u_last) {
+        if (lane == 0) wait_counter(lc + CTR_EXP + u, (unsigned)(I / 8), p.status, &s_abort);
         __syncwarp();
-        item_stamp(p, ii, 2);
-        if (lane == 0) mbar_arrive(&empty[s]);
+        uint8_t* dst = afc + (size_t)warp * M * ass;
+        for (int tok = 0; tok < M; ++tok) {
+          const bool live = P.w[u][tok] != 0.0f;
+          const float4* src = reinterpret_cast<const float4*>(p.a_routed + ((size_t)u * M + tok) * I);
+          float4 v[8];  // I <= 1024: at most 8 float4 per lane
+          float amax = 0.0f;
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int tok = 2 * t + e;
-          if (tok < M) {
-            const float wt = P.w[u][tok];
-            if (wt != 0.0f) {
-              const float f = wt * s_pscale[warp][tok];
-              atomicAdd(p.h + (size_t)tok * H + it.b + g, c[e] * f);
-              atomicAdd(p.h + (size_t)tok * H + it.b + g + 8, c[2 + e] * f);
+          for (int jj = 0; jj < 8; ++jj) {
+            const int c4 = lane + 32 * jj;
+            v[jj] = (live && c4 < I / 4) ? __ldcg(src + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
+            amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v[jj].x), fabsf(v[jj].y)), fmaxf(fabsf(v[jj].z), fabsf(v[jj].w))));
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+          const int sh = f16_range_shift(amax);
+          const float scl = exp2i(sh);
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) {
+            const int c4 = lane + 32 * jj;
+            if (c4 < I / 4) {
+              const __half2 h0 = __floats2half2_rn(v[jj].x * scl, v[jj].y * scl);
+              const __half2 h1 = __floats2half2_rn(v[jj].z * scl, v[jj].w * scl);
+              uint2 u2;
+              u2.x = *reinterpret_cast<const uint32_t*>(&h0);
+              u2.y = *reinterpret_cast<const uint32_t*>(&h1);
+              *reinterpret_cast<uint2*>(dst + tok * ass + 8 * c4) = u2;
             }
           }
+          if (lane == 0) s_pscale[warp][tok] = live ? exp2i(-sh) : 0.0f;
         }
-      } else {
-        // shared W2: 4 output rows (N) against the activation rows m = 2*token + {hi, lo} (M)
-        float c[4] = {0.f, 0.f, 0.f, 0.f};
-        item_stamp(p, ii, 3);
-      if (ring_wait(&full[s], (uint32_t)((ii / S) & 1), p.status, &s_abort)) {
-          item_stamp(p, ii, 1);
-          const uint8_t* src = (g & 1) ? slo : shi;
-          const int t0 = g >> 1, t1 = 4 + (g >> 1);
-          rows4_dot(st, 2u * Is, g < 4 ? g : -1, t0 < M ? src + t0 * sss : nullptr,
-                    t1 < M ? src + t1 * sss : nullptr, Is, c);
-        }
-        __syncwarp();
-        item_stamp(p, ii, 2);
-        if (lane == 0) mbar_arrive(&empty[s]);
-        // hi + lo: rows m = 2tok (lane group g even) and 2tok + 1 (g odd)
+      }
+      csync();
+    }
+    for (long long r = 0; r < W.nC; ++r, ++i) {
+      const uint32_t s0 = ring_take(pos, bytesC, R);
+      if ((int)(i % STEP_CONSUMERS) != warp) continue;
+      const int slot = (int)(i % STEP_SLOTS);
+      const Item it = W.at(p, baseC + r);
+      const int cu = it.a - u_first;  // cache entry
+      const uint8_t* my_af = afc + (size_t)cu * M * ass;
+      float c[4] = {0.f, 0.f, 0.f, 0.f};
+      item_stamp(p, i, 3);
+      if (ring_wait(&full[slot], (uint32_t)((i / STEP_SLOTS) & 1), p.status, &s_abort)) {
+        item_stamp(p, i, 1);
+        const uint8_t* st = ring + s0;
+        const uint8_t* sc = st + 8 * I;  // 16 scale rows of I/32 after the 16 code rows of I/2
+        mxfp4_tile_dot(st + g * (I / 2), st + (8 + g) * (I / 2), sc + g * (I / 32), sc + (8 + g) * (I / 32), I / 32,
+                       my_af, ass, M, c);
+      }
+      __syncwarp();
+      item_stamp(p, i, 2);
+      if (lane == 0) mbar_arrive(&empty[slot]);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) c[e] += __shfl_xor_sync(0xffffffffu, c[e], 4);
-        if ((g & 1) == 0 && t < 2) {
-          const int t0 = g >> 1, t1 = 4 + (g >> 1);
-          if (t0 < M) {
-            atomicAdd(p.h + (size_t)t0 * H + it.a + 2 * t, c[0]);
-            atomicAdd(p.h + (size_t)t0 * H + it.a + 2 * t + 1, c[1]);
-          }
-          if (t1 < M) {
-            atomicAdd(p.h + (size_t)t1 * H + it.a + 2 * t, c[2]);
-            atomicAdd(p.h + (size_t)t1 * H + it.a + 2 * t + 1, c[3]);
+      for (int e = 0; e < 2; ++e) {
+        const int tok = 2 * t + e;
+        if (tok < M) {
+          const float wt = P.w[it.a][tok];
+          if (wt != 0.0f) {
+            const float f = wt * s_pscale[cu][tok];
+            atomicAdd(hout + (size_t)tok * H + it.b + g, c[e] * f);
+            atomicAdd(hout + (size_t)tok * H + it.b + g + 8, c[2 + e] * f);
           }
         }
       }
     }
-    i += nC + W.nS;
     stamp(p, l, 10);
     csync();
     if (tid == 0) signal_counter(lc + CTR_H);
@@ -863,10 +1034,11 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
   if (blockIdx.x != 0) return;
   if (tid == 0) wait_counter(ctr + (size_t)(L - 1) * CTR_PER_LAYER + CTR_H, G, p.status, &s_abort);
   csync();
+  const float* hf = p.h + (size_t)((L - 1) & 1) * M * H;
   for (int tok = 0; tok < M; ++tok) {
     float ss = 0.0f;
-    for (int c = tid; c < H / 4; c += 32 * N_CONSUMERS) {
-      const float4 v = __ldcg(reinterpret_cast<const float4*>(p.h + (size_t)tok * H) + c);
+    for (int c = tid; c < H / 4; c += 32 * STEP_CONSUMERS) {
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(hf + (size_t)tok * H) + c);
       ss = fmaf(v.x, v.x, ss);
       ss = fmaf(v.y, v.y, ss);
       ss = fmaf(v.z, v.z, ss);
@@ -874,18 +1046,18 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    if (lane == 0) s_part[tok * N_CONSUMERS + warp] = ss;
+    if (lane == 0) s_part[tok * STEP_CONSUMERS + warp] = ss;
   }
   csync();
   if (tid < M) {
     float ss = 0.0f;
-    for (int w = 0; w < N_CONSUMERS; ++w) ss += s_part[tid * N_CONSUMERS + w];
+    for (int w = 0; w < STEP_CONSUMERS; ++w) ss += s_part[tid * STEP_CONSUMERS + w];
     s_r[tid] = 1.0f / sqrtf(ss / (float)H + p.eps);
   }
   csync();
-  for (int e = tid; e < M * H; e += 32 * N_CONSUMERS) {
+  for (int e = tid; e < M * H; e += 32 * STEP_CONSUMERS) {
     const int tok = e / H;
-    const float hv = __ldcg(p.h + e);
+    const float hv = __ldcg(hf + e);
     const __nv_bfloat16 v = __float2bfloat16_rn(hv * s_r[tok]);
     p.x_final[e] = v;
     if (p.x_trace) p.x_trace[(size_t)L * M * H + e] = v;
