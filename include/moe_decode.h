@@ -290,6 +290,49 @@ MOE_API moe_status_t decode_step_graph_create(const moe_model_t* model, const vo
 MOE_API moe_status_t decode_step_graph_launch(moe_graph_t graph, moe_stream_t stream);
 MOE_API void decode_step_graph_destroy(moe_graph_t graph);
 
+/* ---------------------------------------------------------------------------
+ * Prefill chunk: one MoE layer for M tokens on the block-scaled tensor cores.
+ * Source: DGX Spark MoE knowledge card (知识卡片：NVIDIA DGX Spark 上提升 MoE 推理吞吐的
+ * 三种方法), 方法/产品要点 items 1 and 3: MXFP4 expert weights, 8 of 512 routed experts
+ * plus one shared BF16 expert.  The pages fix no prefill activation format; the
+ * block-scaled MMA needs MX operands on both sides, so the routed experts take
+ * their activations as MXFP8 (per token, per 32 elements of K: s = clamp(floor(log2
+ * amax) - 8, -127, 127), codes e4m3 RNE-saturating of v * 2^-s; amax = 0 gives
+ * s = -127 and zero codes) -- both x and the SwiGLU output a.  Router and shared
+ * expert run on BF16 operands with fp32 accumulation; the shared activation is
+ * rounded to BF16.
+ * ------------------------------------------------------------------------- */
+
+/* Bytes of workspace moe_prefill_layer needs (0: unsupported shape). */
+MOE_API size_t moe_prefill_workspace_bytes(int M, int H, int I, int E, int top_k, int Is);
+
+/* y[t] = sum_j w[t][j] * W2_e (MXFP8(silu(Wg_e xq) * Wu_e xq)) + Ws2 bf16(silu(Wsg x) * Wsu x),
+ * e = ids[t][j], xq = MXFP8(x[t]); ids/w = top-k of the router logits x Wr^T (largest,
+ * lowest index on ties) and the softmax over the k selected logits.
+ *   x_bf16 [M][H] bf16; w_router_bf16 [E][H]; w13_codes [E][2I][H/2] MXFP4 (rows 0..I-1
+ *   gate, I..2I-1 up; low nibble = even element), w13_scales [E][2I][H/32] E8M0;
+ *   w2_codes [E][H][I/2], w2_scales [E][H][I/32]; shared_w13_bf16 [2Is][H],
+ *   shared_w2_bf16 [H][Is] (both NULL when Is == 0);
+ *   topk_ids_opt [M][k] int32, topk_w_opt [M][k] fp32, logits_opt [M][E] fp32: optional
+ *   outputs (NULL: not written); y [M][H] fp32 out (overwritten).
+ * Limits: M % 128 == 0, 128 <= M <= 16384; H, I multiples of 128 in [128, 4096];
+ *   E % 128 == 0, 128 <= E <= 512; 1 <= top_k <= 8; Is % 64 == 0, 0 <= Is <= 4096.
+ * Pointers 16-byte aligned; w13_codes and w2_codes 32-byte aligned (MOE_ERR_ALIGNMENT).
+ * Asynchronous on `stream`; device-side bounded waits report MOE_ERR_TIMEOUT through
+ * moe_workspace_status.  Caller owns every buffer; nothing is allocated. */
+MOE_API moe_status_t moe_prefill_layer(const void* x_bf16, int M, int H, int I, int E, int top_k,
+                                       const void* w_router_bf16, const uint8_t* w13_codes,
+                                       const uint8_t* w13_scales, const uint8_t* w2_codes,
+                                       const uint8_t* w2_scales, const void* shared_w13_bf16,
+                                       const void* shared_w2_bf16, int Is, int32_t* topk_ids_opt,
+                                       float* topk_w_opt, float* logits_opt, float* y, void* ws,
+                                       size_t ws_bytes, moe_stream_t stream);
+
+/* MXFP8 quantiser of the prefill path on its own: v [M][K] fp32 -> q [M][K] e4m3 codes,
+ * scales [M][K/32] E8M0, by the rule above.  K % 32 == 0; M * K <= 2^31. */
+MOE_API moe_status_t moe_mxfp8_quantize(const float* v, int M, int K, uint8_t* q, uint8_t* scales,
+                                        moe_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -52,6 +52,9 @@ SIGNATURES = {
     "moe_experts_workspace_bytes": (Z, [I, I, I, I, I, I]),
     "moe_mxfp4_experts": (I, [P, I, I, I, I, I, P, P, P, P, P, P, P, P, I, P, P, Z, P]),
     "lm_head_fp8_quantize": (I, [P, I, I, P, P, P]),
+    "moe_prefill_workspace_bytes": (Z, [I, I, I, I, I, I]),
+    "moe_prefill_layer": (I, [P, I, I, I, I, I, P, P, P, P, P, P, P, I, P, P, P, P, P, Z, P]),
+    "moe_mxfp8_quantize": (I, [P, I, I, P, P, P]),
     "lm_head_workspace_bytes": (Z, [I, I, I]),
     "lm_head_fp8_gemv": (I, [P, I, I, I, P, P, P, P, P, Z, P]),
     "lm_head_fp8_gemv_noalloc": (I, [P, I, I, I, P, P, P, P, P]),

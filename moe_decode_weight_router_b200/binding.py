@@ -122,6 +122,49 @@ def moe_mxfp4_experts(x, topk_ids, topk_w, w13c, w13s, w2c, w2s, sw13=None, sw2=
 
 
 # ---------------------------------------------------------------------------
+# prefill chunk (tcgen05 block-scaled path)
+# ---------------------------------------------------------------------------
+def moe_prefill_workspace_bytes(M, H, I, E, top_k, Is) -> int:
+    return _lib().moe_prefill_workspace_bytes(M, H, I, E, top_k, Is)
+
+
+def moe_prefill_layer(x, wr, w13c, w13s, w2c, w2s, sw13=None, sw2=None, *, top_k, ws=None, y=None,
+                      want_routing: bool = True, want_logits: bool = False, stream=None):
+    """One MoE layer over a prefill chunk: bf16 x [M,H] -> (y fp32 [M,H], ids [M,k], w [M,k], logits [M,E]).
+
+    Routing, shared expert and routed experts all run in this call (MXFP8
+    activations for the routed experts); ids/w/logits are None unless asked for."""
+    _dev_bf16(x, "x")
+    M, H = x.shape
+    E, twoI, _ = w13c.shape
+    I = twoI // 2
+    Is = sw13.shape[0] // 2 if sw13 is not None else 0
+    dev = x.device
+    if y is None:
+        y = torch.empty((M, H), dtype=torch.float32, device=dev)
+    ids = torch.empty((M, top_k), dtype=torch.int32, device=dev) if want_routing else None
+    w = torch.empty((M, top_k), dtype=torch.float32, device=dev) if want_routing else None
+    lg = torch.empty((M, E), dtype=torch.float32, device=dev) if want_logits else None
+    if ws is None:
+        ws = _ws(moe_prefill_workspace_bytes(M, H, I, E, top_k, Is), dev)
+    _check("moe_prefill_layer", _lib().moe_prefill_layer(
+        _ptr(x), M, H, I, E, top_k, _ptr(wr), _ptr(w13c), _ptr(w13s), _ptr(w2c), _ptr(w2s), _ptr(sw13), _ptr(sw2),
+        Is, _ptr(ids), _ptr(w), _ptr(lg), _ptr(y), _ptr(ws), ws.numel(), _stream(stream)))
+    return y, ids, w, lg
+
+
+def moe_mxfp8_quantize(v, *, stream=None):
+    """fp32 [M,K] -> (e4m3 codes uint8 [M,K], E8M0 scales uint8 [M,K/32])."""
+    if v.dtype != torch.float32 or not v.is_cuda or not v.is_contiguous():
+        raise TypeError("v: expected a contiguous CUDA float32 tensor")
+    M, K = v.shape
+    q = torch.empty((M, K), dtype=torch.uint8, device=v.device)
+    s = torch.empty((M, K // 32), dtype=torch.uint8, device=v.device)
+    _check("moe_mxfp8_quantize", _lib().moe_mxfp8_quantize(_ptr(v), M, K, _ptr(q), _ptr(s), _stream(stream)))
+    return q, s
+
+
+# ---------------------------------------------------------------------------
 # LM head
 # ---------------------------------------------------------------------------
 def lm_head_fp8_quantize(w: torch.Tensor, *, out=None, stream=None):

@@ -15,6 +15,7 @@
 #include "decode_kernels.cuh"
 #include "lmhead_kernels.cuh"
 #include "step_kernel.cuh"
+#include "prefill_kernels.cuh"
 
 using namespace moe;
 
@@ -41,7 +42,7 @@ struct DevInfo {
   int smem_optin = 0;
   // largest dynamic shared memory per kernel family: the opt-in limit minus the
   // kernel's own static shared memory
-  int dyn_dense = 0, dyn_e13 = 0, dyn_e2 = 0, dyn_lm = 0, dyn_step = 0;
+  int dyn_dense = 0, dyn_e13 = 0, dyn_e2 = 0, dyn_lm = 0, dyn_step = 0, dyn_pf = 0;
   int coop = 0;
 };
 
@@ -74,6 +75,7 @@ moe_status_t dev_info(DevInfo* out) {
     MOE_CUDA(allow_dyn_smem(k_experts2, lim, &d.dyn_e2));
     MOE_CUDA(allow_dyn_smem(k_lm_gemv, lim, &d.dyn_lm));
     MOE_CUDA(allow_dyn_smem(k_step, lim, &d.dyn_step));
+    MOE_CUDA(allow_dyn_smem(k_umma, lim, &d.dyn_pf));
     MOE_CUDA(cudaDeviceGetAttribute(&d.coop, cudaDevAttrCooperativeLaunch, dev));
     cache[dev] = d;
     ready[dev] = true;
@@ -822,3 +824,267 @@ extern "C" moe_status_t lm_head_fp8_gemv_noalloc(const void* x_bf16, int M, int 
   p.status = c.status;
   return launch_lm(p, d, st);
 }
+
+// =============================================================================
+// prefill chunk: one MoE layer for M tokens on tcgen05 (router, shared expert,
+// routed experts with MXFP8 activations)
+// =============================================================================
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn f = [] {
+    void* fp = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fp, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<EncodeTiledFn>(nullptr);
+    return reinterpret_cast<EncodeTiledFn>(fp);
+  }();
+  return f;
+}
+
+// 2-D K-major operand: dims {inner elements, rows}, row pitch in bytes, 128-byte swizzle.
+bool make_map(CUtensorMap* m, CUtensorMapDataType t, const void* base, uint64_t inner, uint64_t rows,
+              uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows) {
+  EncodeTiledFn f = encode_fn();
+  if (!f) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return f(m, t, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+bool ok_pf(int M, int H, int I, int E, int k, int Is) {
+  return M >= 128 && M % 128 == 0 && M <= 16384 && H >= 128 && H % 128 == 0 && H <= 4096 && I >= 128 &&
+         I % 128 == 0 && I <= 4096 && E >= 128 && E % 128 == 0 && E <= 512 && k >= 1 && k <= 8 && Is >= 0 &&
+         Is % 64 == 0 && Is <= 4096;
+}
+
+struct PfWs {
+  int* status;
+  int* counts;  // [E]
+  int* fill;    // [E]
+  int* goff;    // [E+1]
+  int* ntp;     // [E+1]
+  size_t clear_bytes;
+  float* logits;  // [M][E]
+  int32_t* ids;   // [M][k]
+  float* w;       // [M][k]
+  int32_t* g_tok; // [G]
+  float* g_w;     // [G]
+  int32_t* pos;   // [M][k]
+  uint8_t* xq;    // [G][H]
+  uint8_t* xs;    // [G][H/32]
+  __nv_bfloat16* as;  // [M][Is]
+  uint8_t* aq;    // [G][I]
+  uint8_t* aqs;   // [G][I/32]
+  size_t bytes;
+};
+PfWs pf_ws(void* ws, int M, int H, int I, int E, int k, int Is) {
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  PfWs s{};
+  const size_t G = (size_t)M * k;
+  size_t off = 0;
+  s.status = reinterpret_cast<int*>(b);
+  off += CTRL_BYTES;
+  s.counts = reinterpret_cast<int*>(b + off);
+  off += up256((size_t)E * 4);
+  s.clear_bytes = off;
+  s.fill = reinterpret_cast<int*>(b + off);
+  off += up256((size_t)E * 4);
+  s.goff = reinterpret_cast<int*>(b + off);
+  off += up256((size_t)(E + 1) * 4);
+  s.ntp = reinterpret_cast<int*>(b + off);
+  off += up256((size_t)(E + 1) * 4);
+  s.logits = reinterpret_cast<float*>(b + off);
+  off += up256((size_t)M * E * 4);
+  s.ids = reinterpret_cast<int32_t*>(b + off);
+  off += up256(G * 4);
+  s.w = reinterpret_cast<float*>(b + off);
+  off += up256(G * 4);
+  s.g_tok = reinterpret_cast<int32_t*>(b + off);
+  off += up256(G * 4);
+  s.g_w = reinterpret_cast<float*>(b + off);
+  off += up256(G * 4);
+  s.pos = reinterpret_cast<int32_t*>(b + off);
+  off += up256(G * 4);
+  s.xq = b + off;
+  off += up256(G * H);
+  s.xs = b + off;
+  off += up256(G * (H / 32));
+  s.as = reinterpret_cast<__nv_bfloat16*>(b + off);
+  off += up256((size_t)M * (Is > 0 ? Is : 1) * 2);
+  s.aq = b + off;
+  off += up256(G * I);
+  s.aqs = b + off;
+  off += up256(G * (I / 32));
+  s.bytes = off;
+  return s;
+}
+
+moe_status_t launch_umma(PrefillParams& p, const DevInfo& d, cudaStream_t st) {
+  const int stages = (d.dyn_pf - 1024) / PF_STAGE_BYTES;
+  p.stages = stages > PF_MAX_STAGES ? PF_MAX_STAGES : stages;
+  if (p.stages < 2) return MOE_ERR_UNSUPPORTED_SHAPE;
+  const size_t smem = 1024 + (size_t)p.stages * PF_STAGE_BYTES;
+  k_umma<<<d.sms, PF_THREADS, smem, st>>>(p);
+  MOE_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_prefill_workspace_bytes(int M, int H, int I, int E, int top_k, int Is) {
+  if (!ok_pf(M, H, I, E, top_k, Is)) return 0;
+  return pf_ws(nullptr, M, H, I, E, top_k, Is).bytes;
+}
+
+moe_status_t moe_prefill_layer(const void* x_bf16, int M, int H, int I, int E, int top_k, const void* w_router_bf16,
+                               const uint8_t* w13_codes, const uint8_t* w13_scales, const uint8_t* w2_codes,
+                               const uint8_t* w2_scales, const void* shared_w13_bf16, const void* shared_w2_bf16,
+                               int Is, int32_t* topk_ids_opt, float* topk_w_opt, float* logits_opt, float* y,
+                               void* ws, size_t ws_bytes, moe_stream_t stream) {
+  REQ(x_bf16 && w_router_bf16 && w13_codes && w13_scales && w2_codes && w2_scales && y, MOE_ERR_INVALID_ARG);
+  REQ(ok_pf(M, H, I, E, top_k, Is), MOE_ERR_UNSUPPORTED_SHAPE);
+  REQ(Is == 0 || (shared_w13_bf16 && shared_w2_bf16), MOE_ERR_INVALID_ARG);
+  moe_status_t s = check_ptrs_aligned({x_bf16, w_router_bf16, w13_codes, w13_scales, w2_codes, w2_scales,
+                                       shared_w13_bf16, shared_w2_bf16, topk_ids_opt, topk_w_opt, logits_opt, y, ws});
+  if (s != MOE_OK) return s;
+  // the 4-bit tensor-map form reads from 32-byte aligned bases
+  REQ((reinterpret_cast<uintptr_t>(w13_codes) & 31u) == 0 && (reinterpret_cast<uintptr_t>(w2_codes) & 31u) == 0,
+      MOE_ERR_ALIGNMENT);
+  REQ(ws && ws_bytes >= moe_prefill_workspace_bytes(M, H, I, E, top_k, Is), MOE_ERR_WORKSPACE);
+  DevInfo d;
+  if ((s = dev_info(&d)) != MOE_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const PfWs w = pf_ws(ws, M, H, I, E, top_k, Is);
+  const int G = M * top_k;
+  const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(x_bf16);
+  MOE_CUDA(cudaMemsetAsync(ws, 0, w.clear_bytes, st));
+
+  // a1: router logits (bf16 x bf16 on tcgen05), top-k, softmax over the selected
+  PrefillParams p{};
+  p.status = w.status;
+  p.E = E;
+  REQ(make_map(&p.tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w_router_bf16, H, E, (uint64_t)H * 2, 64, 64),
+      MOE_ERR_INVALID_ARG);
+  REQ(make_map(&p.tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, H, M, (uint64_t)H * 2, 64, 32), MOE_ERR_INVALID_ARG);
+  p.mode = PF_ROUTER;
+  p.K = H;
+  p.m_tiles = E / 128;
+  p.M = M;
+  p.out_f32 = w.logits;
+  p.out_ld = E;
+  if ((s = launch_umma(p, d, st)) != MOE_OK) return s;
+  k_pf_topk<<<(M + 7) / 8, 256, 0, st>>>(w.logits, M, E, top_k, w.ids, w.w, w.counts);
+  MOE_CUDA(cudaGetLastError());
+  // a2: grouped rows per expert
+  k_pf_scan<<<1, 1024, 0, st>>>(w.counts, E, w.goff, w.ntp, w.fill);
+  MOE_CUDA(cudaGetLastError());
+  k_pf_scatter<<<(G + 255) / 256, 256, 0, st>>>(w.ids, w.w, M, top_k, w.goff, w.fill, w.g_tok, w.g_w, w.pos);
+  MOE_CUDA(cudaGetLastError());
+  k_pf_quant_x<<<(int)(((long long)M * (H / 32) + 7) / 8), 256, 0, st>>>(x, M, H, top_k, w.pos, w.xq, w.xs);
+  MOE_CUDA(cudaGetLastError());
+
+  // a5: shared expert (bf16): a_s = bf16(silu(Wg x) * Wu x), y = Ws2 a_s
+  if (Is > 0) {
+    PrefillParams q{};
+    q.status = w.status;
+    REQ(make_map(&q.tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, shared_w13_bf16, H, 2 * (uint64_t)Is, (uint64_t)H * 2, 64,
+                 64),
+        MOE_ERR_INVALID_ARG);
+    q.tmB = p.tmB;
+    q.mode = PF_SH13;
+    q.K = H;
+    q.m_tiles = Is / 64;
+    q.up_off = Is;
+    q.M = M;
+    q.out_bf16 = w.as;
+    q.out_ld = Is;
+    if ((s = launch_umma(q, d, st)) != MOE_OK) return s;
+    PrefillParams r{};
+    r.status = w.status;
+    REQ(make_map(&r.tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, shared_w2_bf16, Is, H, (uint64_t)Is * 2, 64, 64),
+        MOE_ERR_INVALID_ARG);
+    REQ(make_map(&r.tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w.as, Is, M, (uint64_t)Is * 2, 64, 32), MOE_ERR_INVALID_ARG);
+    r.mode = PF_SH2;
+    r.K = Is;
+    r.m_tiles = H / 128;
+    r.M = M;
+    r.out_f32 = y;
+    r.out_ld = H;
+    if ((s = launch_umma(r, d, st)) != MOE_OK) return s;
+  } else {
+    MOE_CUDA(cudaMemsetAsync(y, 0, (size_t)M * H * 4, st));
+  }
+
+  // a3: routed W13 + SwiGLU, activation re-quantised to MXFP8 (E2M1 x E4M3 block-scaled)
+  PrefillParams a{};
+  a.status = w.status;
+  REQ(make_map(&a.tmA, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, w13_codes, H, (uint64_t)E * 2 * I, (uint64_t)H / 2, 128,
+               64),
+      MOE_ERR_INVALID_ARG);
+  REQ(make_map(&a.tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.xq, H, G, H, 128, 32), MOE_ERR_INVALID_ARG);
+  a.mode = PF_R13;
+  a.K = H;
+  a.m_tiles = I / 64;
+  a.up_off = I;
+  a.prob_rows = 2 * I;
+  a.E = E;
+  a.ntile_prefix = w.ntp;
+  a.goff = w.goff;
+  a.sfa = w13_scales;
+  a.sfb = w.xs;
+  a.out_q = w.aq;
+  a.out_qs = w.aqs;
+  a.out_ld = I;
+  if ((s = launch_umma(a, d, st)) != MOE_OK) return s;
+
+  // a4: routed W2, weighted by the routing weight and added into y
+  PrefillParams b{};
+  b.status = w.status;
+  REQ(make_map(&b.tmA, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, w2_codes, I, (uint64_t)E * H, (uint64_t)I / 2, 128, 64),
+      MOE_ERR_INVALID_ARG);
+  REQ(make_map(&b.tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.aq, I, G, I, 128, 32), MOE_ERR_INVALID_ARG);
+  b.mode = PF_R2;
+  b.K = I;
+  b.m_tiles = H / 128;
+  b.prob_rows = H;
+  b.E = E;
+  b.ntile_prefix = w.ntp;
+  b.goff = w.goff;
+  b.g_tok = w.g_tok;
+  b.g_w = w.g_w;
+  b.sfa = w2_scales;
+  b.sfb = w.aqs;
+  b.out_f32 = y;
+  b.out_ld = H;
+  if ((s = launch_umma(b, d, st)) != MOE_OK) return s;
+
+  if (topk_ids_opt) MOE_CUDA(cudaMemcpyAsync(topk_ids_opt, w.ids, (size_t)G * 4, cudaMemcpyDeviceToDevice, st));
+  if (topk_w_opt) MOE_CUDA(cudaMemcpyAsync(topk_w_opt, w.w, (size_t)G * 4, cudaMemcpyDeviceToDevice, st));
+  if (logits_opt) MOE_CUDA(cudaMemcpyAsync(logits_opt, w.logits, (size_t)M * E * 4, cudaMemcpyDeviceToDevice, st));
+  return MOE_OK;
+}
+
+moe_status_t moe_mxfp8_quantize(const float* v, int M, int K, uint8_t* q, uint8_t* scales, moe_stream_t stream) {
+  REQ(v && q && scales, MOE_ERR_INVALID_ARG);
+  REQ(M >= 1 && K >= 32 && K % 32 == 0 && (long long)M * K <= (1LL << 31), MOE_ERR_UNSUPPORTED_SHAPE);
+  moe_status_t s = check_ptrs_aligned({v, q, scales});
+  if (s != MOE_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  k_mxfp8_quantize<<<(int)(((long long)M * (K / 32) + 7) / 8), 256, 0, st>>>(v, M, K, q, scales);
+  MOE_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
+
+}  // extern "C"

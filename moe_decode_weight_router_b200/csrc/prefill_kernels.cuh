@@ -1,0 +1,583 @@
+// prefill_kernels.cuh -- one MoE layer over a prefill chunk (M tokens, M a multiple of
+// 128) on the 5th-generation tensor cores.
+//
+// Source: DGX Spark MoE knowledge card (知识卡片：NVIDIA DGX Spark 上提升 MoE 推理吞吐的
+// 三种方法), 方法/产品要点 items 1 and 3 (MXFP4 expert weights, 8 of 512 experts plus one
+// shared expert); the prefill activations are MXFP8 (a power-of-two scale per 32
+// elements along K, e4m3 codes) because the block-scaled MMA takes both operands in
+// an MX format.
+//
+// Every GEMM of the layer is one launch of k_umma, a persistent warp-specialised
+// kernel (one CTA per SM):
+//   warp 4      TMA producer: weight tile (two 64-row boxes, 128 B of K per row) and
+//               activation tile (32-row boxes) per K chunk into a ring of stages;
+//   warp 5      MMA issuer: one elected thread issues tcgen05.mma (M = 128 weight rows,
+//               N = tokens, fp32 accumulator in tensor memory) and commits each stage
+//               back to the producer and each finished tile to the epilogue;
+//   warps 0-3   epilogue: tcgen05.ld of the accumulator (warp w owns TMEM lanes
+//               32w..32w+31), the mode's arithmetic and the global stores; for the
+//               block-scaled modes they also place the tile's E8M0 scale factors in
+//               tensor memory (tcgen05.st) before its MMAs start.
+// Modes: router logits (bf16 x bf16), shared W13 + SwiGLU (bf16), shared W2 (bf16,
+// stores y), routed W13 + SwiGLU + MXFP8 re-quantisation (E2M1 x E4M3 block-scaled),
+// routed W2 with the routing weight, added into y.
+//
+// Shared-memory operand layout: K-major, 128-byte swizzle (rows of 128 bytes, 8-row
+// atoms of 1024 bytes).  E2M1 weights reach shared memory through the tensor map type
+// that leaves an 8-byte gap after every 8 bytes (16 codes), the form the block-scaled
+// MMA reads for 4-bit operands, so a 128-element K chunk is 128 bytes per row for
+// every operand type.  Scale factors in tensor memory: the E8M0 of operand row m,
+// K blocks 4c..4c+3 (one per byte, selected by the instruction's scale-factor id), is
+// the 32-bit word at lane m % 32 + 32q (every q), column base + 4c + m / 32.
+#pragma once
+
+#include <cuda.h>
+
+#include "decode_kernels.cuh"
+
+namespace moe {
+
+enum : int { PF_ROUTER = 0, PF_SH13 = 1, PF_SH2 = 2, PF_R13 = 3, PF_R2 = 4 };
+constexpr int PF_THREADS = 192;        // warps 0-3 epilogue, 4 producer, 5 MMA
+constexpr int PF_BN = 128;             // token tile (MMA N <= 128)
+constexpr int PF_STAGE_BYTES = 32768;  // weight tile 16 KB + token tile 16 KB
+constexpr int PF_MAX_STAGES = 6;
+constexpr int PF_TMEM_COLS = 512;      // accumulator 0..127, SFA 128.., SFB 256..
+constexpr int PF_SFA_COL = 128, PF_SFB_COL = 256;
+constexpr int PF_MAX_CHUNKS = 32;      // K / 128 for the block-scaled modes (SF columns)
+
+struct alignas(64) PrefillParams {
+  CUtensorMap tmA;  // weights: dims {K, rows}, box {64 or 128 elements, 64 rows}
+  CUtensorMap tmB;  // activations: dims {K, rows}, box {.., 32 rows}
+  int mode;
+  int K;
+  int m_tiles;   // weight tiles per problem
+  int up_off;    // 13 modes: row offset of the up half within a problem
+  int prob_rows; // weight rows per problem (expert) for the routed modes
+  int M;         // dense modes: tokens
+  int E;
+  const int* ntile_prefix;  // routed: [E+1] prefix sums of ceil(n_e / 128)
+  const int* goff;          // routed: [E+1] first grouped row of each expert
+  const int32_t* g_tok;     // routed: [G] token of each grouped row
+  const float* g_w;         // routed: [G] routing weight of each grouped row
+  const uint8_t* sfa;       // routed: weight scales [rows][K/32]
+  const uint8_t* sfb;       // routed: activation scales [G][K/32]
+  int out_ld;               // leading dimension of the output
+  float* out_f32;           // router logits [M][E], y [M][H]
+  __nv_bfloat16* out_bf16;  // shared activation [M][Is]
+  uint8_t* out_q;           // routed activation e4m3 [G][I]
+  uint8_t* out_qs;          // routed activation E8M0 [G][I/32]
+  int stages;
+  int* status;
+};
+
+// ---------------------------------------------------------------------------
+// tcgen05 / TMA primitives
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, "
+      "[%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  tc_wait_ld();
+#pragma unroll
+  for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]);
+}
+__device__ __forceinline__ void tmem_st4(uint32_t taddr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+// D[tmem] (+)= A[smem] * B[smem]^T, bf16 x bf16 -> fp32
+__device__ __forceinline__ void umma_bf16(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}\n" ::"r"(d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc), "r"(0u), "r"(0u), "r"(0u), "r"(0u)
+      : "memory");
+}
+// D[tmem] (+)= (A * 2^sfa)[smem] * (B * 2^sfb)[smem]^T, E2M1 x E4M3 with E8M0 per 32 of K
+__device__ __forceinline__ void umma_mx(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc,
+                                        uint32_t tsfa, uint32_t tsfb) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc), "r"(tsfa), "r"(tsfb)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+// K-major operand, 128-byte swizzle: start >> 4, LBO 1 (unused when swizzled), SBO 1024 B
+// between 8-row atoms, descriptor version 1, layout SWIZZLE_128B.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1u << 16) | ((uint64_t)64u << 32) | ((uint64_t)1u << 46) |
+         ((uint64_t)2u << 61);
+}
+// Instruction descriptors (M = 128, both operands K-major).
+__host__ __device__ inline uint32_t idesc_bf16(int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+__host__ __device__ inline uint32_t idesc_mx(int N, uint32_t sf_id) {
+  return (sf_id << 4) | (5u << 7) | (0u << 10) | ((uint32_t)(N >> 3) << 17) | (1u << 23) |
+         ((uint32_t)(128 >> 4) << 24) | (sf_id << 29);
+}
+
+// Bounded mbarrier wait; once any thread of the CTA has given up, every later wait
+// returns false at once, so all roles reach the final block barrier.  The first
+// timeout of a workspace also records where it happened (status[4..7]: wait site,
+// mode, block, parity).
+enum : int { PFW_EMPTY = 1, PFW_DRAIN = 2, PFW_ACC_EMPTY = 3, PFW_SF = 4, PFW_FULL = 5, PFW_ACC_FULL = 6 };
+__device__ __noinline__ bool pf_wait(uint64_t* bar, uint32_t parity, int* status, volatile int* abort_flag,
+                                     int site, int mode) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
+      if (atomicCAS(status, 0, DEV_ERR_TIMEOUT) == 0) {
+        status[4] = site;
+        status[5] = mode;
+        status[6] = (int)blockIdx.x;
+        status[7] = (int)parity;
+      }
+      *abort_flag = 1;
+      return false;
+    }
+  }
+  return true;
+}
+
+// ---------------------------------------------------------------------------
+// work items
+// ---------------------------------------------------------------------------
+struct PfItem {
+  int e;       // expert (routed modes)
+  int mt;      // weight tile
+  int n0;      // first token of the tile within the problem
+  int ncnt;    // tokens in the tile
+  int grow0;   // activation row of token n0
+  int ya0, ya1;  // weight rows of the two 64-row halves
+};
+
+__device__ __forceinline__ bool pf_routed(int mode) { return mode == PF_R13 || mode == PF_R2; }
+__device__ __forceinline__ bool pf_13(int mode) { return mode == PF_SH13 || mode == PF_R13; }
+
+__device__ inline int pf_total_items(const PrefillParams& p) {
+  if (pf_routed(p.mode)) return p.m_tiles * __ldg(p.ntile_prefix + p.E);
+  return p.m_tiles * ((p.M + PF_BN - 1) / PF_BN);
+}
+__device__ inline PfItem pf_item(const PrefillParams& p, int idx) {
+  PfItem it;
+  it.mt = idx % p.m_tiles;
+  const int j = idx / p.m_tiles;
+  int rows0;
+  if (pf_routed(p.mode)) {
+    int lo = 0, hi = p.E;  // largest e with ntile_prefix[e] <= j
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (__ldg(p.ntile_prefix + mid) <= j)
+        lo = mid;
+      else
+        hi = mid;
+    }
+    it.e = lo;
+    it.n0 = (j - __ldg(p.ntile_prefix + lo)) * PF_BN;
+    const int g0 = __ldg(p.goff + lo), ne = __ldg(p.goff + lo + 1) - g0;
+    it.ncnt = min(PF_BN, ne - it.n0);
+    it.grow0 = g0 + it.n0;
+    rows0 = lo * p.prob_rows;
+  } else {
+    it.e = 0;
+    it.n0 = j * PF_BN;
+    it.ncnt = min(PF_BN, p.M - it.n0);
+    it.grow0 = it.n0;
+    rows0 = 0;
+  }
+  if (pf_13(p.mode)) {
+    it.ya0 = rows0 + 64 * it.mt;              // gate rows
+    it.ya1 = rows0 + p.up_off + 64 * it.mt;   // up rows
+  } else {
+    it.ya0 = rows0 + 128 * it.mt;
+    it.ya1 = it.ya0 + 64;
+  }
+  return it;
+}
+
+__device__ __forceinline__ float pf_silu(float g) { return g / (1.0f + expf(-g)); }
+
+// floor(log2(a)) of a finite a > 0, exact (subnormals from the mantissa's top bit).
+__device__ __forceinline__ int floor_log2_f32(float a) {
+  const uint32_t b = __float_as_uint(a);
+  const int e = (int)((b >> 23) & 0xFFu);
+  if (e != 0) return e - 127;
+  return (31 - __clz(b & 0x7FFFFFu)) - 149;
+}
+// MXFP8 scale exponent of a 32-block with max |v| = amax: clamp(floor(log2 amax) - 8).
+__device__ __forceinline__ int mxfp8_exponent(float amax) {
+  if (amax == 0.0f) return -127;
+  int s = floor_log2_f32(amax) - 8;
+  return s < -127 ? -127 : (s > 127 ? 127 : s);
+}
+__device__ __forceinline__ uint8_t e4m3_of(float v) {
+  return (uint8_t)(f32x2_to_e4m3x2(v, 0.0f) & 0xFFu);
+}
+
+// ---------------------------------------------------------------------------
+// k_umma
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ PrefillParams p) {
+  extern __shared__ __align__(1024) uint8_t pf_smem_raw[];
+  // 1024-byte alignment of the stage ring (the 128-byte swizzle atom)
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(pf_smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ uint64_t full[PF_MAX_STAGES], empty[PF_MAX_STAGES];
+  __shared__ uint64_t acc_full, acc_empty, sf_ready;
+  __shared__ uint32_t tmem_base_s;
+  __shared__ volatile int s_abort;
+  __shared__ float xch[2][32][17];  // up-half values handed from warps 2,3 to warps 0,1
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int S = p.stages;
+  const bool mx = pf_routed(p.mode);
+  const int kbox = mx ? 128 : 64;  // K elements per stage (128 bytes per row)
+  const int nch = p.K / kbox;
+  const int total = pf_total_items(p);
+  const int G = gridDim.x;
+
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(&acc_full, 1);
+    mbar_init(&acc_empty, 4);
+    mbar_init(&sf_ready, 4);
+    fence_mbar_init();
+    s_abort = 0;
+  }
+  if (warp == 5) {
+    tmem_alloc(&tmem_base_s, PF_TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = tmem_base_s;
+
+  if (warp == 4) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      long long q = 0;
+      bool ok = true;
+      for (int idx = blockIdx.x; idx < total && ok; idx += G) {
+        const PfItem it = pf_item(p, idx);
+        const int N = (it.ncnt + 15) & ~15;
+        const int nb = (N + 31) / 32;
+        for (int ch = 0; ch < nch; ++ch, ++q) {
+          const int s = (int)(q % S);
+          if (q >= S && !pf_wait(&empty[s], (uint32_t)(((q / S) - 1) & 1), p.status, &s_abort, PFW_EMPTY, p.mode)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + (size_t)s * PF_STAGE_BYTES;
+          // transaction bytes count the global (packed) side: a 64-row box of 128
+          // E2M1 codes is 4 KB although it fills 8 KB of shared memory
+          mbar_arrive_expect_tx(&full[s], (mx ? 8192u : 16384u) + 4096u * (uint32_t)nb);
+          tma_load_2d(st, &p.tmA, ch * kbox, it.ya0, &full[s]);
+          tma_load_2d(st + 8192, &p.tmA, ch * kbox, it.ya1, &full[s]);
+          for (int b = 0; b < nb; ++b) tma_load_2d(st + 16384 + 4096 * b, &p.tmB, ch * kbox, it.grow0 + 32 * b, &full[s]);
+        }
+      }
+      // every copy issued lands before the CTA may finish
+      for (long long j = (q > S ? q - S : 0); j < q; ++j) pf_wait(&full[j % S], (uint32_t)((j / S) & 1), p.status, &s_abort, PFW_DRAIN, p.mode);
+    }
+  } else if (warp == 5) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      long long q = 0;
+      int n_item = 0;
+      bool ok = true;
+      for (int idx = blockIdx.x; idx < total && ok; idx += G, ++n_item) {
+        const PfItem it = pf_item(p, idx);
+        const int N = (it.ncnt + 15) & ~15;
+        if (n_item > 0 && !pf_wait(&acc_empty, (uint32_t)((n_item - 1) & 1), p.status, &s_abort, PFW_ACC_EMPTY, p.mode)) break;
+        if (mx && !pf_wait(&sf_ready, (uint32_t)(n_item & 1), p.status, &s_abort, PFW_SF, p.mode)) break;
+        tc_fence_after();
+        for (int ch = 0; ch < nch; ++ch, ++q) {
+          const int s = (int)(q % S);
+          if (!pf_wait(&full[s], (uint32_t)((q / S) & 1), p.status, &s_abort, PFW_FULL, p.mode)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + (size_t)s * PF_STAGE_BYTES);
+          const uint64_t adesc = sw128_desc(sa), bdesc = sw128_desc(sa + 16384);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint32_t accum = (ch > 0 || k > 0) ? 1u : 0u;
+            // advance 32 bytes of K inside the 128-byte swizzled row
+            if (mx)
+              umma_mx(tbase, adesc + 2u * k, bdesc + 2u * k, idesc_mx(N, (uint32_t)k), accum,
+                      tbase + PF_SFA_COL + 4u * ch, tbase + PF_SFB_COL + 4u * ch);
+            else
+              umma_bf16(tbase, adesc + 2u * k, bdesc + 2u * k, idesc_bf16(N), accum);
+          }
+          tc_commit(&empty[s]);  // the stage returns to the producer once these MMAs are done
+        }
+        if (!ok) break;
+        tc_commit(&acc_full);  // the accumulator is complete
+      }
+    }
+  } else {
+    // ---------------- epilogue warps 0-3 ----------------
+    const int r = lane;
+    const uint32_t lane_base = tbase + ((uint32_t)(32 * warp) << 16);
+    int n_item = 0;
+    for (int idx = blockIdx.x; idx < total; idx += G, ++n_item) {
+      const PfItem it = pf_item(p, idx);
+      if (mx) {
+        // scale factors of this tile (the previous tile's MMAs are complete: its
+        // accumulator was waited for below before this point)
+        const int kb = p.K / 32;
+        const uint8_t* arow[4];
+        const uint8_t* brow[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int m = r + 32 * c;
+          arow[c] = p.sfa + (size_t)(m < 64 ? it.ya0 + m : it.ya1 + (m - 64)) * kb;
+          brow[c] = m < it.ncnt ? p.sfb + (size_t)(it.grow0 + m) * kb : nullptr;
+        }
+        for (int ch = 0; ch < nch; ++ch) {
+          uint32_t wa[4], wb[4];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            wa[c] = __ldg(reinterpret_cast<const uint32_t*>(arow[c] + 4 * ch));
+            wb[c] = brow[c] ? __ldg(reinterpret_cast<const uint32_t*>(brow[c] + 4 * ch)) : 0x7F7F7F7Fu;
+          }
+          tmem_st4(lane_base + PF_SFA_COL + 4 * ch, wa[0], wa[1], wa[2], wa[3]);
+          tmem_st4(lane_base + PF_SFB_COL + 4 * ch, wb[0], wb[1], wb[2], wb[3]);
+        }
+        tc_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sf_ready);
+      }
+      pf_wait(&acc_full, (uint32_t)(n_item & 1), p.status, &s_abort, PFW_ACC_FULL, p.mode);
+      named_barrier(2, 128);  // the four epilogue warps take the same decision below
+      if (s_abort) break;
+      tc_fence_after();
+      for (int j0 = 0; j0 < it.ncnt; j0 += 16) {
+        float v[16];
+        tmem_ld16(lane_base + (uint32_t)j0, v);
+        const int jn = min(16, it.ncnt - j0);
+        if (p.mode == PF_ROUTER || p.mode == PF_SH2) {
+          const int row = 128 * it.mt + 32 * warp + r;
+          for (int j = 0; j < jn; ++j) p.out_f32[(size_t)(it.n0 + j0 + j) * p.out_ld + row] = v[j];
+        } else if (p.mode == PF_R2) {
+          const int row = 128 * it.mt + 32 * warp + r;
+          for (int j = 0; j < jn; ++j) {
+            const int g = it.grow0 + j0 + j;
+            atomicAdd(p.out_f32 + (size_t)__ldg(p.g_tok + g) * p.out_ld + row, __ldg(p.g_w + g) * v[j]);
+          }
+        } else {
+          // 13 modes: warps 0,1 hold gate rows, warps 2,3 the matching up rows
+          if (warp >= 2)
+            for (int j = 0; j < 16; ++j) xch[warp - 2][r][j] = v[j];
+          named_barrier(2, 128);
+          if (warp < 2) {
+            const int i = 64 * it.mt + 32 * warp + r;  // intermediate index
+            float a[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) a[j] = pf_silu(v[j]) * xch[warp][r][j];
+            if (p.mode == PF_SH13) {
+              for (int j = 0; j < jn; ++j) p.out_bf16[(size_t)(it.n0 + j0 + j) * p.out_ld + i] = __float2bfloat16_rn(a[j]);
+            } else {
+              // MXFP8 of each token's 32-block (this warp's 32 rows)
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                float am = fabsf(a[j]);
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+                const int s = mxfp8_exponent(am);
+                if (j < jn) {
+                  const size_t g = (size_t)(it.grow0 + j0 + j);
+                  p.out_q[g * p.out_ld + i] = am == 0.0f ? (uint8_t)0 : e4m3_of(a[j] * exp2i(-s));
+                  if (r == 0) p.out_qs[g * (p.out_ld / 32) + (64 * it.mt + 32 * warp) / 32] = (uint8_t)(s + 127);
+                }
+              }
+            }
+          }
+          named_barrier(2, 128);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tbase, PF_TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// routing and grouping for the chunk
+// ---------------------------------------------------------------------------
+// One warp per token: top-k of logits [M][E] (largest, lowest index on ties), softmax
+// over the selected, per-expert counts.
+__global__ void __launch_bounds__(256) k_pf_topk(const float* __restrict__ logits, int M, int E, int k,
+                                                  int32_t* __restrict__ ids, float* __restrict__ w,
+                                                  int* __restrict__ counts) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (t >= M) return;
+  const float* lr = logits + (size_t)t * E;
+  uint32_t key[16];  // E <= 512
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int e = lane + 32 * i;
+    key[i] = e < E ? float_key(lr[e]) : 0u;
+  }
+  float sel_l = 0.0f;
+  int sel_i = 0;
+  for (int j = 0; j < k; ++j) {
+    uint32_t bk = 0u;
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if (key[i] > bk) {
+        bk = key[i];
+        bi = lane + 32 * i;
+      }
+    const uint32_t mk = __reduce_max_sync(0xffffffffu, bk);
+    const int mi = (int)__reduce_min_sync(0xffffffffu, (unsigned)(bk == mk ? bi : 0x7fffffff));
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if (lane + 32 * i == mi) key[i] = 0u;
+    if (lane == j) {
+      sel_l = key_float(mk);
+      sel_i = mi;
+    }
+  }
+  const float l0 = __shfl_sync(0xffffffffu, sel_l, 0);
+  const float ex = lane < k ? expf(sel_l - l0) : 0.0f;
+  float den = ex;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+  if (lane < k) {
+    ids[(size_t)t * k + lane] = sel_i;
+    w[(size_t)t * k + lane] = ex / den;
+    atomicAdd(counts + sel_i, 1);
+  }
+}
+
+// One block: exclusive prefix of the counts (grouped offsets) and of the 128-token
+// tiles per expert; clears the fill cursors.
+__global__ void __launch_bounds__(1024) k_pf_scan(const int* __restrict__ counts, int E, int* __restrict__ goff,
+                                                   int* __restrict__ ntile_prefix, int* __restrict__ fill) {
+  __shared__ int s_c[1024], s_t[1024];
+  const int e = threadIdx.x;
+  const int c = e < E ? counts[e] : 0;
+  s_c[e] = c;
+  s_t[e] = (c + PF_BN - 1) / PF_BN;
+  __syncthreads();
+  for (int o = 1; o < 1024; o <<= 1) {
+    const int a = e >= o ? s_c[e - o] : 0, b = e >= o ? s_t[e - o] : 0;
+    __syncthreads();
+    s_c[e] += a;
+    s_t[e] += b;
+    __syncthreads();
+  }
+  if (e < E) {
+    goff[e + 1] = s_c[e];
+    ntile_prefix[e + 1] = s_t[e];
+    fill[e] = 0;
+  }
+  if (e == 0) {
+    goff[0] = 0;
+    ntile_prefix[0] = 0;
+  }
+}
+
+// Grouped rows: each (token, selection) gets a slot in its expert's range.
+__global__ void k_pf_scatter(const int32_t* __restrict__ ids, const float* __restrict__ w, int M, int k,
+                             const int* __restrict__ goff, int* __restrict__ fill, int32_t* __restrict__ g_tok,
+                             float* __restrict__ g_w, int32_t* __restrict__ pos) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= M * k) return;
+  const int e = ids[i];
+  const int g = goff[e] + atomicAdd(fill + e, 1);
+  g_tok[g] = i / k;
+  g_w[g] = w[i];
+  pos[i] = g;
+}
+
+// MXFP8 of the chunk's input, written to every grouped row of its token: one warp
+// per (token, 32-block); lane = element.
+__global__ void __launch_bounds__(256) k_pf_quant_x(const __nv_bfloat16* __restrict__ x, int M, int H, int k,
+                                                     const int32_t* __restrict__ pos, uint8_t* __restrict__ xq,
+                                                     uint8_t* __restrict__ xs) {
+  const int lane = threadIdx.x & 31;
+  const long long wi = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int nb = H / 32;
+  if (wi >= (long long)M * nb) return;
+  const int t = (int)(wi / nb), b = (int)(wi % nb);
+  const float v = __bfloat162float(x[(size_t)t * H + 32 * b + lane]);
+  float am = fabsf(v);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+  const int s = mxfp8_exponent(am);
+  const uint8_t q = am == 0.0f ? (uint8_t)0 : e4m3_of(v * exp2i(-s));
+  for (int j = 0; j < k; ++j) {
+    const size_t g = (size_t)pos[(size_t)t * k + j];
+    xq[g * H + 32 * b + lane] = q;
+    if (lane == 0) xs[g * nb + b] = (uint8_t)(s + 127);
+  }
+}
+
+// Stand-alone MXFP8 quantiser of an fp32 matrix [M][K] (codes [M][K], E8M0 [M][K/32]).
+__global__ void __launch_bounds__(256) k_mxfp8_quantize(const float* __restrict__ v, int M, int K,
+                                                         uint8_t* __restrict__ q, uint8_t* __restrict__ se) {
+  const int lane = threadIdx.x & 31;
+  const long long wi = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int nb = K / 32;
+  if (wi >= (long long)M * nb) return;
+  const int t = (int)(wi / nb), b = (int)(wi % nb);
+  const float x = v[(size_t)t * K + 32 * b + lane];
+  float am = fabsf(x);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+  const int s = mxfp8_exponent(am);
+  q[(size_t)t * K + 32 * b + lane] = am == 0.0f ? (uint8_t)0 : e4m3_of(x * exp2i(-s));
+  if (lane == 0) se[(size_t)t * nb + b] = (uint8_t)(s + 127);
+}
+
+}  // namespace moe

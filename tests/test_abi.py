@@ -95,6 +95,40 @@ def test_experts_validation(lib):
     assert call(ws_bytes=need - 1) == 4
 
 
+def test_prefill_validation(lib):
+    need = lib.moe_prefill_workspace_bytes(2048, 2560, 768, 512, 8, 768)
+    assert need > 0
+    assert lib.moe_prefill_workspace_bytes(100, 2560, 768, 512, 8, 768) == 0   # M % 128
+    assert lib.moe_prefill_workspace_bytes(2048, 2560, 768, 1024, 8, 768) == 0  # E > 512
+    args = [A, 2048, 2560, 768, 512, 8, A, A, A, A, A, A, A, 768, None, None, None, A, A, need, None]
+    f = lib.moe_prefill_layer
+
+    def call(**kw):
+        a = list(args)
+        names = ["x", "M", "H", "I", "E", "k", "wr", "w13c", "w13s", "w2c", "w2s", "sw13", "sw2", "Is", "ids", "w",
+                 "logits", "y", "ws", "ws_bytes", "stream"]
+        for k, v in kw.items():
+            a[names.index(k)] = v
+        return f(*a)
+
+    assert call(x=None) == 1
+    assert call(y=None) == 1
+    assert call(sw2=None) == 1           # shared weights are required when Is > 0
+    assert call(M=64) == 2
+    assert call(H=2600) == 2
+    assert call(I=800) == 2
+    assert call(E=640) == 2
+    assert call(k=9) == 2
+    assert call(Is=96) == 2
+    assert call(w13c=A + 16) == 3        # the 4-bit tensor-map form needs 32-byte bases
+    assert call(y=A + 4) == 3
+    assert call(ws_bytes=need - 1) == 4
+    q = lib.moe_mxfp8_quantize
+    assert q(None, 4, 64, A, A, None) == 1
+    assert q(A, 4, 48, A, A, None) == 2
+    assert q(A, 4, 64, A + 2, A, None) == 3
+
+
 def test_lm_head_validation(lib):
     need = lib.lm_head_workspace_bytes(1, 157184, 2560)
     assert need > 0
