@@ -52,6 +52,8 @@ def parse_args():
     ap.add_argument("--ref-layers", type=int, default=4, help="layers per reference-arm step")
     ap.add_argument("--skip-m4", action="store_true")
     ap.add_argument("--per-layer", action="store_true", help="force the three-kernels-per-layer path")
+    ap.add_argument("--skip-prefill", action="store_true", help="skip the prefill-chunk measurement")
+    ap.add_argument("--prefill-m", type=int, default=2048, help="tokens of the prefill chunk")
     return ap.parse_args()
 
 
@@ -316,6 +318,43 @@ def run_ours(args, rank, world, local_rank):
             res["kernels"] = ker
         results[M] = res
 
+    # prefill chunk: one MoE layer for M tokens on the block-scaled tensor cores, each
+    # timed call on the next of the L distinct layers (1.6 GB of experts each, > L2)
+    if not args.skip_prefill:
+        from moe_decode_weight_router_b200 import moe_prefill_layer, moe_prefill_workspace_bytes
+        Mp = args.prefill_m
+        xp = synth.tokens(Mp, S.H, seed, tid=7, device=dev)
+        wsp = torch.empty(moe_prefill_workspace_bytes(Mp, S.H, S.I, S.E, S.k, S.Is), dtype=torch.uint8, device=dev)
+        yp = torch.empty((Mp, S.H), dtype=torch.float32, device=dev)
+        idp = torch.empty((Mp, S.k), dtype=torch.int32, device=dev)
+
+        def pf(l, ids=False):
+            Ly = layers[l % L]
+            return moe_prefill_layer(xp, Ly["wr"], Ly["w13c"], Ly["w13s"], Ly["w2c"], Ly["w2s"], Ly["sw13"],
+                                     Ly["sw2"], top_k=S.k, ws=wsp, y=yp, want_routing=ids)
+        hit = []
+        for i in range(min(L, K + W)):
+            _, ids, _, _ = pf(i, ids=True)
+            hit.append(len(np.unique(ids.cpu().numpy())))
+        for i in range(W):
+            pf(i)
+        torch.cuda.synchronize()
+        barrier()
+        e0.record()
+        for i in range(K):
+            pf(W + i)
+        e1.record()
+        torch.cuda.synchronize()
+        barrier()
+        ms = max_over_ranks(e0.elapsed_time(e1)) / K
+        n_hit = float(np.mean(hit))
+        wbytes = S.E * S.H * 2 + n_hit * S.expert_bytes + 3 * S.Is * S.H * 2
+        abytes = Mp * S.H * 2 + Mp * S.H * 4
+        flops = 2.0 * Mp * S.k * (3 * S.I * S.H) + 2.0 * Mp * (3 * S.Is * S.H) + 2.0 * Mp * S.E * S.H
+        results["prefill"] = {"M": Mp, "us_per_chunk": 1000 * ms, "experts_hit": n_hit,
+                              "weight_bytes": wbytes, "gbps": world * (wbytes + abytes) / (ms * 1e-3) / 1e9,
+                              "tflops": world * flops / (ms * 1e-3) / 1e12, "launches_per_chunk": 10}
+
     # CPU oracle baseline (rank 0, single GPU only): a bounded sample of the same step
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -495,6 +534,11 @@ def main():
                           "frac_of_8tbs": r4["gbps"] / world / NOMINAL_HBM_GBS,
                           "frac_of_measured_hbm": r4["gbps"] / world / hbm,
                           "mean_unique_experts": r4["mean_unique_experts"], "e2e": r4["e2e"], "clocks": r4["clocks"]}
+        if "prefill" in results:
+            rp = results["prefill"]
+            line["prefill"] = dict(rp, frac_of_measured_hbm=rp["gbps"] / world / hbm,
+                                   workload=f"prefill chunk: one MoE layer, M={rp['M']} tokens, MXFP8 activations, "
+                                            "tcgen05 block-scaled MMA")
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

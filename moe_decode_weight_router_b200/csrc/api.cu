@@ -861,6 +861,24 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType t, const void* base, uint64_t 
          CUDA_SUCCESS;
 }
 
+// Bytes per activation-scale row: K/32 rounded up to 16 (rows are bulk-copied).
+int pf_sf_ld(int K) { return (K / 32 + 15) / 16 * 16; }
+
+// Weight operand as {K elements, rows, 2 halves}: one box of {box_inner, 64, 2} brings
+// 64 rows and the 64 rows half_bytes further on (gate and up rows, or the next 64).
+bool make_map_halves(CUtensorMap* m, CUtensorMapDataType t, const void* base, uint64_t inner, uint64_t rows,
+                     uint64_t row_bytes, uint64_t half_bytes, uint32_t box_inner) {
+  EncodeTiledFn f = encode_fn();
+  if (!f) return false;
+  cuuint64_t dims[3] = {inner, rows, 2};
+  cuuint64_t strides[2] = {row_bytes, half_bytes};
+  cuuint32_t box[3] = {box_inner, 64, 2};
+  cuuint32_t es[3] = {1, 1, 1};
+  return f(m, t, 3, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 bool ok_pf(int M, int H, int I, int E, int k, int Is) {
   return M >= 128 && M % 128 == 0 && M <= 16384 && H >= 128 && H % 128 == 0 && H <= 4096 && I >= 128 &&
          I % 128 == 0 && I <= 4096 && E >= 128 && E % 128 == 0 && E <= 512 && k >= 1 && k <= 8 && Is >= 0 &&
@@ -918,22 +936,24 @@ PfWs pf_ws(void* ws, int M, int H, int I, int E, int k, int Is) {
   s.xq = b + off;
   off += up256(G * H);
   s.xs = b + off;
-  off += up256(G * (H / 32));
+  off += up256(G * pf_sf_ld(H));
   s.as = reinterpret_cast<__nv_bfloat16*>(b + off);
   off += up256((size_t)M * (Is > 0 ? Is : 1) * 2);
   s.aq = b + off;
   off += up256(G * I);
   s.aqs = b + off;
-  off += up256(G * (I / 32));
+  off += up256(G * pf_sf_ld(I));
   s.bytes = off;
   return s;
 }
 
 moe_status_t launch_umma(PrefillParams& p, const DevInfo& d, cudaStream_t st) {
-  const int stages = (d.dyn_pf - 1024) / PF_STAGE_BYTES;
+  const size_t sf = (p.mode == PF_R13 || p.mode == PF_R2) ? 2 * (size_t)pf_sf_buf_bytes(p.K, p.sf_ld) : 0;
+  const long long room = (long long)d.dyn_pf - 1024 - (long long)sf;
+  const int stages = room > 0 ? (int)(room / PF_STAGE_BYTES) : 0;
   p.stages = stages > PF_MAX_STAGES ? PF_MAX_STAGES : stages;
   if (p.stages < 2) return MOE_ERR_UNSUPPORTED_SHAPE;
-  const size_t smem = 1024 + (size_t)p.stages * PF_STAGE_BYTES;
+  const size_t smem = 1024 + (size_t)p.stages * PF_STAGE_BYTES + sf;
   k_umma<<<d.sms, PF_THREADS, smem, st>>>(p);
   MOE_CUDA(cudaGetLastError());
   return MOE_OK;
@@ -975,9 +995,10 @@ moe_status_t moe_prefill_layer(const void* x_bf16, int M, int H, int I, int E, i
   PrefillParams p{};
   p.status = w.status;
   p.E = E;
-  REQ(make_map(&p.tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w_router_bf16, H, E, (uint64_t)H * 2, 64, 64),
+  REQ(make_map_halves(&p.tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w_router_bf16, H, E, (uint64_t)H * 2,
+                      (uint64_t)64 * H * 2, 64),
       MOE_ERR_INVALID_ARG);
-  REQ(make_map(&p.tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, H, M, (uint64_t)H * 2, 64, 32), MOE_ERR_INVALID_ARG);
+  REQ(make_map(&p.tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, H, M, (uint64_t)H * 2, 64, 64), MOE_ERR_INVALID_ARG);
   p.mode = PF_ROUTER;
   p.K = H;
   p.m_tiles = E / 128;
@@ -992,15 +1013,16 @@ moe_status_t moe_prefill_layer(const void* x_bf16, int M, int H, int I, int E, i
   MOE_CUDA(cudaGetLastError());
   k_pf_scatter<<<(G + 255) / 256, 256, 0, st>>>(w.ids, w.w, M, top_k, w.goff, w.fill, w.g_tok, w.g_w, w.pos);
   MOE_CUDA(cudaGetLastError());
-  k_pf_quant_x<<<(int)(((long long)M * (H / 32) + 7) / 8), 256, 0, st>>>(x, M, H, top_k, w.pos, w.xq, w.xs);
+  k_pf_quant_x<<<(int)(((long long)M * (H / 32) + 7) / 8), 256, 0, st>>>(x, M, H, top_k, w.pos, w.xq, w.xs,
+                                                                          pf_sf_ld(H));
   MOE_CUDA(cudaGetLastError());
 
   // a5: shared expert (bf16): a_s = bf16(silu(Wg x) * Wu x), y = Ws2 a_s
   if (Is > 0) {
     PrefillParams q{};
     q.status = w.status;
-    REQ(make_map(&q.tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, shared_w13_bf16, H, 2 * (uint64_t)Is, (uint64_t)H * 2, 64,
-                 64),
+    REQ(make_map_halves(&q.tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, shared_w13_bf16, H, 2 * (uint64_t)Is,
+                        (uint64_t)H * 2, (uint64_t)Is * H * 2, 64),
         MOE_ERR_INVALID_ARG);
     q.tmB = p.tmB;
     q.mode = PF_SH13;
@@ -1013,9 +1035,10 @@ moe_status_t moe_prefill_layer(const void* x_bf16, int M, int H, int I, int E, i
     if ((s = launch_umma(q, d, st)) != MOE_OK) return s;
     PrefillParams r{};
     r.status = w.status;
-    REQ(make_map(&r.tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, shared_w2_bf16, Is, H, (uint64_t)Is * 2, 64, 64),
+    REQ(make_map_halves(&r.tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, shared_w2_bf16, Is, H, (uint64_t)Is * 2,
+                        (uint64_t)64 * Is * 2, 64),
         MOE_ERR_INVALID_ARG);
-    REQ(make_map(&r.tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w.as, Is, M, (uint64_t)Is * 2, 64, 32), MOE_ERR_INVALID_ARG);
+    REQ(make_map(&r.tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w.as, Is, M, (uint64_t)Is * 2, 64, 64), MOE_ERR_INVALID_ARG);
     r.mode = PF_SH2;
     r.K = Is;
     r.m_tiles = H / 128;
@@ -1030,10 +1053,10 @@ moe_status_t moe_prefill_layer(const void* x_bf16, int M, int H, int I, int E, i
   // a3: routed W13 + SwiGLU, activation re-quantised to MXFP8 (E2M1 x E4M3 block-scaled)
   PrefillParams a{};
   a.status = w.status;
-  REQ(make_map(&a.tmA, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, w13_codes, H, (uint64_t)E * 2 * I, (uint64_t)H / 2, 128,
-               64),
+  REQ(make_map_halves(&a.tmA, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, w13_codes, H, (uint64_t)E * 2 * I,
+                      (uint64_t)H / 2, (uint64_t)I * (H / 2), 128),
       MOE_ERR_INVALID_ARG);
-  REQ(make_map(&a.tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.xq, H, G, H, 128, 32), MOE_ERR_INVALID_ARG);
+  REQ(make_map(&a.tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.xq, H, G, H, 128, 64), MOE_ERR_INVALID_ARG);
   a.mode = PF_R13;
   a.K = H;
   a.m_tiles = I / 64;
@@ -1042,19 +1065,23 @@ moe_status_t moe_prefill_layer(const void* x_bf16, int M, int H, int I, int E, i
   a.E = E;
   a.ntile_prefix = w.ntp;
   a.goff = w.goff;
+  a.a_codes = w13_codes;
   a.sfa = w13_scales;
   a.sfb = w.xs;
+  a.sf_ld = pf_sf_ld(H);
   a.out_q = w.aq;
   a.out_qs = w.aqs;
+  a.out_qs_ld = pf_sf_ld(I);
   a.out_ld = I;
   if ((s = launch_umma(a, d, st)) != MOE_OK) return s;
 
   // a4: routed W2, weighted by the routing weight and added into y
   PrefillParams b{};
   b.status = w.status;
-  REQ(make_map(&b.tmA, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, w2_codes, I, (uint64_t)E * H, (uint64_t)I / 2, 128, 64),
+  REQ(make_map_halves(&b.tmA, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, w2_codes, I, (uint64_t)E * H, (uint64_t)I / 2,
+                      (uint64_t)64 * (I / 2), 128),
       MOE_ERR_INVALID_ARG);
-  REQ(make_map(&b.tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.aq, I, G, I, 128, 32), MOE_ERR_INVALID_ARG);
+  REQ(make_map(&b.tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.aq, I, G, I, 128, 64), MOE_ERR_INVALID_ARG);
   b.mode = PF_R2;
   b.K = I;
   b.m_tiles = H / 128;
@@ -1064,8 +1091,10 @@ moe_status_t moe_prefill_layer(const void* x_bf16, int M, int H, int I, int E, i
   b.goff = w.goff;
   b.g_tok = w.g_tok;
   b.g_w = w.g_w;
+  b.a_codes = w2_codes;
   b.sfa = w2_scales;
   b.sfb = w.aqs;
+  b.sf_ld = pf_sf_ld(I);
   b.out_f32 = y;
   b.out_ld = H;
   if ((s = launch_umma(b, d, st)) != MOE_OK) return s;

@@ -9,8 +9,10 @@
 //
 // Every GEMM of the layer is one launch of k_umma, a persistent warp-specialised
 // kernel (one CTA per SM):
-//   warp 4      TMA producer: weight tile (two 64-row boxes, 128 B of K per row) and
-//               activation tile (32-row boxes) per K chunk into a ring of stages;
+//   warp 4      TMA producer: per K chunk, one tensor copy for the weight tile (two
+//               64-row halves -- gate/up, or consecutive rows -- through a 3-D map)
+//               and one for the 64-token tile, into a ring of stages (the TMA engine
+//               takes copies at a bounded rate, so every copy moves as much as it can);
 //   warp 5      MMA issuer: one elected thread issues tcgen05.mma (M = 128 weight rows,
 //               N = tokens, fp32 accumulator in tensor memory) and commits each stage
 //               back to the producer and each finished tile to the epilogue;
@@ -39,16 +41,16 @@ namespace moe {
 
 enum : int { PF_ROUTER = 0, PF_SH13 = 1, PF_SH2 = 2, PF_R13 = 3, PF_R2 = 4 };
 constexpr int PF_THREADS = 192;        // warps 0-3 epilogue, 4 producer, 5 MMA
-constexpr int PF_BN = 128;             // token tile (MMA N <= 128)
-constexpr int PF_STAGE_BYTES = 32768;  // weight tile 16 KB + token tile 16 KB
-constexpr int PF_MAX_STAGES = 6;
-constexpr int PF_TMEM_COLS = 512;      // accumulator 0..127, SFA 128.., SFB 256..
-constexpr int PF_SFA_COL = 128, PF_SFB_COL = 256;
+constexpr int PF_BN = 64;              // token tile (MMA N <= 64)
+constexpr int PF_STAGE_BYTES = 24576;  // weight tile 16 KB + token tile 8 KB
+constexpr int PF_MAX_STAGES = 9;
+constexpr int PF_TMEM_COLS = 512;      // accumulators 0..127 and 128..255, SFA 256.., SFB 384..
+constexpr int PF_SFA_COL = 256, PF_SFB_COL = 384;
 constexpr int PF_MAX_CHUNKS = 32;      // K / 128 for the block-scaled modes (SF columns)
 
 struct alignas(64) PrefillParams {
-  CUtensorMap tmA;  // weights: dims {K, rows}, box {64 or 128 elements, 64 rows}
-  CUtensorMap tmB;  // activations: dims {K, rows}, box {.., 32 rows}
+  CUtensorMap tmA;  // weights: dims {K, rows, 2 halves}, box {64 or 128 elements, 64 rows, 2}
+  CUtensorMap tmB;  // activations: dims {K, rows}, box {.., 64 rows}
   int mode;
   int K;
   int m_tiles;   // weight tiles per problem
@@ -56,17 +58,20 @@ struct alignas(64) PrefillParams {
   int prob_rows; // weight rows per problem (expert) for the routed modes
   int M;         // dense modes: tokens
   int E;
+  const uint8_t* a_codes;   // routed: the weight codes the tensor map covers (L2 prefetch of the next tile)
   const int* ntile_prefix;  // routed: [E+1] prefix sums of ceil(n_e / 128)
   const int* goff;          // routed: [E+1] first grouped row of each expert
   const int32_t* g_tok;     // routed: [G] token of each grouped row
   const float* g_w;         // routed: [G] routing weight of each grouped row
   const uint8_t* sfa;       // routed: weight scales [rows][K/32]
-  const uint8_t* sfb;       // routed: activation scales [G][K/32]
+  const uint8_t* sfb;       // routed: activation scales [G][sf_ld]
+  int sf_ld;                // routed: bytes per activation-scale row (K/32 rounded up to 16)
   int out_ld;               // leading dimension of the output
   float* out_f32;           // router logits [M][E], y [M][H]
   __nv_bfloat16* out_bf16;  // shared activation [M][Is]
   uint8_t* out_q;           // routed activation e4m3 [G][I]
-  uint8_t* out_qs;          // routed activation E8M0 [G][I/32]
+  uint8_t* out_qs;          // routed activation E8M0 [G][out_qs_ld]
+  int out_qs_ld;
   int stages;
   int* status;
 };
@@ -126,6 +131,16 @@ __device__ __forceinline__ void umma_mx(uint32_t d, uint64_t adesc, uint64_t bde
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc), "r"(tsfa), "r"(tsfb)
       : "memory");
 }
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+      "[%5];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
@@ -157,7 +172,9 @@ __device__ __noinline__ bool pf_wait(uint64_t* bar, uint32_t parity, int* status
                                      int site, int mode) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity)) {
+  for (unsigned n = 1;; ++n) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((n & 63u) != 0) continue;  // the clock and the flag are read every 64 polls
     if (*abort_flag) return false;
     if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
       if (atomicCAS(status, 0, DEV_ERR_TIMEOUT) == 0) {
@@ -188,11 +205,15 @@ struct PfItem {
 __device__ __forceinline__ bool pf_routed(int mode) { return mode == PF_R13 || mode == PF_R2; }
 __device__ __forceinline__ bool pf_13(int mode) { return mode == PF_SH13 || mode == PF_R13; }
 
-__device__ inline int pf_total_items(const PrefillParams& p) {
-  if (pf_routed(p.mode)) return p.m_tiles * __ldg(p.ntile_prefix + p.E);
+constexpr int PF_MAX_E = 512;
+// Routed modes: tile prefix and grouped offsets are copied to shared memory once per
+// CTA (every role decodes every tile; a search over global memory would put a chain
+// of dependent loads in front of each tile).
+__device__ inline int pf_total_items(const PrefillParams& p, const int* s_ntp) {
+  if (pf_routed(p.mode)) return p.m_tiles * s_ntp[p.E];
   return p.m_tiles * ((p.M + PF_BN - 1) / PF_BN);
 }
-__device__ inline PfItem pf_item(const PrefillParams& p, int idx) {
+__device__ inline PfItem pf_item(const PrefillParams& p, int idx, const int* s_ntp, const int* s_goff) {
   PfItem it;
   it.mt = idx % p.m_tiles;
   const int j = idx / p.m_tiles;
@@ -201,14 +222,14 @@ __device__ inline PfItem pf_item(const PrefillParams& p, int idx) {
     int lo = 0, hi = p.E;  // largest e with ntile_prefix[e] <= j
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
-      if (__ldg(p.ntile_prefix + mid) <= j)
+      if (s_ntp[mid] <= j)
         lo = mid;
       else
         hi = mid;
     }
     it.e = lo;
-    it.n0 = (j - __ldg(p.ntile_prefix + lo)) * PF_BN;
-    const int g0 = __ldg(p.goff + lo), ne = __ldg(p.goff + lo + 1) - g0;
+    it.n0 = (j - s_ntp[lo]) * PF_BN;
+    const int g0 = s_goff[lo], ne = s_goff[lo + 1] - g0;
     it.ncnt = min(PF_BN, ne - it.n0);
     it.grow0 = g0 + it.n0;
     rows0 = lo * p.prob_rows;
@@ -251,31 +272,54 @@ __device__ __forceinline__ uint8_t e4m3_of(float v) {
 // ---------------------------------------------------------------------------
 // k_umma
 // ---------------------------------------------------------------------------
+// Shared memory: the 1024-aligned stage ring (weight tile at +0 and +8192, token tile
+// at +16384 in 32-row boxes of 4096 B), then for the block-scaled modes two buffers of
+// the current tiles' E8M0 rows (weight rows at +0, K/32 bytes each; token rows after
+// them, sf_ld bytes each), filled by the producer with bulk copies.
+__host__ __device__ inline uint32_t pf_sf_buf_bytes(int K, int sf_ld) {
+  const uint32_t a = (uint32_t)(128 * (K / 32) + 15) / 16 * 16;
+  return a + 128u * (uint32_t)sf_ld;
+}
+
 __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ PrefillParams p) {
   extern __shared__ __align__(1024) uint8_t pf_smem_raw[];
-  // 1024-byte alignment of the stage ring (the 128-byte swizzle atom)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(pf_smem_raw) + 1023) & ~uintptr_t(1023));
   __shared__ uint64_t full[PF_MAX_STAGES], empty[PF_MAX_STAGES];
-  __shared__ uint64_t acc_full, acc_empty, sf_ready;
+  __shared__ uint64_t acc_full[2], acc_empty[2], sf_full[2], sf_empty[2], sf_ready;
   __shared__ uint32_t tmem_base_s;
   __shared__ volatile int s_abort;
   __shared__ float xch[2][32][17];  // up-half values handed from warps 2,3 to warps 0,1
+  __shared__ int s_ntp[PF_MAX_E + 1], s_goff[PF_MAX_E + 1];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int S = p.stages;
   const bool mx = pf_routed(p.mode);
   const int kbox = mx ? 128 : 64;  // K elements per stage (128 bytes per row)
   const int nch = p.K / kbox;
-  const int total = pf_total_items(p);
+  if (mx)
+    for (int e = tid; e <= p.E; e += PF_THREADS) {
+      s_ntp[e] = __ldg(p.ntile_prefix + e);
+      s_goff[e] = __ldg(p.goff + e);
+    }
+  __syncthreads();
+  const int total = pf_total_items(p, s_ntp);
   const int G = gridDim.x;
+  const int kb = p.K / 32;  // E8M0 bytes per weight row
+  const uint32_t sfa_bytes = (uint32_t)(128 * kb + 15) / 16 * 16;
+  uint8_t* sfbuf = smem + (size_t)S * PF_STAGE_BYTES;
+  const uint32_t sfbuf_bytes = pf_sf_buf_bytes(p.K, p.sf_ld);
 
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(&acc_full, 1);
-    mbar_init(&acc_empty, 4);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 4);
+      mbar_init(&sf_full[b], 1);
+      mbar_init(&sf_empty[b], 4);
+    }
     mbar_init(&sf_ready, 4);
     fence_mbar_init();
     s_abort = 0;
@@ -293,11 +337,27 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
     // ---------------- TMA producer ----------------
     if (lane == 0) {
       long long q = 0;
+      int n_item = 0;
       bool ok = true;
-      for (int idx = blockIdx.x; idx < total && ok; idx += G) {
-        const PfItem it = pf_item(p, idx);
-        const int N = (it.ncnt + 15) & ~15;
-        const int nb = (N + 31) / 32;
+      for (int idx = blockIdx.x; idx < total && ok; idx += G, ++n_item) {
+        const PfItem it = pf_item(p, idx, s_ntp, s_goff);
+        if (mx) {
+          // this tile's scale rows: weight rows (two 64-row runs or one 128-row run) and
+          // the token rows, into scale buffer n_item & 1
+          const int b = n_item & 1;
+          if (n_item >= 2 && !pf_wait(&sf_empty[b], (uint32_t)(((n_item >> 1) - 1) & 1), p.status, &s_abort,
+                                      PFW_SF, p.mode)) {
+            ok = false;
+            break;
+          }
+          uint8_t* dst = sfbuf + (size_t)b * sfbuf_bytes;
+          const uint32_t half = 64u * (uint32_t)kb, tok = (uint32_t)it.ncnt * (uint32_t)p.sf_ld;
+          mbar_arrive_expect_tx(&sf_full[b], 2 * half + tok);
+          const uint64_t pol = policy_evict_first();
+          bulk_g2s(dst, p.sfa + (size_t)it.ya0 * kb, half, &sf_full[b], pol);
+          bulk_g2s(dst + half, p.sfa + (size_t)it.ya1 * kb, half, &sf_full[b], pol);
+          bulk_g2s(dst + sfa_bytes, p.sfb + (size_t)it.grow0 * p.sf_ld, tok, &sf_full[b], pol);
+        }
         for (int ch = 0; ch < nch; ++ch, ++q) {
           const int s = (int)(q % S);
           if (q >= S && !pf_wait(&empty[s], (uint32_t)(((q / S) - 1) & 1), p.status, &s_abort, PFW_EMPTY, p.mode)) {
@@ -305,16 +365,20 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
             break;
           }
           uint8_t* st = smem + (size_t)s * PF_STAGE_BYTES;
-          // transaction bytes count the global (packed) side: a 64-row box of 128
-          // E2M1 codes is 4 KB although it fills 8 KB of shared memory
-          mbar_arrive_expect_tx(&full[s], (mx ? 8192u : 16384u) + 4096u * (uint32_t)nb);
-          tma_load_2d(st, &p.tmA, ch * kbox, it.ya0, &full[s]);
-          tma_load_2d(st + 8192, &p.tmA, ch * kbox, it.ya1, &full[s]);
-          for (int b = 0; b < nb; ++b) tma_load_2d(st + 16384 + 4096 * b, &p.tmB, ch * kbox, it.grow0 + 32 * b, &full[s]);
+          // transaction bytes count the global (packed) side: 128 rows of 128 E2M1
+          // codes are 8 KB although they fill 16 KB of shared memory; the token box
+          // is always whole (rows past the tensor read as zeros and still count)
+          mbar_arrive_expect_tx(&full[s], (mx ? 8192u : 16384u) + 8192u);
+          tma_load_3d(st, &p.tmA, ch * kbox, it.ya0, 0, &full[s]);
+          tma_load_2d(st + 16384, &p.tmB, ch * kbox, it.grow0, &full[s]);
         }
       }
       // every copy issued lands before the CTA may finish
-      for (long long j = (q > S ? q - S : 0); j < q; ++j) pf_wait(&full[j % S], (uint32_t)((j / S) & 1), p.status, &s_abort, PFW_DRAIN, p.mode);
+      for (long long j = (q > S ? q - S : 0); j < q; ++j)
+        pf_wait(&full[j % S], (uint32_t)((j / S) & 1), p.status, &s_abort, PFW_DRAIN, p.mode);
+      if (mx)
+        for (int j = (n_item > 2 ? n_item - 2 : 0); j < n_item; ++j)
+          pf_wait(&sf_full[j & 1], (uint32_t)((j >> 1) & 1), p.status, &s_abort, PFW_DRAIN, p.mode);
     }
   } else if (warp == 5) {
     // ---------------- MMA issuer ----------------
@@ -323,11 +387,15 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
       int n_item = 0;
       bool ok = true;
       for (int idx = blockIdx.x; idx < total && ok; idx += G, ++n_item) {
-        const PfItem it = pf_item(p, idx);
+        const PfItem it = pf_item(p, idx, s_ntp, s_goff);
         const int N = (it.ncnt + 15) & ~15;
-        if (n_item > 0 && !pf_wait(&acc_empty, (uint32_t)((n_item - 1) & 1), p.status, &s_abort, PFW_ACC_EMPTY, p.mode)) break;
+        const int ab = n_item & 1;
+        if (n_item >= 2 && !pf_wait(&acc_empty[ab], (uint32_t)(((n_item >> 1) - 1) & 1), p.status, &s_abort,
+                                    PFW_ACC_EMPTY, p.mode))
+          break;
         if (mx && !pf_wait(&sf_ready, (uint32_t)(n_item & 1), p.status, &s_abort, PFW_SF, p.mode)) break;
         tc_fence_after();
+        const uint32_t dacc = tbase + 128u * ab;
         for (int ch = 0; ch < nch; ++ch, ++q) {
           const int s = (int)(q % S);
           if (!pf_wait(&full[s], (uint32_t)((q / S) & 1), p.status, &s_abort, PFW_FULL, p.mode)) {
@@ -342,72 +410,84 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
             const uint32_t accum = (ch > 0 || k > 0) ? 1u : 0u;
             // advance 32 bytes of K inside the 128-byte swizzled row
             if (mx)
-              umma_mx(tbase, adesc + 2u * k, bdesc + 2u * k, idesc_mx(N, (uint32_t)k), accum,
+              umma_mx(dacc, adesc + 2u * k, bdesc + 2u * k, idesc_mx(N, (uint32_t)k), accum,
                       tbase + PF_SFA_COL + 4u * ch, tbase + PF_SFB_COL + 4u * ch);
             else
-              umma_bf16(tbase, adesc + 2u * k, bdesc + 2u * k, idesc_bf16(N), accum);
+              umma_bf16(dacc, adesc + 2u * k, bdesc + 2u * k, idesc_bf16(N), accum);
           }
           tc_commit(&empty[s]);  // the stage returns to the producer once these MMAs are done
         }
         if (!ok) break;
-        tc_commit(&acc_full);  // the accumulator is complete
+        tc_commit(&acc_full[ab]);  // accumulator ab is complete (and so are this tile's reads of the scales)
       }
     }
   } else {
     // ---------------- epilogue warps 0-3 ----------------
     const int r = lane;
     const uint32_t lane_base = tbase + ((uint32_t)(32 * warp) << 16);
-    int n_item = 0;
-    for (int idx = blockIdx.x; idx < total; idx += G, ++n_item) {
-      const PfItem it = pf_item(p, idx);
-      if (mx) {
-        // scale factors of this tile (the previous tile's MMAs are complete: its
-        // accumulator was waited for below before this point)
-        const int kb = p.K / 32;
-        const uint8_t* arow[4];
-        const uint8_t* brow[4];
+    // E8M0 words of a tile from its scale buffer into tensor memory (lane r of every
+    // quarter, column base + 4ch + c: operand row r + 32c, K blocks 4ch..4ch+3)
+    auto put_scales = [&](int n_item, const PfItem& it) -> bool {
+      const int b = n_item & 1;
+      if (!pf_wait(&sf_full[b], (uint32_t)((n_item >> 1) & 1), p.status, &s_abort, PFW_SF, p.mode)) return false;
+      const uint8_t* sa = sfbuf + (size_t)b * sfbuf_bytes;
+      const uint8_t* sb = sa + sfa_bytes;
+      for (int ch = 0; ch < nch; ++ch) {
+        uint32_t wa[4], wb[4];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           const int m = r + 32 * c;
-          arow[c] = p.sfa + (size_t)(m < 64 ? it.ya0 + m : it.ya1 + (m - 64)) * kb;
-          brow[c] = m < it.ncnt ? p.sfb + (size_t)(it.grow0 + m) * kb : nullptr;
+          wa[c] = *reinterpret_cast<const uint32_t*>(sa + m * kb + 4 * ch);
+          wb[c] = m < it.ncnt ? *reinterpret_cast<const uint32_t*>(sb + m * p.sf_ld + 4 * ch) : 0x7F7F7F7Fu;
         }
-        for (int ch = 0; ch < nch; ++ch) {
-          uint32_t wa[4], wb[4];
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            wa[c] = __ldg(reinterpret_cast<const uint32_t*>(arow[c] + 4 * ch));
-            wb[c] = brow[c] ? __ldg(reinterpret_cast<const uint32_t*>(brow[c] + 4 * ch)) : 0x7F7F7F7Fu;
-          }
-          tmem_st4(lane_base + PF_SFA_COL + 4 * ch, wa[0], wa[1], wa[2], wa[3]);
-          tmem_st4(lane_base + PF_SFB_COL + 4 * ch, wb[0], wb[1], wb[2], wb[3]);
-        }
-        tc_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sf_ready);
+        tmem_st4(lane_base + PF_SFA_COL + 4 * ch, wa[0], wa[1], wa[2], wa[3]);
+        tmem_st4(lane_base + PF_SFB_COL + 4 * ch, wb[0], wb[1], wb[2], wb[3]);
       }
-      pf_wait(&acc_full, (uint32_t)(n_item & 1), p.status, &s_abort, PFW_ACC_FULL, p.mode);
+      tc_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&sf_ready);
+        mbar_arrive(&sf_empty[b]);
+      }
+      return true;
+    };
+    bool live = true;
+    if (mx && blockIdx.x < total) live = put_scales(0, pf_item(p, blockIdx.x, s_ntp, s_goff));
+    int n_item = 0;
+    for (int idx = blockIdx.x; idx < total; idx += G, ++n_item) {
+      const PfItem it = pf_item(p, idx, s_ntp, s_goff);
+      const int ab = n_item & 1;
+      if (live) pf_wait(&acc_full[ab], (uint32_t)((n_item >> 1) & 1), p.status, &s_abort, PFW_ACC_FULL, p.mode);
       named_barrier(2, 128);  // the four epilogue warps take the same decision below
       if (s_abort) break;
       tc_fence_after();
+      // the MMAs of this tile are complete: the scale columns may take the next tile's
+      if (mx && idx + G < total) live = put_scales(n_item + 1, pf_item(p, idx + G, s_ntp, s_goff));
+      const uint32_t acc_lane = lane_base + 128u * ab;
       for (int j0 = 0; j0 < it.ncnt; j0 += 16) {
         float v[16];
-        tmem_ld16(lane_base + (uint32_t)j0, v);
+        tmem_ld16(acc_lane + (uint32_t)j0, v);
         const int jn = min(16, it.ncnt - j0);
         if (p.mode == PF_ROUTER || p.mode == PF_SH2) {
           const int row = 128 * it.mt + 32 * warp + r;
-          for (int j = 0; j < jn; ++j) p.out_f32[(size_t)(it.n0 + j0 + j) * p.out_ld + row] = v[j];
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (j < jn) p.out_f32[(size_t)(it.n0 + j0 + j) * p.out_ld + row] = v[j];
         } else if (p.mode == PF_R2) {
           const int row = 128 * it.mt + 32 * warp + r;
-          for (int j = 0; j < jn; ++j) {
-            const int g = it.grow0 + j0 + j;
-            atomicAdd(p.out_f32 + (size_t)__ldg(p.g_tok + g) * p.out_ld + row, __ldg(p.g_w + g) * v[j]);
-          }
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (j < jn) {
+              const int g = it.grow0 + j0 + j;
+              atomicAdd(p.out_f32 + (size_t)__ldg(p.g_tok + g) * p.out_ld + row, __ldg(p.g_w + g) * v[j]);
+            }
         } else {
           // 13 modes: warps 0,1 hold gate rows, warps 2,3 the matching up rows
-          if (warp >= 2)
+          if (warp >= 2) {
+#pragma unroll
             for (int j = 0; j < 16; ++j) xch[warp - 2][r][j] = v[j];
+          }
           named_barrier(2, 128);
           if (warp < 2) {
             const int i = 64 * it.mt + 32 * warp + r;  // intermediate index
@@ -415,19 +495,20 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
 #pragma unroll
             for (int j = 0; j < 16; ++j) a[j] = pf_silu(v[j]) * xch[warp][r][j];
             if (p.mode == PF_SH13) {
-              for (int j = 0; j < jn; ++j) p.out_bf16[(size_t)(it.n0 + j0 + j) * p.out_ld + i] = __float2bfloat16_rn(a[j]);
+#pragma unroll
+              for (int j = 0; j < 16; ++j)
+                if (j < jn) p.out_bf16[(size_t)(it.n0 + j0 + j) * p.out_ld + i] = __float2bfloat16_rn(a[j]);
             } else {
-              // MXFP8 of each token's 32-block (this warp's 32 rows)
+              // MXFP8 of each token's 32-block (this warp's 32 rows): the block maximum
+              // of |a| is one warp max over the bit patterns (monotonic for x >= 0)
 #pragma unroll
               for (int j = 0; j < 16; ++j) {
-                float am = fabsf(a[j]);
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+                const float am = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(a[j]))));
                 const int s = mxfp8_exponent(am);
                 if (j < jn) {
                   const size_t g = (size_t)(it.grow0 + j0 + j);
                   p.out_q[g * p.out_ld + i] = am == 0.0f ? (uint8_t)0 : e4m3_of(a[j] * exp2i(-s));
-                  if (r == 0) p.out_qs[g * (p.out_ld / 32) + (64 * it.mt + 32 * warp) / 32] = (uint8_t)(s + 127);
+                  if (r == 0) p.out_qs[g * p.out_qs_ld + (64 * it.mt + 32 * warp) / 32] = (uint8_t)(s + 127);
                 }
               }
             }
@@ -437,7 +518,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty);
+      if (lane == 0) mbar_arrive(&acc_empty[ab]);
     }
   }
   tc_fence_before();
@@ -544,7 +625,7 @@ __global__ void k_pf_scatter(const int32_t* __restrict__ ids, const float* __res
 // per (token, 32-block); lane = element.
 __global__ void __launch_bounds__(256) k_pf_quant_x(const __nv_bfloat16* __restrict__ x, int M, int H, int k,
                                                      const int32_t* __restrict__ pos, uint8_t* __restrict__ xq,
-                                                     uint8_t* __restrict__ xs) {
+                                                     uint8_t* __restrict__ xs, int xs_ld) {
   const int lane = threadIdx.x & 31;
   const long long wi = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int nb = H / 32;
@@ -559,7 +640,7 @@ __global__ void __launch_bounds__(256) k_pf_quant_x(const __nv_bfloat16* __restr
   for (int j = 0; j < k; ++j) {
     const size_t g = (size_t)pos[(size_t)t * k + j];
     xq[g * H + 32 * b + lane] = q;
-    if (lane == 0) xs[g * nb + b] = (uint8_t)(s + 127);
+    if (lane == 0) xs[g * xs_ld + b] = (uint8_t)(s + 127);
   }
 }
 
