@@ -165,6 +165,37 @@ MOE_API moe_status_t lm_head_fp8_gemv(const void* x_bf16, int M, int V, int H, c
                               const float* row_scale, float* logits, int32_t* argmax,
                               void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* Verify window of multi-token prediction, fused into the head's argmax tail (source:
+ * the DGX Spark MoE knowledge card, 方法/产品要点 item 2 -- the window of the last
+ * accepted token and M-1 draft tokens goes through the step at once).  As
+ * lm_head_fp8_gemv for the M window positions, then draft t+1 is accepted while it
+ * equals argmax[t], and argmax at the first mismatch (or after the last draft) is
+ * accepted too:
+ *   drafts [M-1] int32 in; accept [1+M] int32 out: accept[0] = accepted count (1..M),
+ *   accept[1..count] = the accepted tokens.  2 <= M <= 8; other limits as the GEMV. */
+MOE_API moe_status_t lm_head_fp8_verify(const void* x_bf16, int M, int V, int H, const uint8_t* w_e4m3,
+                                        const float* row_scale, const int32_t* drafts, float* logits,
+                                        int32_t* argmax, int32_t* accept, void* ws, size_t ws_bytes,
+                                        moe_stream_t stream);
+
+/* The same head on the BF16 weights it is quantised from (the comparison the FP8
+ * head halves the bytes against; same knowledge card, 方法/产品要点 item 2):
+ *   logits[t][v] = sum_h w_bf16[v][h] * x[t][h] (fp32 accumulation), argmax as above.
+ *   w_bf16 [V][H] bf16; workspace as lm_head_workspace_bytes; limits as the FP8 GEMV. */
+MOE_API moe_status_t lm_head_bf16_gemv(const void* x_bf16, int M, int V, int H, const void* w_bf16,
+                                       float* logits, int32_t* argmax, void* ws, size_t ws_bytes,
+                                       moe_stream_t stream);
+
+/* Sampling of one token per row of fp32 logits [M][V] (the knowledge card's serving
+ * settings: temperature, top-k 29, top-p 0.95), the uniform draw u [M] in [0,1) given:
+ * z = logits / T over the top_k largest logits (ties to the lower index), p = softmax
+ * of z, nucleus = the shortest prefix (in that order) with sum p >= top_p, sample =
+ * the first nucleus token whose cumulative p / sum_nucleus p exceeds u.
+ *   ids [M] int32 out.  1 <= top_k <= 32 (and <= V); T > 0; 0 < top_p <= 1.
+ *   At most 1024 logits may tie at or above the top_k-th value. */
+MOE_API moe_status_t moe_sample(const float* logits, int M, int V, float temperature, int top_k, float top_p,
+                                const float* u, int32_t* ids, moe_stream_t stream);
+
 /* Allocation-free variant of lm_head_fp8_gemv (no counterpart on the pages; it
  * exists for integration).  Some callers cannot hand this library any scratch
  * memory: an operator slot that passes only input and output tensors and has no

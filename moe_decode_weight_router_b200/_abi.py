@@ -57,6 +57,9 @@ SIGNATURES = {
     "moe_mxfp8_quantize": (I, [P, I, I, P, P, P]),
     "lm_head_workspace_bytes": (Z, [I, I, I]),
     "lm_head_fp8_gemv": (I, [P, I, I, I, P, P, P, P, P, Z, P]),
+    "lm_head_fp8_verify": (I, [P, I, I, I, P, P, P, P, P, P, P, Z, P]),
+    "lm_head_bf16_gemv": (I, [P, I, I, I, P, P, P, P, Z, P]),
+    "moe_sample": (I, [P, I, I, ctypes.c_float, I, ctypes.c_float, P, P, P]),
     "lm_head_fp8_gemv_noalloc": (I, [P, I, I, I, P, P, P, P, P]),
     "decode_step_workspace_bytes": (Z, [ctypes.POINTER(Model), I]),
     "decode_step_launch_names": (I, [ctypes.POINTER(Model), I, ctypes.POINTER(ctypes.c_char_p), I]),

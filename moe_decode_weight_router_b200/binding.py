@@ -202,6 +202,55 @@ def lm_head_fp8_gemv(x, q, s, *, want_logits: bool = True, ws=None, out=None, st
     return logits, am
 
 
+def lm_head_fp8_verify(x, q, s, drafts, *, want_logits: bool = False, ws=None, stream=None):
+    """Verify window: (logits or None, argmax int32 [M], accept int32 [1+M]) -- accept[0]
+    is the accepted count, accept[1:1+count] the accepted tokens."""
+    _dev_bf16(x, "x")
+    M, H = x.shape
+    V = q.shape[0]
+    dev = x.device
+    logits = torch.empty((M, V), dtype=torch.float32, device=dev) if want_logits else None
+    am = torch.empty((M,), dtype=torch.int32, device=dev)
+    acc = torch.empty((1 + M,), dtype=torch.int32, device=dev)
+    d = drafts.to(device=dev, dtype=torch.int32).contiguous()
+    if ws is None:
+        ws = _ws(lm_head_workspace_bytes(M, V, H), dev)
+    _check("lm_head_fp8_verify", _lib().lm_head_fp8_verify(_ptr(x), M, V, H, _ptr(q), _ptr(s), _ptr(d), _ptr(logits),
+                                                            _ptr(am), _ptr(acc), _ptr(ws), ws.numel(), _stream(stream)))
+    return logits, am, acc
+
+
+def lm_head_bf16_gemv(x, w, *, want_logits: bool = True, ws=None, out=None, stream=None):
+    """BF16-weight head: (logits fp32 [M,V] or None, argmax int32 [M])."""
+    _dev_bf16(x, "x")
+    _dev_bf16(w, "w")
+    M, H = x.shape
+    V = w.shape[0]
+    dev = x.device
+    if out is None:
+        logits = torch.empty((M, V), dtype=torch.float32, device=dev) if want_logits else None
+        am = torch.empty((M,), dtype=torch.int32, device=dev)
+    else:
+        logits, am = out
+    if ws is None:
+        ws = _ws(lm_head_workspace_bytes(M, V, H), dev)
+    _check("lm_head_bf16_gemv", _lib().lm_head_bf16_gemv(_ptr(x), M, V, H, _ptr(w), _ptr(logits), _ptr(am), _ptr(ws),
+                                                          ws.numel(), _stream(stream)))
+    return logits, am
+
+
+def moe_sample(logits, u, *, temperature: float, top_k: int, top_p: float, stream=None):
+    """One sampled token id per row of fp32 logits [M,V]; u [M] fp32 uniform draws."""
+    if logits.dtype != torch.float32 or not logits.is_cuda or not logits.is_contiguous():
+        raise TypeError("logits: expected a contiguous CUDA float32 tensor")
+    M, V = logits.shape
+    uu = u.to(device=logits.device, dtype=torch.float32).contiguous()
+    ids = torch.empty((M,), dtype=torch.int32, device=logits.device)
+    _check("moe_sample", _lib().moe_sample(_ptr(logits), M, V, float(temperature), int(top_k), float(top_p), _ptr(uu),
+                                           _ptr(ids), _stream(stream)))
+    return ids
+
+
 def lm_head_fp8_gemv_noalloc(x, q, s, *, want_logits: bool = True, out=None, stream=None):
     """As lm_head_fp8_gemv, through the entry point that takes no workspace (the
     library's static per-device control block; calls must not overlap)."""

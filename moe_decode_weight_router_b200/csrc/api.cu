@@ -16,6 +16,7 @@
 #include "lmhead_kernels.cuh"
 #include "step_kernel.cuh"
 #include "prefill_kernels.cuh"
+#include "sample_kernels.cuh"
 
 using namespace moe;
 
@@ -505,6 +506,73 @@ moe_status_t lm_head_fp8_gemv(const void* x_bf16, int M, int V, int H, const uin
   p.counter = c.lm_counter;
   p.status = c.status;
   return launch_lm(p, d, st);
+}
+
+moe_status_t lm_head_fp8_verify(const void* x_bf16, int M, int V, int H, const uint8_t* w_e4m3,
+                                const float* row_scale, const int32_t* drafts, float* logits, int32_t* argmax,
+                                int32_t* accept, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  REQ(x_bf16 && w_e4m3 && row_scale && argmax && drafts && accept, MOE_ERR_INVALID_ARG);
+  REQ(M >= 2 && ok_M(M) && V >= 1 && V <= (1 << 26) && ok_H_lm(H), MOE_ERR_UNSUPPORTED_SHAPE);
+  moe_status_t s = check_ptrs_aligned({x_bf16, w_e4m3, row_scale, logits, argmax, ws});
+  if (s != MOE_OK) return s;
+  REQ(ws && ws_bytes >= lm_head_workspace_bytes(M, V, H), MOE_ERR_WORKSPACE);
+  DevInfo d;
+  if ((s = dev_info(&d)) != MOE_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  Ctrl c = ctrl_of(ws);
+  MOE_CUDA(cudaMemsetAsync(ws, 0, CTRL_BYTES, st));
+  LMParams p{};
+  p.x = static_cast<const __nv_bfloat16*>(x_bf16);
+  p.M = M;
+  p.V = V;
+  p.H = H;
+  p.w = w_e4m3;
+  p.rs = row_scale;
+  p.logits = logits;
+  p.argmax = argmax;
+  p.keys = c.keys;
+  p.counter = c.lm_counter;
+  p.status = c.status;
+  p.drafts = drafts;
+  p.accept = accept;
+  return launch_lm(p, d, st);
+}
+
+moe_status_t lm_head_bf16_gemv(const void* x_bf16, int M, int V, int H, const void* w_bf16, float* logits,
+                               int32_t* argmax, void* ws, size_t ws_bytes, moe_stream_t stream) {
+  REQ(x_bf16 && w_bf16 && argmax, MOE_ERR_INVALID_ARG);
+  REQ(ok_M(M) && V >= 1 && V <= (1 << 26) && ok_H_lm(H), MOE_ERR_UNSUPPORTED_SHAPE);
+  moe_status_t s = check_ptrs_aligned({x_bf16, w_bf16, logits, argmax, ws});
+  if (s != MOE_OK) return s;
+  REQ(ws && ws_bytes >= lm_head_workspace_bytes(M, V, H), MOE_ERR_WORKSPACE);
+  DevInfo d;
+  if ((s = dev_info(&d)) != MOE_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  Ctrl c = ctrl_of(ws);
+  MOE_CUDA(cudaMemsetAsync(ws, 0, CTRL_BYTES, st));
+  const long long T = (V + 15) / 16;
+  const long long want = (T + LMB_WARPS - 1) / LMB_WARPS;
+  const int grid = (int)(want < 4LL * d.sms ? want : 4LL * d.sms);
+  const size_t smem = (size_t)MAX_M * padded_stride(2u * H);
+  k_lm_gemv_bf16<<<grid, 32 * LMB_WARPS, smem, st>>>(static_cast<const __nv_bfloat16*>(x_bf16), M, V, H,
+                                                     static_cast<const __nv_bfloat16*>(w_bf16), logits, argmax, c.keys,
+                                                     c.lm_counter);
+  MOE_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
+
+moe_status_t moe_sample(const float* logits, int M, int V, float temperature, int top_k, float top_p,
+                        const float* u, int32_t* ids, moe_stream_t stream) {
+  REQ(logits && u && ids, MOE_ERR_INVALID_ARG);
+  REQ(M >= 1 && M <= 65535 && V >= 1 && V <= (1 << 26) && top_k >= 1 && top_k <= SAMPLE_MAX_K && top_k <= V,
+      MOE_ERR_UNSUPPORTED_SHAPE);
+  REQ(temperature > 0.0f && top_p > 0.0f && top_p <= 1.0f, MOE_ERR_INVALID_ARG);
+  moe_status_t s = check_ptrs_aligned({logits, u, ids});
+  if (s != MOE_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  k_sample<<<M, SAMPLE_THREADS, 0, st>>>(logits, V, temperature, top_k, top_p, u, ids);
+  MOE_CUDA(cudaGetLastError());
+  return MOE_OK;
 }
 
 static moe_status_t check_model(const moe_model_t* m) {

@@ -73,7 +73,24 @@ struct LMParams {
   unsigned* counter;         // zero on entry
   int* status;
   int stages;
+  const int32_t* drafts;     // optional [M-1]: draft tokens of a verify window (MTP)
+  int32_t* accept;           // [1 + M] when drafts: accepted count, then the accepted tokens
 };
+
+// Multi-token-prediction verify (the window holds the last accepted token and M - 1
+// drafts; the head's argmax at position t predicts the token after it): draft t + 1
+// is accepted while it equals the argmax at t, and the head's own token at the first
+// mismatch (or after the last draft) is accepted with them.  out[0] = accepted count
+// (1..M), out[1..] = the accepted tokens.
+__device__ __forceinline__ void mtp_accept(const int32_t* argmax, const int32_t* drafts, int M, int32_t* out) {
+  int n = 0;
+  while (n < M - 1 && drafts[n] == argmax[n]) {
+    out[1 + n] = drafts[n];
+    ++n;
+  }
+  out[1 + n] = argmax[n];
+  out[0] = n + 1;
+}
 
 __host__ __device__ inline size_t lm_stage_bytes(int H) {
   size_t b = 16 * (size_t)H;  // 16 contiguous rows: one bulk copy per tile
@@ -222,6 +239,113 @@ __global__ void __launch_bounds__(EXPERT_THREADS, 1) k_lm_gemv(LMParams p) {
       p.argmax[tid] = (int32_t)(0xFFFFFFFFu - (uint32_t)(k & 0xFFFFFFFFull));
     }
     if (tid == 0) *p.counter = 0u;
+    if (p.drafts) {
+      named_barrier(1, 32 * N_CONSUMERS);
+      if (tid == 0) mtp_accept(p.argmax, p.drafts, M, p.accept);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// k_lm_gemv_bf16: the same head with the BF16 weights it is quantised from -- the
+// comparison the FP8 head is measured against (twice the bytes per logit).  Eight
+// warps per block, each owning 16-row tiles; rows stream through 128-bit
+// non-allocating loads (two per row per 64 columns, 16 in flight per thread).
+// ---------------------------------------------------------------------------
+constexpr int LMB_WARPS = 8;
+__global__ void __launch_bounds__(32 * LMB_WARPS) k_lm_gemv_bf16(const __nv_bfloat16* __restrict__ x, int M, int V,
+                                                                int H, const __nv_bfloat16* __restrict__ w,
+                                                                float* __restrict__ logits, int32_t* __restrict__ argmax,
+                                                                unsigned long long* keys, unsigned* counter) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ unsigned long long s_best[LMB_WARPS][MAX_M];
+  __shared__ int s_last;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+  const uint32_t xss = padded_stride(2u * H);
+  // activation rows as bf16 (the MMA's B operand), zero rows beyond M
+  for (int i = tid; i < MAX_M * (H / 8); i += blockDim.x) {
+    const int tok = i / (H / 8), c = i % (H / 8);
+    const uint4 v = tok < M ? *reinterpret_cast<const uint4*>(x + (size_t)tok * H + 8 * c) : make_uint4(0, 0, 0, 0);
+    *reinterpret_cast<uint4*>(smem + tok * xss + 16 * c) = v;
+  }
+  __syncthreads();
+  const long long T = (V + 15) / 16;
+  const long long gw = (long long)blockIdx.x * LMB_WARPS + warp, nw = (long long)gridDim.x * LMB_WARPS;
+  unsigned long long bestA = 0ull, bestB = 0ull;
+  const int ta = 2 * t, tb = 2 * t + 1;
+  for (long long tile = gw; tile < T; tile += nw) {
+    const long long v0 = tile * 16;
+    const long long ra = min(v0 + g, (long long)V - 1), rb = min(v0 + g + 8, (long long)V - 1);
+    const uint4* wa = reinterpret_cast<const uint4*>(w + ra * H);
+    const uint4* wb = reinterpret_cast<const uint4*>(w + rb * H);
+    float c4[4][4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) c4[u][0] = c4[u][1] = c4[u][2] = c4[u][3] = 0.0f;
+#pragma unroll 4
+    for (int j = 0; j < H / 64; ++j) {
+      // this thread's 16 columns of the chunk: 64j + 16t .. +15 (two 16-byte pieces per row)
+      const uint4 A0 = ldg128_stream(wa + 8 * j + 2 * t), A0b = ldg128_stream(wa + 8 * j + 2 * t + 1);
+      const uint4 A1 = ldg128_stream(wb + 8 * j + 2 * t), A1b = ldg128_stream(wb + 8 * j + 2 * t + 1);
+      const uint4 X0 = lds128(smem + g * xss + 2 * (64 * j + 16 * t));
+      const uint4 X1 = lds128(smem + g * xss + 2 * (64 * j + 16 * t) + 16);
+      const uint32_t P[8] = {A0.x, A0.y, A0.z, A0.w, A0b.x, A0b.y, A0b.z, A0b.w};
+      const uint32_t Q[8] = {A1.x, A1.y, A1.z, A1.w, A1b.x, A1b.y, A1b.z, A1b.w};
+      const uint32_t X[8] = {X0.x, X0.y, X0.z, X0.w, X1.x, X1.y, X1.z, X1.w};
+#pragma unroll
+      for (int s4 = 0; s4 < 4; ++s4)
+        mma_bf16(c4[s4], P[2 * s4], Q[2 * s4], P[2 * s4 + 1], Q[2 * s4 + 1], X[2 * s4], X[2 * s4 + 1]);
+    }
+    float c[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) c[e] = (c4[0][e] + c4[1][e]) + (c4[2][e] + c4[3][e]);
+    const long long va = v0 + g, vb = v0 + g + 8;
+    if (ta < M) {
+      if (va < V) {
+        if (logits) logits[(size_t)ta * V + va] = c[0];
+        bestA = max(bestA, argmax_key(c[0], (int)va));
+      }
+      if (vb < V) {
+        if (logits) logits[(size_t)ta * V + vb] = c[2];
+        bestA = max(bestA, argmax_key(c[2], (int)vb));
+      }
+    }
+    if (tb < M) {
+      if (va < V) {
+        if (logits) logits[(size_t)tb * V + va] = c[1];
+        bestB = max(bestB, argmax_key(c[1], (int)va));
+      }
+      if (vb < V) {
+        if (logits) logits[(size_t)tb * V + vb] = c[3];
+        bestB = max(bestB, argmax_key(c[3], (int)vb));
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    bestA = max(bestA, __shfl_xor_sync(0xffffffffu, bestA, o));
+    bestB = max(bestB, __shfl_xor_sync(0xffffffffu, bestB, o));
+  }
+  if (g == 0) {
+    s_best[warp][ta] = bestA;
+    s_best[warp][tb] = bestB;
+  }
+  __syncthreads();
+  if (warp == 0 && lane < M) {
+    unsigned long long b = 0ull;
+    for (int w2 = 0; w2 < LMB_WARPS; ++w2) b = max(b, s_best[w2][lane]);
+    if (b) atomicMax(keys + lane, b);
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = (atomicAdd(counter, 1u) == gridDim.x - 1);
+  __syncthreads();
+  if (s_last) {
+    __threadfence();
+    if (tid < M) {
+      const unsigned long long k = atomicExch(keys + tid, 0ull);
+      argmax[tid] = (int32_t)(0xFFFFFFFFu - (uint32_t)(k & 0xFFFFFFFFull));
+    }
+    if (tid == 0) *counter = 0u;
   }
 }
 

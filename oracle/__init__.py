@@ -319,3 +319,89 @@ def decode_step(x0: np.ndarray, layers, lm_q, lm_s, k: int, eps: float = 1e-6, t
     logits, am, gap = lmhead_logits(x, lm_q, lm_s)
     out.update(logits=logits, argmax=am, gap=gap, h=h)
     return out
+
+
+# ---------------------------------------------------------------------------
+# Beyond the step: the verify window, the BF16 head, sampling
+# ---------------------------------------------------------------------------
+def mtp_accept(argmax, drafts):
+    """Multi-token-prediction verify (DGX Spark MoE knowledge card, 方法/产品要点 item 2:
+    a window of the last accepted token plus draft tokens is verified in one step).
+    The head's argmax at window position t is its prediction of the token after t;
+    draft t+1 is accepted while it equals that prediction, and the head's own token
+    at the first mismatch (or after the last draft) is accepted with them.
+    Returns [count, token_1, ..., token_count]."""
+    argmax = [int(a) for a in argmax]
+    drafts = [int(d) for d in drafts]
+    assert len(drafts) == len(argmax) - 1
+    out = []
+    n = 0
+    while n < len(drafts) and drafts[n] == argmax[n]:
+        out.append(drafts[n])
+        n += 1
+    out.append(argmax[n])
+    return [n + 1] + out
+
+
+def lmhead_logits_bf16(x: np.ndarray, w: np.ndarray):
+    """The BF16 head the FP8 head is quantised from (same knowledge card, item 2):
+    logits fp64 [M,V] = W x with bf16 -> fp64 exact operands (a library matmul of the
+    exact values), argmax with ties to the lower index, and the top-2 gap [M]."""
+    x = _c(x, np.uint16)
+    w = _c(w, np.uint16)
+    xf = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    wf = (w.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    logits = xf @ wf.T
+    am = np.argmax(logits, axis=1).astype(np.int32)  # first occurrence = lowest index
+    srt = np.sort(logits, axis=1)
+    gap = srt[:, -1] - srt[:, -2] if logits.shape[1] > 1 else np.full(logits.shape[0], np.inf)
+    return logits, am, gap
+
+
+def sample(logits: np.ndarray, temperature: float, top_k: int, top_p: float, u: np.ndarray):
+    """Temperature / top-k / top-p sampling of one token per row, the random draw
+    u [M] in [0, 1) given (the knowledge card's serving settings: temperature,
+    top-k 29, top-p 0.95).  Reading, step by step in fp64:
+      z = logits / T; S = the top_k largest z (ties to the lower index);
+      p_i = softmax of z over S; order S by (p desc, index asc);
+      nucleus N = the shortest prefix of that order with sum p >= top_p;
+      q = p renormalised over N; the sample is the first i of N (in order) whose
+      cumulative q exceeds u (the last of N if rounding leaves none).
+    Returns (ids int32 [M], margin fp64 [M]): margin = distance of u, and of top_p,
+    to the nearest cumulative boundary -- below ~1e-6 the decision depends on
+    rounding and a comparison is flagged rather than failed."""
+    logits = np.asarray(logits, np.float64)
+    M, V = logits.shape
+    ids = np.zeros(M, np.int32)
+    margin = np.zeros(M, np.float64)
+    for t in range(M):
+        z = logits[t] / float(temperature)
+        order = sorted(range(V), key=lambda i: (-z[i], i))[:top_k]
+        zm = z[order[0]]
+        e = [np.exp(z[i] - zm) for i in order]
+        den = sum(e)
+        p = [v / den for v in e]
+        # (p desc, index asc) is the z order already: p is monotone in z
+        cum, n = 0.0, 0
+        bounds_p = []
+        while True:
+            cum += p[n]
+            bounds_p.append(cum)
+            n += 1
+            if cum >= top_p or n == len(p):
+                break
+        mass = cum
+        q = [v / mass for v in p[:n]]
+        c, pick = 0.0, n - 1
+        bounds_q = []
+        for j in range(n):
+            c += q[j]
+            bounds_q.append(c)
+            if c > u[t]:
+                pick = j
+                break
+        ids[t] = order[pick]
+        m = min(abs(b - u[t]) for b in bounds_q)
+        m = min(m, min(abs(b - top_p) for b in bounds_p))
+        margin[t] = m
+    return ids, margin
