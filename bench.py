@@ -39,6 +39,25 @@ NOMINAL_HBM_GBS = 8000.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 
 
+# DRAM traffic of k_step per layer (read + write) from the ncu capture summarised in
+# profiles/k_step_ling_2layers_m1.md, valid while the kernel sources hash to the value
+# recorded with it (otherwise the roofline's traffic is reported as null).
+KSTEP_TRAFFIC = {"bytes_per_layer": (79.15e6 + 1.95e6) / 2, "sources_sha256_16": "f36f803cdc03fd53",
+                 "sources": ("step_kernel.cuh", "decode_kernels.cuh", "common.cuh")}
+
+
+def kstep_traffic(layers: int):
+    import hashlib
+    d = os.path.join(os.path.dirname(os.path.abspath(__file__)), "moe_decode_weight_router_b200", "csrc")
+    h = hashlib.sha256()
+    for f in KSTEP_TRAFFIC["sources"]:
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(fh.read())
+    if h.hexdigest()[:16] != KSTEP_TRAFFIC["sources_sha256_16"]:
+        return None
+    return KSTEP_TRAFFIC["bytes_per_layer"] * layers
+
+
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -53,6 +72,7 @@ def parse_args():
     ap.add_argument("--skip-m4", action="store_true")
     ap.add_argument("--per-layer", action="store_true", help="force the three-kernels-per-layer path")
     ap.add_argument("--skip-prefill", action="store_true", help="skip the prefill-chunk measurement")
+    ap.add_argument("--skip-head", action="store_true", help="skip the LM-head comparison and verify window")
     ap.add_argument("--prefill-m", type=int, default=2048, help="tokens of the prefill chunk")
     return ap.parse_args()
 
@@ -318,6 +338,45 @@ def run_ours(args, rank, world, local_rank):
             res["kernels"] = ker
         results[M] = res
 
+    # LM head: the FP8 head against the BF16 weights it is quantised from (M=1), and the
+    # multi-token-prediction verify window (M=4) on synthetic drafts
+    if not args.skip_head:
+        from moe_decode_weight_router_b200 import lm_head_bf16_gemv, lm_head_fp8_gemv, lm_head_fp8_verify
+        w_bf = synth.lm_head(V, S.H, seed, device=dev)
+        xh1 = [synth.tokens(1, S.H, seed, tid=300 + i, device=dev) for i in range(K + W)]
+        head_us = {}
+        for name, fn in (("fp8", lambda x: lm_head_fp8_gemv(x, lm_q, lm_s, want_logits=False)),
+                         ("bf16", lambda x: lm_head_bf16_gemv(x, w_bf, want_logits=False))):
+            for i in range(W):
+                fn(xh1[i])
+            torch.cuda.synchronize()
+            e0.record()
+            for i in range(K):
+                fn(xh1[W + i])
+            e1.record()
+            torch.cuda.synchronize()
+            head_us[name] = 1000 * max_over_ranks(e0.elapsed_time(e1)) / K
+        del w_bf
+        torch.cuda.empty_cache()
+        g = torch.Generator(device="cpu")
+        g.manual_seed(seed + 11)
+        accepted = []
+        for i in range(K + W):
+            x4 = synth.tokens(4, S.H, seed, tid=500 + i, device=dev)
+            _, am4 = lm_head_fp8_gemv(x4, lm_q, lm_s, want_logits=False)
+            am4 = am4.cpu()
+            drafts = am4[:3].clone()
+            keep = torch.rand(3, generator=g) < 0.7
+            drafts[~keep] = torch.randint(0, V, (int((~keep).sum()),), generator=g, dtype=torch.int32)
+            _, _, acc = lm_head_fp8_verify(x4, lm_q, lm_s, drafts)
+            accepted.append(int(acc[0].item()))
+        results["head"] = {"fp8_us": head_us["fp8"], "bf16_us": head_us["bf16"],
+                           "bf16_over_fp8": head_us["bf16"] / head_us["fp8"],
+                           "fp8_gbps": (V * S.H + 4 * V) / (head_us["fp8"] * 1e-6) / 1e9,
+                           "bf16_gbps": (2 * V * S.H) / (head_us["bf16"] * 1e-6) / 1e9,
+                           "mtp_mean_accept": float(np.mean(accepted)),
+                           "mtp_drafts": "each of 3 drafts copies the head's token with probability 0.7, else random"}
+
     # prefill chunk: one MoE layer for M tokens on the block-scaled tensor cores, each
     # timed call on the next of the L distinct layers (1.6 GB of experts each, > L2)
     if not args.skip_prefill:
@@ -508,8 +567,10 @@ def main():
         roof = None
         if dom:
             ach = ker[dom]["gbps"]
+            traffic = kstep_traffic(args.layers) if dom == "k_step" else None
             roof = {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
-                    "traffic": None, "peak_source": f"{src} hbm_gbs (copy, burst)"}
+                    "traffic": traffic, "traffic_unit": "bytes per launch (ncu dram read + write)",
+                    "peak_source": f"{src} hbm_gbs (copy, burst)"}
         line = {
             "metric": METRIC, "value": r1["gbps"], "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": r1["ms_per_step"], "us_per_step": r1["us_per_step"],
@@ -534,6 +595,8 @@ def main():
                           "frac_of_8tbs": r4["gbps"] / world / NOMINAL_HBM_GBS,
                           "frac_of_measured_hbm": r4["gbps"] / world / hbm,
                           "mean_unique_experts": r4["mean_unique_experts"], "e2e": r4["e2e"], "clocks": r4["clocks"]}
+        if "head" in results:
+            line["lm_head"] = results["head"]
         if "prefill" in results:
             rp = results["prefill"]
             line["prefill"] = dict(rp, frac_of_measured_hbm=rp["gbps"] / world / hbm,
