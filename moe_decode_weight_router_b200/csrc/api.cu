@@ -256,19 +256,6 @@ bool use_persistent(const moe_model_t& m, int M, const DevInfo& d, uint32_t* rin
   return ring >= (size_t)N_CONSUMERS * step_max_item_bytes(m.H, m.I, m.Is);
 }
 
-// Bound on the bytes a block keeps in flight in the persistent step (MOE_STEP_INFLIGHT_KB
-// overrides; 0 = the whole ring).  Enough to keep HBM streaming, small enough that the
-// loads and polls of the dependency chain do not wait behind a queue of weight copies.
-uint32_t step_inflight_bytes() {
-  static const uint32_t v = [] {
-    const char* e = getenv("MOE_STEP_INFLIGHT_KB");
-    long kb = e ? strtol(e, nullptr, 10) : 0;
-    if (kb < 0) kb = 0;
-    return (uint32_t)kb * 1024u;
-  }();
-  return v;
-}
-
 moe_status_t launch_step(const StepParams& sp, const DevInfo& d, cudaStream_t st) {
   const size_t smem = STEP_FIXED + (size_t)sp.ring_bytes + sp.act_bytes;
   cudaLaunchConfig_t cfg{};
@@ -666,7 +653,6 @@ moe_status_t decode_step(const moe_model_t* model, const void* x_bf16, int M, fl
     sp.x_final = w.x_final;
     sp.logits = w.tlogits;
     sp.a_shared = w.tshared;
-    sp.inflight_bytes = step_inflight_bytes();
     sp.a_routed = w.a_routed;
     sp.ctr = w.ctr;
     sp.status = c.status;

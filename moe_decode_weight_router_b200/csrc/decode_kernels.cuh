@@ -429,9 +429,86 @@ __device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
 //   xb: f16 activation rows (stride xss bytes), token n at xb + n*xss
 // Latency: the next group's codes and scales are loaded while this group computes;
 // each group issues its 32 conversions back to back, then 8 MMAs into 4 accumulators.
+// Rows with a multiple of 8 scale blocks (every Ling-shaped tile): two groups per
+// iteration into eight accumulators, the scale maxima from 32-bit words.
+__device__ __forceinline__ void mxfp4_tile_dot_x2(const uint8_t* codes_g, const uint8_t* codes_g8,
+                                                  const uint8_t* sc_g, const uint8_t* sc_g8, int nb,
+                                                  const uint8_t* xb, uint32_t xss, int M, float (&c)[4]) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+  uint32_t ref_g, ref_g8;
+  {
+    uint32_t a = 0u, b = 0u;
+    const uint32_t* ga = reinterpret_cast<const uint32_t*>(sc_g);
+    const uint32_t* gb = reinterpret_cast<const uint32_t*>(sc_g8);
+    for (int i = t; i < nb / 4; i += 4) {
+      a = __vmaxu4(a, ga[i]);
+      b = __vmaxu4(b, gb[i]);
+    }
+    a = __vmaxu4(a, __shfl_xor_sync(0xffffffffu, a, 1));
+    b = __vmaxu4(b, __shfl_xor_sync(0xffffffffu, b, 1));
+    a = __vmaxu4(a, __shfl_xor_sync(0xffffffffu, a, 2));
+    b = __vmaxu4(b, __shfl_xor_sync(0xffffffffu, b, 2));
+    ref_g = max(max(a & 0xFFu, (a >> 8) & 0xFFu), max((a >> 16) & 0xFFu, a >> 24));
+    ref_g8 = max(max(b & 0xFFu, (b >> 8) & 0xFFu), max((b >> 16) & 0xFFu, b >> 24));
+  }
+  const bool xact = g < M;
+  const uint8_t* xrow = xb + g * xss;
+  float acc[8][4];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) acc[u][0] = acc[u][1] = acc[u][2] = acc[u][3] = 0.0f;
+  for (int q = 0; q < nb / 4; q += 2) {
+    uint4 A0[2], A1[2], X[2][4];
+    uint32_t e0[2], e1[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int beta = 4 * (q + h) + t;
+      A0[h] = lds128(codes_g + 16 * beta);
+      A1[h] = lds128(codes_g8 + 16 * beta);
+      e0[h] = sc_g[beta];
+      e1[h] = sc_g8[beta];
+#pragma unroll
+      for (int wd = 0; wd < 4; ++wd) X[h][wd] = xact ? lds128(xrow + 64 * beta + 16 * wd) : zero;
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t f0 = pow2_f16x2((int)e0[h] - (int)ref_g), f1 = pow2_f16x2((int)e1[h] - (int)ref_g8);
+      uint32_t hh[16], kk[16];
+      const uint32_t a0w[4] = {A0[h].x, A0[h].y, A0[h].z, A0[h].w};
+      const uint32_t a1w[4] = {A1[h].x, A1[h].y, A1[h].z, A1[h].w};
+#pragma unroll
+      for (int wd = 0; wd < 4; ++wd) {
+        e2m1x8_to_f16x2(a0w[wd], hh[4 * wd], hh[4 * wd + 1], hh[4 * wd + 2], hh[4 * wd + 3]);
+        e2m1x8_to_f16x2(a1w[wd], kk[4 * wd], kk[4 * wd + 1], kk[4 * wd + 2], kk[4 * wd + 3]);
+      }
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        hh[j] = hmul2_u32(hh[j], f0);
+        kk[j] = hmul2_u32(kk[j], f1);
+      }
+#pragma unroll
+      for (int wd = 0; wd < 4; ++wd) {
+        mma_f16(acc[4 * h + wd], hh[4 * wd], kk[4 * wd], hh[4 * wd + 1], kk[4 * wd + 1], X[h][wd].x, X[h][wd].y);
+        mma_f16(acc[4 * h + wd], hh[4 * wd + 2], kk[4 * wd + 2], hh[4 * wd + 3], kk[4 * wd + 3], X[h][wd].z,
+                X[h][wd].w);
+      }
+    }
+  }
+  const float r0 = e8m0_to_f32(ref_g), r1 = e8m0_to_f32(ref_g8);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float sum = ((acc[0][e] + acc[1][e]) + (acc[2][e] + acc[3][e])) + ((acc[4][e] + acc[5][e]) + (acc[6][e] + acc[7][e]));
+    c[e] = sum * (e < 2 ? r0 : r1);
+  }
+}
+
 __device__ __forceinline__ void mxfp4_tile_dot(const uint8_t* codes_g, const uint8_t* codes_g8,
                                                const uint8_t* sc_g, const uint8_t* sc_g8, int nb,
                                                const uint8_t* xb, uint32_t xss, int M, float (&c)[4]) {
+  if ((nb & 7) == 0 && ((reinterpret_cast<uintptr_t>(sc_g) | reinterpret_cast<uintptr_t>(sc_g8)) & 3u) == 0) {
+    mxfp4_tile_dot_x2(codes_g, codes_g8, sc_g, sc_g8, nb, xb, xss, M, c);
+    return;
+  }
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const int nq = (nb + 3) / 4;
   const uint4 zero = make_uint4(0u, 0u, 0u, 0u);

@@ -65,7 +65,6 @@ struct StepParams {
   float eps;
   uint32_t ring_bytes;
   uint32_t act_bytes;
-  uint32_t inflight_bytes;    // producer cap on copied-but-not-landed bytes (0: the ring)
   const __nv_bfloat16* x_in;  // [M][H]
   float* h;                   // [2][M][H] residual stream, buffer l & 1 is layer l's output
   __nv_bfloat16* x_final;     // [M][H] LM-head input
@@ -92,12 +91,13 @@ __device__ __forceinline__ void stamp(const StepParams& p, int l, int slot) {
   if (tid != 0 && tid != 32 * STEP_CONSUMERS) return;
   p.timeline[((size_t)(last ? 1 : 0) * p.L + l) * 16 + slot] = globaltimer_ns();
 }
-// Profiling: block 0's first STEP_ITEM_LOG ring items -- (issued, data ready, done,
-// consumer started waiting) stamps after the [2][L][16] phase stamps.
-constexpr int STEP_ITEM_LOG = 4096;
+// Profiling: block 0's first STEP_ITEM_LOG ring items, 8 stamps each after the
+// [2][L][16] phase stamps: 0 copies issued, 1 data seen by the consumer, 2 consumer
+// done, 3 consumer started waiting, 4 producer entered issue().
+constexpr int STEP_ITEM_LOG = 2048;
 __device__ __forceinline__ void item_stamp(const StepParams& p, long long i, int which) {
   if (!p.timeline || blockIdx.x != 0 || i >= STEP_ITEM_LOG || (threadIdx.x & 31) != 0) return;
-  p.timeline[(size_t)2 * p.L * 16 + (size_t)i * 4 + which] = globaltimer_ns();
+  p.timeline[(size_t)2 * p.L * 16 + (size_t)i * 8 + which] = globaltimer_ns();
 }
 
 // ---------------------------------------------------------------------------
@@ -143,13 +143,20 @@ __host__ __device__ inline uint32_t step_act_bytes(int M, int H, int I, int Is) 
   if (c > a) a = c;
   return (a + 127) / 128 * 128;
 }
-// Deterministic placement in the byte ring (producer and every consumer warp walk
-// the same item sequence and compute the same offsets): an item that would cross
-// the end starts over at 0.
-__device__ __forceinline__ uint32_t ring_take(uint32_t& pos, uint32_t n, uint32_t R) {
-  const uint32_t s = pos + n <= R ? pos : 0u;
-  pos = s + n;
-  return s;
+// Deterministic placement in the byte ring on monotonic virtual byte positions (the
+// producer and every consumer warp walk the same item sequence and compute the same
+// offsets): an item that would cross the end of the ring starts at the next multiple
+// of R.  Returns the ring offset; *vstart receives the item's virtual start.
+__device__ __forceinline__ uint32_t ring_take(unsigned long long& vpos, uint32_t n, uint32_t R,
+                                              unsigned long long* vstart = nullptr) {
+  uint32_t off = (uint32_t)(vpos % R);
+  if (off + n > R) {
+    vpos += R - off;
+    off = 0u;
+  }
+  if (vstart) *vstart = vpos;
+  vpos += n;
+  return off;
 }
 
 // ---------------------------------------------------------------------------
@@ -312,6 +319,29 @@ struct Work {
   }
 };
 
+// Consecutive routed tiles of one expert travel as one ring item (their rows are
+// contiguous in HBM: one copy per run instead of one per tile).  Walks tiles
+// x .. end-1 of the block's range (T tiles per expert), at most cap per group.
+struct GroupWalk {
+  long long x, end;
+  int T, cap;
+  __device__ bool next(int& u, int& r0, int& nt) {
+    if (x >= end) return false;
+    u = (int)(x / T);
+    r0 = (int)(x - (long long)u * T);
+    const long long lim = min(end, (long long)(u + 1) * T);
+    nt = (int)min((long long)cap, lim - x);
+    x += nt;
+    return true;
+  }
+};
+// Tiles per group: a third of the ring at most, so two groups and the smaller items
+// around them are in flight together.
+__host__ __device__ inline int step_group_cap(uint32_t R, uint32_t tile_bytes, int maxcap) {
+  const int c = (int)(R / (3u * tile_bytes));
+  return c < 1 ? 1 : (c > maxcap ? maxcap : c);
+}
+
 // ---------------------------------------------------------------------------
 // producer side
 // ---------------------------------------------------------------------------
@@ -321,34 +351,29 @@ struct Producer {
   uint32_t R;
   uint64_t* full;
   uint64_t* empty;
-  uint32_t* fs;  // [STEP_SLOTS] ring start / end of the items in flight (lane 0)
-  uint32_t* fe;
+  unsigned long long* vst;  // [STEP_SLOTS] virtual start of the items in flight (lane 0)
   uint64_t pol;
-  long long i;        // next ring item
-  long long oldest;   // oldest item whose release lane 0 has not seen yet
-  long long land;     // oldest item lane 0 has not seen land yet
-  uint32_t pos;       // ring placement cursor
-  uint32_t inflight;  // bytes copied but not seen landed (lane 0)
-  uint32_t cap;       // bound on inflight: enough to keep HBM busy, no more, so that
-                      // the latency-bound loads of the dependency chain do not queue
+  long long i;               // next ring item
+  long long oldest;          // oldest item whose release lane 0 has not seen yet
+  unsigned long long vpos;   // virtual placement cursor
   volatile int* abort_flag;
   int lane;
 
-  // Run by all 32 lanes of the producer warp: lane 0 frees the item's bytes (waits
-  // for the release of the oldest items until neither their bytes nor their
-  // barrier slot are needed), waits until the bytes in flight leave room under the
-  // cap, and arms the barrier, then one lane per contiguous run issues its bulk
-  // copy.  Items in flight occupy one arc of the ring in allocation order, so the
-  // items the new one overlaps are always the oldest.
-  __device__ bool issue(const LayerPtrs& Lp, const Plan& P, const Item& it) {
-    const uint32_t n = step_item_bytes(it.type, p.H, p.I, p.Is);
-    const uint32_t s0 = ring_take(pos, n, R);
-    const int slot = (int)(i % STEP_SLOTS);
+  // Run by all 32 lanes of the producer warp: lane 0 waits, in FIFO order, for the
+  // release of the oldest items until the new item and every item still in flight
+  // fit in one ring-length window of virtual bytes (then no two overlap in the ring)
+  // and the new item's barrier slot is free, and arms the barrier; then one lane per
+  // contiguous run issues its bulk copy.
+  __device__ bool acquire(uint32_t n, uint32_t& s0, int& slot) {
+    item_stamp(p, i, 4);
+    unsigned long long vs;
+    s0 = ring_take(vpos, n, R, &vs);
+    slot = (int)(i % STEP_SLOTS);
     int ok = 1;
     if (lane == 0) {
       while (oldest < i) {
         const int os = (int)(oldest % STEP_SLOTS);
-        const bool need = (i - oldest >= STEP_SLOTS) || (fs[os] < s0 + n && s0 < fe[os]);
+        const bool need = (i - oldest >= STEP_SLOTS) || (vs + n - vst[os] > R);
         if (!need) break;
         if (!ring_wait(&empty[os], (uint32_t)((oldest / STEP_SLOTS) & 1), p.status, abort_flag)) {
           ok = 0;
@@ -356,28 +381,60 @@ struct Producer {
         }
         ++oldest;
       }
-      // released items have landed (their slots still hold their extents: slot i % 32
-      // is the only one rewritten below, and it belonged to item i - 32 < oldest)
-      for (; land < oldest; ++land) inflight -= fe[land % STEP_SLOTS] - fs[land % STEP_SLOTS];
-      while (ok && land < i && inflight + n > cap) {
-        const int ls = (int)(land % STEP_SLOTS);
-        if (!ring_wait(&full[ls], (uint32_t)((land / STEP_SLOTS) & 1), p.status, abort_flag)) {
-          ok = 0;
-          break;
-        }
-        inflight -= fe[ls] - fs[ls];
-        ++land;
-      }
-      fs[slot] = s0;
-      fe[slot] = s0 + n;
-      inflight += n;
+      vst[slot] = vs;
     }
     ok = __shfl_sync(0xffffffffu, ok, 0);
-    if (!ok) return false;
+    if (ok) item_stamp(p, i, 0);
+    return ok != 0;
+  }
+
+  // routed W13 group: tiles r0 .. r0+nt-1 (8 gate + 8 up rows each) of expert slot u;
+  // layout [gate codes][up codes][gate scales][up scales], nt*8 rows each
+  __device__ bool issue_b(const LayerPtrs& Lp, const Plan& P, int u, int r0, int nt) {
+    const int H = p.H, I = p.I;
+    const uint32_t codes = (uint32_t)nt * 8u * (H / 2), scales = (uint32_t)nt * 8u * (H / 32);
+    uint32_t s0;
+    int slot;
+    if (!acquire(2 * codes + 2 * scales, s0, slot)) return false;
     uint8_t* st = ring + s0;
     uint64_t* fb = &full[slot];
-    const int H = p.H, I = p.I, Is = p.Is;
-    item_stamp(p, i, 0);
+    const size_t row = (size_t)P.ids[u] * 2 * I + 8 * (size_t)r0;
+    if (lane == 0) mbar_arrive_expect_tx(fb, 2 * codes + 2 * scales);
+    __syncwarp();
+    if (lane == 0) bulk_g2s(st, Lp.w13c + row * (H / 2), codes, fb, pol);
+    if (lane == 1) bulk_g2s(st + codes, Lp.w13c + (row + I) * (H / 2), codes, fb, pol);
+    if (lane == 2) bulk_g2s(st + 2 * codes, Lp.w13s + row * (H / 32), scales, fb, pol);
+    if (lane == 3) bulk_g2s(st + 2 * codes + scales, Lp.w13s + (row + I) * (H / 32), scales, fb, pol);
+    ++i;
+    return true;
+  }
+  // routed W2 group: tiles c0 .. c0+nt-1 (16 output rows each) of expert slot u;
+  // layout [codes][scales], nt*16 rows each
+  __device__ bool issue_c(const LayerPtrs& Lp, const Plan& P, int u, int c0, int nt) {
+    const int H = p.H, I = p.I;
+    const uint32_t codes = (uint32_t)nt * 16u * (I / 2), scales = (uint32_t)nt * 16u * (I / 32);
+    uint32_t s0;
+    int slot;
+    if (!acquire(codes + scales, s0, slot)) return false;
+    uint8_t* st = ring + s0;
+    uint64_t* fb = &full[slot];
+    const size_t row = (size_t)P.ids[u] * H + 16 * (size_t)c0;
+    if (lane == 0) mbar_arrive_expect_tx(fb, codes + scales);
+    __syncwarp();
+    if (lane == 0) bulk_g2s(st, Lp.w2c + row * (I / 2), codes, fb, pol);
+    if (lane == 1) bulk_g2s(st + codes, Lp.w2s + row * (I / 32), scales, fb, pol);
+    ++i;
+    return true;
+  }
+
+  // router / shared items (one tile each)
+  __device__ bool issue(const LayerPtrs& Lp, const Plan& P, const Item& it) {
+    uint32_t s0;
+    int slot;
+    if (!acquire(step_item_bytes(it.type, p.H, p.I, p.Is), s0, slot)) return false;
+    uint8_t* st = ring + s0;
+    uint64_t* fb = &full[slot];
+    const int H = p.H, Is = p.Is;
     if (it.type == IT_A) {
       const int nr = p.E / 4;
       if (lane == 0) mbar_arrive_expect_tx(fb, 4u * 2u * H);
@@ -389,26 +446,10 @@ struct Producer {
         if (lane == 0) bulk_g2s(st, Lp.sw13 + (size_t)2 * sh * H, 2u * 2u * H, fb, pol);
         if (lane == 1) bulk_g2s(st + 4 * H, Lp.sw13 + (size_t)(Is + 2 * sh) * H, 2u * 2u * H, fb, pol);
       }
-    } else if (it.type == IT_CS) {
+    } else {
       if (lane == 0) mbar_arrive_expect_tx(fb, 4u * 2u * Is);
       __syncwarp();
       if (lane == 0) bulk_g2s(st, Lp.sw2 + (size_t)it.a * Is, 4u * 2u * Is, fb, pol);
-    } else if (it.type == IT_B) {
-      const size_t e2I = (size_t)P.ids[it.a] * 2 * I;
-      const uint32_t runb = 8u * (H / 2), scb = 8u * (H / 32);
-      if (lane == 0) mbar_arrive_expect_tx(fb, 2 * runb + 2 * scb);
-      __syncwarp();
-      if (lane == 0) bulk_g2s(st, Lp.w13c + (e2I + it.b) * (H / 2), runb, fb, pol);
-      if (lane == 1) bulk_g2s(st + runb, Lp.w13c + (e2I + I + it.b) * (H / 2), runb, fb, pol);
-      if (lane == 2) bulk_g2s(st + 2 * runb, Lp.w13s + (e2I + it.b) * (H / 32), scb, fb, pol);
-      if (lane == 3) bulk_g2s(st + 2 * runb + scb, Lp.w13s + (e2I + I + it.b) * (H / 32), scb, fb, pol);
-    } else {
-      const size_t eH = (size_t)P.ids[it.a] * H;
-      const uint32_t runb = 16u * (I / 2), scb = 16u * (I / 32);
-      if (lane == 0) mbar_arrive_expect_tx(fb, runb + scb);
-      __syncwarp();
-      if (lane == 0) bulk_g2s(st, Lp.w2c + (eH + it.b) * (I / 2), runb, fb, pol);
-      if (lane == 1) bulk_g2s(st + runb, Lp.w2s + (eH + it.b) * (I / 32), scb, fb, pol);
     }
     ++i;
     return true;
@@ -717,7 +758,8 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
   __shared__ int s_sh[MAX_M];
   __shared__ uint32_t s_ck[MAX_M * STEP_CONSUMERS * 8];
   __shared__ int32_t s_ci[MAX_M * STEP_CONSUMERS * 8];
-  __shared__ uint32_t s_fs[STEP_SLOTS], s_fe[STEP_SLOTS];
+  __shared__ unsigned long long s_vst[STEP_SLOTS];
+  __shared__ int s_gdone[STEP_SLOTS];  // tiles of a grouped ring item finished so far
   __shared__ volatile int s_abort;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -741,6 +783,7 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
   uint8_t* afc = act;                     // CR phase: routed a of the block's experts [CR_CACHE][M][ass]
   const uint32_t bytesA = step_item_bytes(IT_A, H, I, Is), bytesS = step_item_bytes(IT_CS, H, I, Is);
   const uint32_t bytesB = step_item_bytes(IT_B, H, I, Is), bytesC = step_item_bytes(IT_CR, H, I, Is);
+  const int capB = step_group_cap(R, bytesB, 8), capC = step_group_cap(R, bytesC, 16);
 
   if (tid == 0) {
     for (int s = 0; s < STEP_SLOTS; ++s) {
@@ -749,6 +792,7 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
     }
     mbar_init(plan_bar, 1);
     mbar_init(hinit_bar, 1);
+    for (int s = 0; s < STEP_SLOTS; ++s) s_gdone[s] = 0;
     fence_mbar_init();
     s_abort = 0;
   }
@@ -756,8 +800,7 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
 
   // ---------------- producer ----------------
   if (warp == STEP_CONSUMERS) {
-    Producer pr{p,  ring, R,  full, empty, s_fs, s_fe, policy_evict_first(), 0, 0, 0, 0u, 0u,
-                p.inflight_bytes ? p.inflight_bytes : R, &s_abort, lane};
+    Producer pr{p, ring, R, full, empty, s_vst, policy_evict_first(), 0, 0, 0ull, &s_abort, lane};
     bool ok = true;
     for (int l = 0; l < L && ok; ++l) {
       const LayerPtrs& Lp = p.layer[l];
@@ -778,8 +821,13 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
       if (!__shfl_sync(0xffffffffu, got, 0)) break;
       stamp(p, l, 13);
       W.init_routed(p, P.n_unique);
-      const long long nR = W.nB + W.nC;
-      for (long long r = 0; r < nR && ok; ++r) ok = pr.issue(Lp, P, W.at(p, W.nA + W.nS + r));
+      {
+        int u, r0, nt;
+        GroupWalk gb{W.b0, W.b0 + W.nB, p.I / 8, capB};
+        while (ok && gb.next(u, r0, nt)) ok = pr.issue_b(Lp, P, u, r0, nt);
+        GroupWalk gc{W.c0, W.c0 + W.nC, p.H / 16, capC};
+        while (ok && gc.next(u, r0, nt)) ok = pr.issue_c(Lp, P, u, r0, nt);
+      }
       stamp(p, l, 14);
     }
     // every copy issued lands before the block may exit
@@ -792,7 +840,7 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
   // ---------------- consumers ----------------
   unsigned* ctr = p.ctr;
   long long i = 0;   // ring item
-  uint32_t pos = 0;  // ring placement cursor (same walk as the producer's)
+  unsigned long long pos = 0;  // virtual ring cursor (same walk as the producer's)
   for (int l = 0; l < L; ++l) {
     unsigned* lc = ctr + (size_t)l * CTR_PER_LAYER;
     float* hout = p.h + (size_t)(l & 1) * M * H;
@@ -916,32 +964,53 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
     stamp(p, l, 7);
 
     // ---- B: routed W13 + SwiGLU ----
+    // Groups of consecutive tiles of one expert share a ring item; tile j of a group
+    // (global tile tc + j of this phase) is computed by warp (tc + j) % 8, and the last
+    // warp to finish a group releases it.
     W.init_routed(p, P.n_unique);
-    for (long long r = 0; r < W.nB; ++r, ++i) {
-      const uint32_t s0 = ring_take(pos, bytesB, R);
-      if ((int)(i % STEP_CONSUMERS) != warp) continue;
-      const int slot = (int)(i % STEP_SLOTS);
-      const Item it = W.at(p, W.nA + W.nS + r);
-      float c[4] = {0.f, 0.f, 0.f, 0.f};
-      item_stamp(p, i, 3);
-      if (ring_wait(&full[slot], (uint32_t)((i / STEP_SLOTS) & 1), p.status, &s_abort)) {
-        item_stamp(p, i, 1);
-        const uint8_t* st = ring + s0;
-        const uint8_t* sc = st + 8 * H;  // 16 scale rows of H/32 after the 16 code rows of H/2
-        mxfp4_tile_dot(st + g * (H / 2), st + (8 + g) * (H / 2), sc + g * (H / 32), sc + (8 + g) * (H / 32), H / 32,
-                       xf16, xss, M, c);
-      }
-      __syncwarp();
-      item_stamp(p, i, 2);
-      if (lane == 0) mbar_arrive(&empty[slot]);
+    {
+      GroupWalk gb{W.b0, W.b0 + W.nB, p.I / 8, capB};
+      int u, r0, nt, tc = 0;
+      while (gb.next(u, r0, nt)) {
+        const uint32_t codes = (uint32_t)nt * 8u * (H / 2), scales = (uint32_t)nt * 8u * (H / 32);
+        const uint32_t s0 = ring_take(pos, 2 * codes + 2 * scales, R);
+        const int slot = (int)(i % STEP_SLOTS);
+        const int j0 = ((warp - tc) % STEP_CONSUMERS + STEP_CONSUMERS) % STEP_CONSUMERS;
+        if (j0 < nt) {
+          item_stamp(p, i, 3);
+          const bool ready = ring_wait(&full[slot], (uint32_t)((i / STEP_SLOTS) & 1), p.status, &s_abort);
+          item_stamp(p, i, 1);
+          const uint8_t* gate = ring + s0;
+          const uint8_t* up = gate + codes;
+          const uint8_t* gs = gate + 2 * codes;
+          const uint8_t* us = gs + scales;
+          int mine = 0;
+          for (int j = j0; j < nt; j += STEP_CONSUMERS, ++mine) {
+            float c[4] = {0.f, 0.f, 0.f, 0.f};
+            if (ready) {
+              const int rg = 8 * j + g;  // tile row: gate row and up row of intermediate 8 (r0 + j) + g
+              mxfp4_tile_dot(gate + rg * (H / 2), up + rg * (H / 2), gs + rg * (H / 32), us + rg * (H / 32), H / 32,
+                             xf16, xss, M, c);
+            }
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int tok = 2 * t + e;  // rows g (gate) and g+8 (up) of intermediate index it.b + g
-        if (tok < M)
-          p.a_routed[((size_t)it.a * M + tok) * I + it.b + g] = silu_f32(c[e] * s_inv[tok]) * (c[2 + e] * s_inv[tok]);
+            for (int e = 0; e < 2; ++e) {
+              const int tok = 2 * t + e;
+              if (tok < M)
+                p.a_routed[((size_t)u * M + tok) * I + 8 * (r0 + j) + g] =
+                    silu_f32(c[e] * s_inv[tok]) * (c[2 + e] * s_inv[tok]);
+            }
+            __syncwarp();
+            if (lane == 0) signal_counter(lc + CTR_EXP + u);
+          }
+          item_stamp(p, i, 2);
+          if (lane == 0 && atomicAdd(&s_gdone[slot], mine) + mine == nt) {
+            s_gdone[slot] = 0;
+            mbar_arrive(&empty[slot]);
+          }
+        }
+        tc += nt;
+        ++i;
       }
-      __syncwarp();
-      if (lane == 0) signal_counter(lc + CTR_EXP + it.a);
     }
     stamp(p, l, 8);
     csync();  // xf16 and the shared halves are dead: the routed-W2 activation copies take the region
@@ -992,36 +1061,52 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
       }
       csync();
     }
-    for (long long r = 0; r < W.nC; ++r, ++i) {
-      const uint32_t s0 = ring_take(pos, bytesC, R);
-      if ((int)(i % STEP_CONSUMERS) != warp) continue;
-      const int slot = (int)(i % STEP_SLOTS);
-      const Item it = W.at(p, baseC + r);
-      const int cu = it.a - u_first;  // cache entry
-      const uint8_t* my_af = afc + (size_t)cu * M * ass;
-      float c[4] = {0.f, 0.f, 0.f, 0.f};
-      item_stamp(p, i, 3);
-      if (ring_wait(&full[slot], (uint32_t)((i / STEP_SLOTS) & 1), p.status, &s_abort)) {
-        item_stamp(p, i, 1);
-        const uint8_t* st = ring + s0;
-        const uint8_t* sc = st + 8 * I;  // 16 scale rows of I/32 after the 16 code rows of I/2
-        mxfp4_tile_dot(st + g * (I / 2), st + (8 + g) * (I / 2), sc + g * (I / 32), sc + (8 + g) * (I / 32), I / 32,
-                       my_af, ass, M, c);
-      }
-      __syncwarp();
-      item_stamp(p, i, 2);
-      if (lane == 0) mbar_arrive(&empty[slot]);
+    {
+      GroupWalk gc{W.c0, W.c0 + W.nC, p.H / 16, capC};
+      int u, c0, nt, tc = 0;
+      while (gc.next(u, c0, nt)) {
+        const uint32_t codes = (uint32_t)nt * 16u * (I / 2), scales = (uint32_t)nt * 16u * (I / 32);
+        const uint32_t s0 = ring_take(pos, codes + scales, R);
+        const int slot = (int)(i % STEP_SLOTS);
+        const int j0 = ((warp - tc) % STEP_CONSUMERS + STEP_CONSUMERS) % STEP_CONSUMERS;
+        if (j0 < nt) {
+          const int cu = u - u_first;  // cache entry
+          const uint8_t* my_af = afc + (size_t)cu * M * ass;
+          item_stamp(p, i, 3);
+          const bool ready = ring_wait(&full[slot], (uint32_t)((i / STEP_SLOTS) & 1), p.status, &s_abort);
+          item_stamp(p, i, 1);
+          const uint8_t* cd = ring + s0;
+          const uint8_t* sc = cd + codes;
+          int mine = 0;
+          for (int j = j0; j < nt; j += STEP_CONSUMERS, ++mine) {
+            float c[4] = {0.f, 0.f, 0.f, 0.f};
+            const int rg = 16 * j + g;  // tile rows rg and rg + 8: output rows 16 (c0 + j) + g (+8)
+            if (ready)
+              mxfp4_tile_dot(cd + rg * (I / 2), cd + (rg + 8) * (I / 2), sc + rg * (I / 32), sc + (rg + 8) * (I / 32),
+                             I / 32, my_af, ass, M, c);
+            const int h0 = 16 * (c0 + j) + g;
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int tok = 2 * t + e;
-        if (tok < M) {
-          const float wt = P.w[it.a][tok];
-          if (wt != 0.0f) {
-            const float f = wt * s_pscale[cu][tok];
-            atomicAdd(hout + (size_t)tok * H + it.b + g, c[e] * f);
-            atomicAdd(hout + (size_t)tok * H + it.b + g + 8, c[2 + e] * f);
+            for (int e = 0; e < 2; ++e) {
+              const int tok = 2 * t + e;
+              if (tok < M) {
+                const float wt = P.w[u][tok];
+                if (wt != 0.0f) {
+                  const float f = wt * s_pscale[cu][tok];
+                  atomicAdd(hout + (size_t)tok * H + h0, c[e] * f);
+                  atomicAdd(hout + (size_t)tok * H + h0 + 8, c[2 + e] * f);
+                }
+              }
+            }
+          }
+          __syncwarp();
+          item_stamp(p, i, 2);
+          if (lane == 0 && atomicAdd(&s_gdone[slot], mine) + mine == nt) {
+            s_gdone[slot] = 0;
+            mbar_arrive(&empty[slot]);
           }
         }
+        tc += nt;
+        ++i;
       }
     }
     stamp(p, l, 10);
