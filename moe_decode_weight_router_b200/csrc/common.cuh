@@ -128,6 +128,37 @@ __device__ __forceinline__ float e8m0_to_f32(uint32_t e) {
 // 2^k as fp32 for |k| <= 126.
 __device__ __forceinline__ float exp2i(int k) { return __uint_as_float(static_cast<uint32_t>(k + 127) << 23); }
 
+// Mixed-precision multiply-add: one 16-bit half of each packed operand, product exact
+// in fp32, one fp32 rounding (d = a * b + c).
+__device__ __forceinline__ float fma_f16_lo(uint32_t a2, uint32_t b2, float c) {
+  float d;
+  asm("{\n\t.reg .f16 a0, a1, b0, b1;\n\tmov.b32 {a0, a1}, %1;\n\tmov.b32 {b0, b1}, %2;\n\t"
+      "fma.rn.f32.f16 %0, a0, b0, %3;\n\t}"
+      : "=f"(d) : "r"(a2), "r"(b2), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float fma_f16_hi(uint32_t a2, uint32_t b2, float c) {
+  float d;
+  asm("{\n\t.reg .f16 a0, a1, b0, b1;\n\tmov.b32 {a0, a1}, %1;\n\tmov.b32 {b0, b1}, %2;\n\t"
+      "fma.rn.f32.f16 %0, a1, b1, %3;\n\t}"
+      : "=f"(d) : "r"(a2), "r"(b2), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float fma_bf16_lo(uint32_t a2, uint32_t b2, float c) {
+  float d;
+  asm("{\n\t.reg .b16 a0, a1, b0, b1;\n\tmov.b32 {a0, a1}, %1;\n\tmov.b32 {b0, b1}, %2;\n\t"
+      "fma.rn.f32.bf16 %0, a0, b0, %3;\n\t}"
+      : "=f"(d) : "r"(a2), "r"(b2), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float fma_bf16_hi(uint32_t a2, uint32_t b2, float c) {
+  float d;
+  asm("{\n\t.reg .b16 a0, a1, b0, b1;\n\tmov.b32 {a0, a1}, %1;\n\tmov.b32 {b0, b1}, %2;\n\t"
+      "fma.rn.f32.bf16 %0, a1, b1, %3;\n\t}"
+      : "=f"(d) : "r"(a2), "r"(b2), "f"(c));
+  return d;
+}
+
 // Power-of-two exponent p with amax * 2^p in [2^14, 2^15): moves a row into the
 // f16 range without touching its significands.  0 for amax == 0.
 __device__ __forceinline__ int f16_range_shift(float amax) {

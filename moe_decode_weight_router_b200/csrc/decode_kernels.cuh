@@ -502,9 +502,60 @@ __device__ __forceinline__ void mxfp4_tile_dot_x2(const uint8_t* codes_g, const 
   }
 }
 
+// One token (M = 1) on the CUDA cores: a single activation column leaves 7/8 of each
+// m16n8k16 product idle, so thread (g, t) instead multiplies its blocks t, t+4, ... of
+// rows g and g+8 against the token directly -- codes widened to f16 pairs as above,
+// exact f16 x f16 products summed in fp32 per block, the block's E8M0 scale applied as
+// an exact power of two.  The four t lanes then sum their partials, so every lane of
+// group g returns c0 = row g, c2 = row g+8 (c1 = c3 = 0: there is no second token).
+__device__ __forceinline__ void mxfp4_tile_dot_m1(const uint8_t* codes_g, const uint8_t* codes_g8,
+                                                  const uint8_t* sc_g, const uint8_t* sc_g8, int nb,
+                                                  const uint8_t* xb, float (&c)[4]) {
+  const int t = threadIdx.x & 3;
+  float a0 = 0.0f, a1 = 0.0f;
+#pragma unroll 2
+  for (int b = t; b < nb; b += 4) {
+    const uint4 X0 = lds128(xb + 64 * b), X1 = lds128(xb + 64 * b + 16);
+    const uint4 X2 = lds128(xb + 64 * b + 32), X3 = lds128(xb + 64 * b + 48);
+    const uint32_t xw[16] = {X0.x, X0.y, X0.z, X0.w, X1.x, X1.y, X1.z, X1.w,
+                             X2.x, X2.y, X2.z, X2.w, X3.x, X3.y, X3.z, X3.w};
+    const uint4 C0 = lds128(codes_g + 16 * b), C1 = lds128(codes_g8 + 16 * b);
+    const float f0 = e8m0_to_f32(sc_g[b]), f1 = e8m0_to_f32(sc_g8[b]);
+    const uint32_t w0[4] = {C0.x, C0.y, C0.z, C0.w}, w1[4] = {C1.x, C1.y, C1.z, C1.w};
+    uint32_t h0[16], h1[16];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      e2m1x8_to_f16x2(w0[k], h0[4 * k], h0[4 * k + 1], h0[4 * k + 2], h0[4 * k + 3]);
+      e2m1x8_to_f16x2(w1[k], h1[4 * k], h1[4 * k + 1], h1[4 * k + 2], h1[4 * k + 3]);
+    }
+    float p0 = 0.0f, p1 = 0.0f, p2 = 0.0f, p3 = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      p0 = fma_f16_lo(h0[j], xw[j], p0);
+      p1 = fma_f16_hi(h0[j], xw[j], p1);
+      p2 = fma_f16_lo(h1[j], xw[j], p2);
+      p3 = fma_f16_hi(h1[j], xw[j], p3);
+    }
+    a0 = fmaf(p0 + p1, f0, a0);
+    a1 = fmaf(p2 + p3, f1, a1);
+  }
+  a0 += __shfl_xor_sync(0xffffffffu, a0, 1);
+  a1 += __shfl_xor_sync(0xffffffffu, a1, 1);
+  a0 += __shfl_xor_sync(0xffffffffu, a0, 2);
+  a1 += __shfl_xor_sync(0xffffffffu, a1, 2);
+  c[0] = a0;
+  c[1] = 0.0f;
+  c[2] = a1;
+  c[3] = 0.0f;
+}
+
 __device__ __forceinline__ void mxfp4_tile_dot(const uint8_t* codes_g, const uint8_t* codes_g8,
                                                const uint8_t* sc_g, const uint8_t* sc_g8, int nb,
                                                const uint8_t* xb, uint32_t xss, int M, float (&c)[4]) {
+  if (M == 1) {
+    mxfp4_tile_dot_m1(codes_g, codes_g8, sc_g, sc_g8, nb, xb, c);
+    return;
+  }
   if ((nb & 7) == 0 && ((reinterpret_cast<uintptr_t>(sc_g) | reinterpret_cast<uintptr_t>(sc_g8)) & 3u) == 0) {
     mxfp4_tile_dot_x2(codes_g, codes_g8, sc_g, sc_g8, nb, xb, xss, M, c);
     return;

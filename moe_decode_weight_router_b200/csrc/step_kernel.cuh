@@ -745,6 +745,55 @@ __device__ __forceinline__ void rows4_dot(const uint8_t* wrows, uint32_t wstride
   for (int e = 0; e < 4; ++e) c[e] = (c4[0][e] + c4[1][e]) + (c4[2][e] + c4[3][e]);
 }
 
+// One token (M = 1) on the CUDA cores: column n of the four reads shared-memory row
+// (rmap >> 4n) & 3; lane L covers K columns 8L + 256j.  Exact bf16 products summed in
+// fp32 against act0 (plus act1 when given: a hi/lo split of one fp32 row); every lane
+// returns all four column sums.
+__device__ __forceinline__ void rows4_dot_m1(const uint8_t* wrows, uint32_t wstride, uint32_t rmap,
+                                             const uint8_t* act0, const uint8_t* act1, int K, float (&o)[4]) {
+  const int lane = threadIdx.x & 31;
+  float a[4][2];
+#pragma unroll
+  for (int n = 0; n < 4; ++n) a[n][0] = a[n][1] = 0.0f;
+  const uint8_t* wr[4];
+#pragma unroll
+  for (int n = 0; n < 4; ++n) wr[n] = wrows + (size_t)((rmap >> (4 * n)) & 3u) * wstride;
+#pragma unroll 2
+  for (int k = 8 * lane; k < K; k += 256) {
+    const uint4 X = lds128(act0 + 2 * k);
+    const uint32_t xw[4] = {X.x, X.y, X.z, X.w};
+    uint32_t yw[4] = {0u, 0u, 0u, 0u};
+    if (act1) {
+      const uint4 Y = lds128(act1 + 2 * k);
+      yw[0] = Y.x; yw[1] = Y.y; yw[2] = Y.z; yw[3] = Y.w;
+    }
+#pragma unroll
+    for (int n = 0; n < 4; ++n) {
+      const uint4 W = lds128(wr[n] + 2 * k);
+      const uint32_t ww[4] = {W.x, W.y, W.z, W.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        a[n][0] = fma_bf16_lo(ww[j], xw[j], a[n][0]);
+        a[n][1] = fma_bf16_hi(ww[j], xw[j], a[n][1]);
+      }
+      if (act1) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          a[n][0] = fma_bf16_lo(ww[j], yw[j], a[n][0]);
+          a[n][1] = fma_bf16_hi(ww[j], yw[j], a[n][1]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int n = 0; n < 4; ++n) {
+    float v = a[n][0] + a[n][1];
+#pragma unroll
+    for (int s = 16; s > 0; s >>= 1) v += __shfl_xor_sync(0xffffffffu, v, s);
+    o[n] = v;
+  }
+}
+
 __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant__ StepParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ Plan P;
@@ -880,8 +929,15 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
         item_stamp(p, i, 1);
         // shared items: columns (0,1,2,3) = (gate 2s, up 2s, gate 2s+1, up 2s+1) from
         // smem rows (0, 2, 1, 3), so a thread's two columns are a (gate, up) pair
-        const int wrow = g < 4 ? (router ? g : ((g & 1) ? 2 : 0) + (g >> 1)) : -1;
-        rows4_dot(ring + s0, 2u * H, wrow, g < M ? xb16 + g * xss : nullptr, nullptr, H, c);
+        if (M == 1) {
+          float o[4];
+          rows4_dot_m1(ring + s0, 2u * H, router ? 0x3210u : 0x3120u, xb16, nullptr, H, o);
+          c[0] = t == 0 ? o[0] : o[2];
+          c[1] = t == 0 ? o[1] : o[3];
+        } else {
+          const int wrow = g < 4 ? (router ? g : ((g & 1) ? 2 : 0) + (g >> 1)) : -1;
+          rows4_dot(ring + s0, 2u * H, wrow, g < M ? xb16 + g * xss : nullptr, nullptr, H, c);
+        }
       }
       __syncwarp();
       item_stamp(p, i, 2);
@@ -938,10 +994,18 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
       item_stamp(p, i, 3);
       if (ring_wait(&full[slot], (uint32_t)((i / STEP_SLOTS) & 1), p.status, &s_abort)) {
         item_stamp(p, i, 1);
-        const uint8_t* src = (g & 1) ? slo : shi;
-        const int t0 = g >> 1, t1 = 4 + (g >> 1);
-        rows4_dot(ring + s0, 2u * Is, g < 4 ? g : -1, t0 < M ? src + t0 * sss : nullptr,
-                  t1 < M ? src + t1 * sss : nullptr, Is, c);
+        if (M == 1) {
+          // the full hi + lo sum lands in lane group 0; group 1 adds zeros below
+          float o[4];
+          rows4_dot_m1(ring + s0, 2u * Is, 0x3210u, shi, slo, Is, o);
+          c[0] = g == 0 ? (t == 0 ? o[0] : o[2]) : 0.0f;
+          c[1] = g == 0 ? (t == 0 ? o[1] : o[3]) : 0.0f;
+        } else {
+          const uint8_t* src = (g & 1) ? slo : shi;
+          const int t0 = g >> 1, t1 = 4 + (g >> 1);
+          rows4_dot(ring + s0, 2u * Is, g < 4 ? g : -1, t0 < M ? src + t0 * sss : nullptr,
+                    t1 < M ? src + t1 * sss : nullptr, Is, c);
+        }
       }
       __syncwarp();
       item_stamp(p, i, 2);
