@@ -276,8 +276,8 @@ enum { MOE_STEP_AUTO = 0, MOE_STEP_PER_LAYER = 1 };
  *     (decode_step_launch_names gives the launches).
  *   timeline: NULL or [2*L*16 + 4*4096] uint64 %globaltimer stamps (ns), for profiling
  *     the persistent path: [2][L][16] phase boundaries of blocks 0 and G-1, then block 0's
- *     first 2048 weight items, 8 stamps each (issued, data ready, done, wait started,
- *     producer entered, 3 unused). */
+ *     first 2048 weight items, 8 stamps each (window acquired, data ready, done, wait
+ *     started, producer entered, copies issued, 2 unused). */
 typedef struct {
   void* x;
   float* h;

@@ -48,7 +48,8 @@ constexpr int STEP_SLOTS = 32;  // ring items in flight at most (one full/empty 
 constexpr int CTR_H = 2, CTR_HINIT = 3, CTR_EXP = 4;  // slots 0-1 unused
 constexpr int CTR_PER_LAYER = CTR_EXP + MAX_SLOTS;
 constexpr size_t STEP_FIXED = 1024;  // full[32], empty[32], plan and h-init barriers
-constexpr int STAGE_REG_F4 = 4;      // residual float4s a consumer thread keeps in registers (M = 1 at H = 2560)
+constexpr int STAGE_REG_F4 = 4;  // residual float4s a consumer thread keeps in registers (M = 1 at H = 2560)
+constexpr int STAGE_BATCH = 5;   // larger inputs: residual loads a thread keeps in flight
 
 struct LayerPtrs {
   const __nv_bfloat16* wr;
@@ -267,8 +268,8 @@ struct Item {
 struct Work {
   int nA;             // A items of this block
   int nS;             // shared-W2 items of this block
-  long long b0, nB;   // routed W13 range
-  long long c0, nC;   // routed W2 range
+  int b0, nB;         // routed W13 range
+  int c0, nC;         // routed W2 range
   __device__ void init_fixed(const StepParams& p) {
     const int c = blockIdx.x, G = gridDim.x;
     const int TA = p.E / 4 + p.Is / 2;
@@ -279,11 +280,12 @@ struct Work {
     b0 = c0 = 0;
   }
   __device__ void init_routed(const StepParams& p, int n_unique) {
-    const long long c = blockIdx.x, G = gridDim.x;
-    const long long TB = (long long)n_unique * (p.I / 8);
+    // n_unique <= MAX_SLOTS: tiles per expert * n_unique * blocks stays far below 2^31
+    const int c = blockIdx.x, G = gridDim.x;
+    const int TB = n_unique * (p.I / 8);
     b0 = TB * c / G;
     nB = TB * (c + 1) / G - b0;
-    const long long TC = (long long)n_unique * (p.H / 16);
+    const int TC = n_unique * (p.H / 16);
     c0 = TC * c / G;
     nC = TC * (c + 1) / G - c0;
   }
@@ -323,14 +325,14 @@ struct Work {
 // contiguous in HBM: one copy per run instead of one per tile).  Walks tiles
 // x .. end-1 of the block's range (T tiles per expert), at most cap per group.
 struct GroupWalk {
-  long long x, end;
+  int x, end;
   int T, cap;
   __device__ bool next(int& u, int& r0, int& nt) {
     if (x >= end) return false;
-    u = (int)(x / T);
-    r0 = (int)(x - (long long)u * T);
-    const long long lim = min(end, (long long)(u + 1) * T);
-    nt = (int)min((long long)cap, lim - x);
+    u = x / T;
+    r0 = x - u * T;
+    const int lim = min(end, (u + 1) * T);
+    nt = min(cap, lim - x);
     x += nt;
     return true;
   }
@@ -405,6 +407,7 @@ struct Producer {
     if (lane == 1) bulk_g2s(st + codes, Lp.w13c + (row + I) * (H / 2), codes, fb, pol);
     if (lane == 2) bulk_g2s(st + 2 * codes, Lp.w13s + row * (H / 32), scales, fb, pol);
     if (lane == 3) bulk_g2s(st + 2 * codes + scales, Lp.w13s + (row + I) * (H / 32), scales, fb, pol);
+    item_stamp(p, i, 5);
     ++i;
     return true;
   }
@@ -423,6 +426,7 @@ struct Producer {
     __syncwarp();
     if (lane == 0) bulk_g2s(st, Lp.w2c + row * (I / 2), codes, fb, pol);
     if (lane == 1) bulk_g2s(st + codes, Lp.w2s + row * (I / 32), scales, fb, pol);
+    item_stamp(p, i, 5);
     ++i;
     return true;
   }
@@ -451,6 +455,7 @@ struct Producer {
       __syncwarp();
       if (lane == 0) bulk_g2s(st, Lp.sw2 + (size_t)it.a * Is, 4u * 2u * Is, fb, pol);
     }
+    item_stamp(p, i, 5);
     ++i;
     return true;
   }
@@ -554,24 +559,51 @@ __device__ void stage_layer_input(const StepParams& p, int l, const float* hin, 
       }
     }
   } else {
-    for (int tok = 0; tok < M; ++tok) {
-      float ss = 0.0f, am = 0.0f;
-      for (int c = tid; c < per; c += nt) {
-        const int q = tok * per + c;
-        const float4 w = load_residual4(p, l, hin, q);
-        if (q >= q0 && q < q1) hout4[q] = w;
-        accumulate4(w, ss, am);
-      }
+    // Streamed in batches of STAGE_BATCH independent loads.  H/4 is a multiple of 32,
+    // so the 32 consecutive q of a warp share one token, and a thread's q only grow:
+    // each warp meets each of its tokens in one run and reduces it when the run ends.
+    for (int e = tid; e < M * STEP_CONSUMERS; e += nt) {
+      s_part[e] = 0.0f;
+      s_amx[e] = 0.0f;
+    }
+    csync();
+    int cur = -1;
+    float ss = 0.0f, am = 0.0f;
+    auto flush = [&]() {
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) {
         ss += __shfl_xor_sync(0xffffffffu, ss, o);
         am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
       }
       if (lane == 0) {
-        s_part[tok * STEP_CONSUMERS + warp] = ss;
-        s_amx[tok * STEP_CONSUMERS + warp] = am;
+        s_part[cur * STEP_CONSUMERS + warp] = ss;
+        s_amx[cur * STEP_CONSUMERS + warp] = am;
+      }
+    };
+    for (int qb = tid; qb < Q; qb += STAGE_BATCH * nt) {
+      float4 w[STAGE_BATCH];
+#pragma unroll
+      for (int j = 0; j < STAGE_BATCH; ++j) {
+        const int q = qb + j * nt;
+        w[j] = q < Q ? load_residual4(p, l, hin, q) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int j = 0; j < STAGE_BATCH; ++j) {
+        const int q = qb + j * nt;
+        if (q < Q) {  // uniform across the warp (Q is a multiple of 32)
+          const int tok = q / per;
+          if (tok != cur) {
+            if (cur >= 0) flush();
+            cur = tok;
+            ss = 0.0f;
+            am = 0.0f;
+          }
+          if (q >= q0 && q < q1) hout4[q] = w[j];
+          accumulate4(w[j], ss, am);
+        }
       }
     }
+    if (cur >= 0) flush();
   }
   csync();
   if (tid < M) {
@@ -593,9 +625,21 @@ __device__ void stage_layer_input(const StepParams& p, int l, const float* hin, 
       if (tq[j] < M)
         write_layer_input4(xb16, xf16, tq[j] * xss + 8 * cq[j], v[j], s_r[tq[j]], exp2i(s_sh[tq[j]]));
   } else {
-    for (int q = tid; q < Q; q += nt) {
-      const int tok = q / per, c = q - tok * per;
-      write_layer_input4(xb16, xf16, tok * xss + 8 * c, load_residual4(p, l, hin, q), s_r[tok], exp2i(s_sh[tok]));
+    for (int qb = tid; qb < Q; qb += STAGE_BATCH * nt) {
+      float4 w[STAGE_BATCH];
+#pragma unroll
+      for (int j = 0; j < STAGE_BATCH; ++j) {
+        const int q = qb + j * nt;
+        w[j] = q < Q ? load_residual4(p, l, hin, q) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int j = 0; j < STAGE_BATCH; ++j) {
+        const int q = qb + j * nt;
+        if (q < Q) {
+          const int tok = q / per, c = q - tok * per;
+          write_layer_input4(xb16, xf16, tok * xss + 8 * c, w[j], s_r[tok], exp2i(s_sh[tok]));
+        }
+      }
     }
   }
   csync();  // also orders this block's slice stores before the h-init hand-off
@@ -603,16 +647,21 @@ __device__ void stage_layer_input(const StepParams& p, int l, const float* hin, 
 
 // Top-k of every token from the complete router logits (same rule as k_dense:
 // largest logit, lowest index on ties), then the union plan.  The 8 consumer warps
-// each take an eighth of the experts and keep their own top-k (a global top-k
-// element is always in its part's top-k, ties included), then one warp per token
-// merges the 8k candidates.
+// form TG token groups x EP expert parts (TG the largest power of two <= min(M, 8)
+// whose parts hold at most 256 experts): each keeps its part's top-k of its tokens
+// (a global top-k element is always in its part's top-k, ties included), then one
+// warp per token merges the EP*k candidates.
 __device__ void step_topk(const StepParams& p, int l, Plan& P, int32_t* s_ids, float* s_wts, uint32_t* s_ck,
                           int32_t* s_ci, volatile int* s_abort_ptr) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int E = p.E, k = p.k, M = p.M;
-  const int per = (E + STEP_CONSUMERS - 1) / STEP_CONSUMERS;  // experts per warp (<= 256)
-  const int e0 = warp * per;
-  for (int tok = 0; tok < M; ++tok) {
+  int TG = 1;
+  while (2 * TG <= M && 2 * TG <= STEP_CONSUMERS && E <= 256 * (STEP_CONSUMERS / (2 * TG))) TG *= 2;
+  const int EP = STEP_CONSUMERS / TG;
+  const int per = (E + EP - 1) / EP;  // experts per part (<= 256)
+  const int part = warp % EP;
+  const int e0 = part * per;
+  for (int tok = warp / EP; tok < M; tok += TG) {
     uint32_t key[8];
     {
       const unsigned long long* w[8];
@@ -646,15 +695,15 @@ __device__ void step_topk(const StepParams& p, int l, Plan& P, int32_t* s_ids, f
         for (int i = 0; i < 8; ++i)
           if (e0 + lane + 32 * i == mi) key[i] = 0u;
         if (lane == 0) {
-          s_ck[(tok * STEP_CONSUMERS + warp) * 8 + j] = mk;
-          s_ci[(tok * STEP_CONSUMERS + warp) * 8 + j] = mk ? mi : 0x7fffffff;
+          s_ck[(tok * STEP_CONSUMERS + part) * 8 + j] = mk;
+          s_ci[(tok * STEP_CONSUMERS + part) * 8 + j] = mk ? mi : 0x7fffffff;
         }
       }
     }
   }
   csync();
   for (int tok = warp; tok < M; tok += STEP_CONSUMERS) {
-    const int nc = STEP_CONSUMERS * k;  // <= 64 candidates, two per lane
+    const int nc = EP * k;  // <= 64 candidates, two per lane
     uint32_t ck[2] = {0u, 0u};
     int ci[2] = {0x7fffffff, 0x7fffffff};
 #pragma unroll
@@ -870,6 +919,7 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
       if (!__shfl_sync(0xffffffffu, got, 0)) break;
       stamp(p, l, 13);
       W.init_routed(p, P.n_unique);
+      stamp(p, l, 15);
       {
         int u, r0, nt;
         GroupWalk gb{W.b0, W.b0 + W.nB, p.I / 8, capB};
