@@ -42,7 +42,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 # DRAM traffic of k_step per layer (read + write) from the ncu capture summarised in
 # profiles/k_step_ling_2layers_m1.md, valid while the kernel sources hash to the value
 # recorded with it (otherwise the roofline's traffic is reported as null).
-KSTEP_TRAFFIC = {"bytes_per_layer": (79.14e6 + 2.01e6) / 2, "sources_sha256_16": "e4142767afffce3a",
+KSTEP_TRAFFIC = {"bytes_per_layer": (79.14e6 + 1.88e6) / 2, "sources_sha256_16": "c6720a0d82a49ca8",
                  "sources": ("step_kernel.cuh", "decode_kernels.cuh", "common.cuh")}
 
 
