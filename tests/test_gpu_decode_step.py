@@ -109,6 +109,22 @@ def test_tiny_chain_free_running_matches_oracle_chain():
         assert_rows_close(res["logits"].cpu().numpy(), out["logits"], what="free-running logits")
 
 
+@pytest.mark.parametrize("M", [2, 3, 5, 8])
+def test_ling_shaped_short_chain_every_window(M):
+    """Three Ling-shaped layers (H 2560: the layer input of two or more tokens no longer
+    fits the registers and is streamed; the top-k splits its warps into token groups x
+    expert parts) at the verify-window sizes the tiny chain does not reach; every
+    layer and the head are recomputed by the oracle."""
+    S = synth.LING
+    model = _model(S, 3, 1000, 51 + M)
+    x = synth.tokens(M, S.H, 51 + M, device="cuda")
+    assert decode_step_launch_names(model, M) == ["k_step", "k_lm_gemv"]
+    res = decode_step(model, x, trace=True)
+    torch.cuda.synchronize()
+    assert workspace_status(res["ws"]) == 0
+    _check_step(model, S, x, res, range(3))
+
+
 @pytest.mark.parametrize("M,path", [(1, "persistent"), (4, "persistent"), (1, "per_layer")])
 def test_ling_42_layers_sampled(M, path):
     """Full size: 42 distinct Ling-shaped layers (~67 GB MXFP4) and the 157,184 x 2,560
