@@ -901,16 +901,19 @@ EncodeTiledFn encode_fn() {
   return f;
 }
 
-// 2-D K-major operand: dims {inner elements, rows}, row pitch in bytes, 128-byte swizzle.
+// Activation operand, K-major in chunks of box_inner elements (chunk_bytes in HBM):
+// dims {chunk, rows, K / chunk}, box {chunk, 64 rows, kc}, 128-byte swizzle.  The chunk
+// index is the outermost dimension although its stride is the smallest, so kc chunks
+// arrive as kc consecutive swizzled tiles.
 bool make_map(CUtensorMap* m, CUtensorMapDataType t, const void* base, uint64_t inner, uint64_t rows,
-              uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows) {
+              uint64_t row_bytes, uint32_t box_inner, uint64_t chunk_bytes, int kc) {
   EncodeTiledFn f = encode_fn();
   if (!f) return false;
-  cuuint64_t dims[2] = {inner, rows};
-  cuuint64_t strides[1] = {row_bytes};
-  cuuint32_t box[2] = {box_inner, box_rows};
-  cuuint32_t es[2] = {1, 1};
-  return f(m, t, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+  cuuint64_t dims[3] = {box_inner, rows, inner / box_inner};
+  cuuint64_t strides[2] = {row_bytes, chunk_bytes};
+  cuuint32_t box[3] = {box_inner, 64, (cuuint32_t)kc};
+  cuuint32_t es[3] = {1, 1, 1};
+  return f(m, t, 3, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
          CUDA_SUCCESS;
 }
@@ -918,20 +921,24 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType t, const void* base, uint64_t 
 // Bytes per activation-scale row: K/32 rounded up to 16 (rows are bulk-copied).
 int pf_sf_ld(int K) { return (K / 32 + 15) / 16 * 16; }
 
-// Weight operand as {K elements, rows, 2 halves}: one box of {box_inner, 64, 2} brings
-// 64 rows and the 64 rows half_bytes further on (gate and up rows, or the next 64).
+// Weight operand as {chunk, rows, 2 halves, K / chunk}: one box of {chunk, 64, 2, kc}
+// brings 64 rows and the 64 rows half_bytes further on (gate and up rows, or the next
+// 64) for kc consecutive K chunks.  Fewer, larger copies: each tensor copy costs the copy
+// engine a fixed fraction of a microsecond besides its bytes.
 bool make_map_halves(CUtensorMap* m, CUtensorMapDataType t, const void* base, uint64_t inner, uint64_t rows,
-                     uint64_t row_bytes, uint64_t half_bytes, uint32_t box_inner) {
+                     uint64_t row_bytes, uint64_t half_bytes, uint32_t box_inner, uint64_t chunk_bytes, int kc) {
   EncodeTiledFn f = encode_fn();
   if (!f) return false;
-  cuuint64_t dims[3] = {inner, rows, 2};
-  cuuint64_t strides[2] = {row_bytes, half_bytes};
-  cuuint32_t box[3] = {box_inner, 64, 2};
-  cuuint32_t es[3] = {1, 1, 1};
-  return f(m, t, 3, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+  cuuint64_t dims[4] = {box_inner, rows, 2, inner / box_inner};
+  cuuint64_t strides[3] = {row_bytes, half_bytes, chunk_bytes};
+  cuuint32_t box[4] = {box_inner, 64, 2, (cuuint32_t)kc};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return f(m, t, 4, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
          CUDA_SUCCESS;
 }
+// K chunks per stage of a k_umma launch: two when they divide the chunk count.
+int pf_kc(int K, int kbox) { return ((K / kbox) % 2 == 0) ? 2 : 1; }
 
 bool ok_pf(int M, int H, int I, int E, int k, int Is) {
   return M >= 128 && M % 128 == 0 && M <= 16384 && H >= 128 && H % 128 == 0 && H <= 4096 && I >= 128 &&
@@ -1004,10 +1011,11 @@ PfWs pf_ws(void* ws, int M, int H, int I, int E, int k, int Is) {
 moe_status_t launch_umma(PrefillParams& p, const DevInfo& d, cudaStream_t st) {
   const size_t sf = (p.mode == PF_R13 || p.mode == PF_R2) ? 2 * (size_t)pf_sf_buf_bytes(p.K, p.sf_ld) : 0;
   const long long room = (long long)d.dyn_pf - 1024 - (long long)sf;
-  const int stages = room > 0 ? (int)(room / PF_STAGE_BYTES) : 0;
+  const long long stage = (long long)PF_STAGE_BYTES * p.kc;
+  const int stages = room > 0 ? (int)(room / stage) : 0;
   p.stages = stages > PF_MAX_STAGES ? PF_MAX_STAGES : stages;
   if (p.stages < 2) return MOE_ERR_UNSUPPORTED_SHAPE;
-  const size_t smem = 1024 + (size_t)p.stages * PF_STAGE_BYTES + sf;
+  const size_t smem = 1024 + (size_t)p.stages * stage + sf;
   k_umma<<<d.sms, PF_THREADS, smem, st>>>(p);
   MOE_CUDA(cudaGetLastError());
   return MOE_OK;
@@ -1049,10 +1057,12 @@ moe_status_t moe_prefill_layer(const void* x_bf16, int M, int H, int I, int E, i
   PrefillParams p{};
   p.status = w.status;
   p.E = E;
+  p.kc = pf_kc(H, 64);
   REQ(make_map_halves(&p.tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w_router_bf16, H, E, (uint64_t)H * 2,
-                      (uint64_t)64 * H * 2, 64),
+                      (uint64_t)64 * H * 2, 64, 128, p.kc),
       MOE_ERR_INVALID_ARG);
-  REQ(make_map(&p.tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, H, M, (uint64_t)H * 2, 64, 64), MOE_ERR_INVALID_ARG);
+  REQ(make_map(&p.tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, H, M, (uint64_t)H * 2, 64, 128, p.kc),
+      MOE_ERR_INVALID_ARG);
   p.mode = PF_ROUTER;
   p.K = H;
   p.m_tiles = E / 128;
@@ -1075,8 +1085,9 @@ moe_status_t moe_prefill_layer(const void* x_bf16, int M, int H, int I, int E, i
   if (Is > 0) {
     PrefillParams q{};
     q.status = w.status;
+    q.kc = p.kc;  // K = H as for the router: the token map is shared
     REQ(make_map_halves(&q.tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, shared_w13_bf16, H, 2 * (uint64_t)Is,
-                        (uint64_t)H * 2, (uint64_t)Is * H * 2, 64),
+                        (uint64_t)H * 2, (uint64_t)Is * H * 2, 64, 128, q.kc),
         MOE_ERR_INVALID_ARG);
     q.tmB = p.tmB;
     q.mode = PF_SH13;
@@ -1089,10 +1100,12 @@ moe_status_t moe_prefill_layer(const void* x_bf16, int M, int H, int I, int E, i
     if ((s = launch_umma(q, d, st)) != MOE_OK) return s;
     PrefillParams r{};
     r.status = w.status;
+    r.kc = pf_kc(Is, 64);
     REQ(make_map_halves(&r.tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, shared_w2_bf16, Is, H, (uint64_t)Is * 2,
-                        (uint64_t)64 * Is * 2, 64),
+                        (uint64_t)64 * Is * 2, 64, 128, r.kc),
         MOE_ERR_INVALID_ARG);
-    REQ(make_map(&r.tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w.as, Is, M, (uint64_t)Is * 2, 64, 64), MOE_ERR_INVALID_ARG);
+    REQ(make_map(&r.tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w.as, Is, M, (uint64_t)Is * 2, 64, 128, r.kc),
+        MOE_ERR_INVALID_ARG);
     r.mode = PF_SH2;
     r.K = Is;
     r.m_tiles = H / 128;
@@ -1107,10 +1120,11 @@ moe_status_t moe_prefill_layer(const void* x_bf16, int M, int H, int I, int E, i
   // a3: routed W13 + SwiGLU, activation re-quantised to MXFP8 (E2M1 x E4M3 block-scaled)
   PrefillParams a{};
   a.status = w.status;
+  a.kc = pf_kc(H, 128);
   REQ(make_map_halves(&a.tmA, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, w13_codes, H, (uint64_t)E * 2 * I,
-                      (uint64_t)H / 2, (uint64_t)I * (H / 2), 128),
+                      (uint64_t)H / 2, (uint64_t)I * (H / 2), 128, 64, a.kc),
       MOE_ERR_INVALID_ARG);
-  REQ(make_map(&a.tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.xq, H, G, H, 128, 64), MOE_ERR_INVALID_ARG);
+  REQ(make_map(&a.tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.xq, H, G, H, 128, 128, a.kc), MOE_ERR_INVALID_ARG);
   a.mode = PF_R13;
   a.K = H;
   a.m_tiles = I / 64;
@@ -1132,10 +1146,11 @@ moe_status_t moe_prefill_layer(const void* x_bf16, int M, int H, int I, int E, i
   // a4: routed W2, weighted by the routing weight and added into y
   PrefillParams b{};
   b.status = w.status;
+  b.kc = pf_kc(I, 128);
   REQ(make_map_halves(&b.tmA, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, w2_codes, I, (uint64_t)E * H, (uint64_t)I / 2,
-                      (uint64_t)64 * (I / 2), 128),
+                      (uint64_t)64 * (I / 2), 128, 64, b.kc),
       MOE_ERR_INVALID_ARG);
-  REQ(make_map(&b.tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.aq, I, G, I, 128, 64), MOE_ERR_INVALID_ARG);
+  REQ(make_map(&b.tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.aq, I, G, I, 128, 128, b.kc), MOE_ERR_INVALID_ARG);
   b.mode = PF_R2;
   b.K = I;
   b.m_tiles = H / 128;

@@ -42,15 +42,18 @@ namespace moe {
 enum : int { PF_ROUTER = 0, PF_SH13 = 1, PF_SH2 = 2, PF_R13 = 3, PF_R2 = 4 };
 constexpr int PF_THREADS = 192;        // warps 0-3 epilogue, 4 producer, 5 MMA
 constexpr int PF_BN = 64;              // token tile (MMA N <= 64)
-constexpr int PF_STAGE_BYTES = 24576;  // weight tile 16 KB + token tile 8 KB
+constexpr int PF_STAGE_BYTES = 24576;  // per K chunk: weight tile 16 KB + token tile 8 KB
 constexpr int PF_MAX_STAGES = 9;
 constexpr int PF_TMEM_COLS = 512;      // accumulators 0..127 and 128..255, SFA 256.., SFB 384..
 constexpr int PF_SFA_COL = 256, PF_SFB_COL = 384;
 constexpr int PF_MAX_CHUNKS = 32;      // K / 128 for the block-scaled modes (SF columns)
 
 struct alignas(64) PrefillParams {
-  CUtensorMap tmA;  // weights: dims {K, rows, 2 halves}, box {64 or 128 elements, 64 rows, 2}
-  CUtensorMap tmB;  // activations: dims {K, rows}, box {.., 64 rows}
+  // Both maps put the K chunk (64 bf16 or 128 E2M1 / E4M3 elements: 128 bytes a row in
+  // shared memory) in an outer dimension, so one copy brings kc chunks, each landing as
+  // the swizzled tile one chunk of MMAs reads.
+  CUtensorMap tmA;  // weights: dims {chunk, rows, 2 halves, K / chunk}, box {chunk, 64, 2, kc}
+  CUtensorMap tmB;  // activations: dims {chunk, rows, K / chunk}, box {chunk, 64, kc}
   int mode;
   int K;
   int m_tiles;   // weight tiles per problem
@@ -73,6 +76,7 @@ struct alignas(64) PrefillParams {
   uint8_t* out_qs;          // routed activation E8M0 [G][out_qs_ld]
   int out_qs_ld;
   int stages;
+  int kc;  // K chunks per pipeline stage (one copy per operand per stage)
   int* status;
 };
 
@@ -139,6 +143,14 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, i
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
       "[%5];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, int x, int y, int z, int w,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], "
+      "[%6];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar))
       : "memory");
 }
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
@@ -272,8 +284,8 @@ __device__ __forceinline__ uint8_t e4m3_of(float v) {
 // ---------------------------------------------------------------------------
 // k_umma
 // ---------------------------------------------------------------------------
-// Shared memory: the 1024-aligned stage ring (weight tile at +0 and +8192, token tile
-// at +16384 in 32-row boxes of 4096 B), then for the block-scaled modes two buffers of
+// Shared memory: the 1024-aligned stage ring (kc chunks a stage: chunk c's weight tile
+// at +16384 c, its token tile at +16384 kc + 8192 c), then for the block-scaled modes two buffers of
 // the current tiles' E8M0 rows (weight rows at +0, K/32 bytes each; token rows after
 // them, sf_ld bytes each), filled by the producer with bulk copies.
 __host__ __device__ inline uint32_t pf_sf_buf_bytes(int K, int sf_ld) {
@@ -294,8 +306,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int S = p.stages;
   const bool mx = pf_routed(p.mode);
-  const int kbox = mx ? 128 : 64;  // K elements per stage (128 bytes per row)
+  const int kbox = mx ? 128 : 64;  // K elements per chunk (128 bytes per row)
   const int nch = p.K / kbox;
+  const int KC = p.kc;             // chunks per stage (divides nch)
+  const size_t stage_bytes = (size_t)PF_STAGE_BYTES * KC;
   if (mx)
     for (int e = tid; e <= p.E; e += PF_THREADS) {
       s_ntp[e] = __ldg(p.ntile_prefix + e);
@@ -306,7 +320,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
   const int G = gridDim.x;
   const int kb = p.K / 32;  // E8M0 bytes per weight row
   const uint32_t sfa_bytes = (uint32_t)(128 * kb + 15) / 16 * 16;
-  uint8_t* sfbuf = smem + (size_t)S * PF_STAGE_BYTES;
+  uint8_t* sfbuf = smem + (size_t)S * stage_bytes;
   const uint32_t sfbuf_bytes = pf_sf_buf_bytes(p.K, p.sf_ld);
 
   if (tid == 0) {
@@ -358,19 +372,19 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
           bulk_g2s(dst + half, p.sfa + (size_t)it.ya1 * kb, half, &sf_full[b], pol);
           bulk_g2s(dst + sfa_bytes, p.sfb + (size_t)it.grow0 * p.sf_ld, tok, &sf_full[b], pol);
         }
-        for (int ch = 0; ch < nch; ++ch, ++q) {
+        for (int ch = 0; ch < nch; ch += KC, ++q) {
           const int s = (int)(q % S);
           if (q >= S && !pf_wait(&empty[s], (uint32_t)(((q / S) - 1) & 1), p.status, &s_abort, PFW_EMPTY, p.mode)) {
             ok = false;
             break;
           }
-          uint8_t* st = smem + (size_t)s * PF_STAGE_BYTES;
+          uint8_t* st = smem + (size_t)s * stage_bytes;
           // transaction bytes count the global (packed) side: 128 rows of 128 E2M1
           // codes are 8 KB although they fill 16 KB of shared memory; the token box
           // is always whole (rows past the tensor read as zeros and still count)
-          mbar_arrive_expect_tx(&full[s], (mx ? 8192u : 16384u) + 8192u);
-          tma_load_3d(st, &p.tmA, ch * kbox, it.ya0, 0, &full[s]);
-          tma_load_2d(st + 16384, &p.tmB, ch * kbox, it.grow0, &full[s]);
+          mbar_arrive_expect_tx(&full[s], (uint32_t)KC * ((mx ? 8192u : 16384u) + 8192u));
+          tma_load_4d(st, &p.tmA, 0, it.ya0, 0, ch, &full[s]);
+          tma_load_3d(st + 16384 * KC, &p.tmB, 0, it.grow0, ch, &full[s]);
         }
       }
       // every copy issued lands before the CTA may finish
@@ -396,24 +410,27 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
         if (mx && !pf_wait(&sf_ready, (uint32_t)(n_item & 1), p.status, &s_abort, PFW_SF, p.mode)) break;
         tc_fence_after();
         const uint32_t dacc = tbase + 128u * ab;
-        for (int ch = 0; ch < nch; ++ch, ++q) {
+        for (int ch = 0; ch < nch; ch += KC, ++q) {
           const int s = (int)(q % S);
           if (!pf_wait(&full[s], (uint32_t)((q / S) & 1), p.status, &s_abort, PFW_FULL, p.mode)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sa = smem_u32(smem + (size_t)s * PF_STAGE_BYTES);
-          const uint64_t adesc = sw128_desc(sa), bdesc = sw128_desc(sa + 16384);
+          const uint32_t sa = smem_u32(smem + (size_t)s * stage_bytes);
+          for (int c = 0; c < KC; ++c) {
+            const uint64_t adesc = sw128_desc(sa + 16384u * c), bdesc = sw128_desc(sa + 16384u * KC + 8192u * c);
+            const uint32_t chc = (uint32_t)(ch + c);
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint32_t accum = (ch > 0 || k > 0) ? 1u : 0u;
-            // advance 32 bytes of K inside the 128-byte swizzled row
-            if (mx)
-              umma_mx(dacc, adesc + 2u * k, bdesc + 2u * k, idesc_mx(N, (uint32_t)k), accum,
-                      tbase + PF_SFA_COL + 4u * ch, tbase + PF_SFB_COL + 4u * ch);
-            else
-              umma_bf16(dacc, adesc + 2u * k, bdesc + 2u * k, idesc_bf16(N), accum);
+            for (int k = 0; k < 4; ++k) {
+              const uint32_t accum = (chc > 0 || k > 0) ? 1u : 0u;
+              // advance 32 bytes of K inside the 128-byte swizzled row
+              if (mx)
+                umma_mx(dacc, adesc + 2u * k, bdesc + 2u * k, idesc_mx(N, (uint32_t)k), accum,
+                        tbase + PF_SFA_COL + 4u * chc, tbase + PF_SFB_COL + 4u * chc);
+              else
+                umma_bf16(dacc, adesc + 2u * k, bdesc + 2u * k, idesc_bf16(N), accum);
+            }
           }
           tc_commit(&empty[s]);  // the stage returns to the producer once these MMAs are done
         }
