@@ -177,6 +177,33 @@ class Clocks:
 
 
 # ---------------------------------------------------------------------------
+# replicas: the only cross-rank steps are a barrier and two scalar reductions
+# ---------------------------------------------------------------------------
+def rank_barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def rank_reduce(v, world, device, op):
+    """max or sum of a per-rank scalar over the ranks (float64 on `device`)."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
+    return t.item()
+
+
+def replica_gbps(bytes_per_rank, ms_per_rank, world, device):
+    """Whole-job rate of N replicas: the bytes all ranks moved over the slowest rank's time."""
+    ms = rank_reduce(ms_per_rank, world, device, "max")
+    total = rank_reduce(float(bytes_per_rank), world, device, "sum")
+    return total / (ms * 1e-3) / 1e9, ms, total
+
+
+# ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
 def run_ours(args, rank, world, local_rank):
@@ -204,22 +231,13 @@ def run_ours(args, rank, world, local_rank):
     model = DecodeModel(layers=layers, lm_q=lm_q, lm_s=lm_s, top_k=S.k, step_path=1 if args.per_layer else 0)
 
     def barrier():
-        if world > 1:
-            dist.barrier()
+        rank_barrier(world)
 
     def max_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return t.item()
+        return rank_reduce(v, world, dev, "max")
 
     def sum_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.SUM)
-        return t.item()
+        return rank_reduce(v, world, dev, "sum")
 
     K, W = args.steps, args.warmup
     props = torch.cuda.get_device_properties(dev)
