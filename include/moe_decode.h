@@ -109,7 +109,7 @@ MOE_API moe_status_t moe_route(const void* x_bf16, int M, int H, const void* w_r
 /* Routed MXFP4 experts + BF16 shared expert (knowledge card, methods item 1)  */
 /* ------------------------------------------------------------------------- */
 
-/* Bytes of workspace moe_mxfp4_experts needs. */
+/* Bytes of workspace moe_mxfp4_experts needs (0 for an unsupported shape). */
 MOE_API size_t moe_experts_workspace_bytes(int M, int H, int I, int E, int top_k, int Is);
 
 /* One MoE layer for M tokens under a given routing:
@@ -132,7 +132,14 @@ MOE_API size_t moe_experts_workspace_bytes(int M, int H, int I, int E, int top_k
  * out of bounds).  A token listing the same expert twice gives it both weights.
  * Limits: 1 <= M <= 8 (decode / verify windows); H % 64 == 0, 64 <= H <= 4096;
  *         I % 32 == 0, 32 <= I <= 1024; Is % 32 == 0, 0 <= Is <= 1024;
- *         E % 16 == 0, 16 <= E <= 1024; 1 <= top_k <= min(8, E). */
+ *         E % 16 == 0, 16 <= E <= 1024; 1 <= top_k <= min(8, E).
+ * A chunk -- M a multiple of 128, 128 <= M <= 16384 -- takes the prefill chunk's
+ * block-scaled tcgen05 path under the given routing instead: the activations x and
+ * silu(g)*u are quantised to MXFP8 (E4M3 with an E8M0 scale per 32: scale exponent
+ * floor(log2 amax) - 8, clamped to [-127, 127]) before the E2M1 x E4M3 products; shapes
+ * as moe_prefill_layer (H, I multiples of 128 up to 4096; E a multiple of 128 up to 512;
+ * Is a multiple of 64), w13_codes and w2_codes 32-byte aligned, workspace from
+ * moe_experts_workspace_bytes with the same M. */
 MOE_API moe_status_t moe_mxfp4_experts(const void* x_bf16, int M, int H, int I, int E, int top_k,
                                const int32_t* topk_ids, const float* topk_w,
                                const uint8_t* w13_codes, const uint8_t* w13_scales,

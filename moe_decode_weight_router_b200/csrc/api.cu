@@ -310,6 +310,16 @@ moe_status_t check_layer_buf(const moe_buf_t& b, int fmt, bool required) {
   return MOE_OK;
 }
 
+
+// The chunk path (M > MAX_M) of moe_mxfp4_experts, with the prefill machinery below.
+bool ok_pf(int M, int H, int I, int E, int k, int Is);
+size_t pf_ws_bytes(int M, int H, int I, int E, int k, int Is);
+moe_status_t experts_chunk(const void* x_bf16, int M, int H, int I, int E, int top_k, const int32_t* topk_ids,
+                           const float* topk_w, const uint8_t* w13_codes, const uint8_t* w13_scales,
+                           const uint8_t* w2_codes, const uint8_t* w2_scales, const void* shared_w13_bf16,
+                           const void* shared_w2_bf16, int Is, float* y, void* ws, size_t ws_bytes,
+                           moe_stream_t stream);
+
 }  // namespace
 
 extern "C" {
@@ -375,6 +385,7 @@ moe_status_t moe_route(const void* x_bf16, int M, int H, const void* w_router_bf
 }
 
 size_t moe_experts_workspace_bytes(int M, int H, int I, int E, int top_k, int Is) {
+  if (M > MAX_M) return ok_pf(M, H, I, E, top_k, Is) ? pf_ws_bytes(M, H, I, E, top_k, Is) : 0;
   if (!ok_M(M) || !ok_H(H) || !ok_I(I) || !ok_E(E) || !ok_k(top_k, E) || !ok_Is(Is)) return 0;
   return experts_ws(nullptr, M, H, I, E, top_k, Is).bytes;
 }
@@ -385,11 +396,14 @@ moe_status_t moe_mxfp4_experts(const void* x_bf16, int M, int H, int I, int E, i
                                const void* shared_w13_bf16, const void* shared_w2_bf16, int Is, float* y,
                                void* ws, size_t ws_bytes, moe_stream_t stream) {
   REQ(x_bf16 && topk_ids && topk_w && w13_codes && w13_scales && w2_codes && w2_scales && y, MOE_ERR_INVALID_ARG);
-  REQ(ok_M(M) && ok_H(H) && ok_I(I) && ok_E(E) && ok_k(top_k, E) && ok_Is(Is), MOE_ERR_UNSUPPORTED_SHAPE);
   REQ((Is == 0) == (shared_w13_bf16 == nullptr) && (Is == 0) == (shared_w2_bf16 == nullptr), MOE_ERR_INVALID_ARG);
   moe_status_t s = check_ptrs_aligned({x_bf16, topk_ids, topk_w, w13_codes, w13_scales, w2_codes, w2_scales,
                                        shared_w13_bf16, shared_w2_bf16, y, ws});
   if (s != MOE_OK) return s;
+  if (M > MAX_M)  // a chunk: block-scaled tcgen05 GEMMs on MXFP8 activations
+    return experts_chunk(x_bf16, M, H, I, E, top_k, topk_ids, topk_w, w13_codes, w13_scales, w2_codes, w2_scales,
+                         shared_w13_bf16, shared_w2_bf16, Is, y, ws, ws_bytes, stream);
+  REQ(ok_M(M) && ok_H(H) && ok_I(I) && ok_E(E) && ok_k(top_k, E) && ok_Is(Is), MOE_ERR_UNSUPPORTED_SHAPE);
   const size_t need = moe_experts_workspace_bytes(M, H, I, E, top_k, Is);
   REQ(ws && ws_bytes >= need, MOE_ERR_WORKSPACE);
   DevInfo d;
@@ -1021,61 +1035,22 @@ moe_status_t launch_umma(PrefillParams& p, const DevInfo& d, cudaStream_t st) {
   return MOE_OK;
 }
 
-}  // namespace
+size_t pf_ws_bytes(int M, int H, int I, int E, int k, int Is) { return pf_ws(nullptr, M, H, I, E, k, Is).bytes; }
 
-extern "C" {
-
-size_t moe_prefill_workspace_bytes(int M, int H, int I, int E, int top_k, int Is) {
-  if (!ok_pf(M, H, I, E, top_k, Is)) return 0;
-  return pf_ws(nullptr, M, H, I, E, top_k, Is).bytes;
-}
-
-moe_status_t moe_prefill_layer(const void* x_bf16, int M, int H, int I, int E, int top_k, const void* w_router_bf16,
-                               const uint8_t* w13_codes, const uint8_t* w13_scales, const uint8_t* w2_codes,
-                               const uint8_t* w2_scales, const void* shared_w13_bf16, const void* shared_w2_bf16,
-                               int Is, int32_t* topk_ids_opt, float* topk_w_opt, float* logits_opt, float* y,
-                               void* ws, size_t ws_bytes, moe_stream_t stream) {
-  REQ(x_bf16 && w_router_bf16 && w13_codes && w13_scales && w2_codes && w2_scales && y, MOE_ERR_INVALID_ARG);
-  REQ(ok_pf(M, H, I, E, top_k, Is), MOE_ERR_UNSUPPORTED_SHAPE);
-  REQ(Is == 0 || (shared_w13_bf16 && shared_w2_bf16), MOE_ERR_INVALID_ARG);
-  moe_status_t s = check_ptrs_aligned({x_bf16, w_router_bf16, w13_codes, w13_scales, w2_codes, w2_scales,
-                                       shared_w13_bf16, shared_w2_bf16, topk_ids_opt, topk_w_opt, logits_opt, y, ws});
-  if (s != MOE_OK) return s;
-  // the 4-bit tensor-map form reads from 32-byte aligned bases
-  REQ((reinterpret_cast<uintptr_t>(w13_codes) & 31u) == 0 && (reinterpret_cast<uintptr_t>(w2_codes) & 31u) == 0,
-      MOE_ERR_ALIGNMENT);
-  REQ(ws && ws_bytes >= moe_prefill_workspace_bytes(M, H, I, E, top_k, Is), MOE_ERR_WORKSPACE);
-  DevInfo d;
-  if ((s = dev_info(&d)) != MOE_OK) return s;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const PfWs w = pf_ws(ws, M, H, I, E, top_k, Is);
+// a2-a5 of a chunk whose routing (ids, wts [M][top_k], per-expert counts in w.counts) is
+// known: grouped rows per expert, MXFP8 activations, shared expert, routed W13 + SwiGLU,
+// routed W2 into y.  Ids outside [0, E) contribute nothing.
+moe_status_t pf_experts(const __nv_bfloat16* x, int M, int H, int I, int E, int top_k, const int32_t* ids,
+                        const float* wts, const uint8_t* w13_codes, const uint8_t* w13_scales,
+                        const uint8_t* w2_codes, const uint8_t* w2_scales, const void* shared_w13_bf16,
+                        const void* shared_w2_bf16, int Is, float* y, const PfWs& w, const DevInfo& d,
+                        cudaStream_t st) {
+  moe_status_t s = MOE_OK;
   const int G = M * top_k;
-  const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(x_bf16);
-  MOE_CUDA(cudaMemsetAsync(ws, 0, w.clear_bytes, st));
-
-  // a1: router logits (bf16 x bf16 on tcgen05), top-k, softmax over the selected
-  PrefillParams p{};
-  p.status = w.status;
-  p.E = E;
-  p.kc = pf_kc(H, 64);
-  REQ(make_map_halves(&p.tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w_router_bf16, H, E, (uint64_t)H * 2,
-                      (uint64_t)64 * H * 2, 64, 128, p.kc),
-      MOE_ERR_INVALID_ARG);
-  REQ(make_map(&p.tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, H, M, (uint64_t)H * 2, 64, 128, p.kc),
-      MOE_ERR_INVALID_ARG);
-  p.mode = PF_ROUTER;
-  p.K = H;
-  p.m_tiles = E / 128;
-  p.M = M;
-  p.out_f32 = w.logits;
-  p.out_ld = E;
-  if ((s = launch_umma(p, d, st)) != MOE_OK) return s;
-  k_pf_topk<<<(M + 7) / 8, 256, 0, st>>>(w.logits, M, E, top_k, w.ids, w.w, w.counts);
-  MOE_CUDA(cudaGetLastError());
   // a2: grouped rows per expert
   k_pf_scan<<<1, 1024, 0, st>>>(w.counts, E, w.goff, w.ntp, w.fill);
   MOE_CUDA(cudaGetLastError());
-  k_pf_scatter<<<(G + 255) / 256, 256, 0, st>>>(w.ids, w.w, M, top_k, w.goff, w.fill, w.g_tok, w.g_w, w.pos);
+  k_pf_scatter<<<(G + 255) / 256, 256, 0, st>>>(ids, wts, M, top_k, E, w.goff, w.fill, w.g_tok, w.g_w, w.pos);
   MOE_CUDA(cudaGetLastError());
   k_pf_quant_x<<<(int)(((long long)M * (H / 32) + 7) / 8), 256, 0, st>>>(x, M, H, top_k, w.pos, w.xq, w.xs,
                                                                           pf_sf_ld(H));
@@ -1085,11 +1060,12 @@ moe_status_t moe_prefill_layer(const void* x_bf16, int M, int H, int I, int E, i
   if (Is > 0) {
     PrefillParams q{};
     q.status = w.status;
-    q.kc = p.kc;  // K = H as for the router: the token map is shared
+    q.kc = pf_kc(H, 64);
     REQ(make_map_halves(&q.tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, shared_w13_bf16, H, 2 * (uint64_t)Is,
                         (uint64_t)H * 2, (uint64_t)Is * H * 2, 64, 128, q.kc),
         MOE_ERR_INVALID_ARG);
-    q.tmB = p.tmB;
+    REQ(make_map(&q.tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, H, M, (uint64_t)H * 2, 64, 128, q.kc),
+        MOE_ERR_INVALID_ARG);
     q.mode = PF_SH13;
     q.K = H;
     q.m_tiles = Is / 64;
@@ -1167,6 +1143,87 @@ moe_status_t moe_prefill_layer(const void* x_bf16, int M, int H, int I, int E, i
   b.out_f32 = y;
   b.out_ld = H;
   if ((s = launch_umma(b, d, st)) != MOE_OK) return s;
+
+  return MOE_OK;
+}
+
+// Chunk path of moe_mxfp4_experts: the routing is the caller's.
+moe_status_t experts_chunk(const void* x_bf16, int M, int H, int I, int E, int top_k, const int32_t* topk_ids,
+                           const float* topk_w, const uint8_t* w13_codes, const uint8_t* w13_scales,
+                           const uint8_t* w2_codes, const uint8_t* w2_scales, const void* shared_w13_bf16,
+                           const void* shared_w2_bf16, int Is, float* y, void* ws, size_t ws_bytes,
+                           moe_stream_t stream) {
+  REQ(ok_pf(M, H, I, E, top_k, Is), MOE_ERR_UNSUPPORTED_SHAPE);
+  REQ((reinterpret_cast<uintptr_t>(w13_codes) & 31u) == 0 && (reinterpret_cast<uintptr_t>(w2_codes) & 31u) == 0,
+      MOE_ERR_ALIGNMENT);
+  REQ(ws && ws_bytes >= pf_ws(nullptr, M, H, I, E, top_k, Is).bytes, MOE_ERR_WORKSPACE);
+  DevInfo d;
+  moe_status_t s;
+  if ((s = dev_info(&d)) != MOE_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const PfWs w = pf_ws(ws, M, H, I, E, top_k, Is);
+  MOE_CUDA(cudaMemsetAsync(ws, 0, w.clear_bytes, st));
+  const int G = M * top_k;
+  k_pf_count<<<(G + 255) / 256, 256, 0, st>>>(topk_ids, G, E, w.counts);
+  MOE_CUDA(cudaGetLastError());
+  return pf_experts(static_cast<const __nv_bfloat16*>(x_bf16), M, H, I, E, top_k, topk_ids, topk_w, w13_codes,
+                    w13_scales, w2_codes, w2_scales, shared_w13_bf16, shared_w2_bf16, Is, y, w, d, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_prefill_workspace_bytes(int M, int H, int I, int E, int top_k, int Is) {
+  if (!ok_pf(M, H, I, E, top_k, Is)) return 0;
+  return pf_ws(nullptr, M, H, I, E, top_k, Is).bytes;
+}
+
+moe_status_t moe_prefill_layer(const void* x_bf16, int M, int H, int I, int E, int top_k, const void* w_router_bf16,
+                               const uint8_t* w13_codes, const uint8_t* w13_scales, const uint8_t* w2_codes,
+                               const uint8_t* w2_scales, const void* shared_w13_bf16, const void* shared_w2_bf16,
+                               int Is, int32_t* topk_ids_opt, float* topk_w_opt, float* logits_opt, float* y,
+                               void* ws, size_t ws_bytes, moe_stream_t stream) {
+  REQ(x_bf16 && w_router_bf16 && w13_codes && w13_scales && w2_codes && w2_scales && y, MOE_ERR_INVALID_ARG);
+  REQ(ok_pf(M, H, I, E, top_k, Is), MOE_ERR_UNSUPPORTED_SHAPE);
+  REQ(Is == 0 || (shared_w13_bf16 && shared_w2_bf16), MOE_ERR_INVALID_ARG);
+  moe_status_t s = check_ptrs_aligned({x_bf16, w_router_bf16, w13_codes, w13_scales, w2_codes, w2_scales,
+                                       shared_w13_bf16, shared_w2_bf16, topk_ids_opt, topk_w_opt, logits_opt, y, ws});
+  if (s != MOE_OK) return s;
+  // the 4-bit tensor-map form reads from 32-byte aligned bases
+  REQ((reinterpret_cast<uintptr_t>(w13_codes) & 31u) == 0 && (reinterpret_cast<uintptr_t>(w2_codes) & 31u) == 0,
+      MOE_ERR_ALIGNMENT);
+  REQ(ws && ws_bytes >= moe_prefill_workspace_bytes(M, H, I, E, top_k, Is), MOE_ERR_WORKSPACE);
+  DevInfo d;
+  if ((s = dev_info(&d)) != MOE_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const PfWs w = pf_ws(ws, M, H, I, E, top_k, Is);
+  const int G = M * top_k;
+  const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(x_bf16);
+  MOE_CUDA(cudaMemsetAsync(ws, 0, w.clear_bytes, st));
+
+  // a1: router logits (bf16 x bf16 on tcgen05), top-k, softmax over the selected
+  PrefillParams p{};
+  p.status = w.status;
+  p.E = E;
+  p.kc = pf_kc(H, 64);
+  REQ(make_map_halves(&p.tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w_router_bf16, H, E, (uint64_t)H * 2,
+                      (uint64_t)64 * H * 2, 64, 128, p.kc),
+      MOE_ERR_INVALID_ARG);
+  REQ(make_map(&p.tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, H, M, (uint64_t)H * 2, 64, 128, p.kc),
+      MOE_ERR_INVALID_ARG);
+  p.mode = PF_ROUTER;
+  p.K = H;
+  p.m_tiles = E / 128;
+  p.M = M;
+  p.out_f32 = w.logits;
+  p.out_ld = E;
+  if ((s = launch_umma(p, d, st)) != MOE_OK) return s;
+  k_pf_topk<<<(M + 7) / 8, 256, 0, st>>>(w.logits, M, E, top_k, w.ids, w.w, w.counts);
+  MOE_CUDA(cudaGetLastError());
+  if ((s = pf_experts(x, M, H, I, E, top_k, w.ids, w.w, w13_codes, w13_scales, w2_codes, w2_scales,
+                      shared_w13_bf16, shared_w2_bf16, Is, y, w, d, st)) != MOE_OK)
+    return s;
 
   if (topk_ids_opt) MOE_CUDA(cudaMemcpyAsync(topk_ids_opt, w.ids, (size_t)G * 4, cudaMemcpyDeviceToDevice, st));
   if (topk_w_opt) MOE_CUDA(cudaMemcpyAsync(topk_w_opt, w.w, (size_t)G * 4, cudaMemcpyDeviceToDevice, st));

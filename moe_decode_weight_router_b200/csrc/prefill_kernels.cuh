@@ -625,13 +625,27 @@ __global__ void __launch_bounds__(1024) k_pf_scan(const int* __restrict__ counts
   }
 }
 
-// Grouped rows: each (token, selection) gets a slot in its expert's range.
-__global__ void k_pf_scatter(const int32_t* __restrict__ ids, const float* __restrict__ w, int M, int k,
+// Per-expert counts of a routing given by the caller (ids outside [0, E) count for
+// nothing, as in the decode path).
+__global__ void k_pf_count(const int32_t* __restrict__ ids, int n, int E, int* __restrict__ counts) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const int e = ids[i];
+  if (e >= 0 && e < E) atomicAdd(counts + e, 1);
+}
+
+// Grouped rows: each (token, selection) gets a slot in its expert's range (pos -1 for an
+// id outside [0, E)).
+__global__ void k_pf_scatter(const int32_t* __restrict__ ids, const float* __restrict__ w, int M, int k, int E,
                              const int* __restrict__ goff, int* __restrict__ fill, int32_t* __restrict__ g_tok,
                              float* __restrict__ g_w, int32_t* __restrict__ pos) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= M * k) return;
   const int e = ids[i];
+  if (e < 0 || e >= E) {
+    pos[i] = -1;
+    return;
+  }
   const int g = goff[e] + atomicAdd(fill + e, 1);
   g_tok[g] = i / k;
   g_w[g] = w[i];
@@ -655,7 +669,9 @@ __global__ void __launch_bounds__(256) k_pf_quant_x(const __nv_bfloat16* __restr
   const int s = mxfp8_exponent(am);
   const uint8_t q = am == 0.0f ? (uint8_t)0 : e4m3_of(v * exp2i(-s));
   for (int j = 0; j < k; ++j) {
-    const size_t g = (size_t)pos[(size_t)t * k + j];
+    const int gi = pos[(size_t)t * k + j];
+    if (gi < 0) continue;
+    const size_t g = (size_t)gi;
     xq[g * H + 32 * b + lane] = q;
     if (lane == 0) xs[g * xs_ld + b] = (uint8_t)(s + 127);
   }

@@ -93,6 +93,13 @@ def test_experts_validation(lib):
     assert call(H=8192) == 2
     assert call(w2s=A + 8) == 3
     assert call(ws_bytes=need - 1) == 4
+    # a chunk (M a multiple of 128) takes the block-scaled path under the caller's routing
+    chunk = lib.moe_experts_workspace_bytes(2048, 2560, 768, 512, 8, 768)
+    assert chunk == lib.moe_prefill_workspace_bytes(2048, 2560, 768, 512, 8, 768) > 0
+    assert lib.moe_experts_workspace_bytes(200, 2560, 768, 512, 8, 768) == 0
+    assert call(M=200) == 2
+    assert call(M=2048, ws_bytes=chunk - 1) == 4
+    assert call(M=2048, ws_bytes=chunk, w13c=A + 16) == 3   # 32-byte bases for the 4-bit tensor maps
 
 
 def test_prefill_validation(lib):

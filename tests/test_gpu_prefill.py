@@ -13,7 +13,8 @@ import pytest
 import torch
 
 import oracle
-from moe_decode_weight_router_b200 import moe_mxfp8_quantize, moe_prefill_layer, synth, workspace_status
+from moe_decode_weight_router_b200 import (moe_experts_workspace_bytes, moe_mxfp4_experts, moe_mxfp8_quantize,
+                                           moe_prefill_layer, synth, workspace_status)
 from moe_decode_weight_router_b200.binding import moe_prefill_workspace_bytes
 from tests._gpu import MARGIN_FLAG, assert_rows_close, need_gpu
 
@@ -120,3 +121,29 @@ def test_prefill_ling_chunk():
     toks = np.array(sorted(sample))
     ref = oracle.moe_layer_prefill(synth.bits(x), ids, w.astype(np.float64), _fetch(L), _shared(L), toks)
     assert_rows_close(y[toks], ref, what="prefill layer output (Ling)")
+
+
+def test_experts_chunk_under_given_routing():
+    # moe_mxfp4_experts with M a multiple of 128: the caller's routing (distinct random
+    # experts per token, random positive weights, two ids outside [0, E) that must add
+    # nothing) through the block-scaled path; every token row against the oracle
+    M = 256
+    L = synth.layer(SMALL, 9, device="cuda")
+    x = synth.tokens(M, SMALL.H, 9, device="cuda")
+    rng = np.random.default_rng(9)
+    ids = np.stack([rng.choice(SMALL.E, SMALL.k, replace=False) for _ in range(M)]).astype(np.int32)
+    w = rng.uniform(0.05, 1.0, size=(M, SMALL.k)).astype(np.float32)
+    ids[5, 2] = -1
+    ids[7, 0] = SMALL.E
+    ws = torch.empty(moe_experts_workspace_bytes(M, SMALL.H, SMALL.I, SMALL.E, SMALL.k, SMALL.Is),
+                     dtype=torch.uint8, device="cuda")
+    y = moe_mxfp4_experts(x, torch.from_numpy(ids).cuda(), torch.from_numpy(w).cuda(), L["w13c"], L["w13s"],
+                          L["w2c"], L["w2s"], L["sw13"], L["sw2"], ws=ws)
+    torch.cuda.synchronize()
+    assert workspace_status(ws) == 0
+    ids_o, w_o = ids.copy(), w.astype(np.float64)
+    bad = (ids_o < 0) | (ids_o >= SMALL.E)
+    ids_o[bad] = 0
+    w_o[bad] = 0.0
+    ref = oracle.moe_layer_prefill(synth.bits(x), ids_o, w_o, _fetch(L), _shared(L), np.arange(M))
+    assert_rows_close(y.cpu().numpy(), ref, what="experts chunk under given routing")
