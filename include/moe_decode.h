@@ -277,10 +277,11 @@ enum { MOE_STEP_AUTO = 0, MOE_STEP_PER_LAYER = 1 };
  *   ids [L][M][top_k] int32, w [L][M][top_k] fp32: each layer's routing
  *   events: NULL or an array of n_events cudaEvent_t handles (host array, created by
  *     the caller) recorded on the step's stream around every kernel: events[2i] before
- *     and events[2i+1] after launch i, launches ordered (router+shared W13, routed W13,
- *     W2+combine) per layer, then the final RMSNorm, then the LM head; 3L+2 launches.
- *     Fewer events than 2 x (launch count) record the first n_events/2 launches only
- *     (decode_step_launch_names gives the launches).
+ *     and events[2i+1] after launch i, in the order decode_step_launch_names gives: the
+ *     persistent kernel then the LM head (2 launches), or on the per-layer path (router +
+ *     shared W13, routed W13, W2 + combine) per layer, the final RMSNorm and the LM head
+ *     (3L+2 launches).  Fewer events than 2 x (launch count) record the first
+ *     n_events/2 launches only.
  *   timeline: NULL or [2*L*16 + 4*4096] uint64 %globaltimer stamps (ns), for profiling
  *     the persistent path: [2][L][16] phase boundaries of blocks 0 and G-1, then block 0's
  *     first 2048 weight items, 8 stamps each (window acquired, data ready, done, wait
@@ -317,8 +318,9 @@ MOE_API moe_status_t decode_step(const moe_model_t* model, const void* x_bf16, i
                          int32_t* argmax, const moe_trace_t* trace_opt, void* ws,
                          size_t ws_bytes, moe_stream_t stream);
 
-/* A whole decode step captured once as a CUDA graph (about 3 launches per layer),
- * replayed with a single launch.  The graph binds the given x, logits, argmax and
+/* A whole decode step captured once as a CUDA graph (the workspace clear and the
+ * step's kernels: 2 on the persistent path, 3L+2 on the per-layer one), replayed with
+ * a single launch.  The graph binds the given x, logits, argmax and
  * workspace pointers: refill x in place between launches.  The handle is a small
  * host object owned by the caller (decode_step_graph_destroy); no device memory is
  * allocated.  The model's buffers must stay valid while the handle lives. */
