@@ -1109,7 +1109,6 @@ moe_status_t pf_experts(const __nv_bfloat16* x, int M, int H, int I, int E, int 
   a.E = E;
   a.ntile_prefix = w.ntp;
   a.goff = w.goff;
-  a.a_codes = w13_codes;
   a.sfa = w13_scales;
   a.sfb = w.xs;
   a.sf_ld = pf_sf_ld(H);
@@ -1136,7 +1135,6 @@ moe_status_t pf_experts(const __nv_bfloat16* x, int M, int H, int I, int E, int 
   b.goff = w.goff;
   b.g_tok = w.g_tok;
   b.g_w = w.g_w;
-  b.a_codes = w2_codes;
   b.sfa = w2_scales;
   b.sfb = w.aqs;
   b.sf_ld = pf_sf_ld(I);

@@ -61,7 +61,6 @@ struct alignas(64) PrefillParams {
   int prob_rows; // weight rows per problem (expert) for the routed modes
   int M;         // dense modes: tokens
   int E;
-  const uint8_t* a_codes;   // routed: the weight codes the tensor map covers (L2 prefetch of the next tile)
   const int* ntile_prefix;  // routed: [E+1] prefix sums of ceil(n_e / 128)
   const int* goff;          // routed: [E+1] first grouped row of each expert
   const int32_t* g_tok;     // routed: [G] token of each grouped row
@@ -135,9 +134,6 @@ __device__ __forceinline__ void umma_mx(uint32_t d, uint64_t adesc, uint64_t bde
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc), "r"(tsfa), "r"(tsfb)
       : "memory");
 }
-__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar) {
   asm volatile(
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
@@ -151,13 +147,6 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, i
       "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], "
       "[%6];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar))
-      : "memory");
-}
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
-          smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
       : "memory");
 }
 // K-major operand, 128-byte swizzle: start >> 4, LBO 1 (unused when swizzled), SBO 1024 B
