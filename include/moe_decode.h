@@ -282,10 +282,13 @@ enum { MOE_STEP_AUTO = 0, MOE_STEP_PER_LAYER = 1 };
  *     shared W13, routed W13, W2 + combine) per layer, the final RMSNorm and the LM head
  *     (3L+2 launches).  Fewer events than 2 x (launch count) record the first
  *     n_events/2 launches only.
- *   timeline: NULL or [2*L*16 + 4*4096] uint64 %globaltimer stamps (ns), for profiling
- *     the persistent path: [2][L][16] phase boundaries of blocks 0 and G-1, then block 0's
- *     first 2048 weight items, 8 stamps each (window acquired, data ready, done, wait
- *     started, producer entered, copies issued, 2 unused). */
+ *   timeline: NULL or [2*L*16 + 4*4096 + G*L*16] uint64 %globaltimer stamps (ns), G the
+ *     device's SM count, for profiling the persistent path: [2][L][16] phase boundaries of
+ *     blocks 0 and G-1, then block 0's first 2048 weight items, 8 stamps each (window
+ *     acquired, data ready, done, wait started, producer entered, copies issued, 2 unused),
+ *     then [G][L][16] phase ends of every block (residual seen, input staged, router item
+ *     published, router/shared-W13 items done, plan built, shared W2 done, routed W13
+ *     done, routed W2 done, then finer marks inside the top-k and the staging). */
 typedef struct {
   void* x;
   float* h;

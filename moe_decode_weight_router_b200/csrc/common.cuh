@@ -57,6 +57,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// As mbar_try_wait, but the thread may be suspended in hardware for up to ns
+// nanoseconds until the phase completes, instead of spinning.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
 // Wait for the phase with the given parity to complete.  Bounded: after
 // WAIT_LIMIT_NS it records DEV_ERR_TIMEOUT in *status and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status) {
@@ -160,13 +173,25 @@ __device__ __forceinline__ float fma_bf16_hi(uint32_t a2, uint32_t b2, float c) 
 }
 
 // Power-of-two exponent p with amax * 2^p in [2^14, 2^15): moves a row into the
-// f16 range without touching its significands.  0 for amax == 0.
+// f16 range without touching its significands.  0 for amax == 0 or not finite.
+// Every positive finite fp32 amax gives p in [-113, 163].
 __device__ __forceinline__ int f16_range_shift(float amax) {
-  if (!(amax > 0.0f) || !(amax < 3.0e38f)) return 0;
+  if (!(amax > 0.0f) || !(amax <= 3.4028235e38f)) return 0;
   int e;
   (void)frexpf(amax, &e);  // amax = f 2^e, f in [0.5, 1): floor(log2 amax) = e - 1
-  int p = 14 - (e - 1);
-  return p < -100 ? -100 : (p > 100 ? 100 : p);
+  return 14 - (e - 1);
+}
+// v * 2^k for |k| <= 252 as two exact power-of-two multiplications (each factor is a
+// normal fp32 number): exact unless the result itself leaves the fp32 range.
+__device__ __forceinline__ float mul_pow2(float v, int k) {
+  const int k1 = k / 2;
+  return (v * exp2i(k1)) * exp2i(k - k1);
+}
+// 2^d as fp32: exact for d in [-149, 127] (subnormal below -126), 0 below, 2^127 above.
+__device__ __forceinline__ float pow2_clamped(int d) {
+  if (d > 127) d = 127;
+  if (d >= -126) return __uint_as_float(static_cast<uint32_t>(d + 127) << 23);
+  return d >= -149 ? __uint_as_float(1u << (d + 149)) : 0.0f;
 }
 
 // ---------------------------------------------------------------------------

@@ -342,12 +342,12 @@ __global__ void __launch_bounds__(DENSE_THREADS) k_dense(DenseParams p) {
 // ---------------------------------------------------------------------------
 // Shared pieces of the streamed expert kernels
 // ---------------------------------------------------------------------------
-// f16 copy of x scaled per token by a power of two (exact), for the f16 tensor-core
-// operand; inv[t] undoes the scaling.  Run by the NC consumer warps.
+// f16 copy of x scaled per token by a power of two (exact), for the f16 products;
+// shift[t] receives token t's exponent sh (x_t * 2^sh has its largest magnitude in
+// [2^14, 2^15)).  Run by the N_CONSUMERS consumer warps.
 __device__ __forceinline__ void stage_x_f16(const __nv_bfloat16* x, int M, int H, uint8_t* xs, uint32_t xss,
-                                            float* inv) {
+                                            int* shift) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  __shared__ int s_shift[MAX_M];
   for (int tok = warp; tok < MAX_M; tok += N_CONSUMERS) {
     float amax = 0.0f;
     if (tok < M)
@@ -359,11 +359,7 @@ __device__ __forceinline__ void stage_x_f16(const __nv_bfloat16* x, int M, int H
       }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    if (lane == 0) {
-      const int sh = f16_range_shift(amax);
-      s_shift[tok] = sh;
-      inv[tok] = exp2i(-sh);
-    }
+    if (lane == 0) shift[tok] = f16_range_shift(amax);
   }
   named_barrier(1, 32 * N_CONSUMERS);
   for (int i = tid; i < MAX_M * (H / 8); i += 32 * N_CONSUMERS) {
@@ -371,12 +367,12 @@ __device__ __forceinline__ void stage_x_f16(const __nv_bfloat16* x, int M, int H
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
     if (tok < M) {
       v = *reinterpret_cast<const uint4*>(x + (size_t)tok * H + 8 * c);
-      const float sc = exp2i(s_shift[tok]);
+      const int sh = shift[tok];
       uint32_t* w = reinterpret_cast<uint32_t*>(&v);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&w[j]);
-        const __half2 hh = __floats2half2_rn(__low2float(b) * sc, __high2float(b) * sc);
+        const __half2 hh = __floats2half2_rn(mul_pow2(__low2float(b), sh), mul_pow2(__high2float(b), sh));
         w[j] = *reinterpret_cast<const uint32_t*>(&hh);
       }
     }
@@ -385,30 +381,55 @@ __device__ __forceinline__ void stage_x_f16(const __nv_bfloat16* x, int M, int H
   named_barrier(1, 32 * N_CONSUMERS);
 }
 
-// Largest E8M0 scale byte of a row, for rows g and g+8 (the 4 lanes of a lane
-// group split the row's bytes and combine with two shuffles).
-__device__ __forceinline__ void row_scale_max(const uint8_t* sc_g, const uint8_t* sc_g8, int nb, uint32_t& mg,
-                                              uint32_t& mg8) {
+// Largest and smallest E8M0 scale byte of rows g and g+8 (the 4 lanes of a lane group
+// split the row's bytes, 32-bit words when the row allows, and combine with two
+// shuffles).  Every lane of group g returns its rows' values.
+__device__ __forceinline__ void row_scale_range(const uint8_t* sc_g, const uint8_t* sc_g8, int nb, uint32_t& mx_g,
+                                                uint32_t& mx_g8, uint32_t& mn_g, uint32_t& mn_g8) {
   const int t = threadIdx.x & 3;
-  uint32_t a = 0u, b = 0u;
-  for (int i = t; i < nb; i += 4) {
-    a = max(a, (uint32_t)sc_g[i]);
-    b = max(b, (uint32_t)sc_g8[i]);
+  uint32_t a = 0u, b = 0u, c = 0xFFFFFFFFu, d = 0xFFFFFFFFu;
+  if ((nb & 3) == 0 && ((reinterpret_cast<uintptr_t>(sc_g) | reinterpret_cast<uintptr_t>(sc_g8)) & 3u) == 0) {
+    const uint32_t* ga = reinterpret_cast<const uint32_t*>(sc_g);
+    const uint32_t* gb = reinterpret_cast<const uint32_t*>(sc_g8);
+    for (int i = t; i < nb / 4; i += 4) {
+      const uint32_t wa = ga[i], wb = gb[i];
+      a = __vmaxu4(a, wa);
+      b = __vmaxu4(b, wb);
+      c = __vminu4(c, wa);
+      d = __vminu4(d, wb);
+    }
+  } else {
+    for (int i = t; i < nb; i += 4) {
+      const uint32_t wa = sc_g[i] * 0x01010101u, wb = sc_g8[i] * 0x01010101u;
+      a = __vmaxu4(a, wa);
+      b = __vmaxu4(b, wb);
+      c = __vminu4(c, wa);
+      d = __vminu4(d, wb);
+    }
   }
-  a = max(a, __shfl_xor_sync(0xffffffffu, a, 1));
-  b = max(b, __shfl_xor_sync(0xffffffffu, b, 1));
-  a = max(a, __shfl_xor_sync(0xffffffffu, a, 2));
-  b = max(b, __shfl_xor_sync(0xffffffffu, b, 2));
-  mg = a;
-  mg8 = b;
+#pragma unroll
+  for (int o = 1; o <= 2; o <<= 1) {
+    a = __vmaxu4(a, __shfl_xor_sync(0xffffffffu, a, o));
+    b = __vmaxu4(b, __shfl_xor_sync(0xffffffffu, b, o));
+    c = __vminu4(c, __shfl_xor_sync(0xffffffffu, c, o));
+    d = __vminu4(d, __shfl_xor_sync(0xffffffffu, d, o));
+  }
+  mx_g = max(max(a & 0xFFu, (a >> 8) & 0xFFu), max((a >> 16) & 0xFFu, a >> 24));
+  mx_g8 = max(max(b & 0xFFu, (b >> 8) & 0xFFu), max((b >> 16) & 0xFFu, b >> 24));
+  mn_g = min(min(c & 0xFFu, (c >> 8) & 0xFFu), min((c >> 16) & 0xFFu, c >> 24));
+  mn_g8 = min(min(d & 0xFFu, (d >> 8) & 0xFFu), min((d >> 16) & 0xFFu, d >> 24));
 }
 
-// f16x2 of 2^d in both halves, d = e - ref <= 0: normal for d >= -14, subnormal
-// down to 2^-24, 0 below.  Exact wherever it is not 0.
+// f16x2 of 2^d in both halves, d = e - ref in [-23, 0]: normal for d >= -14,
+// subnormal below.  Every E2M1 value times 2^d is then an exact f16 number (its
+// lowest set bit is 2^(d-1) >= 2^-24, the f16 subnormal step).
 __device__ __forceinline__ uint32_t pow2_f16x2(int d) {
   uint32_t b = d >= -14 ? (uint32_t)(d + 15) << 10 : (d >= -24 ? 1u << (d + 24) : 0u);
   return b | (b << 16);
 }
+// Largest scale span (row maximum minus row minimum exponent) over which folding the
+// block scales into the f16 codes, relative to the row maximum, stays exact.
+constexpr int FOLD_SPAN = 23;
 
 __device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
   uint32_t r;
@@ -416,42 +437,29 @@ __device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
   return r;
 }
 
+// Activations of the MXFP4 products are f16 rows scaled per token by 2^sh (sh from
+// f16_range_shift of the row's largest magnitude): the tile products below return
+// results in the true units, the shift undone together with the weight scales.
+
 // The warp's 16 x K MXFP4 tile (rows g and g+8 of each lane group) against up to 8
-// token columns.  Thread (g, t) owns scale block 4q+t of both rows: its 32 codes per
-// row widen to f16 with the hardware e2m1x2 conversion and are multiplied by
-// 2^(e - e_ref) with e_ref the row's largest scale -- an exact power-of-two
-// rescaling (blocks more than 2^23 below the row maximum flush to zero: an error
-// below 2^-20 of the row's largest block).  Every MMA column is then one token and
-// the fp32 accumulators run over the whole row; 2^(e_ref - 127) is applied at the
-// end.  c[]: c0 (row g, token 2t), c1 (row g, token 2t+1), c2 (row g+8, token 2t),
+// token columns on the warp tensor core.  Thread (g, t) owns scale block 4q+t of both
+// rows: its 32 codes per row widen to f16 with the hardware e2m1x2 conversion and are
+// multiplied by 2^(e - e_ref) with e_ref the row's largest scale -- exact because the
+// caller only takes this path when every row's scale span is at most FOLD_SPAN.  Every
+// MMA column is one token and the fp32 accumulators run over the whole row; the factor
+// 2^(e_ref - 127 - sh_token) is applied once at the end (ldexpf: exact, any range).
+// c[]: c0 (row g, token 2t), c1 (row g, token 2t+1), c2 (row g+8, token 2t),
 // c3 (row g+8, token 2t+1).  Tokens >= M read zeros.
 //   codes_g/codes_g8: row g / row g+8 codes in shared memory; sc_g/sc_g8: their scales
-//   xb: f16 activation rows (stride xss bytes), token n at xb + n*xss
-// Latency: the next group's codes and scales are loaded while this group computes;
-// each group issues its 32 conversions back to back, then 8 MMAs into 4 accumulators.
+//   xb: f16 activation rows (stride xss bytes), token n at xb + n*xss, shift xsh[n]
 // Rows with a multiple of 8 scale blocks (every Ling-shaped tile): two groups per
-// iteration into eight accumulators, the scale maxima from 32-bit words.
+// iteration into eight accumulators.
 __device__ __forceinline__ void mxfp4_tile_dot_x2(const uint8_t* codes_g, const uint8_t* codes_g8,
                                                   const uint8_t* sc_g, const uint8_t* sc_g8, int nb,
-                                                  const uint8_t* xb, uint32_t xss, int M, float (&c)[4]) {
+                                                  const uint8_t* xb, uint32_t xss, int M, uint32_t ref_g,
+                                                  uint32_t ref_g8, float (&acc_out)[4]) {
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
-  uint32_t ref_g, ref_g8;
-  {
-    uint32_t a = 0u, b = 0u;
-    const uint32_t* ga = reinterpret_cast<const uint32_t*>(sc_g);
-    const uint32_t* gb = reinterpret_cast<const uint32_t*>(sc_g8);
-    for (int i = t; i < nb / 4; i += 4) {
-      a = __vmaxu4(a, ga[i]);
-      b = __vmaxu4(b, gb[i]);
-    }
-    a = __vmaxu4(a, __shfl_xor_sync(0xffffffffu, a, 1));
-    b = __vmaxu4(b, __shfl_xor_sync(0xffffffffu, b, 1));
-    a = __vmaxu4(a, __shfl_xor_sync(0xffffffffu, a, 2));
-    b = __vmaxu4(b, __shfl_xor_sync(0xffffffffu, b, 2));
-    ref_g = max(max(a & 0xFFu, (a >> 8) & 0xFFu), max((a >> 16) & 0xFFu, a >> 24));
-    ref_g8 = max(max(b & 0xFFu, (b >> 8) & 0xFFu), max((b >> 16) & 0xFFu, b >> 24));
-  }
   const bool xact = g < M;
   const uint8_t* xrow = xb + g * xss;
   float acc[8][4];
@@ -494,77 +502,20 @@ __device__ __forceinline__ void mxfp4_tile_dot_x2(const uint8_t* codes_g, const 
       }
     }
   }
-  const float r0 = e8m0_to_f32(ref_g), r1 = e8m0_to_f32(ref_g8);
 #pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    const float sum = ((acc[0][e] + acc[1][e]) + (acc[2][e] + acc[3][e])) + ((acc[4][e] + acc[5][e]) + (acc[6][e] + acc[7][e]));
-    c[e] = sum * (e < 2 ? r0 : r1);
-  }
+  for (int e = 0; e < 4; ++e)
+    acc_out[e] = ((acc[0][e] + acc[1][e]) + (acc[2][e] + acc[3][e])) + ((acc[4][e] + acc[5][e]) + (acc[6][e] + acc[7][e]));
 }
 
-// One token (M = 1) on the CUDA cores: a single activation column leaves 7/8 of each
-// m16n8k16 product idle, so thread (g, t) instead multiplies its blocks t, t+4, ... of
-// rows g and g+8 against the token directly -- codes widened to f16 pairs as above,
-// exact f16 x f16 products summed in fp32 per block, the block's E8M0 scale applied as
-// an exact power of two.  The four t lanes then sum their partials, so every lane of
-// group g returns c0 = row g, c2 = row g+8 (c1 = c3 = 0: there is no second token).
-__device__ __forceinline__ void mxfp4_tile_dot_m1(const uint8_t* codes_g, const uint8_t* codes_g8,
+// Any row shape: one group per iteration, the next group's codes and scales loaded
+// while this one computes.  Same contract as mxfp4_tile_dot_x2.
+__device__ __forceinline__ void mxfp4_tile_dot_x1(const uint8_t* codes_g, const uint8_t* codes_g8,
                                                   const uint8_t* sc_g, const uint8_t* sc_g8, int nb,
-                                                  const uint8_t* xb, float (&c)[4]) {
-  const int t = threadIdx.x & 3;
-  float a0 = 0.0f, a1 = 0.0f;
-#pragma unroll 2
-  for (int b = t; b < nb; b += 4) {
-    const uint4 X0 = lds128(xb + 64 * b), X1 = lds128(xb + 64 * b + 16);
-    const uint4 X2 = lds128(xb + 64 * b + 32), X3 = lds128(xb + 64 * b + 48);
-    const uint32_t xw[16] = {X0.x, X0.y, X0.z, X0.w, X1.x, X1.y, X1.z, X1.w,
-                             X2.x, X2.y, X2.z, X2.w, X3.x, X3.y, X3.z, X3.w};
-    const uint4 C0 = lds128(codes_g + 16 * b), C1 = lds128(codes_g8 + 16 * b);
-    const float f0 = e8m0_to_f32(sc_g[b]), f1 = e8m0_to_f32(sc_g8[b]);
-    const uint32_t w0[4] = {C0.x, C0.y, C0.z, C0.w}, w1[4] = {C1.x, C1.y, C1.z, C1.w};
-    uint32_t h0[16], h1[16];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      e2m1x8_to_f16x2(w0[k], h0[4 * k], h0[4 * k + 1], h0[4 * k + 2], h0[4 * k + 3]);
-      e2m1x8_to_f16x2(w1[k], h1[4 * k], h1[4 * k + 1], h1[4 * k + 2], h1[4 * k + 3]);
-    }
-    float p0 = 0.0f, p1 = 0.0f, p2 = 0.0f, p3 = 0.0f;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      p0 = fma_f16_lo(h0[j], xw[j], p0);
-      p1 = fma_f16_hi(h0[j], xw[j], p1);
-      p2 = fma_f16_lo(h1[j], xw[j], p2);
-      p3 = fma_f16_hi(h1[j], xw[j], p3);
-    }
-    a0 = fmaf(p0 + p1, f0, a0);
-    a1 = fmaf(p2 + p3, f1, a1);
-  }
-  a0 += __shfl_xor_sync(0xffffffffu, a0, 1);
-  a1 += __shfl_xor_sync(0xffffffffu, a1, 1);
-  a0 += __shfl_xor_sync(0xffffffffu, a0, 2);
-  a1 += __shfl_xor_sync(0xffffffffu, a1, 2);
-  c[0] = a0;
-  c[1] = 0.0f;
-  c[2] = a1;
-  c[3] = 0.0f;
-}
-
-__device__ __forceinline__ void mxfp4_tile_dot(const uint8_t* codes_g, const uint8_t* codes_g8,
-                                               const uint8_t* sc_g, const uint8_t* sc_g8, int nb,
-                                               const uint8_t* xb, uint32_t xss, int M, float (&c)[4]) {
-  if (M == 1) {
-    mxfp4_tile_dot_m1(codes_g, codes_g8, sc_g, sc_g8, nb, xb, c);
-    return;
-  }
-  if ((nb & 7) == 0 && ((reinterpret_cast<uintptr_t>(sc_g) | reinterpret_cast<uintptr_t>(sc_g8)) & 3u) == 0) {
-    mxfp4_tile_dot_x2(codes_g, codes_g8, sc_g, sc_g8, nb, xb, xss, M, c);
-    return;
-  }
+                                                  const uint8_t* xb, uint32_t xss, int M, uint32_t ref_g,
+                                                  uint32_t ref_g8, float (&acc_out)[4]) {
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const int nq = (nb + 3) / 4;
   const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
-  uint32_t ref_g, ref_g8;
-  row_scale_max(sc_g, sc_g8, nb, ref_g, ref_g8);
   const bool xact = g < M;
   const uint8_t* xrow = xb + g * xss;
   float acc[4][4];
@@ -576,8 +527,8 @@ __device__ __forceinline__ void mxfp4_tile_dot(const uint8_t* codes_g, const uin
     const bool v = t < nb;
     nA0 = v ? lds128(codes_g + 16 * t) : zero;
     nA1 = v ? lds128(codes_g8 + 16 * t) : zero;
-    ns0 = v ? sc_g[t] : 0u;
-    ns1 = v ? sc_g8[t] : 0u;
+    ns0 = v ? sc_g[t] : ref_g;
+    ns1 = v ? sc_g8[t] : ref_g8;
   }
   for (int q = 0; q < nq; ++q) {
     const uint4 A0 = nA0, A1 = nA1;
@@ -588,8 +539,8 @@ __device__ __forceinline__ void mxfp4_tile_dot(const uint8_t* codes_g, const uin
       const bool v = b2 < nb;
       nA0 = v ? lds128(codes_g + 16 * b2) : zero;
       nA1 = v ? lds128(codes_g8 + 16 * b2) : zero;
-      ns0 = v ? sc_g[b2] : 0u;
-      ns1 = v ? sc_g8[b2] : 0u;
+      ns0 = v ? sc_g[b2] : ref_g;
+      ns1 = v ? sc_g8[b2] : ref_g8;
     }
     const bool valid = beta < nb;
     uint4 X[4];
@@ -615,11 +566,148 @@ __device__ __forceinline__ void mxfp4_tile_dot(const uint8_t* codes_g, const uin
       mma_f16(acc[wd], h[4 * wd + 2], k[4 * wd + 2], h[4 * wd + 3], k[4 * wd + 3], X[wd].z, X[wd].w);
     }
   }
-  const float r0 = e8m0_to_f32(ref_g), r1 = e8m0_to_f32(ref_g8);
-  c[0] = ((acc[0][0] + acc[1][0]) + (acc[2][0] + acc[3][0])) * r0;
-  c[1] = ((acc[0][1] + acc[1][1]) + (acc[2][1] + acc[3][1])) * r0;
-  c[2] = ((acc[0][2] + acc[1][2]) + (acc[2][2] + acc[3][2])) * r1;
-  c[3] = ((acc[0][3] + acc[1][3]) + (acc[2][3] + acc[3][3])) * r1;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) acc_out[e] = (acc[0][e] + acc[1][e]) + (acc[2][e] + acc[3][e]);
+}
+
+// One token on the CUDA cores: a single activation column leaves 7/8 of each m16n8k16
+// product idle, so thread (g, t) instead multiplies its blocks t, t+4, ... of rows g
+// and g+8 against the token directly -- codes widened to f16 pairs as above, exact
+// f16 x f16 products summed in fp32 per block, then the block's factor
+// 2^(e - 127 - sh) applied in fp32.  FAST: the caller has checked that every block's
+// e - sh lies in [1, 254], so the factor is the normal number with exponent byte e - sh;
+// otherwise each factor is built clamped (exact down to 2^-149, the only losses being
+// block contributions outside the fp32 range).  The four t lanes then sum their
+// partials, so every lane of group g returns a0 = row g, a1 = row g+8.
+template <bool FAST>
+__device__ __forceinline__ void mxfp4_rows_m1(const uint8_t* codes_g, const uint8_t* codes_g8, const uint8_t* sc_g,
+                                              const uint8_t* sc_g8, int nb, const uint8_t* xb, int sh, float& r0,
+                                              float& r1) {
+  const int t = threadIdx.x & 3;
+  float a0 = 0.0f, a1 = 0.0f;
+#pragma unroll 2
+  for (int b = t; b < nb; b += 4) {
+    const uint4 X0 = lds128(xb + 64 * b), X1 = lds128(xb + 64 * b + 16);
+    const uint4 X2 = lds128(xb + 64 * b + 32), X3 = lds128(xb + 64 * b + 48);
+    const uint32_t xw[16] = {X0.x, X0.y, X0.z, X0.w, X1.x, X1.y, X1.z, X1.w,
+                             X2.x, X2.y, X2.z, X2.w, X3.x, X3.y, X3.z, X3.w};
+    const uint4 C0 = lds128(codes_g + 16 * b), C1 = lds128(codes_g8 + 16 * b);
+    float f0, f1;
+    if (FAST) {
+      f0 = __uint_as_float((uint32_t)((int)sc_g[b] - sh) << 23);
+      f1 = __uint_as_float((uint32_t)((int)sc_g8[b] - sh) << 23);
+    } else {
+      f0 = pow2_clamped((int)sc_g[b] - 127 - sh);
+      f1 = pow2_clamped((int)sc_g8[b] - 127 - sh);
+    }
+    const uint32_t w0[4] = {C0.x, C0.y, C0.z, C0.w}, w1[4] = {C1.x, C1.y, C1.z, C1.w};
+    uint32_t h0[16], h1[16];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      e2m1x8_to_f16x2(w0[k], h0[4 * k], h0[4 * k + 1], h0[4 * k + 2], h0[4 * k + 3]);
+      e2m1x8_to_f16x2(w1[k], h1[4 * k], h1[4 * k + 1], h1[4 * k + 2], h1[4 * k + 3]);
+    }
+    float p0 = 0.0f, p1 = 0.0f, p2 = 0.0f, p3 = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      p0 = fma_f16_lo(h0[j], xw[j], p0);
+      p1 = fma_f16_hi(h0[j], xw[j], p1);
+      p2 = fma_f16_lo(h1[j], xw[j], p2);
+      p3 = fma_f16_hi(h1[j], xw[j], p3);
+    }
+    a0 = fmaf(p0 + p1, f0, a0);
+    a1 = fmaf(p2 + p3, f1, a1);
+  }
+  a0 += __shfl_xor_sync(0xffffffffu, a0, 1);
+  a1 += __shfl_xor_sync(0xffffffffu, a1, 1);
+  a0 += __shfl_xor_sync(0xffffffffu, a0, 2);
+  a1 += __shfl_xor_sync(0xffffffffu, a1, 2);
+  r0 = a0;
+  r1 = a1;
+}
+
+// The clamped-factor rows (rare: block exponents outside the fast range), out of line.
+__device__ __noinline__ void mxfp4_rows_m1_safe(const uint8_t* codes_g, const uint8_t* codes_g8, const uint8_t* sc_g,
+                                                const uint8_t* sc_g8, int nb, const uint8_t* xb, int sh, float& r0,
+                                                float& r1) {
+  mxfp4_rows_m1<false>(codes_g, codes_g8, sc_g, sc_g8, nb, xb, sh, r0, r1);
+}
+// A window tile whose rows span more than FOLD_SPAN scale exponents: exact per-block
+// fp32 scaling, one token at a time (rare; out of line).
+__device__ __noinline__ void mxfp4_tile_dot_wide(const uint8_t* codes_g, const uint8_t* codes_g8, const uint8_t* sc_g,
+                                                 const uint8_t* sc_g8, int nb, const uint8_t* xb, uint32_t xss, int M,
+                                                 const int* xsh, float* c) {
+  const int t = threadIdx.x & 3;
+  c[0] = c[1] = c[2] = c[3] = 0.0f;
+  for (int m = 0; m < M; ++m) {
+    float r0, r1;
+    mxfp4_rows_m1<false>(codes_g, codes_g8, sc_g, sc_g8, nb, xb + m * xss, xsh[m], r0, r1);
+    if (m == 2 * t) {
+      c[0] = r0;
+      c[2] = r1;
+    } else if (m == 2 * t + 1) {
+      c[1] = r0;
+      c[3] = r1;
+    }
+  }
+}
+
+// A window (M >= 2) tile on the warp tensor core; see mxfp4_tile_dot.
+__device__ __forceinline__ void mxfp4_tile_dot_win(const uint8_t* codes_g, const uint8_t* codes_g8,
+                                                   const uint8_t* sc_g, const uint8_t* sc_g8, int nb,
+                                                   const uint8_t* xb, uint32_t xss, int M, const int* xsh,
+                                                   float (&c)[4]) {
+  const int t = threadIdx.x & 3;
+  uint32_t mx_g, mx_g8, mn_g, mn_g8;
+  row_scale_range(sc_g, sc_g8, nb, mx_g, mx_g8, mn_g, mn_g8);
+  const bool fold = __all_sync(0xffffffffu, (int)(mx_g - mn_g) <= FOLD_SPAN && (int)(mx_g8 - mn_g8) <= FOLD_SPAN);
+  if (!fold) {
+    mxfp4_tile_dot_wide(codes_g, codes_g8, sc_g, sc_g8, nb, xb, xss, M, xsh, c);
+    return;
+  }
+  float acc[4];
+  if ((nb & 7) == 0 && ((reinterpret_cast<uintptr_t>(sc_g) | reinterpret_cast<uintptr_t>(sc_g8)) & 3u) == 0)
+    mxfp4_tile_dot_x2(codes_g, codes_g8, sc_g, sc_g8, nb, xb, xss, M, mx_g, mx_g8, acc);
+  else
+    mxfp4_tile_dot_x1(codes_g, codes_g8, sc_g, sc_g8, nb, xb, xss, M, mx_g, mx_g8, acc);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int tok = 2 * t + (e & 1);
+    const int ref = (int)(e < 2 ? mx_g : mx_g8);
+    c[e] = tok < M ? ldexpf(acc[e], ref - 127 - xsh[tok]) : 0.0f;
+  }
+}
+
+// The warp's 16-row MXFP4 tile (rows g and g+8 of each lane group, nb scale blocks of
+// 32) against M <= 8 f16 activation rows xb (stride xss, token n scaled by 2^xsh[n]).
+// Returns the products in true units, c as the m16n8 C layout: c0 (row g, token 2t),
+// c1 (row g, token 2t+1), c2 (row g+8, token 2t), c3 (row g+8, token 2t+1); for M = 1
+// every lane of group g returns c0 = row g, c2 = row g+8 (c1 = c3 = 0).
+// Paths (warp-uniform): M = 1 on the CUDA cores; M > 1 on the warp tensor core with
+// the scales folded into the codes when every row's scale span is at most FOLD_SPAN,
+// otherwise token by token on the CUDA cores (exact for any E8M0 scales).
+__device__ __forceinline__ void mxfp4_tile_dot(const uint8_t* codes_g, const uint8_t* codes_g8,
+                                               const uint8_t* sc_g, const uint8_t* sc_g8, int nb,
+                                               const uint8_t* xb, uint32_t xss, int M, const int* xsh,
+                                               float (&c)[4]) {
+  if (M > 1) {
+    mxfp4_tile_dot_win(codes_g, codes_g8, sc_g, sc_g8, nb, xb, xss, M, xsh, c);
+    return;
+  }
+  uint32_t mx_g, mx_g8, mn_g, mn_g8;
+  row_scale_range(sc_g, sc_g8, nb, mx_g, mx_g8, mn_g, mn_g8);
+  const int sh = xsh[0];
+  // the fast factor needs 1 <= e - sh <= 254 for every block of both rows
+  const bool fast = __all_sync(0xffffffffu, (int)min(mn_g, mn_g8) - sh >= 1 && (int)max(mx_g, mx_g8) - sh <= 254);
+  float r0, r1;
+  if (fast)
+    mxfp4_rows_m1<true>(codes_g, codes_g8, sc_g, sc_g8, nb, xb, sh, r0, r1);
+  else
+    mxfp4_rows_m1_safe(codes_g, codes_g8, sc_g, sc_g8, nb, xb, sh, r0, r1);
+  c[0] = r0;
+  c[1] = 0.0f;
+  c[2] = r1;
+  c[3] = 0.0f;
 }
 
 // ---------------------------------------------------------------------------
@@ -648,7 +736,7 @@ __host__ __device__ inline size_t e13_fixed_bytes(int H) { return 128 + 8 * (siz
 __global__ void __launch_bounds__(EXPERT_THREADS, 1) k_experts13(E13Params p) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ Plan P;
-  __shared__ float s_inv[MAX_M];
+  __shared__ int s_sh[MAX_M];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
   const int M = p.M, H = p.H, I = p.I, S = p.stages;
@@ -700,7 +788,7 @@ __global__ void __launch_bounds__(EXPERT_THREADS, 1) k_experts13(E13Params p) {
     return;
   }
 
-  stage_x_f16(p.x, M, H, xs, xss, s_inv);
+  stage_x_f16(p.x, M, H, xs, xss, s_sh);
   for (int i = warp; i < nloc; i += N_CONSUMERS) {
     const int s = i % S;
     if (!mbar_wait(&full[s], (i / S) & 1, p.status)) return;
@@ -709,14 +797,13 @@ __global__ void __launch_bounds__(EXPERT_THREADS, 1) k_experts13(E13Params p) {
     const uint8_t* st = stages + s * sbytes;
     float c[4];
     mxfp4_tile_dot(st + g * cs, st + (8 + g) * cs, st + 16 * cs + g * (H / 32), st + 16 * cs + (8 + g) * (H / 32),
-                   nb, xs, xss, M, c);
+                   nb, xs, xss, M, s_sh, c);
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
       const int tok = 2 * t + e;  // rows g (gate) and g+8 (up) of intermediate index r0 + g
-      if (tok < M)
-        p.a_routed[((size_t)u * M + tok) * I + r0 + g] = silu_f32(c[e] * s_inv[tok]) * (c[2 + e] * s_inv[tok]);
+      if (tok < M) p.a_routed[((size_t)u * M + tok) * I + r0 + g] = silu_f32(c[e]) * c[2 + e];
     }
   }
 }
@@ -758,7 +845,7 @@ __host__ __device__ inline size_t e2_fixed_bytes(int M, int I, int Is) {
 __global__ void __launch_bounds__(EXPERT_THREADS, 1) k_experts2(E2Params p) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ Plan P;
-  __shared__ float s_pscale[E2_MAX_LOCAL_SLOTS][MAX_M];
+  __shared__ int s_ash[E2_MAX_LOCAL_SLOTS][MAX_M];  // f16 shift of each staged routed activation
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
   const int M = p.M, H = p.H, I = p.I, Is = p.Is, S = p.stages;
@@ -841,13 +928,12 @@ __global__ void __launch_bounds__(EXPERT_THREADS, 1) k_experts2(E2Params p) {
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
       const int sh = f16_range_shift(amax);
-      const float sc = exp2i(sh);
       for (int i = lane; i < I / 2; i += 32) {
         __half2 v = __floats2half2_rn(0.0f, 0.0f);
-        if (live) v = __floats2half2_rn(src[2 * i] * sc, src[2 * i + 1] * sc);
+        if (live) v = __floats2half2_rn(mul_pow2(src[2 * i], sh), mul_pow2(src[2 * i + 1], sh));
         *reinterpret_cast<__half2*>(dst + 4 * i) = v;
       }
-      if (lane == 0) s_pscale[uu][tok] = live ? exp2i(-sh) : 0.0f;
+      if (lane == 0) s_ash[uu][tok] = sh;
     }
     if (Is > 0 && end > Tr) {
       for (int i = tid; i < MAX_M * Is; i += 32 * N_CONSUMERS) {
@@ -872,7 +958,7 @@ __global__ void __launch_bounds__(EXPERT_THREADS, 1) k_experts2(E2Params p) {
       const int uu = u - u_lo;
       float c[4];
       mxfp4_tile_dot(st + g * cs, st + (8 + g) * cs, st + 16 * cs + g * (I / 32), st + 16 * cs + (8 + g) * (I / 32),
-                     nb, af + (size_t)uu * MAX_M * ass, ass, M, c);
+                     nb, af + (size_t)uu * MAX_M * ass, ass, M, s_ash[uu], c);
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
 #pragma unroll
@@ -881,9 +967,8 @@ __global__ void __launch_bounds__(EXPERT_THREADS, 1) k_experts2(E2Params p) {
         if (tok < M) {
           const float wt = P.w[u][tok];
           if (wt != 0.0f) {
-            const float f = wt * s_pscale[uu][tok];
-            atomicAdd(p.out + (size_t)tok * H + h0 + g, c[e] * f);
-            atomicAdd(p.out + (size_t)tok * H + h0 + g + 8, c[2 + e] * f);
+            atomicAdd(p.out + (size_t)tok * H + h0 + g, c[e] * wt);
+            atomicAdd(p.out + (size_t)tok * H + h0 + g + 8, c[2 + e] * wt);
           }
         }
       }

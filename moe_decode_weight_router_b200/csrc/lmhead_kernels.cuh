@@ -104,7 +104,8 @@ __device__ __forceinline__ unsigned long long argmax_key(float v, int idx) {
 
 __global__ void __launch_bounds__(EXPERT_THREADS, 1) k_lm_gemv(LMParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ float s_inv[MAX_M];
+  __shared__ int s_sh[MAX_M];
+  __shared__ float s_inv[2][MAX_M];  // 2^-sh as two exact factors
   __shared__ unsigned long long s_best[N_CONSUMERS][MAX_M];
   __shared__ int s_last;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -148,7 +149,13 @@ __global__ void __launch_bounds__(EXPERT_THREADS, 1) k_lm_gemv(LMParams p) {
     return;
   }
 
-  stage_x_f16(p.x, M, H, xs, xss, s_inv);
+  stage_x_f16(p.x, M, H, xs, xss, s_sh);
+  if (tid < MAX_M) {
+    const int k = -s_sh[tid], k1 = k / 2;
+    s_inv[0][tid] = exp2i(k1);
+    s_inv[1][tid] = exp2i(k - k1);
+  }
+  named_barrier(1, 32 * N_CONSUMERS);
   unsigned long long bestA = 0ull, bestB = 0ull;  // tokens 2t and 2t+1
   const int ta = 2 * t, tb = 2 * t + 1;
   for (int i = warp; i < nloc; i += N_CONSUMERS) {
@@ -190,7 +197,8 @@ __global__ void __launch_bounds__(EXPERT_THREADS, 1) k_lm_gemv(LMParams p) {
     const float rsa = va < V ? __ldg(p.rs + va) : 0.0f;
     const float rsb = vb < V ? __ldg(p.rs + vb) : 0.0f;
     if (ta < M) {
-      const float la = c[0] * rsa * s_inv[ta], lb = c[2] * rsb * s_inv[ta];
+      const float ia = s_inv[0][ta], ib = s_inv[1][ta];
+      const float la = ((c[0] * ia) * ib) * rsa, lb = ((c[2] * ia) * ib) * rsb;
       if (va < V) {
         if (p.logits) p.logits[(size_t)ta * V + va] = la;
         bestA = max(bestA, argmax_key(la, (int)va));
@@ -201,7 +209,8 @@ __global__ void __launch_bounds__(EXPERT_THREADS, 1) k_lm_gemv(LMParams p) {
       }
     }
     if (tb < M) {
-      const float la = c[1] * rsa * s_inv[tb], lb = c[3] * rsb * s_inv[tb];
+      const float ia = s_inv[0][tb], ib = s_inv[1][tb];
+      const float la = ((c[1] * ia) * ib) * rsa, lb = ((c[3] * ia) * ib) * rsb;
       if (va < V) {
         if (p.logits) p.logits[(size_t)tb * V + va] = la;
         bestB = max(bestB, argmax_key(la, (int)va));

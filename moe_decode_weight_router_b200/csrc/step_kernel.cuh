@@ -42,12 +42,15 @@ namespace moe {
 
 constexpr int STEP_MAX_LAYERS = 64;
 constexpr int STEP_CONSUMERS = 8;  // consumer warps: two per SM sub-partition, to hide latency
-constexpr int STEP_THREADS = 32 * (STEP_CONSUMERS + 1);
+// Consumer warps 0-7, warp 8 the routed-item producer, warp 9 (one-token kernel) the
+// producer of the routing-independent items.
+constexpr int STEP_THREADS = 32 * (STEP_CONSUMERS + 2);
+constexpr int STEP_FIX_MAX = 8;  // routing-independent items of one kind per block and layer
 constexpr int CR_CACHE = 4;         // routed experts whose W2 activation a block keeps staged
 constexpr int STEP_SLOTS = 32;  // ring items in flight at most (one full/empty mbarrier pair each)
 constexpr int CTR_H = 2, CTR_HINIT = 3, CTR_EXP = 4;  // slots 0-1 unused
 constexpr int CTR_PER_LAYER = CTR_EXP + MAX_SLOTS;
-constexpr size_t STEP_FIXED = 1024;  // full[32], empty[32], plan and h-init barriers
+constexpr size_t STEP_FIXED = 1024;  // full/empty[32], plan, h-init, A and CS full/empty[8] barriers
 constexpr int STAGE_REG_F4 = 4;  // residual float4s a consumer thread keeps in registers (M = 1 at H = 2560)
 constexpr int STAGE_BATCH = 5;   // larger inputs: residual loads a thread keeps in flight
 
@@ -66,6 +69,8 @@ struct StepParams {
   float eps;
   uint32_t ring_bytes;
   uint32_t act_bytes;
+  uint32_t fixa_bytes;  // one-token kernel: region of this block's router/shared-W13 items (0: in the ring)
+  uint32_t fixs_bytes;  // one-token kernel: region of this block's shared-W2 items (0: in the ring)
   const __nv_bfloat16* x_in;  // [M][H]
   float* h;                   // [2][M][H] residual stream, buffer l & 1 is layer l's output
   __nv_bfloat16* x_final;     // [M][H] LM-head input
@@ -84,8 +89,11 @@ struct StepParams {
 
 // Profiling stamp: block 0 and the last block record %globaltimer at phase
 // boundaries (slots 0-11 by consumer thread 0, 12-15 by producer lane 0).
+__device__ __noinline__ void stamp_write(const StepParams& p, int l, int slot);
 __device__ __forceinline__ void stamp(const StepParams& p, int l, int slot) {
-  if (!p.timeline) return;
+  if (p.timeline) stamp_write(p, l, slot);
+}
+__device__ __noinline__ void stamp_write(const StepParams& p, int l, int slot) {
   const bool first = blockIdx.x == 0, last = blockIdx.x == gridDim.x - 1;
   if (!first && !last) return;
   const int tid = threadIdx.x;
@@ -96,9 +104,23 @@ __device__ __forceinline__ void stamp(const StepParams& p, int l, int slot) {
 // [2][L][16] phase stamps: 0 copies issued, 1 data seen by the consumer, 2 consumer
 // done, 3 consumer started waiting, 4 producer entered issue().
 constexpr int STEP_ITEM_LOG = 2048;
-__device__ __forceinline__ void item_stamp(const StepParams& p, long long i, int which) {
-  if (!p.timeline || blockIdx.x != 0 || i >= STEP_ITEM_LOG || (threadIdx.x & 31) != 0) return;
+__device__ __noinline__ void item_stamp_write(const StepParams& p, long long i, int which) {
+  if (blockIdx.x != 0 || i >= STEP_ITEM_LOG || (threadIdx.x & 31) != 0) return;
   p.timeline[(size_t)2 * p.L * 16 + (size_t)i * 8 + which] = globaltimer_ns();
+}
+__device__ __forceinline__ void item_stamp(const StepParams& p, long long i, int which) {
+  if (p.timeline) item_stamp_write(p, i, which);
+}
+// Profiling: every block's own phase ends, [G][L][16] after the item log (written by
+// the calling thread): 0 residual seen, 1 layer input staged, 2 router item published,
+// 3 router/shared-W13 items done, 4 routing plan built, 5 shared W2 done, 6 routed W13
+// done, 7 routed W2 done; 8-12 finer marks inside the top-k; 13-15 data arrivals.
+__device__ __noinline__ void blk_stamp_write(const StepParams& p, int l, int slot) {
+  p.timeline[(size_t)2 * p.L * 16 + (size_t)STEP_ITEM_LOG * 8 + ((size_t)blockIdx.x * p.L + l) * 16 + slot] =
+      globaltimer_ns();
+}
+__device__ __forceinline__ void blk_stamp(const StepParams& p, int l, int slot) {
+  if (p.timeline) blk_stamp_write(p, l, slot);
 }
 
 // ---------------------------------------------------------------------------
@@ -147,17 +169,24 @@ __host__ __device__ inline uint32_t step_act_bytes(int M, int H, int I, int Is) 
 // Deterministic placement in the byte ring on monotonic virtual byte positions (the
 // producer and every consumer warp walk the same item sequence and compute the same
 // offsets): an item that would cross the end of the ring starts at the next multiple
-// of R.  Returns the ring offset; *vstart receives the item's virtual start.
-__device__ __forceinline__ uint32_t ring_take(unsigned long long& vpos, uint32_t n, uint32_t R,
+// of R.  The cursor keeps the ring offset beside the virtual position, so placing an
+// item needs no division.  Returns the ring offset; *vstart receives the virtual start.
+struct RingCursor {
+  unsigned long long v;  // virtual byte position
+  uint32_t off;          // v % R
+};
+__device__ __forceinline__ uint32_t ring_take(RingCursor& c, uint32_t n, uint32_t R,
                                               unsigned long long* vstart = nullptr) {
-  uint32_t off = (uint32_t)(vpos % R);
-  if (off + n > R) {
-    vpos += R - off;
-    off = 0u;
+  if (c.off + n > R) {
+    c.v += R - c.off;
+    c.off = 0u;
   }
-  if (vstart) *vstart = vpos;
-  vpos += n;
-  return off;
+  const uint32_t o = c.off;
+  if (vstart) *vstart = c.v;
+  c.v += n;
+  c.off += n;
+  if (c.off == R) c.off = 0u;
+  return o;
 }
 
 // ---------------------------------------------------------------------------
@@ -204,12 +233,17 @@ __device__ __noinline__ bool wait_counter(const unsigned* c, unsigned target, in
     }
   }
 }
-// mbarrier wait that also honours the block's abort flag.
+// mbarrier wait that also honours the block's abort flag: the first try inline, the
+// bounded loop out of line.
+__device__ __noinline__ bool ring_wait_slow(uint64_t* bar, uint32_t parity, int* status, volatile int* abort_flag);
 __device__ __forceinline__ bool ring_wait(uint64_t* bar, uint32_t parity, int* status, volatile int* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
+  return ring_wait_slow(bar, parity, status, abort_flag);
+}
+__device__ __noinline__ bool ring_wait_slow(uint64_t* bar, uint32_t parity, int* status, volatile int* abort_flag) {
   const unsigned long long t0 = globaltimer_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, 500u)) return true;  // suspended, not spinning
     if (*abort_flag) return false;
     if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
       atomicCAS(status, 0, DEV_ERR_TIMEOUT);
@@ -217,6 +251,12 @@ __device__ __forceinline__ bool ring_wait(uint64_t* bar, uint32_t parity, int* s
       return false;
     }
   }
+}
+// The same wait for a whole warp: lane 0 waits, the others take its answer.
+__device__ __forceinline__ bool warp_ring_wait(uint64_t* bar, uint32_t parity, int* status, volatile int* abort_flag) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) ok = ring_wait(bar, parity, status, abort_flag) ? 1 : 0;
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 // Gives up the whole step: records the timeout once and raises the block's abort flag.
 __device__ __noinline__ void step_give_up(int* status, volatile int* abort_flag) {
@@ -357,7 +397,7 @@ struct Producer {
   uint64_t pol;
   long long i;               // next ring item
   long long oldest;          // oldest item whose release lane 0 has not seen yet
-  unsigned long long vpos;   // virtual placement cursor
+  RingCursor vpos;           // virtual placement cursor
   volatile int* abort_flag;
   int lane;
 
@@ -431,13 +471,18 @@ struct Producer {
     return true;
   }
 
-  // router / shared items (one tile each)
+  // router / shared items (one tile each) through the ring
   __device__ bool issue(const LayerPtrs& Lp, const Plan& P, const Item& it) {
     uint32_t s0;
     int slot;
     if (!acquire(step_item_bytes(it.type, p.H, p.I, p.Is), s0, slot)) return false;
-    uint8_t* st = ring + s0;
-    uint64_t* fb = &full[slot];
+    copy_item(Lp, it, ring + s0, &full[slot]);
+    item_stamp(p, i, 5);
+    ++i;
+    return true;
+  }
+  // the copies of one router / shared item into st, completing on fb
+  __device__ void copy_item(const LayerPtrs& Lp, const Item& it, uint8_t* st, uint64_t* fb) {
     const int H = p.H, Is = p.Is;
     if (it.type == IT_A) {
       const int nr = p.E / 4;
@@ -455,9 +500,6 @@ struct Producer {
       __syncwarp();
       if (lane == 0) bulk_g2s(st, Lp.sw2 + (size_t)it.a * Is, 4u * 2u * Is, fb, pol);
     }
-    item_stamp(p, i, 5);
-    ++i;
-    return true;
   }
 };
 
@@ -486,19 +528,32 @@ __device__ __forceinline__ float4 load_residual4(const StepParams& p, int l, con
   }
   return __ldcg(reinterpret_cast<const float4*>(hin) + q);
 }
-__device__ __forceinline__ void write_layer_input4(uint8_t* xb16, uint8_t* xf16, uint32_t off, float4 v, float r,
-                                                   float sc) {
+// Byte offset of element e of a one-token f16 activation row held chunk-major:
+// chunk w (elements 8w..8w+7) of scale block b at (w * nb + b) * 16.  Lanes that walk
+// consecutive blocks then read consecutive 16-byte chunks (no bank conflicts).
+__device__ __forceinline__ uint32_t chunk_major_off(int e, int nb) {
+  return (uint32_t)((((e >> 3) & 3) * nb + (e >> 5)) * 16 + (e & 7) * 2);
+}
+
+__device__ __forceinline__ void write_layer_input4(uint8_t* xb16, uint8_t* xf16, uint32_t off, uint32_t off16, float4 v,
+                                                   float r, int sh) {
   const __nv_bfloat162 a = __floats2bfloat162_rn(v.x * r, v.y * r);
   const __nv_bfloat162 b = __floats2bfloat162_rn(v.z * r, v.w * r);
   uint2 u;
   u.x = *reinterpret_cast<const uint32_t*>(&a);
   u.y = *reinterpret_cast<const uint32_t*>(&b);
   *reinterpret_cast<uint2*>(xb16 + off) = u;
-  const __half2 ha = __floats2half2_rn(__low2float(a) * sc, __high2float(a) * sc);
-  const __half2 hb = __floats2half2_rn(__low2float(b) * sc, __high2float(b) * sc);
+  const __half2 ha = __floats2half2_rn(mul_pow2(__low2float(a), sh), mul_pow2(__high2float(a), sh));
+  const __half2 hb = __floats2half2_rn(mul_pow2(__low2float(b), sh), mul_pow2(__high2float(b), sh));
   u.x = *reinterpret_cast<const uint32_t*>(&ha);
   u.y = *reinterpret_cast<const uint32_t*>(&hb);
-  *reinterpret_cast<uint2*>(xf16 + off) = u;
+  *reinterpret_cast<uint2*>(xf16 + off16) = u;
+}
+// f16 offset of float4 column c of token tok: chunk-major for one token (the lanes-along-K
+// products), row-major (stride xss) for a window (the tensor-core tiles).
+template <bool ONE>
+__device__ __forceinline__ uint32_t xf16_off(int H, uint32_t xss, int tok, int c) {
+  return ONE ? chunk_major_off(4 * c, H / 32) : tok * xss + 8 * c;
 }
 __device__ __forceinline__ void accumulate4(float4 v, float& ss, float& am) {
   ss = fmaf(v.x, v.x, ss);
@@ -508,15 +563,17 @@ __device__ __forceinline__ void accumulate4(float4 v, float& ss, float& am) {
   am = fmaxf(am, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
 }
 
+// [q0, q1): this block's slice of the residual's float4s (copied into hout).
+template <bool ONE>
 __device__ void stage_layer_input(const StepParams& p, int l, const float* hin, float* hout, uint8_t* xb16,
                                   uint8_t* xf16, uint32_t xss, float* s_part, float* s_amx, float* s_r, int* s_sh,
-                                  float* s_inv) {
+                                  int q0, int q1) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int M = p.M, H = p.H, nt = 32 * STEP_CONSUMERS;
+  const int M = ONE ? 1 : p.M, H = p.H, nt = 32 * STEP_CONSUMERS;
   const int per = H / 4, Q = M * per;  // float4s per token / in total
-  const int q0 = (int)((long long)Q * blockIdx.x / gridDim.x), q1 = (int)((long long)Q * (blockIdx.x + 1) / gridDim.x);
+
   float4* hout4 = reinterpret_cast<float4*>(hout);
-  const bool inreg = Q <= STAGE_REG_F4 * nt;
+  const bool inreg = ONE || Q <= STAGE_REG_F4 * nt;  // one token: H <= 4096 always fits
   float4 v[STAGE_REG_F4];
   int tq[STAGE_REG_F4], cq[STAGE_REG_F4];  // token and float4 column of q = tid + nt*j
   if (inreg) {
@@ -614,16 +671,15 @@ __device__ void stage_layer_input(const StepParams& p, int l, const float* hin, 
     }
     const float r = l == 0 ? 1.0f : 1.0f / sqrtf(ss / (float)H + p.eps);
     s_r[tid] = r;
-    const int sh = f16_range_shift(__bfloat162float(__float2bfloat16_rn(am * r)));
-    s_sh[tid] = sh;
-    s_inv[tid] = exp2i(-sh);
+    s_sh[tid] = f16_range_shift(__bfloat162float(__float2bfloat16_rn(am * r)));
   }
   csync();
   if (inreg) {
 #pragma unroll
     for (int j = 0; j < STAGE_REG_F4; ++j)
       if (tq[j] < M)
-        write_layer_input4(xb16, xf16, tq[j] * xss + 8 * cq[j], v[j], s_r[tq[j]], exp2i(s_sh[tq[j]]));
+        write_layer_input4(xb16, xf16, tq[j] * xss + 8 * cq[j], xf16_off<ONE>(H, xss, tq[j], cq[j]), v[j], s_r[tq[j]],
+                           s_sh[tq[j]]);
   } else {
     for (int qb = tid; qb < Q; qb += STAGE_BATCH * nt) {
       float4 w[STAGE_BATCH];
@@ -637,7 +693,7 @@ __device__ void stage_layer_input(const StepParams& p, int l, const float* hin, 
         const int q = qb + j * nt;
         if (q < Q) {
           const int tok = q / per, c = q - tok * per;
-          write_layer_input4(xb16, xf16, tok * xss + 8 * c, w[j], s_r[tok], exp2i(s_sh[tok]));
+          write_layer_input4(xb16, xf16, tok * xss + 8 * c, xf16_off<ONE>(H, xss, tok, c), w[j], s_r[tok], s_sh[tok]);
         }
       }
     }
@@ -646,95 +702,131 @@ __device__ void stage_layer_input(const StepParams& p, int l, const float* hin, 
 }
 
 // Top-k of every token from the complete router logits (same rule as k_dense:
-// largest logit, lowest index on ties), then the union plan.  The 8 consumer warps
-// form TG token groups x EP expert parts (TG the largest power of two <= min(M, 8)
-// whose parts hold at most 256 experts): each keeps its part's top-k of its tokens
-// (a global top-k element is always in its part's top-k, ties included), then one
-// warp per token merges the EP*k candidates.
-__device__ void step_topk(const StepParams& p, int l, Plan& P, int32_t* s_ids, float* s_wts, uint32_t* s_ck,
-                          int32_t* s_ci, volatile int* s_abort_ptr) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int E = p.E, k = p.k, M = p.M;
-  int TG = 1;
-  while (2 * TG <= M && 2 * TG <= STEP_CONSUMERS && E <= 256 * (STEP_CONSUMERS / (2 * TG))) TG *= 2;
-  const int EP = STEP_CONSUMERS / TG;
-  const int per = (E + EP - 1) / EP;  // experts per part (<= 256)
-  const int part = warp % EP;
-  const int e0 = part * per;
-  for (int tok = warp / EP; tok < M; tok += TG) {
-    uint32_t key[8];
-    {
-      const unsigned long long* w[8];
-      int n = 0;
+// largest logit, lowest index on ties), then the union plan.  Candidates are ranked
+// by one 64-bit order key, (logit key << 32) | ~expert, so a larger order key is the
+// better candidate and no two are equal.
+__device__ __forceinline__ unsigned long long order_key(uint32_t key, int e) {
+  return ((unsigned long long)key << 32) | (unsigned long long)(~(uint32_t)e);
+}
+constexpr int TOPK_CAND = 32;  // survivors ranked directly (one per lane)
+
+// Exact k-round selection over all E logits of token tok by one warp (the path for
+// tokens whose logits cluster above the survivor bound): each round takes the
+// largest remaining order key.  Writes the k order keys, best first, to sel[].
+__device__ __noinline__ void topk_token_full(const StepParams& p, int l, int tok, unsigned long long* sel,
+                                             volatile int* abort_flag) {
+  const int lane = threadIdx.x & 31, E = p.E;
+  uint32_t key[32];  // expert lane + 32 i (E <= 1024)
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int off = lane + 32 * i, e = e0 + off;
-        w[i] = p.logits + tok * E + e;
-        if (off < per && e < E) n = i + 1;  // valid columns are a prefix
-      }
-      float lv[8];
-      if (!await_tagged(w, n, (uint32_t)l + 1u, lv, p.status, s_abort_ptr))
-        n = 0;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) key[i] = i < n ? float_key(lv[i]) : 0u;
-    }
+  for (int i = 0; i < 32; i += 8) {
+    const unsigned long long* w[8];
+    int n = 0;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      if (j < k) {
-        uint32_t bk = 0u;
-        int bi = 0x7fffffff;
+      const int e = lane + 32 * (i + j);
+      w[j] = p.logits + (size_t)tok * E + (e < E ? e : 0);
+      if (e < E) n = j + 1;
+    }
+    float lv[8];
+    if (!await_tagged(w, n, (uint32_t)l + 1u, lv, p.status, abort_flag)) n = 0;
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          if (key[i] > bk) {
-            bk = key[i];
-            bi = e0 + lane + 32 * i;
-          }
-        const uint32_t mk = __reduce_max_sync(0xffffffffu, bk);
-        const int mi = (int)__reduce_min_sync(0xffffffffu, (unsigned)(bk == mk ? bi : 0x7fffffff));
+    for (int j = 0; j < 8; ++j) key[i + j] = j < n ? float_key(lv[j]) : 0u;
+  }
+  for (int j = 0; j < p.k; ++j) {
+    uint32_t bk = 0u;
+    int bi = 0x7fffffff;
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          if (e0 + lane + 32 * i == mi) key[i] = 0u;
-        if (lane == 0) {
-          s_ck[(tok * STEP_CONSUMERS + part) * 8 + j] = mk;
-          s_ci[(tok * STEP_CONSUMERS + part) * 8 + j] = mk ? mi : 0x7fffffff;
-        }
+    for (int i = 0; i < 32; ++i)
+      if (key[i] > bk) {  // strict: the first (lowest) index wins a tie within the lane
+        bk = key[i];
+        bi = lane + 32 * i;
+      }
+    const uint32_t mk = __reduce_max_sync(0xffffffffu, bk);
+    const int mi = (int)__reduce_min_sync(0xffffffffu, (unsigned)(bk == mk ? bi : 0x7fffffff));
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if (lane + 32 * i == mi) key[i] = 0u;
+    if (lane == 0) sel[j] = order_key(mk, mi);
+  }
+}
+
+// The 8 consumer warps split the experts: warp w holds experts [w*per, (w+1)*per),
+// per = E/8, at most 4 per lane, of every token.  The smallest of the 8 warp maxima
+// is a lower bound for the k-th largest logit (k <= 8, and the maxima are 8 distinct
+// experts), so only logits at or above it can be selected: those are gathered per
+// token, and when at most TOPK_CAND survive, each survivor's rank is the number of
+// survivors whose order key is larger.  Otherwise the token's warp runs the exact
+// k-round selection.  Warp t then forms token t's softmax over its selected logits.
+template <bool ONE>
+__device__ void step_topk(const StepParams& p, int l, Plan& P, int32_t* s_ids, float* s_wts, uint32_t* s_wmax,
+                          int* s_ncand, unsigned long long* s_cand, unsigned long long* s_sel,
+                          volatile int* s_abort_ptr) {
+  constexpr int MT = ONE ? 1 : MAX_M;  // tokens held in registers
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
+  const int E = p.E, k = p.k, M = ONE ? 1 : p.M;
+  const int per = E / STEP_CONSUMERS;  // E % 16 == 0: every warp holds >= 2 experts
+  const int e0 = warp * per;
+  if (tid < MAX_M) s_ncand[tid] = 0;
+  uint32_t key[MT][4];
+#pragma unroll
+  for (int tok = 0; tok < MT; ++tok) {
+    if (tok >= M) break;
+    const unsigned long long* w[8];
+    int n = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int off = lane + 32 * i;
+      w[i] = p.logits + (size_t)tok * E + e0 + (off < per ? off : 0);
+      if (i < 4 && off < per) n = i + 1;  // valid columns are a prefix
+    }
+    float lv[8];
+    if (!await_tagged(w, n, (uint32_t)l + 1u, lv, p.status, s_abort_ptr)) n = 0;
+    uint32_t mx = 0u;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      key[tok][i] = i < n ? float_key(lv[i]) : 0u;
+      mx = max(mx, key[tok][i]);
+    }
+    mx = __reduce_max_sync(0xffffffffu, mx);
+    if (lane == 0) s_wmax[tok * STEP_CONSUMERS + warp] = mx;
+  }
+  if (tid == 0) blk_stamp(p, l, 8);
+  csync();
+#pragma unroll
+  for (int tok = 0; tok < MT; ++tok) {
+    if (tok >= M) break;
+    uint32_t bound = 0xFFFFFFFFu;
+#pragma unroll
+    for (int w = 0; w < STEP_CONSUMERS; ++w) bound = min(bound, s_wmax[tok * STEP_CONSUMERS + w]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int off = lane + 32 * i;
+      if (off < per && key[tok][i] >= bound) {
+        const int pos = atomicAdd(&s_ncand[tok], 1);
+        if (pos < TOPK_CAND) s_cand[tok * TOPK_CAND + pos] = order_key(key[tok][i], e0 + off);
       }
     }
   }
+  if (tid == 0) blk_stamp(p, l, 9);
   csync();
+  if (tid == 0) blk_stamp(p, l, 10);
   for (int tok = warp; tok < M; tok += STEP_CONSUMERS) {
-    const int nc = EP * k;  // <= 64 candidates, two per lane
-    uint32_t ck[2] = {0u, 0u};
-    int ci[2] = {0x7fffffff, 0x7fffffff};
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const int c = lane + 32 * r;
-      if (c < nc) {
-        ck[r] = s_ck[(tok * STEP_CONSUMERS + c / k) * 8 + c % k];
-        ci[r] = s_ci[(tok * STEP_CONSUMERS + c / k) * 8 + c % k];
-      }
+    unsigned long long* sel = s_sel + tok * 8;
+    const int n = s_ncand[tok];
+    if (n <= TOPK_CAND) {
+      const unsigned long long* cand = s_cand + tok * TOPK_CAND;
+      const unsigned long long mine = lane < n ? cand[lane] : 0ull;
+      int rank = 0;
+      for (int j = 0; j < n; ++j) rank += cand[j] > mine ? 1 : 0;
+      if (lane < n && rank < k) sel[rank] = mine;
+    } else {
+      topk_token_full(p, l, tok, sel, s_abort_ptr);
     }
-    int sel_id = 0;
-    uint32_t sel_key = 0u;
-    for (int j = 0; j < k; ++j) {
-      const int b = (ck[1] > ck[0] || (ck[1] == ck[0] && ci[1] < ci[0])) ? 1 : 0;
-      const uint32_t bk = b ? ck[1] : ck[0];
-      const int bi = b ? ci[1] : ci[0];
-      const uint32_t mk = __reduce_max_sync(0xffffffffu, bk);
-      const int mi = (int)__reduce_min_sync(0xffffffffu, (unsigned)(bk == mk ? bi : 0x7fffffff));
-#pragma unroll
-      for (int r = 0; r < 2; ++r)
-        if (ck[r] == mk && ci[r] == mi) {
-          ck[r] = 0u;
-          ci[r] = 0x7fffffff;
-        }
-      if (lane == j) {
-        sel_id = mi;
-        sel_key = mk;
-      }
-    }
+    __syncwarp();
     // lane j holds the j-th selection; softmax over the selected logits
-    const float lj = key_float(sel_key);
+    const unsigned long long sj = lane < k ? sel[lane] : 0ull;
+    const int sel_id = (int)(~(uint32_t)sj);
+    const float lj = key_float((uint32_t)(sj >> 32));
     const float l0 = __shfl_sync(0xffffffffu, lj, 0);
     const float ex = lane < k ? expf(lj - l0) : 0.0f;
     float den = ex;
@@ -751,9 +843,90 @@ __device__ void step_topk(const StepParams& p, int l, Plan& P, int32_t* s_ids, f
       }
     }
   }
+  if (threadIdx.x == 0) blk_stamp(p, l, 11);
   csync();
   if (warp == 0) build_plan(P, s_ids, s_wts, M, k, E);
+  if (threadIdx.x == 0) blk_stamp(p, l, 12);
   csync();
+}
+
+// ---------------------------------------------------------------------------
+// one-token MXFP4 row products (the routed experts at M = 1)
+// ---------------------------------------------------------------------------
+// R MXFP4 rows (codes rows[q], E8M0 scales scs[q], nb blocks of 32) against one f16
+// activation row xc (chunk-major, scaled by 2^sh), lanes along K: each group of LPR
+// lanes takes blocks l, l+LPR, ... (l = lane % LPR) of all R rows, so the activation
+// chunks load once for R rows.  Products exact in fp32, summed per block; the block
+// factor 2^(e - 127 - sh) applied in fp32.  Fast factors (SAFE false) are the normal
+// number with exponent byte e - sh; a block with e - sh outside [1, 254] sets `bad`
+// and the caller repeats the rows with SAFE (clamped factors, exact down to 2^-149).
+// Every lane of the group returns the R row sums.  All 32 lanes must call it.
+template <int LPR, int R, bool SAFE>
+__device__ __forceinline__ void rows_dot_m1(const uint8_t* const (&rows)[R], const uint8_t* const (&scs)[R], int nb,
+                                            const uint8_t* xc, int sh, bool& bad, float (&out)[R]) {
+  const int l = threadIdx.x & (LPR - 1);
+  float a[R];
+#pragma unroll
+  for (int q = 0; q < R; ++q) a[q] = 0.0f;
+  // one block per iteration, not unrolled: the loop is entered once per row set, and a
+  // compact body stays in the instruction cache
+#pragma unroll 1
+  for (int b = l; b < nb; b += LPR) {
+    uint32_t xw[16];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const uint4 X = lds128(xc + (w * nb + b) * 16);
+      xw[4 * w] = X.x;
+      xw[4 * w + 1] = X.y;
+      xw[4 * w + 2] = X.z;
+      xw[4 * w + 3] = X.w;
+    }
+#pragma unroll
+    for (int q = 0; q < R; ++q) {
+      const uint4 C = lds128(rows[q] + 16 * b);
+      const int e = scs[q][b];
+      float f;
+      if (SAFE) {
+        f = pow2_clamped(e - 127 - sh);
+      } else {
+        const int d = e - sh;
+        bad |= (unsigned)(d - 1) > 253u;
+        f = __uint_as_float((uint32_t)d << 23);
+      }
+      const uint32_t cw[4] = {C.x, C.y, C.z, C.w};
+      uint32_t hv[16];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) e2m1x8_to_f16x2(cw[k], hv[4 * k], hv[4 * k + 1], hv[4 * k + 2], hv[4 * k + 3]);
+      float p0 = 0.0f, p1 = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        p0 = fma_f16_lo(hv[j], xw[j], p0);
+        p1 = fma_f16_hi(hv[j], xw[j], p1);
+      }
+      a[q] = fmaf(p0 + p1, f, a[q]);
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < R; ++q) {
+#pragma unroll
+    for (int o = LPR / 2; o > 0; o >>= 1) a[q] += __shfl_xor_sync(0xffffffffu, a[q], o);
+    out[q] = a[q];
+  }
+}
+template <int LPR, int R>
+__device__ __noinline__ void rows_dot_m1_safe(const uint8_t* const (&rows)[R], const uint8_t* const (&scs)[R], int nb,
+                                              const uint8_t* xc, int sh, float (&out)[R]) {
+  bool bad = false;
+  rows_dot_m1<LPR, R, true>(rows, scs, nb, xc, sh, bad, out);
+}
+// rows_dot_m1 with the fast factors, repeated out of line with exact clamped ones when
+// any lane of the warp met a block outside the fast range.
+template <int LPR, int R>
+__device__ __forceinline__ void rows_dot_m1_exact(const uint8_t* const (&rows)[R], const uint8_t* const (&scs)[R], int nb,
+                                                  const uint8_t* xc, int sh, float (&out)[R]) {
+  bool bad = false;
+  rows_dot_m1<LPR, R, false>(rows, scs, nb, xc, sh, bad, out);
+  if (__any_sync(0xffffffffu, bad)) rows_dot_m1_safe<LPR, R>(rows, scs, nb, xc, sh, out);
 }
 
 // ---------------------------------------------------------------------------
@@ -843,39 +1016,50 @@ __device__ __forceinline__ void rows4_dot_m1(const uint8_t* wrows, uint32_t wstr
   }
 }
 
+// ONE: the one-token instantiation (lanes-along-K products, chunk-major activations);
+// otherwise a verify window of M >= 2 tokens (tensor-core tiles).  Separate
+// instantiations keep each one's code small enough for the instruction caches.
+template <bool ONE>
 __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant__ StepParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ Plan P;
   __shared__ float s_part[MAX_M * STEP_CONSUMERS];
   __shared__ float s_r[MAX_M];
-  __shared__ float s_inv[MAX_M];
-  __shared__ float s_pscale[CR_CACHE][MAX_M];
+  __shared__ int s_ash[CR_CACHE][MAX_M];  // f16 shift of each staged routed activation
   __shared__ int32_t s_ids[MAX_SLOTS];
   __shared__ float s_wts[MAX_SLOTS];
   __shared__ float s_amx[MAX_M * STEP_CONSUMERS];
   __shared__ int s_sh[MAX_M];
-  __shared__ uint32_t s_ck[MAX_M * STEP_CONSUMERS * 8];
-  __shared__ int32_t s_ci[MAX_M * STEP_CONSUMERS * 8];
+  __shared__ uint32_t s_wmax[MAX_M * STEP_CONSUMERS];
+  __shared__ int s_ncand[MAX_M];
+  __shared__ unsigned long long s_cand[MAX_M * TOPK_CAND];
+  __shared__ unsigned long long s_sel[MAX_M * 8];
   __shared__ unsigned long long s_vst[STEP_SLOTS];
   __shared__ int s_gdone[STEP_SLOTS];  // tiles of a grouped ring item finished so far
   __shared__ volatile int s_abort;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
-  const int M = p.M, H = p.H, I = p.I, Is = p.Is, L = p.L;
+  const int M = ONE ? 1 : p.M, H = p.H, I = p.I, Is = p.Is, L = p.L;
   const uint32_t R = p.ring_bytes;
   const unsigned G = gridDim.x;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);
   uint64_t* empty = full + STEP_SLOTS;
   uint64_t* plan_bar = empty + STEP_SLOTS;  // consumers -> producer: this layer's plan is built
   uint64_t* hinit_bar = plan_bar + 1;       // consumers -> producer: this block's h slice is copied
-  uint8_t* ring = smem + STEP_FIXED;
+  uint64_t* fullA = hinit_bar + 1;          // one token: fixed router/shared-W13 slots
+  uint64_t* emptyA = fullA + STEP_FIX_MAX;
+  uint64_t* fullS = emptyA + STEP_FIX_MAX;  // one token: fixed shared-W2 slots
+  uint64_t* emptyS = fullS + STEP_FIX_MAX;
+  uint8_t* fixA = smem + STEP_FIXED;
+  uint8_t* fixS = fixA + p.fixa_bytes;
+  uint8_t* ring = fixS + p.fixs_bytes;
   uint8_t* act = ring + R;
   const uint32_t xss = padded_stride(2u * H);
   const uint32_t sss = Is > 0 ? padded_stride(2u * Is) : 0u;
   const uint32_t ass = padded_stride(2u * I);
   uint8_t* xb16 = act;                    // A phase: bf16 x rows [M][xss]
-  uint8_t* xf16 = act + (size_t)M * xss;  // B phase: f16 x rows  [M][xss]
+  uint8_t* xf16 = act + (size_t)M * xss;  // B phase: f16 x rows  [M][xss] (one token: chunk-major)
   uint8_t* shi = step_shared_over_xb16(H, Is) ? act : act + 2 * (size_t)M * xss;  // CS: shared a, bf16 hi
   uint8_t* slo = shi + (size_t)M * sss;                                            //     bf16 lo
   uint8_t* afc = act;                     // CR phase: routed a of the block's experts [CR_CACHE][M][ass]
@@ -890,22 +1074,80 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
     }
     mbar_init(plan_bar, 1);
     mbar_init(hinit_bar, 1);
+    for (int s = 0; s < STEP_FIX_MAX; ++s) {
+      mbar_init(&fullA[s], 1);
+      mbar_init(&emptyA[s], 1);
+      mbar_init(&fullS[s], 1);
+      mbar_init(&emptyS[s], 1);
+    }
     for (int s = 0; s < STEP_SLOTS; ++s) s_gdone[s] = 0;
     fence_mbar_init();
     s_abort = 0;
   }
   __syncthreads();
 
-  // ---------------- producer ----------------
+  // ---------------- producer of the routing-independent items (one token) ----------------
+  // Router / shared-W13 items and shared-W2 items of layer l go to their fixed slots as
+  // soon as the consumers have released the slot's layer l-1 copy, so each layer's are
+  // in shared memory (or on their way) while the layer before is still routing.
+  if (warp == STEP_CONSUMERS + 1) {
+    if constexpr (ONE) {
+      Producer pr{p, ring, R, full, empty, s_vst, policy_evict_first(), 0, 0, RingCursor{0ull, 0u}, &s_abort, lane};
+      Work W;
+      W.init_fixed(p);
+      int la = 0, ls = 0;  // layers issued completely (A slots / S slots); the slots of layer la / ls partly
+      int ja = 0, js = 0;  // slots issued of the partial layer
+      bool ok = true;
+      for (int l = 0; l < L && ok; ++l) {
+        const LayerPtrs& Lp = p.layer[l];
+        for (ja = 0; ja < W.nA; ++ja) {
+          if (l > 0 && lane == 0) ok = ring_wait(&emptyA[ja], (uint32_t)((l - 1) & 1), p.status, &s_abort);
+          ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+          if (!ok) break;
+          pr.copy_item(Lp, W.at(p, ja), fixA + (size_t)ja * bytesA, &fullA[ja]);
+        }
+        if (!ok) break;
+        la = l + 1;
+        ja = 0;
+        for (js = 0; js < W.nS; ++js) {
+          if (l > 0 && lane == 0) ok = ring_wait(&emptyS[js], (uint32_t)((l - 1) & 1), p.status, &s_abort);
+          ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+          if (!ok) break;
+          pr.copy_item(Lp, W.at(p, W.nA + js), fixS + (size_t)js * bytesS, &fullS[js]);
+        }
+        if (!ok) break;
+        ls = l + 1;
+        js = 0;
+      }
+      // every copy issued lands before the block may exit: slot j's last copy belongs
+      // to layer la (j < ja, a partly issued layer) or la - 1
+      if (lane == 0) {
+        for (int j = 0; j < W.nA; ++j) {
+          const int n = la + (j < ja ? 1 : 0);
+          if (n > 0) drain_wait(&fullA[j], (uint32_t)((n - 1) & 1));
+        }
+        for (int j = 0; j < W.nS; ++j) {
+          const int n = ls + (j < js ? 1 : 0);
+          if (n > 0) drain_wait(&fullS[j], (uint32_t)((n - 1) & 1));
+        }
+      }
+    }
+    return;
+  }
+
+  // ---------------- producer of the ring ----------------
+  // One token: routed items only.  A window: every item of the layer in ring order.
   if (warp == STEP_CONSUMERS) {
-    Producer pr{p, ring, R, full, empty, s_vst, policy_evict_first(), 0, 0, 0ull, &s_abort, lane};
+    Producer pr{p, ring, R, full, empty, s_vst, policy_evict_first(), 0, 0, RingCursor{0ull, 0u}, &s_abort, lane};
     bool ok = true;
     for (int l = 0; l < L && ok; ++l) {
       const LayerPtrs& Lp = p.layer[l];
       Work W;
       W.init_fixed(p);
-      for (int r = 0; r < W.nA + W.nS && ok; ++r) ok = pr.issue(Lp, P, W.at(p, r));
-      if (!ok) break;
+      if constexpr (!ONE) {
+        for (int r = 0; r < W.nA + W.nS && ok; ++r) ok = pr.issue(Lp, P, W.at(p, r));
+        if (!ok) break;
+      }
       stamp(p, l, 12);
       int got = 1;
       // the consumers' slice copy of h (ordered before their arrive by a block
@@ -938,8 +1180,10 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
 
   // ---------------- consumers ----------------
   unsigned* ctr = p.ctr;
+  const int QH = M * (H / 4);  // float4s of the residual
+  const int slice_q0 = (int)((long long)QH * blockIdx.x / G), slice_q1 = (int)((long long)QH * (blockIdx.x + 1) / G);
   long long i = 0;   // ring item
-  unsigned long long pos = 0;  // virtual ring cursor (same walk as the producer's)
+  RingCursor pos{0ull, 0u};  // virtual ring cursor (same walk as the producer's)
   for (int l = 0; l < L; ++l) {
     unsigned* lc = ctr + (size_t)l * CTR_PER_LAYER;
     float* hout = p.h + (size_t)(l & 1) * M * H;
@@ -950,9 +1194,11 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
       csync();
     }
     stamp(p, l, 1);
-    stage_layer_input(p, l, hin, hout, xb16, xf16, xss, s_part, s_amx, s_r, s_sh, s_inv);
+    if (tid == 0) blk_stamp(p, l, 0);
+    stage_layer_input<ONE>(p, l, hin, hout, xb16, xf16, xss, s_part, s_amx, s_r, s_sh, slice_q0, slice_q1);
     if (tid == 0) mbar_arrive(hinit_bar);
     stamp(p, l, 2);
+    if (tid == 0) blk_stamp(p, l, 1);
     if (blockIdx.x == 0 && (p.x_trace || p.h_trace)) {
       for (int e = tid; e < M * H; e += 32 * STEP_CONSUMERS) {
         const int tok = e / H, c = e % H;
@@ -964,125 +1210,214 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
     }
 
     // ---- A: router items (4 experts) and shared-W13 items (2 gate + 2 up rows) ----
+    // One token: item r in fixed slot r on warp r; a window: through the ring.
     Work W;
     W.init_fixed(p);
     const int nr = p.E / 4;
-    for (int r = 0; r < W.nA; ++r, ++i) {
-      const uint32_t s0 = ring_take(pos, bytesA, R);
-      if ((int)(i % STEP_CONSUMERS) != warp) continue;
-      const int slot = (int)(i % STEP_SLOTS);
+    for (int r = 0; r < W.nA; ++r) {
+      const uint8_t* src;
+      uint64_t* eb;
+      bool ready;
+      if constexpr (ONE) {
+        if (r % STEP_CONSUMERS != warp) continue;
+        src = fixA + (size_t)r * bytesA;
+        eb = &emptyA[r];
+        ready = ring_wait(&fullA[r], (uint32_t)(l & 1), p.status, &s_abort);
+      } else {
+        const uint32_t s0 = ring_take(pos, bytesA, R);
+        const long long ii = i++;
+        if ((int)(ii % STEP_CONSUMERS) != warp) continue;
+        const int slot = (int)(ii % STEP_SLOTS);
+        src = ring + s0;
+        eb = &empty[slot];
+        item_stamp(p, ii, 3);
+        ready = ring_wait(&full[slot], (uint32_t)((ii / STEP_SLOTS) & 1), p.status, &s_abort);
+      }
+      ready = __all_sync(0xffffffffu, ready);
       const Item it = W.at(p, r);
       const bool router = it.a < nr;
       float c[4] = {0.f, 0.f, 0.f, 0.f};
-      item_stamp(p, i, 3);
-      if (ring_wait(&full[slot], (uint32_t)((i / STEP_SLOTS) & 1), p.status, &s_abort)) {
-        item_stamp(p, i, 1);
+      if (ready) {
         // shared items: columns (0,1,2,3) = (gate 2s, up 2s, gate 2s+1, up 2s+1) from
         // smem rows (0, 2, 1, 3), so a thread's two columns are a (gate, up) pair
-        if (M == 1) {
+        if constexpr (ONE) {
           float o[4];
-          rows4_dot_m1(ring + s0, 2u * H, router ? 0x3210u : 0x3120u, xb16, nullptr, H, o);
+          rows4_dot_m1(src, 2u * H, router ? 0x3210u : 0x3120u, xb16, nullptr, H, o);
           c[0] = t == 0 ? o[0] : o[2];
           c[1] = t == 0 ? o[1] : o[3];
         } else {
           const int wrow = g < 4 ? (router ? g : ((g & 1) ? 2 : 0) + (g >> 1)) : -1;
-          rows4_dot(ring + s0, 2u * H, wrow, g < M ? xb16 + g * xss : nullptr, nullptr, H, c);
+          rows4_dot(src, 2u * H, wrow, g < M ? xb16 + g * xss : nullptr, nullptr, H, c);
         }
       }
       __syncwarp();
-      item_stamp(p, i, 2);
-      if (lane == 0) mbar_arrive(&empty[slot]);
+      if (lane == 0) mbar_arrive(eb);
       if (t < 2 && g < M) {
         const uint32_t tag = (uint32_t)l + 1u;
         if (router) {
           st_tagged(p.logits + g * p.E + 4 * it.a + 2 * t, c[0], tag);
           st_tagged(p.logits + g * p.E + 4 * it.a + 2 * t + 1, c[1], tag);
+          if (lane == 0) blk_stamp(p, l, 2);
         } else {
           st_tagged(p.a_shared + g * Is + 2 * (it.a - nr) + t, silu_f32(c[0]) * c[1], tag);
         }
       }
     }
     stamp(p, l, 3);
+    if (tid == 0) blk_stamp(p, l, 3);
 
     // ---- top-k and plan (every block, identical; polls the tagged logits) ----
     stamp(p, l, 4);
-    step_topk(p, l, P, s_ids, s_wts, s_ck, s_ci, &s_abort);
+    step_topk<ONE>(p, l, P, s_ids, s_wts, s_wmax, s_ncand, s_cand, s_sel, &s_abort);
     if (tid == 0) mbar_arrive(plan_bar);
     stamp(p, l, 5);
+    if (tid == 0) blk_stamp(p, l, 4);
 
     // ---- CS: shared W2 (activation as bf16 hi + lo), accumulated into h ----
-    if (W.nS > 0) {
-      for (int e = tid; e < M * (Is / 8); e += 32 * STEP_CONSUMERS) {
-        const int tok = e / (Is / 8), c8 = e % (Is / 8);
-        const unsigned long long* w[8];
+    // A window runs it here, ahead of the routed tiles whose copies it waits for; one
+    // token runs it after the routed W13 (its items are already in their slots), to
+    // fill the wait for the routed activations.
+    auto shared_w2 = [&]() {
+      if (W.nS > 0) {
+        for (int e = tid; e < M * (Is / 8); e += 32 * STEP_CONSUMERS) {
+          const int tok = e / (Is / 8), c8 = e % (Is / 8);
+          const unsigned long long* w[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) w[j] = p.a_shared + (size_t)tok * Is + 8 * c8 + j;
-        float a8[8];
-        if (!await_tagged(w, 8, (uint32_t)l + 1u, a8, p.status, &s_abort)) {
+          for (int j = 0; j < 8; ++j) w[j] = p.a_shared + (size_t)tok * Is + 8 * c8 + j;
+          float a8[8];
+          if (!await_tagged(w, 8, (uint32_t)l + 1u, a8, p.status, &s_abort)) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) a8[j] = 0.0f;
-        }
+            for (int j = 0; j < 8; ++j) a8[j] = 0.0f;
+          }
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const __nv_bfloat16 hi = __float2bfloat16_rn(a8[j]);
-          const __nv_bfloat16 lo = __float2bfloat16_rn(a8[j] - __bfloat162float(hi));
-          *reinterpret_cast<__nv_bfloat16*>(shi + tok * sss + 2 * (8 * c8 + j)) = hi;
-          *reinterpret_cast<__nv_bfloat16*>(slo + tok * sss + 2 * (8 * c8 + j)) = lo;
+          for (int j = 0; j < 8; ++j) {
+            const __nv_bfloat16 hi = __float2bfloat16_rn(a8[j]);
+            const __nv_bfloat16 lo = __float2bfloat16_rn(a8[j] - __bfloat162float(hi));
+            *reinterpret_cast<__nv_bfloat16*>(shi + tok * sss + 2 * (8 * c8 + j)) = hi;
+            *reinterpret_cast<__nv_bfloat16*>(slo + tok * sss + 2 * (8 * c8 + j)) = lo;
+          }
         }
       }
-    }
-    if (tid == 0) wait_counter(lc + CTR_HINIT, G, p.status, &s_abort);  // every slice of h initialised
-    csync();
-    stamp(p, l, 6);
-    for (int r = 0; r < W.nS; ++r, ++i) {
-      const uint32_t s0 = ring_take(pos, bytesS, R);
-      if ((int)(i % STEP_CONSUMERS) != warp) continue;
-      const int slot = (int)(i % STEP_SLOTS);
-      const Item it = W.at(p, W.nA + r);
-      // 4 output rows (N) against the activation rows m = 2*token + {hi, lo} (M)
-      float c[4] = {0.f, 0.f, 0.f, 0.f};
-      item_stamp(p, i, 3);
-      if (ring_wait(&full[slot], (uint32_t)((i / STEP_SLOTS) & 1), p.status, &s_abort)) {
-        item_stamp(p, i, 1);
-        if (M == 1) {
-          // the full hi + lo sum lands in lane group 0; group 1 adds zeros below
-          float o[4];
-          rows4_dot_m1(ring + s0, 2u * Is, 0x3210u, shi, slo, Is, o);
-          c[0] = g == 0 ? (t == 0 ? o[0] : o[2]) : 0.0f;
-          c[1] = g == 0 ? (t == 0 ? o[1] : o[3]) : 0.0f;
+      if (tid == 0) wait_counter(lc + CTR_HINIT, G, p.status, &s_abort);  // every slice of h initialised
+      csync();
+      stamp(p, l, 6);
+      for (int r = 0; r < W.nS; ++r) {
+        const uint8_t* src;
+        uint64_t* eb;
+        bool ready;
+        if constexpr (ONE) {
+          if ((r + 4) % STEP_CONSUMERS != warp) continue;
+          src = fixS + (size_t)r * bytesS;
+          eb = &emptyS[r];
+          ready = ring_wait(&fullS[r], (uint32_t)(l & 1), p.status, &s_abort);
         } else {
-          const uint8_t* src = (g & 1) ? slo : shi;
-          const int t0 = g >> 1, t1 = 4 + (g >> 1);
-          rows4_dot(ring + s0, 2u * Is, g < 4 ? g : -1, t0 < M ? src + t0 * sss : nullptr,
-                    t1 < M ? src + t1 * sss : nullptr, Is, c);
+          const uint32_t s0 = ring_take(pos, bytesS, R);
+          const long long ii = i++;
+          if ((int)(ii % STEP_CONSUMERS) != warp) continue;
+          const int slot = (int)(ii % STEP_SLOTS);
+          src = ring + s0;
+          eb = &empty[slot];
+          item_stamp(p, ii, 3);
+          ready = ring_wait(&full[slot], (uint32_t)((ii / STEP_SLOTS) & 1), p.status, &s_abort);
         }
-      }
-      __syncwarp();
-      item_stamp(p, i, 2);
-      if (lane == 0) mbar_arrive(&empty[slot]);
-      // hi + lo: rows m = 2tok (lane group g even) and 2tok + 1 (g odd)
+        ready = __all_sync(0xffffffffu, ready);
+        const Item it = W.at(p, W.nA + r);
+        // 4 output rows (N) against the activation rows m = 2*token + {hi, lo} (M)
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+        if (ready) {
+          if constexpr (ONE) {
+            // the full hi + lo sum lands in lane group 0; group 1 adds zeros below
+            float o[4];
+            rows4_dot_m1(src, 2u * Is, 0x3210u, shi, slo, Is, o);
+            c[0] = g == 0 ? (t == 0 ? o[0] : o[2]) : 0.0f;
+            c[1] = g == 0 ? (t == 0 ? o[1] : o[3]) : 0.0f;
+          } else {
+            const uint8_t* sa = (g & 1) ? slo : shi;
+            const int t0 = g >> 1, t1 = 4 + (g >> 1);
+            rows4_dot(src, 2u * Is, g < 4 ? g : -1, t0 < M ? sa + t0 * sss : nullptr,
+                      t1 < M ? sa + t1 * sss : nullptr, Is, c);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(eb);
+        // hi + lo: rows m = 2tok (lane group g even) and 2tok + 1 (g odd)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) c[e] += __shfl_xor_sync(0xffffffffu, c[e], 4);
-      if ((g & 1) == 0 && t < 2) {
-        const int t0 = g >> 1, t1 = 4 + (g >> 1);
-        if (t0 < M) {
-          atomicAdd(hout + (size_t)t0 * H + it.a + 2 * t, c[0]);
-          atomicAdd(hout + (size_t)t0 * H + it.a + 2 * t + 1, c[1]);
-        }
-        if (t1 < M) {
-          atomicAdd(hout + (size_t)t1 * H + it.a + 2 * t, c[2]);
-          atomicAdd(hout + (size_t)t1 * H + it.a + 2 * t + 1, c[3]);
+        for (int e = 0; e < 4; ++e) c[e] += __shfl_xor_sync(0xffffffffu, c[e], 4);
+        if ((g & 1) == 0 && t < 2) {
+          const int t0 = g >> 1, t1 = 4 + (g >> 1);
+          if (t0 < M) {
+            atomicAdd(hout + (size_t)t0 * H + it.a + 2 * t, c[0]);
+            atomicAdd(hout + (size_t)t0 * H + it.a + 2 * t + 1, c[1]);
+          }
+          if (t1 < M) {
+            atomicAdd(hout + (size_t)t1 * H + it.a + 2 * t, c[2]);
+            atomicAdd(hout + (size_t)t1 * H + it.a + 2 * t + 1, c[3]);
+          }
         }
       }
-    }
-    stamp(p, l, 7);
+      stamp(p, l, 7);
+      if (tid == 0) blk_stamp(p, l, 5);
+    };
+    if constexpr (!ONE) shared_w2();
 
     // ---- B: routed W13 + SwiGLU ----
-    // Groups of consecutive tiles of one expert share a ring item; tile j of a group
-    // (global tile tc + j of this phase) is computed by warp (tc + j) % 8, and the last
-    // warp to finish a group releases it.
+    // Groups of consecutive tiles of one expert share a ring item.  One token: the
+    // units (gate row, up row of one intermediate index) of the block's range go
+    // round-robin to the 16 half-warps, each unit a lanes-along-K product over its two
+    // rows.  A window: tile j of a group (global tile tc + j of this phase) is computed
+    // by warp (tc + j) % 8 on the tensor core.  The last warp to finish a group's
+    // share releases the group; expert u's counter reaches I (one token: units) or
+    // I/8 (a window: tiles) when its activations are complete.
     W.init_routed(p, P.n_unique);
-    {
+    if constexpr (ONE) {
+      GroupWalk gb{W.b0, W.b0 + W.nB, p.I / 8, capB};
+      int u, r0, nt, q0 = 0;
+      const int hw = 2 * warp + (lane >> 4);  // half-warp 0..15
+      while (gb.next(u, r0, nt)) {
+        const uint32_t codes = (uint32_t)nt * 8u * (H / 2), scales = (uint32_t)nt * 8u * (H / 32);
+        const uint32_t s0 = ring_take(pos, 2 * codes + 2 * scales, R);
+        const int slot = (int)(i % STEP_SLOTS);
+        const int U = 8 * nt;
+        const int f = ((hw - q0) % 16 + 16) % 16;  // my first unit of the group
+        const int nmine = f < U ? (U - 1 - f) / 16 + 1 : 0;
+        const int nw = max(__shfl_sync(0xffffffffu, nmine, 0), __shfl_sync(0xffffffffu, nmine, 16));
+        if (nw > 0) {
+          item_stamp(p, i, 3);
+          const bool ready =
+              __all_sync(0xffffffffu, ring_wait(&full[slot], (uint32_t)((i / STEP_SLOTS) & 1), p.status, &s_abort));
+          item_stamp(p, i, 1);
+          const uint8_t* gate = ring + s0;
+          const uint8_t* up = gate + codes;
+          const uint8_t* gs = gate + 2 * codes;
+          const uint8_t* us = gs + scales;
+          for (int m = 0; m < nw; ++m) {
+            const int q = f + 16 * m;
+            const bool live = q < U;
+            const int qq = live ? q : 0;
+            const uint8_t* const rows[2] = {gate + qq * (H / 2), up + qq * (H / 2)};
+            const uint8_t* const scs[2] = {gs + qq * (H / 32), us + qq * (H / 32)};
+            float r[2] = {0.0f, 0.0f};
+            if (ready) rows_dot_m1_exact<16, 2>(rows, scs, H / 32, xf16, s_sh[0], r);
+            if (live && (lane & 15) == 0) p.a_routed[(size_t)u * I + 8 * r0 + q] = silu_f32(r[0]) * r[1];
+          }
+          __syncwarp();
+          item_stamp(p, i, 2);
+          const int done = __shfl_sync(0xffffffffu, nmine, 0) + __shfl_sync(0xffffffffu, nmine, 16);
+          if (lane == 0) {
+            if (done > 0) {
+              __threadfence();
+              atomicAdd(lc + CTR_EXP + u, (unsigned)done);
+            }
+            if (atomicAdd(&s_gdone[slot], done) + done == U) {
+              s_gdone[slot] = 0;
+              mbar_arrive(&empty[slot]);
+            }
+          }
+        }
+        q0 += U;
+        ++i;
+      }
+    } else {
       GroupWalk gb{W.b0, W.b0 + W.nB, p.I / 8, capB};
       int u, r0, nt, tc = 0;
       while (gb.next(u, r0, nt)) {
@@ -1103,15 +1438,14 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
             float c[4] = {0.f, 0.f, 0.f, 0.f};
             if (ready) {
               const int rg = 8 * j + g;  // tile row: gate row and up row of intermediate 8 (r0 + j) + g
-              mxfp4_tile_dot(gate + rg * (H / 2), up + rg * (H / 2), gs + rg * (H / 32), us + rg * (H / 32), H / 32,
-                             xf16, xss, M, c);
+              mxfp4_tile_dot_win(gate + rg * (H / 2), up + rg * (H / 2), gs + rg * (H / 32), us + rg * (H / 32),
+                                 H / 32, xf16, xss, M, s_sh, c);
             }
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
               const int tok = 2 * t + e;
               if (tok < M)
-                p.a_routed[((size_t)u * M + tok) * I + 8 * (r0 + j) + g] =
-                    silu_f32(c[e] * s_inv[tok]) * (c[2 + e] * s_inv[tok]);
+                p.a_routed[((size_t)u * M + tok) * I + 8 * (r0 + j) + g] = silu_f32(c[e]) * c[2 + e];
             }
             __syncwarp();
             if (lane == 0) signal_counter(lc + CTR_EXP + u);
@@ -1127,6 +1461,8 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
       }
     }
     stamp(p, l, 8);
+    if (tid == 0) blk_stamp(p, l, 6);
+    if constexpr (ONE) shared_w2();
     csync();  // xf16 and the shared halves are dead: the routed-W2 activation copies take the region
     stamp(p, l, 9);
 
@@ -1140,7 +1476,7 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
       const int u_last = W.at(p, baseC + W.nC - 1).a;
       const int u = u_first + warp;
       if (warp < CR_CACHE && u <= u_last) {
-        if (lane == 0) wait_counter(lc + CTR_EXP + u, (unsigned)(I / 8), p.status, &s_abort);
+        if (lane == 0) wait_counter(lc + CTR_EXP + u, (unsigned)(ONE ? I : I / 8), p.status, &s_abort);
         __syncwarp();
         uint8_t* dst = afc + (size_t)warp * M * ass;
         for (int tok = 0; tok < M; ++tok) {
@@ -1157,25 +1493,75 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
           const int sh = f16_range_shift(amax);
-          const float scl = exp2i(sh);
 #pragma unroll
           for (int jj = 0; jj < 8; ++jj) {
             const int c4 = lane + 32 * jj;
             if (c4 < I / 4) {
-              const __half2 h0 = __floats2half2_rn(v[jj].x * scl, v[jj].y * scl);
-              const __half2 h1 = __floats2half2_rn(v[jj].z * scl, v[jj].w * scl);
+              const __half2 h0 = __floats2half2_rn(mul_pow2(v[jj].x, sh), mul_pow2(v[jj].y, sh));
+              const __half2 h1 = __floats2half2_rn(mul_pow2(v[jj].z, sh), mul_pow2(v[jj].w, sh));
               uint2 u2;
               u2.x = *reinterpret_cast<const uint32_t*>(&h0);
               u2.y = *reinterpret_cast<const uint32_t*>(&h1);
-              *reinterpret_cast<uint2*>(dst + tok * ass + 8 * c4) = u2;
+              *reinterpret_cast<uint2*>(dst + (ONE ? chunk_major_off(4 * c4, I / 32) : tok * ass + 8 * c4)) = u2;
             }
           }
-          if (lane == 0) s_pscale[warp][tok] = live ? exp2i(-sh) : 0.0f;
+          if (lane == 0) s_ash[warp][tok] = sh;
         }
       }
       csync();
     }
-    {
+    if constexpr (ONE) {
+      // one token: the block's W2 rows go round-robin to 32 row slots of 8 lanes (4
+      // per warp), each slot taking its rows of a group two at a time (same expert:
+      // the activation chunks load once for both), lanes along K
+      GroupWalk gc{W.c0, W.c0 + W.nC, p.H / 16, capC};
+      int u, c0, nt, q0 = 0;
+      const int rs = 4 * warp + (lane >> 3);  // row slot 0..31
+      while (gc.next(u, c0, nt)) {
+        const uint32_t codes = (uint32_t)nt * 16u * (I / 2), scales = (uint32_t)nt * 16u * (I / 32);
+        const uint32_t s0 = ring_take(pos, codes + scales, R);
+        const int slot = (int)(i % STEP_SLOTS);
+        const int Rg = 16 * nt;
+        const int f = ((rs - q0) % 32 + 32) % 32;  // my first row of the group
+        const int nmine = f < Rg ? (Rg - 1 - f) / 32 + 1 : 0;
+        int nw = max(nmine, __shfl_xor_sync(0xffffffffu, nmine, 8));
+        nw = max(nw, __shfl_xor_sync(0xffffffffu, nw, 16));
+        if (nw > 0) {
+          const int cu = u - u_first;  // cache entry
+          const uint8_t* my_af = afc + (size_t)cu * ass;
+          item_stamp(p, i, 3);
+          const bool ready =
+              __all_sync(0xffffffffu, ring_wait(&full[slot], (uint32_t)((i / STEP_SLOTS) & 1), p.status, &s_abort));
+          item_stamp(p, i, 1);
+          const uint8_t* cd = ring + s0;
+          const uint8_t* sc = cd + codes;
+          const float wt = P.w[u][0];
+          for (int m = 0; m < nw; m += 2) {
+            const int qa = f + 32 * m, qb = qa + 32;
+            const bool la = qa < Rg, lb = qb < Rg;
+            const int ra = la ? qa : 0, rb = lb ? qb : 0;
+            const uint8_t* const rows[2] = {cd + ra * (I / 2), cd + rb * (I / 2)};
+            const uint8_t* const scs[2] = {sc + ra * (I / 32), sc + rb * (I / 32)};
+            float r[2] = {0.0f, 0.0f};
+            if (ready) rows_dot_m1_exact<8, 2>(rows, scs, I / 32, my_af, s_ash[cu][0], r);
+            if ((lane & 7) == 0 && wt != 0.0f) {
+              if (la) atomicAdd(hout + 16 * c0 + qa, r[0] * wt);
+              if (lb) atomicAdd(hout + 16 * c0 + qb, r[1] * wt);
+            }
+          }
+          __syncwarp();
+          item_stamp(p, i, 2);
+          int done = nmine + __shfl_xor_sync(0xffffffffu, nmine, 8);
+          done += __shfl_xor_sync(0xffffffffu, done, 16);
+          if (lane == 0 && atomicAdd(&s_gdone[slot], done) + done == Rg) {
+            s_gdone[slot] = 0;
+            mbar_arrive(&empty[slot]);
+          }
+        }
+        q0 += Rg;
+        ++i;
+      }
+    } else {
       GroupWalk gc{W.c0, W.c0 + W.nC, p.H / 16, capC};
       int u, c0, nt, tc = 0;
       while (gc.next(u, c0, nt)) {
@@ -1196,8 +1582,8 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
             float c[4] = {0.f, 0.f, 0.f, 0.f};
             const int rg = 16 * j + g;  // tile rows rg and rg + 8: output rows 16 (c0 + j) + g (+8)
             if (ready)
-              mxfp4_tile_dot(cd + rg * (I / 2), cd + (rg + 8) * (I / 2), sc + rg * (I / 32), sc + (rg + 8) * (I / 32),
-                             I / 32, my_af, ass, M, c);
+              mxfp4_tile_dot_win(cd + rg * (I / 2), cd + (rg + 8) * (I / 2), sc + rg * (I / 32),
+                                 sc + (rg + 8) * (I / 32), I / 32, my_af, ass, M, s_ash[cu], c);
             const int h0 = 16 * (c0 + j) + g;
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
@@ -1205,9 +1591,8 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
               if (tok < M) {
                 const float wt = P.w[u][tok];
                 if (wt != 0.0f) {
-                  const float f = wt * s_pscale[cu][tok];
-                  atomicAdd(hout + (size_t)tok * H + h0, c[e] * f);
-                  atomicAdd(hout + (size_t)tok * H + h0 + 8, c[2 + e] * f);
+                  atomicAdd(hout + (size_t)tok * H + h0, c[e] * wt);
+                  atomicAdd(hout + (size_t)tok * H + h0 + 8, c[2 + e] * wt);
                 }
               }
             }
@@ -1225,6 +1610,7 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
     }
     stamp(p, l, 10);
     csync();
+    if (tid == 0) blk_stamp(p, l, 7);
     if (tid == 0) signal_counter(lc + CTR_H);
     stamp(p, l, 11);
   }

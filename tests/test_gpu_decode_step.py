@@ -45,6 +45,7 @@ def _check_step(model, shape, x, res, layers_to_check):
     xt = res["x_trace"]
     ht = res["h_trace"].cpu().numpy()
     ids_t = res["ids_trace"].cpu().numpy()
+    w_t = res["w_trace"].cpu().numpy()
     L = len(model.layers)
     M = x.shape[0]
     np.testing.assert_array_equal(synth.bits(xt[0]), synth.bits(x))
@@ -52,14 +53,16 @@ def _check_step(model, shape, x, res, layers_to_check):
     for l in layers_to_check:
         Ly = model.layers[l]
         xl = synth.bits(xt[l])
-        o_ids, o_w, _, margin = oracle.route(xl, synth.bits(Ly["wr"]), shape.k)
+        o_ids, o_w, o_lg, margin = oracle.route(xl, synth.bits(Ly["wr"]), shape.k)
         ids_use = o_ids.copy()
         for t in range(M):
             if margin[t] >= MARGIN_FLAG:
                 assert list(ids_t[l, t]) == list(o_ids[t]), (l, t)
             else:
                 ids_use[t] = ids_t[l, t]  # flagged near-tie: follow the GPU's choice
-        w_use = oracle.softmax_weights_at(oracle.route(xl, synth.bits(Ly["wr"]), shape.k)[2], ids_use)
+        w_use = oracle.softmax_weights_at(o_lg, ids_use)
+        # the routing weights the step used, against the oracle's softmax at the same ids
+        np.testing.assert_allclose(w_t[l], w_use, rtol=1e-5, atol=1e-6, err_msg=f"layer {l} routing weights")
         y_ref = oracle.moe_layer(xl, ids_use, w_use, _fetch(Ly),
                                  {"sw13": synth.bits(Ly["sw13"]), "sw2": synth.bits(Ly["sw2"])})
         dh = ht[l + 1].astype(np.float64) - ht[l].astype(np.float64)
@@ -96,17 +99,26 @@ def test_tiny_chain_all_layers(M, path):
 
 
 def test_tiny_chain_free_running_matches_oracle_chain():
+    """The step run free (no teacher forcing) against the oracle's own chain.  A
+    near-tie routing decision anywhere in the chain would let the two follow different
+    experts legitimately, so the seed is the first of a fixed list whose oracle chain
+    has no decision closer than the flag margin; the test fails if none has."""
     S = synth.TINY
-    model = _model(S, 3, 1000, 31)
-    x = synth.tokens(2, S.H, 31, device="cuda")
+    for seed in range(31, 39):
+        model = _model(S, 3, 1000, seed)
+        x = synth.tokens(2, S.H, seed, device="cuda")
+        spec = [{"wr": synth.bits(L["wr"]), "experts": _fetch(L),
+                 "shared": {"sw13": synth.bits(L["sw13"]), "sw2": synth.bits(L["sw2"])}} for L in model.layers]
+        out = oracle.decode_step(synth.bits(x), spec, synth.bits(model.lm_q), model.lm_s.cpu().numpy(), S.k)
+        if all(np.all(m >= MARGIN_FLAG) for m in out["margin"]):
+            break
+    else:
+        pytest.fail("no seed in 31..38 gives a chain without near-tie routing decisions")
     res = decode_step(model, x, trace=True)
     torch.cuda.synchronize()
-    spec = [{"wr": synth.bits(L["wr"]), "experts": _fetch(L),
-             "shared": {"sw13": synth.bits(L["sw13"]), "sw2": synth.bits(L["sw2"])}} for L in model.layers]
-    out = oracle.decode_step(synth.bits(x), spec, synth.bits(model.lm_q), model.lm_s.cpu().numpy(), S.k)
-    if all(np.all(m >= MARGIN_FLAG) for m in out["margin"]):
-        assert_rows_close(res["h_trace"][-1].cpu().numpy(), out["h"], what="free-running h_L")
-        assert_rows_close(res["logits"].cpu().numpy(), out["logits"], what="free-running logits")
+    np.testing.assert_array_equal(res["ids_trace"].cpu().numpy(), np.stack(out["ids"]))
+    assert_rows_close(res["h_trace"][-1].cpu().numpy(), out["h"], what="free-running h_L")
+    assert_rows_close(res["logits"].cpu().numpy(), out["logits"], what="free-running logits")
 
 
 @pytest.mark.parametrize("M", [2, 3, 5, 8])
