@@ -74,7 +74,7 @@ typedef enum {
 /* Human-readable name of a status value (static storage). */
 MOE_API const char* moe_status_string(int status);
 /* ABI version of this header: MOE_ABI_VERSION. */
-#define MOE_ABI_VERSION 1
+#define MOE_ABI_VERSION 2
 MOE_API int moe_abi_version(void);
 /* cudaError_t of the last MOE_ERR_CUDA returned on the calling thread (0 if none). */
 MOE_API int moe_last_cuda_error(void);
@@ -288,7 +288,13 @@ enum { MOE_STEP_AUTO = 0, MOE_STEP_PER_LAYER = 1 };
  *     acquired, data ready, done, wait started, producer entered, copies issued, 2 unused),
  *     then [G][L][16] phase ends of every block (residual seen, input staged, router item
  *     published, router/shared-W13 items done, plan built, shared W2 done, routed W13
- *     done, routed W2 done, then finer marks inside the top-k and the staging). */
+ *     done, routed W2 done, then finer marks inside the top-k and data arrivals).
+ *   wait_limit_ns: 0, or a shorter limit for every bounded device wait of the step (the
+ *     default is 2 s): for testing the timeout path only.
+ *   hold_layer: 0, or l + 1 to make the persistent step never publish layer l's residual,
+ *     so the next wait on it can only time out: with a short wait_limit_ns this drives
+ *     the step's timeout path (MOE_ERR_TIMEOUT from moe_workspace_status; the kernels
+ *     return early, every output is then undefined).  Ignored on the per-layer path. */
 typedef struct {
   void* x;
   float* h;
@@ -297,6 +303,8 @@ typedef struct {
   void** events;
   int n_events;
   unsigned long long* timeline;
+  unsigned long long wait_limit_ns;
+  int hold_layer;
 } moe_trace_t;
 
 MOE_API size_t decode_step_workspace_bytes(const moe_model_t* model, int M);

@@ -38,7 +38,7 @@ STEP_AUTO, STEP_PER_LAYER = 0, 1
 
 class Trace(ctypes.Structure):
     _fields_ = [("x", P), ("h", P), ("ids", P), ("w", P), ("events", ctypes.POINTER(P)), ("n_events", I),
-                ("timeline", P)]
+                ("timeline", P), ("wait_limit_ns", ctypes.c_ulonglong), ("hold_layer", I)]
 
 
 # name -> (restype, argtypes); every symbol the header declares

@@ -334,11 +334,13 @@ def _event_array(events):
 
 
 def decode_step(model: DecodeModel, x: torch.Tensor, *, want_logits: bool = True, trace: bool = False, ws=None,
-                out=None, stream=None, events=None, timeline=None):
+                out=None, stream=None, events=None, timeline=None, wait_limit_ns: int = 0, hold_layer=None):
     """One decode step.  Returns dict(logits, argmax[, trace tensors]).
 
     ``events``: optional list of torch.cuda.Event(enable_timing=True), recorded in
-    pairs around each kernel launch of the step (see moe_trace_t)."""
+    pairs around each kernel launch of the step (see moe_trace_t).  ``wait_limit_ns`` and
+    ``hold_layer`` exercise the timeout path (a layer whose residual is never published,
+    and a short limit on every bounded device wait): testing only."""
     _dev_bf16(x, "x")
     M, H = x.shape
     dev = x.device
@@ -363,10 +365,13 @@ def decode_step(model: DecodeModel, x: torch.Tensor, *, want_logits: bool = True
                         res["w_trace"].data_ptr(), evs, nev)
     elif evs is not None:
         tr = _abi.Trace(None, None, None, None, evs, nev)
-    if timeline is not None:
+    if timeline is not None or wait_limit_ns or hold_layer is not None:
         if tr is None:
             tr = _abi.Trace(None, None, None, None, None, 0)
-        tr.timeline = timeline.data_ptr()
+        if timeline is not None:
+            tr.timeline = timeline.data_ptr()
+        tr.wait_limit_ns = int(wait_limit_ns)
+        tr.hold_layer = 0 if hold_layer is None else int(hold_layer) + 1
     if ws is None:
         ws = _ws(_lib().decode_step_workspace_bytes(ctypes.byref(m), M), dev)
     _check("decode_step", _lib().decode_step(ctypes.byref(m), _ptr(x), M, _ptr(logits), _ptr(am),

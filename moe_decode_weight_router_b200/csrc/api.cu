@@ -16,7 +16,6 @@
 #include "decode_kernels.cuh"
 #include "lmhead_kernels.cuh"
 #include "step_kernel.cuh"
-#include "step1_kernel.cuh"
 #include "prefill_kernels.cuh"
 #include "sample_kernels.cuh"
 
@@ -78,7 +77,7 @@ moe_status_t dev_info(DevInfo* out) {
     MOE_CUDA(allow_dyn_smem(k_experts2, lim, &d.dyn_e2));
     MOE_CUDA(allow_dyn_smem(k_lm_gemv, lim, &d.dyn_lm));
     MOE_CUDA(allow_dyn_smem(k_step<false>, lim, &d.dyn_step));
-    MOE_CUDA(allow_dyn_smem(k_step1, lim, &d.dyn_step));
+    MOE_CUDA(allow_dyn_smem(k_step<true>, lim, &d.dyn_step));
     MOE_CUDA(allow_dyn_smem(k_umma, lim, &d.dyn_pf));
     MOE_CUDA(cudaDeviceGetAttribute(&d.coop, cudaDevAttrCooperativeLaunch, dev));
     cache[dev] = d;
@@ -242,47 +241,25 @@ moe_status_t launch_lm(LMParams p, const DevInfo& d, cudaStream_t st) {
 // STEP_MAX_LAYERS layers, H a multiple of 128 (router/shared tiles split into four
 // 32-column-aligned quarters), cooperative launch available, and a shared-memory
 // ring next to the activation region that holds at least N_CONSUMERS of the
-// largest items (one per consumer warp in flight).  For one token the block's
-// router/shared-W13 items and shared-W2 items (at most STEP_FIX_MAX of each) have
-// fixed regions of their own and the ring carries the routed items only.
-struct StepLayout {
-  bool one = false;  // the one-token kernel (k_step1)
-  uint32_t ring = 0, fixa = 0, fixs = 0;
-};
-bool use_persistent(const moe_model_t& m, int M, const DevInfo& d, StepLayout* lay) {
+// largest items (one per consumer warp in flight).
+bool use_persistent(const moe_model_t& m, int M, const DevInfo& d, uint32_t* ring_bytes) {
   if (m.step_path == MOE_STEP_PER_LAYER) return false;
   if (m.n_layers > STEP_MAX_LAYERS || m.H % 128 != 0 || !d.coop) return false;
-  const size_t act = step_act_bytes(M, m.H, m.I, m.Is);
-  StepLayout L;
-  if (M == 1) {
-    // one token: contiguous per-block shares in regions X and Y; the routed ranges
-    // span at most two experts (k * I <= I * SMs), and the shared-W2 activation
-    // halves fit over the dead bf16 layer input
-    const Step1Sizes z = step1_sizes(m.H, m.I, m.Is, m.E, m.top_k, d.sms);
-    if (z.nu > m.I || z.nw > m.H || !step_shared_over_xb16(m.H, m.Is)) return false;
-    const size_t smem = STEP_FIXED + (size_t)z.x_bytes + z.y_bytes + act;
-    if (smem > (size_t)d.dyn_step) return false;
-    L.one = true;
-    L.fixa = z.x_bytes;
-    L.fixs = z.y_bytes;
-    *lay = L;
-    return true;
-  }
-  const size_t fixed = STEP_FIXED + act;
+  const size_t fixed = STEP_FIXED + step_act_bytes(M, m.H, m.I, m.Is);
   if ((size_t)d.dyn_step <= fixed) return false;
-  L.ring = (uint32_t)(((size_t)d.dyn_step - fixed) / 128 * 128);
-  *lay = L;
+  const size_t ring = ((size_t)d.dyn_step - fixed) / 128 * 128;
+  *ring_bytes = (uint32_t)ring;
   // a block's contiguous routed-W2 range of n items (H/16 per expert) touches at most
   // (n - 2) / (H/16) + 2 experts; their activations must fit the block's cache
   const long long T = m.H / 16;
   const long long n = ((long long)slots_of(M, m.E, m.top_k) * T + d.sms - 1) / d.sms;
   const long long span = n <= 1 ? 1 : (n - 2) / T + 2;
   if (span > CR_CACHE) return false;
-  return L.ring >= (size_t)N_CONSUMERS * step_max_item_bytes(m.H, m.I, m.Is);
+  return ring >= (size_t)N_CONSUMERS * step_max_item_bytes(m.H, m.I, m.Is);
 }
 
 moe_status_t launch_step(const StepParams& sp, const DevInfo& d, cudaStream_t st) {
-  const size_t smem = STEP_FIXED + (size_t)sp.fixa_bytes + sp.fixs_bytes + sp.ring_bytes + sp.act_bytes;
+  const size_t smem = STEP_FIXED + (size_t)sp.ring_bytes + sp.act_bytes;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(d.sms);
   cfg.blockDim = dim3(STEP_THREADS);
@@ -294,11 +271,14 @@ moe_status_t launch_step(const StepParams& sp, const DevInfo& d, cudaStream_t st
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (sp.M == 1)
-    MOE_CUDA(cudaLaunchKernelEx(&cfg, k_step1, sp));
+    MOE_CUDA(cudaLaunchKernelEx(&cfg, k_step<true>, sp));
   else
     MOE_CUDA(cudaLaunchKernelEx(&cfg, k_step<false>, sp));
   return MOE_OK;
 }
+
+// One 64-bit word written on the stream (capturable): the test wait limit of a control block.
+__global__ void k_set_u64(unsigned long long* p, unsigned long long v) { *p = v; }
 
 // Records events[2i] / events[2i+1] around launch i when the caller asked for them.
 struct EventHook {
@@ -645,8 +625,8 @@ int decode_step_launch_names(const moe_model_t* model, int M, const char** names
     if (names && n < max_names) names[n] = nm;
     ++n;
   };
-  StepLayout lay;
-  if (use_persistent(*model, M, d, &lay)) {
+  uint32_t ring_bytes = 0;
+  if (use_persistent(*model, M, d, &ring_bytes)) {
     put("k_step");
   } else {
     for (int l = 0; l < model->n_layers; ++l) {
@@ -682,13 +662,17 @@ moe_status_t decode_step(const moe_model_t* model, const void* x_bf16, int M, fl
   Ctrl c = ctrl_of(ws);
   StepWs w = step_ws(ws, L, M, H, I, E, k, Is);
   MOE_CUDA(cudaMemsetAsync(ws, 0, w.ctrl_bytes, st));
+  if (tr.wait_limit_ns) {
+    k_set_u64<<<1, 1, 0, st>>>(reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(ws) + 16), tr.wait_limit_ns);
+    MOE_CUDA(cudaGetLastError());
+  }
   const __nv_bfloat16* x_in = static_cast<const __nv_bfloat16*>(x_bf16);
   __nv_bfloat16* xt = static_cast<__nv_bfloat16*>(tr.x);
   EventHook hook;
   hook.ev = reinterpret_cast<cudaEvent_t*>(tr.events);
   hook.n = tr.events ? tr.n_events : 0;
-  StepLayout lay;
-  if (use_persistent(*model, M, d, &lay)) {
+  uint32_t ring_bytes = 0;
+  if (use_persistent(*model, M, d, &ring_bytes)) {
     StepParams sp{};
     sp.L = L;
     sp.M = M;
@@ -698,9 +682,7 @@ moe_status_t decode_step(const moe_model_t* model, const void* x_bf16, int M, fl
     sp.k = k;
     sp.Is = Is;
     sp.eps = model->rms_eps;
-    sp.ring_bytes = lay.ring;
-    sp.fixa_bytes = lay.fixa;
-    sp.fixs_bytes = lay.fixs;
+    sp.ring_bytes = ring_bytes;
     sp.act_bytes = step_act_bytes(M, H, I, Is);
     sp.x_in = x_in;
     sp.h = w.h;
@@ -715,6 +697,7 @@ moe_status_t decode_step(const moe_model_t* model, const void* x_bf16, int M, fl
     sp.ids_trace = tr.ids;
     sp.w_trace = tr.w;
     sp.timeline = tr.timeline;
+    sp.hold_layer = tr.hold_layer - 1;
     for (int l = 0; l < L; ++l) {
       const moe_layer_t& Ly = model->layers[l];
       sp.layer[l] = LayerPtrs{static_cast<const __nv_bfloat16*>(Ly.router.ptr),

@@ -16,9 +16,17 @@ namespace moe {
 // Device-side error codes written to the workspace status word.
 enum : int { DEV_OK = 0, DEV_ERR_TIMEOUT = 7 };
 
-// Every spin-wait gives up after this many nanoseconds of %globaltimer, sets the
-// status word and lets the kernel return instead of hanging the GPU.
+// Every spin-wait gives up after a bounded time of %globaltimer, sets the status word
+// and lets the kernel return instead of hanging the GPU.  The status word is the first
+// word of a 256-byte control block; the 64-bit word 16 bytes after it holds the limit
+// in nanoseconds (0: WAIT_LIMIT_NS).  Callers shorten it only to test the timeout path.
 constexpr unsigned long long WAIT_LIMIT_NS = 2000000000ull;  // 2 s
+__device__ __forceinline__ unsigned long long wait_limit(const int* status) {
+  if (!status) return WAIT_LIMIT_NS;
+  const unsigned long long v =
+      *reinterpret_cast<const volatile unsigned long long*>(reinterpret_cast<const char*>(status) + 16);
+  return v ? v : WAIT_LIMIT_NS;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -74,10 +82,10 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
 // WAIT_LIMIT_NS it records DEV_ERR_TIMEOUT in *status and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status) {
   if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = globaltimer_ns();
+  const unsigned long long t0 = globaltimer_ns(), lim = wait_limit(status);
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
+    if (globaltimer_ns() - t0 > lim) {
       if (status) atomicExch(status, DEV_ERR_TIMEOUT);
       return false;
     }

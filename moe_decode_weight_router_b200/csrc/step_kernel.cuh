@@ -42,15 +42,12 @@ namespace moe {
 
 constexpr int STEP_MAX_LAYERS = 64;
 constexpr int STEP_CONSUMERS = 8;  // consumer warps: two per SM sub-partition, to hide latency
-// Consumer warps 0-7, warp 8 the routed-item producer, warp 9 (one-token kernel) the
-// producer of the routing-independent items.
-constexpr int STEP_THREADS = 32 * (STEP_CONSUMERS + 2);
-constexpr int STEP_FIX_MAX = 8;  // routing-independent items of one kind per block and layer
+constexpr int STEP_THREADS = 32 * (STEP_CONSUMERS + 1);  // consumer warps 0-7, producer warp 8
 constexpr int CR_CACHE = 4;         // routed experts whose W2 activation a block keeps staged
 constexpr int STEP_SLOTS = 32;  // ring items in flight at most (one full/empty mbarrier pair each)
 constexpr int CTR_H = 2, CTR_HINIT = 3, CTR_EXP = 4;  // slots 0-1 unused
 constexpr int CTR_PER_LAYER = CTR_EXP + MAX_SLOTS;
-constexpr size_t STEP_FIXED = 1024;  // full/empty[32], plan, h-init, A and CS full/empty[8] barriers
+constexpr size_t STEP_FIXED = 1024;  // full[32], empty[32], plan and h-init barriers
 constexpr int STAGE_REG_F4 = 4;  // residual float4s a consumer thread keeps in registers (M = 1 at H = 2560)
 constexpr int STAGE_BATCH = 5;   // larger inputs: residual loads a thread keeps in flight
 
@@ -69,8 +66,6 @@ struct StepParams {
   float eps;
   uint32_t ring_bytes;
   uint32_t act_bytes;
-  uint32_t fixa_bytes;  // one-token kernel: region of this block's router/shared-W13 items (0: in the ring)
-  uint32_t fixs_bytes;  // one-token kernel: region of this block's shared-W2 items (0: in the ring)
   const __nv_bfloat16* x_in;  // [M][H]
   float* h;                   // [2][M][H] residual stream, buffer l & 1 is layer l's output
   __nv_bfloat16* x_final;     // [M][H] LM-head input
@@ -84,6 +79,7 @@ struct StepParams {
   int32_t* ids_trace;
   float* w_trace;
   unsigned long long* timeline;  // optional [2][L][16] %globaltimer stamps (blocks 0 and G-1)
+  int hold_layer;                // testing the timeout path: this layer's residual is never published (-1: none)
   LayerPtrs layer[STEP_MAX_LAYERS];
 };
 
@@ -221,12 +217,12 @@ __device__ __forceinline__ void signal_counter(unsigned* c) {
 __device__ __noinline__ bool wait_counter(const unsigned* c, unsigned target, int* status, volatile int* abort_flag) {
   if (*abort_flag) return false;
   if (ld_acquire_u32(c) >= target) return true;
-  const unsigned long long t0 = globaltimer_ns();
+  const unsigned long long t0 = globaltimer_ns(), lim = wait_limit(status);
   while (true) {
     __nanosleep(32);
     if (ld_acquire_u32(c) >= target) return true;
     if (*abort_flag) return false;
-    if (ld_volatile_i32(status) != 0 || globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
+    if (ld_volatile_i32(status) != 0 || globaltimer_ns() - t0 > lim) {
       atomicCAS(status, 0, DEV_ERR_TIMEOUT);
       *abort_flag = 1;
       return false;
@@ -241,11 +237,11 @@ __device__ __forceinline__ bool ring_wait(uint64_t* bar, uint32_t parity, int* s
   return ring_wait_slow(bar, parity, status, abort_flag);
 }
 __device__ __noinline__ bool ring_wait_slow(uint64_t* bar, uint32_t parity, int* status, volatile int* abort_flag) {
-  const unsigned long long t0 = globaltimer_ns();
+  const unsigned long long t0 = globaltimer_ns(), lim = wait_limit(status);
   while (true) {
     if (mbar_try_wait_sleep(bar, parity, 500u)) return true;  // suspended, not spinning
     if (*abort_flag) return false;
-    if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
+    if (globaltimer_ns() - t0 > lim) {
       atomicCAS(status, 0, DEV_ERR_TIMEOUT);
       *abort_flag = 1;
       return false;
@@ -278,7 +274,7 @@ __device__ __forceinline__ bool await_tagged(const unsigned long long* const* w,
     if (ok) break;
     if (*abort_flag) return false;
     if (t0 == 0) t0 = globaltimer_ns();
-    if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
+    if (globaltimer_ns() - t0 > wait_limit(status)) {
       step_give_up(status, abort_flag);
       return false;
     }
@@ -290,10 +286,11 @@ __device__ __forceinline__ bool await_tagged(const unsigned long long* const* w,
   return true;
 }
 // Time-bounded wait for a copy to land, used only when the block is about to exit
-// (the abort flag is ignored: copies in flight must finish before shared memory goes).
+// (the abort flag is ignored: copies in flight must finish before shared memory goes;
+// the full default limit, whatever the test limit, since a copy in flight always lands).
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   const unsigned long long t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity))
+  while (!mbar_try_wait_sleep(bar, parity, 500u))
     if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) return;
 }
 
@@ -508,6 +505,19 @@ struct Producer {
 // ---------------------------------------------------------------------------
 // Consumer-only barrier (the 4 consumer warps; the producer never joins).
 __device__ __forceinline__ void csync() { named_barrier(1, 32 * STEP_CONSUMERS); }
+// Consumer barrier that also returns, to every consumer thread, whether any of them
+// passed a true predicate (one decision for the whole block: leaving a loop on it
+// never splits the consumers across a later barrier).
+__device__ __forceinline__ bool csync_or(bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, %2, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(32 * STEP_CONSUMERS)
+      : "memory");
+  return r != 0;
+}
 
 // The layer input in two forms: bf16 x_l (router / shared-expert operand) at
 // xb16 and f16 x_l scaled by a per-token power of two (MXFP4 operand) at xf16.
@@ -823,9 +833,11 @@ __device__ void step_topk(const StepParams& p, int l, Plan& P, int32_t* s_ids, f
       topk_token_full(p, l, tok, sel, s_abort_ptr);
     }
     __syncwarp();
-    // lane j holds the j-th selection; softmax over the selected logits
+    // lane j holds the j-th selection; softmax over the selected logits.  An id outside
+    // [0, E) (only after a failed wait) is replaced by 0 so nothing reads out of bounds.
     const unsigned long long sj = lane < k ? sel[lane] : 0ull;
-    const int sel_id = (int)(~(uint32_t)sj);
+    int sel_id = (int)(~(uint32_t)sj);
+    sel_id = (unsigned)sel_id < (unsigned)E ? sel_id : 0;
     const float lj = key_float((uint32_t)(sj >> 32));
     const float l0 = __shfl_sync(0xffffffffu, lj, 0);
     const float ex = lane < k ? expf(lj - l0) : 0.0f;
@@ -927,6 +939,157 @@ __device__ __forceinline__ void rows_dot_m1_exact(const uint8_t* const (&rows)[R
   bool bad = false;
   rows_dot_m1<LPR, R, false>(rows, scs, nb, xc, sh, bad, out);
   if (__any_sync(0xffffffffu, bad)) rows_dot_m1_safe<LPR, R>(rows, scs, nb, xc, sh, out);
+}
+
+// The one-token layer input: x = bf16(RMSNorm(h)) (layer 0: the given x) as bf16 at xb16
+// and as f16 scaled by 2^sh (largest magnitude in [2^14, 2^15)) chunk-major at xf16; the
+// same pass copies this block's slice [q0, q1) of h into hout.  Every thread forms the
+// norm and the shift from the 8 warp partials in the same order, so every block gets
+// the same bits (each block takes the top-k itself).  One barrier.
+__device__ void stage1(const StepParams& p, int l, const float* hin, float* hout, uint8_t* xb16, uint8_t* xf16,
+                       float* s_part, float* s_amx, int* s_sh, int q0, int q1) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nt = 32 * STEP_CONSUMERS;
+  const int H = p.H, Q = H / 4, nb = H / 32;
+  float4 v[STAGE_REG_F4];
+  float ss = 0.0f, am = 0.0f;
+#pragma unroll
+  for (int j = 0; j < STAGE_REG_F4; ++j) {
+    const int q = tid + nt * j;
+    v[j] = q < Q ? load_residual4(p, l, hin, q) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+#pragma unroll
+  for (int j = 0; j < STAGE_REG_F4; ++j) {
+    const int q = tid + nt * j;
+    if (q >= q0 && q < q1) reinterpret_cast<float4*>(hout)[q] = v[j];
+    accumulate4(v[j], ss, am);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+  }
+  if (lane == 0) {
+    s_part[warp] = ss;
+    s_amx[warp] = am;
+  }
+  csync();
+  float t = 0.0f, a = 0.0f;
+#pragma unroll
+  for (int w = 0; w < STEP_CONSUMERS; ++w) {
+    t += s_part[w];
+    a = fmaxf(a, s_amx[w]);
+  }
+  const float r = l == 0 ? 1.0f : 1.0f / sqrtf(t / (float)H + p.eps);
+  const int sh = f16_range_shift(__bfloat162float(__float2bfloat16_rn(a * r)));
+  if (tid == 0) s_sh[0] = sh;
+  const float f1 = exp2i(sh / 2), f2 = exp2i(sh - sh / 2);
+#pragma unroll
+  for (int j = 0; j < STAGE_REG_F4; ++j) {
+    const int q = tid + nt * j;
+    if (q < Q) {
+      const __nv_bfloat162 b0 = __floats2bfloat162_rn(v[j].x * r, v[j].y * r);
+      const __nv_bfloat162 b1 = __floats2bfloat162_rn(v[j].z * r, v[j].w * r);
+      uint2 u;
+      u.x = *reinterpret_cast<const uint32_t*>(&b0);
+      u.y = *reinterpret_cast<const uint32_t*>(&b1);
+      *reinterpret_cast<uint2*>(xb16 + 8 * q) = u;
+      const __half2 h0 = __floats2half2_rn((__low2float(b0) * f1) * f2, (__high2float(b0) * f1) * f2);
+      const __half2 h1 = __floats2half2_rn((__low2float(b1) * f1) * f2, (__high2float(b1) * f1) * f2);
+      u.x = *reinterpret_cast<const uint32_t*>(&h0);
+      u.y = *reinterpret_cast<const uint32_t*>(&h1);
+      *reinterpret_cast<uint2*>(xf16 + chunk_major_off(4 * q, nb)) = u;
+    }
+  }
+  csync();  // also orders this block's slice stores before the h-init hand-off
+}
+
+// One token's top-k and routing plan.  Warp w holds experts [w*per, (w+1)*per),
+// per = E/8 (at most 4 per lane); the smallest of the 8 warp maxima bounds the k-th
+// largest logit, the survivors (at most TOPK_CAND, else the exact k-round selection)
+// are ranked by their order keys, and warp 0 writes the plan directly: the k selected
+// experts are distinct, so slot i holds the i-th smallest id with its weight.
+__device__ void topk1(const StepParams& p, int l, Plan& P, uint32_t* s_wmax, int* s_ncand,
+                      unsigned long long* s_cand, unsigned long long* s_sel, volatile int* s_abort_ptr) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
+  const int E = p.E, k = p.k;
+  const int per = E / STEP_CONSUMERS;
+  const int e0 = warp * per;
+  if (tid == 0) s_ncand[0] = 0;
+  uint32_t key[4];
+  {
+    const unsigned long long* w[8];
+    int n = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int off = lane + 32 * i;
+      w[i] = p.logits + e0 + (i < 4 && off < per ? off : 0);
+      if (i < 4 && off < per) n = i + 1;
+    }
+    float lv[8];
+    if (!await_tagged(w, n, (uint32_t)l + 1u, lv, p.status, s_abort_ptr)) n = 0;
+    uint32_t mx = 0u;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      key[i] = i < n ? float_key(lv[i]) : 0u;
+      mx = max(mx, key[i]);
+    }
+    mx = __reduce_max_sync(0xffffffffu, mx);
+    if (lane == 0) s_wmax[warp] = mx;
+  }
+  if (tid == 0) blk_stamp(p, l, 8);
+  csync();
+  uint32_t bound = 0xFFFFFFFFu;
+#pragma unroll
+  for (int w = 0; w < STEP_CONSUMERS; ++w) bound = min(bound, s_wmax[w]);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int off = lane + 32 * i;
+    if (off < per && key[i] >= bound) {
+      const int pos = atomicAdd(&s_ncand[0], 1);
+      if (pos < TOPK_CAND) s_cand[pos] = order_key(key[i], e0 + off);
+    }
+  }
+  if (tid == 0) blk_stamp(p, l, 9);
+  csync();
+  if (warp == 0) {
+    const int n = s_ncand[0];
+    if (n <= TOPK_CAND) {
+      const unsigned long long mine = lane < n ? s_cand[lane] : 0ull;
+      int rank = 0;
+      for (int j = 0; j < n; ++j) rank += s_cand[j] > mine ? 1 : 0;
+      if (lane < n && rank < k) s_sel[rank] = mine;
+    } else {
+      topk_token_full(p, l, 0, s_sel, s_abort_ptr);
+    }
+    __syncwarp();
+    // lane j holds the j-th selection; softmax over the selected logits
+    // an id outside [0, E) (only after a failed wait) is replaced by 0: nothing reads out of bounds
+    const unsigned long long sj = lane < k ? s_sel[lane] : 0ull;
+    int id = (int)(~(uint32_t)sj);
+    id = (unsigned)id < (unsigned)E ? id : 0;
+    const float lj = key_float((uint32_t)(sj >> 32));
+    const float l0 = __shfl_sync(0xffffffffu, lj, 0);
+    const float ex = lane < k ? expf(lj - l0) : 0.0f;
+    float den = ex;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+    const float wj = ex / den;
+    // plan: slot = number of selected ids below this one
+    int slot = 0;
+    for (int i = 0; i < k; ++i) slot += __shfl_sync(0xffffffffu, id, i) < id ? 1 : 0;
+    if (lane < k) {
+      P.ids[slot] = id;
+      P.w[slot][0] = wj;
+      if (blockIdx.x == 0) {
+        const size_t o = (size_t)l * k + lane;
+        if (p.ids_trace) p.ids_trace[o] = id;
+        if (p.w_trace) p.w_trace[o] = wj;
+      }
+    }
+    if (lane == 0) P.n_unique = k;
+  }
+  if (tid == 0) blk_stamp(p, l, 12);
+  csync();
 }
 
 // ---------------------------------------------------------------------------
@@ -1047,13 +1210,7 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
   uint64_t* empty = full + STEP_SLOTS;
   uint64_t* plan_bar = empty + STEP_SLOTS;  // consumers -> producer: this layer's plan is built
   uint64_t* hinit_bar = plan_bar + 1;       // consumers -> producer: this block's h slice is copied
-  uint64_t* fullA = hinit_bar + 1;          // one token: fixed router/shared-W13 slots
-  uint64_t* emptyA = fullA + STEP_FIX_MAX;
-  uint64_t* fullS = emptyA + STEP_FIX_MAX;  // one token: fixed shared-W2 slots
-  uint64_t* emptyS = fullS + STEP_FIX_MAX;
-  uint8_t* fixA = smem + STEP_FIXED;
-  uint8_t* fixS = fixA + p.fixa_bytes;
-  uint8_t* ring = fixS + p.fixs_bytes;
+  uint8_t* ring = smem + STEP_FIXED;
   uint8_t* act = ring + R;
   const uint32_t xss = padded_stride(2u * H);
   const uint32_t sss = Is > 0 ? padded_stride(2u * Is) : 0u;
@@ -1074,69 +1231,13 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
     }
     mbar_init(plan_bar, 1);
     mbar_init(hinit_bar, 1);
-    for (int s = 0; s < STEP_FIX_MAX; ++s) {
-      mbar_init(&fullA[s], 1);
-      mbar_init(&emptyA[s], 1);
-      mbar_init(&fullS[s], 1);
-      mbar_init(&emptyS[s], 1);
-    }
     for (int s = 0; s < STEP_SLOTS; ++s) s_gdone[s] = 0;
     fence_mbar_init();
     s_abort = 0;
   }
   __syncthreads();
 
-  // ---------------- producer of the routing-independent items (one token) ----------------
-  // Router / shared-W13 items and shared-W2 items of layer l go to their fixed slots as
-  // soon as the consumers have released the slot's layer l-1 copy, so each layer's are
-  // in shared memory (or on their way) while the layer before is still routing.
-  if (warp == STEP_CONSUMERS + 1) {
-    if constexpr (ONE) {
-      Producer pr{p, ring, R, full, empty, s_vst, policy_evict_first(), 0, 0, RingCursor{0ull, 0u}, &s_abort, lane};
-      Work W;
-      W.init_fixed(p);
-      int la = 0, ls = 0;  // layers issued completely (A slots / S slots); the slots of layer la / ls partly
-      int ja = 0, js = 0;  // slots issued of the partial layer
-      bool ok = true;
-      for (int l = 0; l < L && ok; ++l) {
-        const LayerPtrs& Lp = p.layer[l];
-        for (ja = 0; ja < W.nA; ++ja) {
-          if (l > 0 && lane == 0) ok = ring_wait(&emptyA[ja], (uint32_t)((l - 1) & 1), p.status, &s_abort);
-          ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-          if (!ok) break;
-          pr.copy_item(Lp, W.at(p, ja), fixA + (size_t)ja * bytesA, &fullA[ja]);
-        }
-        if (!ok) break;
-        la = l + 1;
-        ja = 0;
-        for (js = 0; js < W.nS; ++js) {
-          if (l > 0 && lane == 0) ok = ring_wait(&emptyS[js], (uint32_t)((l - 1) & 1), p.status, &s_abort);
-          ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-          if (!ok) break;
-          pr.copy_item(Lp, W.at(p, W.nA + js), fixS + (size_t)js * bytesS, &fullS[js]);
-        }
-        if (!ok) break;
-        ls = l + 1;
-        js = 0;
-      }
-      // every copy issued lands before the block may exit: slot j's last copy belongs
-      // to layer la (j < ja, a partly issued layer) or la - 1
-      if (lane == 0) {
-        for (int j = 0; j < W.nA; ++j) {
-          const int n = la + (j < ja ? 1 : 0);
-          if (n > 0) drain_wait(&fullA[j], (uint32_t)((n - 1) & 1));
-        }
-        for (int j = 0; j < W.nS; ++j) {
-          const int n = ls + (j < js ? 1 : 0);
-          if (n > 0) drain_wait(&fullS[j], (uint32_t)((n - 1) & 1));
-        }
-      }
-    }
-    return;
-  }
-
-  // ---------------- producer of the ring ----------------
-  // One token: routed items only.  A window: every item of the layer in ring order.
+  // ---------------- producer ----------------
   if (warp == STEP_CONSUMERS) {
     Producer pr{p, ring, R, full, empty, s_vst, policy_evict_first(), 0, 0, RingCursor{0ull, 0u}, &s_abort, lane};
     bool ok = true;
@@ -1144,10 +1245,8 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
       const LayerPtrs& Lp = p.layer[l];
       Work W;
       W.init_fixed(p);
-      if constexpr (!ONE) {
-        for (int r = 0; r < W.nA + W.nS && ok; ++r) ok = pr.issue(Lp, P, W.at(p, r));
-        if (!ok) break;
-      }
+      for (int r = 0; r < W.nA + W.nS && ok; ++r) ok = pr.issue(Lp, P, W.at(p, r));
+      if (!ok) break;
       stamp(p, l, 12);
       int got = 1;
       // the consumers' slice copy of h (ordered before their arrive by a block
@@ -1195,7 +1294,10 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
     }
     stamp(p, l, 1);
     if (tid == 0) blk_stamp(p, l, 0);
-    stage_layer_input<ONE>(p, l, hin, hout, xb16, xf16, xss, s_part, s_amx, s_r, s_sh, slice_q0, slice_q1);
+    if constexpr (ONE)
+      stage1(p, l, hin, hout, xb16, xf16, s_part, s_amx, s_sh, slice_q0, slice_q1);
+    else
+      stage_layer_input<ONE>(p, l, hin, hout, xb16, xf16, xss, s_part, s_amx, s_r, s_sh, slice_q0, slice_q1);
     if (tid == 0) mbar_arrive(hinit_bar);
     stamp(p, l, 2);
     if (tid == 0) blk_stamp(p, l, 1);
@@ -1210,7 +1312,6 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
     }
 
     // ---- A: router items (4 experts) and shared-W13 items (2 gate + 2 up rows) ----
-    // One token: item r in fixed slot r on warp r; a window: through the ring.
     Work W;
     W.init_fixed(p);
     const int nr = p.E / 4;
@@ -1218,12 +1319,7 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
       const uint8_t* src;
       uint64_t* eb;
       bool ready;
-      if constexpr (ONE) {
-        if (r % STEP_CONSUMERS != warp) continue;
-        src = fixA + (size_t)r * bytesA;
-        eb = &emptyA[r];
-        ready = ring_wait(&fullA[r], (uint32_t)(l & 1), p.status, &s_abort);
-      } else {
+      {
         const uint32_t s0 = ring_take(pos, bytesA, R);
         const long long ii = i++;
         if ((int)(ii % STEP_CONSUMERS) != warp) continue;
@@ -1268,16 +1364,17 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
 
     // ---- top-k and plan (every block, identical; polls the tagged logits) ----
     stamp(p, l, 4);
-    step_topk<ONE>(p, l, P, s_ids, s_wts, s_wmax, s_ncand, s_cand, s_sel, &s_abort);
+    if constexpr (ONE)
+      topk1(p, l, P, s_wmax, s_ncand, s_cand, s_sel, &s_abort);
+    else
+      step_topk<ONE>(p, l, P, s_ids, s_wts, s_wmax, s_ncand, s_cand, s_sel, &s_abort);
     if (tid == 0) mbar_arrive(plan_bar);
     stamp(p, l, 5);
     if (tid == 0) blk_stamp(p, l, 4);
 
-    // ---- CS: shared W2 (activation as bf16 hi + lo), accumulated into h ----
-    // A window runs it here, ahead of the routed tiles whose copies it waits for; one
-    // token runs it after the routed W13 (its items are already in their slots), to
-    // fill the wait for the routed activations.
-    auto shared_w2 = [&]() {
+    // ---- CS: shared W2 (activation as bf16 hi + lo), accumulated into h, ahead of the
+    //      routed tiles whose copies it waits for ----
+    {
       if (W.nS > 0) {
         for (int e = tid; e < M * (Is / 8); e += 32 * STEP_CONSUMERS) {
           const int tok = e / (Is / 8), c8 = e % (Is / 8);
@@ -1305,12 +1402,7 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
         const uint8_t* src;
         uint64_t* eb;
         bool ready;
-        if constexpr (ONE) {
-          if ((r + 4) % STEP_CONSUMERS != warp) continue;
-          src = fixS + (size_t)r * bytesS;
-          eb = &emptyS[r];
-          ready = ring_wait(&fullS[r], (uint32_t)(l & 1), p.status, &s_abort);
-        } else {
+        {
           const uint32_t s0 = ring_take(pos, bytesS, R);
           const long long ii = i++;
           if ((int)(ii % STEP_CONSUMERS) != warp) continue;
@@ -1357,8 +1449,7 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
       }
       stamp(p, l, 7);
       if (tid == 0) blk_stamp(p, l, 5);
-    };
-    if constexpr (!ONE) shared_w2();
+    }
 
     // ---- B: routed W13 + SwiGLU ----
     // Groups of consecutive tiles of one expert share a ring item.  One token: the
@@ -1462,7 +1553,6 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
     }
     stamp(p, l, 8);
     if (tid == 0) blk_stamp(p, l, 6);
-    if constexpr (ONE) shared_w2();
     csync();  // xf16 and the shared halves are dead: the routed-W2 activation copies take the region
     stamp(p, l, 9);
 
@@ -1611,7 +1701,7 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
     stamp(p, l, 10);
     csync();
     if (tid == 0) blk_stamp(p, l, 7);
-    if (tid == 0) signal_counter(lc + CTR_H);
+    if (tid == 0 && l != p.hold_layer) signal_counter(lc + CTR_H);
     stamp(p, l, 11);
   }
 

@@ -39,7 +39,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings_and_version(lib):
-    assert lib.moe_abi_version() == 1
+    assert lib.moe_abi_version() == 2
     for code, name in _abi.STATUS_NAMES.items():
         assert lib.moe_status_string(code).decode() == name
 
