@@ -627,14 +627,14 @@ __device__ __forceinline__ void mxfp4_rows_m1(const uint8_t* codes_g, const uint
 }
 
 // The clamped-factor rows (rare: block exponents outside the fast range), out of line.
-__device__ __noinline__ void mxfp4_rows_m1_safe(const uint8_t* codes_g, const uint8_t* codes_g8, const uint8_t* sc_g,
+__device__ __forceinline__ void mxfp4_rows_m1_safe(const uint8_t* codes_g, const uint8_t* codes_g8, const uint8_t* sc_g,
                                                 const uint8_t* sc_g8, int nb, const uint8_t* xb, int sh, float& r0,
                                                 float& r1) {
   mxfp4_rows_m1<false>(codes_g, codes_g8, sc_g, sc_g8, nb, xb, sh, r0, r1);
 }
 // A window tile whose rows span more than FOLD_SPAN scale exponents: exact per-block
 // fp32 scaling, one token at a time (rare; out of line).
-__device__ __noinline__ void mxfp4_tile_dot_wide(const uint8_t* codes_g, const uint8_t* codes_g8, const uint8_t* sc_g,
+__device__ __forceinline__ void mxfp4_tile_dot_wide(const uint8_t* codes_g, const uint8_t* codes_g8, const uint8_t* sc_g,
                                                  const uint8_t* sc_g8, int nb, const uint8_t* xb, uint32_t xss, int M,
                                                  const int* xsh, float* c) {
   const int t = threadIdx.x & 3;
@@ -674,7 +674,10 @@ __device__ __forceinline__ void mxfp4_tile_dot_win(const uint8_t* codes_g, const
   for (int e = 0; e < 4; ++e) {
     const int tok = 2 * t + (e & 1);
     const int ref = (int)(e < 2 ? mx_g : mx_g8);
-    c[e] = tok < M ? ldexpf(acc[e], ref - 127 - xsh[tok]) : 0.0f;
+    // 2^(ref - 127 - sh) as two exact power-of-two factors (|exponent| <= 290; a result
+    // below 2^-252 of the fp32 sum is zero in fp32 anyway)
+    const int d = tok < M ? max(ref - 127 - xsh[tok], -252) : 0;
+    c[e] = tok < M ? mul_pow2(acc[e], d) : 0.0f;
   }
 }
 

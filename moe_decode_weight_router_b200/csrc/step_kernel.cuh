@@ -231,15 +231,15 @@ __device__ __noinline__ bool wait_counter(const unsigned* c, unsigned target, in
 }
 // mbarrier wait that also honours the block's abort flag: the first try inline, the
 // bounded loop out of line.
-__device__ __noinline__ bool ring_wait_slow(uint64_t* bar, uint32_t parity, int* status, volatile int* abort_flag);
+__device__ __forceinline__ bool ring_wait_slow(uint64_t* bar, uint32_t parity, int* status, volatile int* abort_flag);
 __device__ __forceinline__ bool ring_wait(uint64_t* bar, uint32_t parity, int* status, volatile int* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
   return ring_wait_slow(bar, parity, status, abort_flag);
 }
-__device__ __noinline__ bool ring_wait_slow(uint64_t* bar, uint32_t parity, int* status, volatile int* abort_flag) {
+__device__ __forceinline__ bool ring_wait_slow(uint64_t* bar, uint32_t parity, int* status, volatile int* abort_flag) {
   const unsigned long long t0 = globaltimer_ns(), lim = wait_limit(status);
   while (true) {
-    if (mbar_try_wait_sleep(bar, parity, 500u)) return true;  // suspended, not spinning
+    if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
     if (globaltimer_ns() - t0 > lim) {
       atomicCAS(status, 0, DEV_ERR_TIMEOUT);
@@ -760,85 +760,99 @@ __device__ __noinline__ void topk_token_full(const StepParams& p, int l, int tok
   }
 }
 
-// The 8 consumer warps split the experts: warp w holds experts [w*per, (w+1)*per),
-// per = E/8, at most 4 per lane, of every token.  The smallest of the 8 warp maxima
-// is a lower bound for the k-th largest logit (k <= 8, and the maxima are 8 distinct
-// experts), so only logits at or above it can be selected: those are gathered per
-// token, and when at most TOPK_CAND survive, each survivor's rank is the number of
-// survivors whose order key is larger.  Otherwise the token's warp runs the exact
-// k-round selection.  Warp t then forms token t's softmax over its selected logits.
-template <bool ONE>
-__device__ void step_topk(const StepParams& p, int l, Plan& P, int32_t* s_ids, float* s_wts, uint32_t* s_wmax,
-                          int* s_ncand, unsigned long long* s_cand, unsigned long long* s_sel,
-                          volatile int* s_abort_ptr) {
-  constexpr int MT = ONE ? 1 : MAX_M;  // tokens held in registers
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
-  const int E = p.E, k = p.k, M = ONE ? 1 : p.M;
-  const int per = E / STEP_CONSUMERS;  // E % 16 == 0: every warp holds >= 2 experts
-  const int e0 = warp * per;
-  if (tid < MAX_M) s_ncand[tid] = 0;
-  uint32_t key[MT][4];
+// Top-k of a window of tokens from the complete router logits (same rule as k_dense:
+// largest logit, lowest index on ties), then the union plan.  The 8 consumer warps
+// form TG token groups x EP expert parts (TG the largest power of two <= min(M, 8)
+// whose parts hold at most 256 experts): each keeps its part's top-k of its tokens
+// (a global top-k element is always in its part's top-k, ties included), then one
+// warp per token merges the EP*k candidates.
+__device__ void step_topk_win(const StepParams& p, int l, Plan& P, int32_t* s_ids, float* s_wts, uint32_t* s_ck,
+                          int32_t* s_ci, volatile int* s_abort_ptr) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int E = p.E, k = p.k, M = p.M;
+  int TG = 1;
+  while (2 * TG <= M && 2 * TG <= STEP_CONSUMERS && E <= 256 * (STEP_CONSUMERS / (2 * TG))) TG *= 2;
+  const int EP = STEP_CONSUMERS / TG;
+  const int per = (E + EP - 1) / EP;  // experts per part (<= 256)
+  const int part = warp % EP;
+  const int e0 = part * per;
+  for (int tok = warp / EP; tok < M; tok += TG) {
+    uint32_t key[8];
+    {
+      const unsigned long long* w[8];
+      int n = 0;
 #pragma unroll
-  for (int tok = 0; tok < MT; ++tok) {
-    if (tok >= M) break;
-    const unsigned long long* w[8];
-    int n = 0;
+      for (int i = 0; i < 8; ++i) {
+        const int off = lane + 32 * i, e = e0 + off;
+        w[i] = p.logits + tok * E + e;
+        if (off < per && e < E) n = i + 1;  // valid columns are a prefix
+      }
+      float lv[8];
+      if (!await_tagged(w, n, (uint32_t)l + 1u, lv, p.status, s_abort_ptr))
+        n = 0;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int off = lane + 32 * i;
-      w[i] = p.logits + (size_t)tok * E + e0 + (off < per ? off : 0);
-      if (i < 4 && off < per) n = i + 1;  // valid columns are a prefix
+      for (int i = 0; i < 8; ++i) key[i] = i < n ? float_key(lv[i]) : 0u;
     }
-    float lv[8];
-    if (!await_tagged(w, n, (uint32_t)l + 1u, lv, p.status, s_abort_ptr)) n = 0;
-    uint32_t mx = 0u;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      key[tok][i] = i < n ? float_key(lv[i]) : 0u;
-      mx = max(mx, key[tok][i]);
-    }
-    mx = __reduce_max_sync(0xffffffffu, mx);
-    if (lane == 0) s_wmax[tok * STEP_CONSUMERS + warp] = mx;
-  }
-  if (tid == 0) blk_stamp(p, l, 8);
-  csync();
+    for (int j = 0; j < 8; ++j) {
+      if (j < k) {
+        uint32_t bk = 0u;
+        int bi = 0x7fffffff;
 #pragma unroll
-  for (int tok = 0; tok < MT; ++tok) {
-    if (tok >= M) break;
-    uint32_t bound = 0xFFFFFFFFu;
+        for (int i = 0; i < 8; ++i)
+          if (key[i] > bk) {
+            bk = key[i];
+            bi = e0 + lane + 32 * i;
+          }
+        const uint32_t mk = __reduce_max_sync(0xffffffffu, bk);
+        const int mi = (int)__reduce_min_sync(0xffffffffu, (unsigned)(bk == mk ? bi : 0x7fffffff));
 #pragma unroll
-    for (int w = 0; w < STEP_CONSUMERS; ++w) bound = min(bound, s_wmax[tok * STEP_CONSUMERS + w]);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int off = lane + 32 * i;
-      if (off < per && key[tok][i] >= bound) {
-        const int pos = atomicAdd(&s_ncand[tok], 1);
-        if (pos < TOPK_CAND) s_cand[tok * TOPK_CAND + pos] = order_key(key[tok][i], e0 + off);
+        for (int i = 0; i < 8; ++i)
+          if (e0 + lane + 32 * i == mi) key[i] = 0u;
+        if (lane == 0) {
+          s_ck[(tok * STEP_CONSUMERS + part) * 8 + j] = mk;
+          s_ci[(tok * STEP_CONSUMERS + part) * 8 + j] = mk ? mi : 0x7fffffff;
+        }
       }
     }
   }
-  if (tid == 0) blk_stamp(p, l, 9);
   csync();
-  if (tid == 0) blk_stamp(p, l, 10);
   for (int tok = warp; tok < M; tok += STEP_CONSUMERS) {
-    unsigned long long* sel = s_sel + tok * 8;
-    const int n = s_ncand[tok];
-    if (n <= TOPK_CAND) {
-      const unsigned long long* cand = s_cand + tok * TOPK_CAND;
-      const unsigned long long mine = lane < n ? cand[lane] : 0ull;
-      int rank = 0;
-      for (int j = 0; j < n; ++j) rank += cand[j] > mine ? 1 : 0;
-      if (lane < n && rank < k) sel[rank] = mine;
-    } else {
-      topk_token_full(p, l, tok, sel, s_abort_ptr);
+    const int nc = EP * k;  // <= 64 candidates, two per lane
+    uint32_t ck[2] = {0u, 0u};
+    int ci[2] = {0x7fffffff, 0x7fffffff};
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int c = lane + 32 * r;
+      if (c < nc) {
+        ck[r] = s_ck[(tok * STEP_CONSUMERS + c / k) * 8 + c % k];
+        ci[r] = s_ci[(tok * STEP_CONSUMERS + c / k) * 8 + c % k];
+      }
     }
-    __syncwarp();
-    // lane j holds the j-th selection; softmax over the selected logits.  An id outside
-    // [0, E) (only after a failed wait) is replaced by 0 so nothing reads out of bounds.
-    const unsigned long long sj = lane < k ? sel[lane] : 0ull;
-    int sel_id = (int)(~(uint32_t)sj);
+    int sel_id = 0;
+    uint32_t sel_key = 0u;
+    for (int j = 0; j < k; ++j) {
+      const int b = (ck[1] > ck[0] || (ck[1] == ck[0] && ci[1] < ci[0])) ? 1 : 0;
+      const uint32_t bk = b ? ck[1] : ck[0];
+      const int bi = b ? ci[1] : ci[0];
+      const uint32_t mk = __reduce_max_sync(0xffffffffu, bk);
+      const int mi = (int)__reduce_min_sync(0xffffffffu, (unsigned)(bk == mk ? bi : 0x7fffffff));
+#pragma unroll
+      for (int r = 0; r < 2; ++r)
+        if (ck[r] == mk && ci[r] == mi) {
+          ck[r] = 0u;
+          ci[r] = 0x7fffffff;
+        }
+      if (lane == j) {
+        sel_id = mi;
+        sel_key = mk;
+      }
+    }
+    // an id outside [0, E) (only after a failed wait) is replaced by 0: nothing reads
+    // out of bounds while the step winds down
     sel_id = (unsigned)sel_id < (unsigned)E ? sel_id : 0;
-    const float lj = key_float((uint32_t)(sj >> 32));
+    // lane j holds the j-th selection; softmax over the selected logits
+    const float lj = key_float(sel_key);
     const float l0 = __shfl_sync(0xffffffffu, lj, 0);
     const float ex = lane < k ? expf(lj - l0) : 0.0f;
     float den = ex;
@@ -855,10 +869,8 @@ __device__ void step_topk(const StepParams& p, int l, Plan& P, int32_t* s_ids, f
       }
     }
   }
-  if (threadIdx.x == 0) blk_stamp(p, l, 11);
   csync();
   if (warp == 0) build_plan(P, s_ids, s_wts, M, k, E);
-  if (threadIdx.x == 0) blk_stamp(p, l, 12);
   csync();
 }
 
@@ -926,7 +938,7 @@ __device__ __forceinline__ void rows_dot_m1(const uint8_t* const (&rows)[R], con
   }
 }
 template <int LPR, int R>
-__device__ __noinline__ void rows_dot_m1_safe(const uint8_t* const (&rows)[R], const uint8_t* const (&scs)[R], int nb,
+__device__ __forceinline__ void rows_dot_m1_safe(const uint8_t* const (&rows)[R], const uint8_t* const (&scs)[R], int nb,
                                               const uint8_t* xc, int sh, float (&out)[R]) {
   bool bad = false;
   rows_dot_m1<LPR, R, true>(rows, scs, nb, xc, sh, bad, out);
@@ -1194,6 +1206,8 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
   __shared__ float s_amx[MAX_M * STEP_CONSUMERS];
   __shared__ int s_sh[MAX_M];
   __shared__ uint32_t s_wmax[MAX_M * STEP_CONSUMERS];
+  __shared__ uint32_t s_ck[ONE ? 1 : MAX_M * STEP_CONSUMERS * 8];
+  __shared__ int32_t s_ci[ONE ? 1 : MAX_M * STEP_CONSUMERS * 8];
   __shared__ int s_ncand[MAX_M];
   __shared__ unsigned long long s_cand[MAX_M * TOPK_CAND];
   __shared__ unsigned long long s_sel[MAX_M * 8];
@@ -1367,7 +1381,7 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
     if constexpr (ONE)
       topk1(p, l, P, s_wmax, s_ncand, s_cand, s_sel, &s_abort);
     else
-      step_topk<ONE>(p, l, P, s_ids, s_wts, s_wmax, s_ncand, s_cand, s_sel, &s_abort);
+      step_topk_win(p, l, P, s_ids, s_wts, s_ck, s_ci, &s_abort);
     if (tid == 0) mbar_arrive(plan_bar);
     stamp(p, l, 5);
     if (tid == 0) blk_stamp(p, l, 4);
