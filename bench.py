@@ -39,10 +39,11 @@ NOMINAL_HBM_GBS = 8000.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 
 
-# DRAM traffic of k_step per layer (read + write) from the ncu capture summarised in
-# profiles/k_step_ling_2layers_m1.md, valid while the kernel sources hash to the value
-# recorded with it (otherwise the roofline's traffic is reported as null).
-KSTEP_TRAFFIC = {"bytes_per_layer": (79.14e6 + 1.88e6) / 2, "sources_sha256_16": "c6720a0d82a49ca8",
+# DRAM traffic of k_step per layer (read + write): an ncu capture (dram__bytes_read.sum +
+# dram__bytes_write.sum, the second k_step launch) of `bench.py --probe-window one
+# --layers 2`, valid while the kernel sources hash to the value recorded with it
+# (otherwise the roofline's traffic is reported as null).
+KSTEP_TRAFFIC = {"bytes_per_layer": (79129344 + 1415168) / 2, "sources_sha256_16": "a40b6b55d5f031c1",
                  "sources": ("step_kernel.cuh", "decode_kernels.cuh", "common.cuh")}
 
 
@@ -74,6 +75,10 @@ def parse_args():
     ap.add_argument("--skip-prefill", action="store_true", help="skip the prefill-chunk measurement")
     ap.add_argument("--skip-head", action="store_true", help="skip the LM-head comparison and verify window")
     ap.add_argument("--prefill-m", type=int, default=2048, help="tokens of the prefill chunk")
+    ap.add_argument("--probe-window", choices=["one", "random", "identical", "disjoint"], default=None,
+                    help="byte-accounting probe: one decode step of --layers layers (M=1 for 'one', else an "
+                         "M=4 window under the given routing), run twice (the second k_step launch is the "
+                         "one to capture); prints its routing and algorithmic bytes")
     return ap.parse_args()
 
 
@@ -446,6 +451,7 @@ def run_ours(args, rank, world, local_rank):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(model, S, V, args.cpu_budget)
+        cpu.update(cpu_baseline_legs(model, S, args.cpu_budget / 4))
     return results, cpu
 
 
@@ -512,6 +518,86 @@ def cpu_baseline(model, S, V, budget_s):
                       f"{t_all:.2f} s of oracle time (host copies of the weights excluded)"}
 
 
+def cpu_baseline_legs(model, S, budget_s):
+    """The other oracle legs of the CPU plan, each a bounded sample of its workload:
+    one_core  -- the M = 1 step on one host thread (chained layers until budget_s, then
+                 8,192 LM-head rows), GB/s over the algorithmic bytes covered;
+    m4        -- the M = 4 verify window on all threads (chained layers, routing from
+                 the chain), GB/s over the bytes of the distinct experts it touched;
+    prefill   -- one M = 2048 prefill chunk of layer 0 (MXFP8 activations): the router
+                 over every token, then the layer output of a sample of tokens; the
+                 chunk time is the router time plus the per-token time x 2048."""
+    import numpy as np
+    import torch
+
+    import oracle
+    from moe_decode_weight_router_b200 import synth
+
+    def fetch_of(Ly):
+        def fetch(lst):
+            idx = torch.tensor(lst, dtype=torch.long, device=Ly["w13c"].device)
+            return {n: synth.bits(Ly[n].index_select(0, idx)) for n in ("w13c", "w13s", "w2c", "w2s")}
+        return fetch
+
+    def chain(M, threads, head_rows):
+        oracle.set_threads(threads)
+        x = synth.bits(synth.tokens(M, S.H, 8 + M, tid=901))
+        h = None
+        t_all, nb, n_done = 0.0, 0, 0
+        for Ly in model.layers:
+            wr = synth.bits(Ly["wr"])
+            shared = {"sw13": synth.bits(Ly["sw13"]), "sw2": synth.bits(Ly["sw2"])}
+            t0 = time.perf_counter()
+            ids, w, _, _ = oracle.route(x, wr, S.k)
+            t1 = time.perf_counter()
+            ex = fetch_of(Ly)(sorted(set(ids.reshape(-1).tolist())))
+            t2 = time.perf_counter()
+            y = oracle.moe_layer(x, ids, w, _remap(ex, ids), shared)
+            h = (np.vectorize(oracle.bf16_value)(x) if h is None else h) + y
+            x = oracle.rmsnorm_bf16(h)
+            t3 = time.perf_counter()
+            t_all += (t1 - t0) + (t3 - t2)
+            nb += layer_bytes(S, M, len(np.unique(ids)))
+            n_done += 1
+            if t_all > budget_s:
+                break
+        if head_rows:
+            q = synth.bits(model.lm_q[:head_rows])
+            sc = model.lm_s[:head_rows].cpu().numpy()
+            t0 = time.perf_counter()
+            oracle.lmhead_logits(x, q, sc)
+            t_all += time.perf_counter() - t0
+            nb += lm_bytes(head_rows, S.H, M)
+        return nb / t_all / 1e9, n_done, t_all
+
+    legs = {}
+    n = _threads()
+    v, nl, t = chain(1, 1, 8192)
+    legs["one_core"] = {"value": v, "unit": "GB/s", "cores": 1,
+                        "sample": f"{nl} chained Ling layers at M=1 + LM-head rows [0,8192); {t:.2f} s"}
+    v, nl, t = chain(4, n, 0)
+    legs["m4"] = {"value": v, "unit": "GB/s", "cores": n,
+                  "sample": f"{nl} chained Ling layers at M=4 (routing from the chain); {t:.2f} s"}
+    oracle.set_threads(n)
+    # prefill chunk: router over all 2048 tokens, then a sample of tokens' layer outputs
+    Mp, ns = 2048, 16
+    Ly = model.layers[0]
+    x = synth.bits(synth.tokens(Mp, S.H, 11, tid=902))
+    t0 = time.perf_counter()
+    ids, w, _, _ = oracle.route(x, synth.bits(Ly["wr"]), S.k)
+    t_route = time.perf_counter() - t0
+    tokens = np.arange(0, Mp, Mp // ns, dtype=np.int32)[:ns]
+    ex = fetch_of(Ly)(sorted(set(ids[tokens].reshape(-1).tolist())))
+    shared = {"sw13": synth.bits(Ly["sw13"]), "sw2": synth.bits(Ly["sw2"])}
+    t0 = time.perf_counter()
+    oracle.moe_layer_prefill(x, ids, w, _remap(ex, ids[tokens]), shared, tokens)
+    t_tok = (time.perf_counter() - t0) / ns
+    legs["prefill"] = {"us_per_chunk": 1e6 * (t_route + t_tok * Mp), "unit": "us", "cores": n,
+                       "sample": f"router over {Mp} tokens ({t_route:.2f} s) + layer output of {ns} sampled tokens "
+                                 f"({t_tok * 1e3:.1f} ms per token), extrapolated to the {Mp}-token chunk"}
+    return legs
+
+
 def _remap(ex, ids):
     """Expert arrays fetched for sorted(set(ids)) re-indexed by expert id for the oracle."""
     uniq = sorted(set(ids.reshape(-1).tolist()))
@@ -566,8 +652,53 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def probe_window(args):
+    """The verify window (M = 4) under a forced routing, for the byte accounting of the
+    persistent step: 'identical' repeats one token (every token takes the same 8 experts
+    in every layer); 'disjoint' gives token t a large component on hidden dimension t and
+    every layer's experts 8t..8t+7 a large router weight on that dimension (each token
+    takes its own 8: 32 distinct experts per layer); 'random' is the benchmark's window;
+    'one' is the benchmark's one-token step.  Prints the distinct experts of every layer
+    and the algorithmic bytes per layer."""
+    import numpy as np
+    import torch
+
+    from moe_decode_weight_router_b200 import DecodeModel, decode_step, synth
+    from moe_decode_weight_router_b200 import build as _b
+
+    _b.build()
+    S, dev = synth.LING, "cuda"
+    M = 1 if args.probe_window == "one" else 4
+    layers = [synth.layer(S, args.seed, l, device=dev) for l in range(args.layers)]
+    x = synth.tokens(M, S.H, args.seed, tid=5, device=dev)
+    if args.probe_window == "identical":
+        x = x[0:1].repeat(M, 1).contiguous()
+    elif args.probe_window == "disjoint":
+        x[:, :M] = 0
+        for t in range(M):
+            x[t, t] = 50.0
+        for Ly in layers:
+            for t in range(M):
+                Ly["wr"][8 * t:8 * t + 8, t] = 2.0
+    q = synth.e4m3_codes((synth.VOCAB, S.H), args.seed, device=dev)
+    s = synth.row_scales(synth.VOCAB, args.seed, device=dev)
+    model = DecodeModel(layers=layers, lm_q=q, lm_s=s, top_k=S.k)
+    res = None
+    for _ in range(2):
+        res = decode_step(model, x, trace=True, ws=None if res is None else res["ws"])
+    torch.cuda.synchronize()
+    ids = res["ids_trace"].cpu().numpy()
+    distinct = [int(len(np.unique(ids[l]))) for l in range(args.layers)]
+    print(json.dumps({"probe_window": args.probe_window, "M": M, "layers": args.layers,
+                      "distinct_experts_per_layer": distinct,
+                      "algorithmic_bytes_per_layer": [layer_bytes(S, M, d) for d in distinct]}))
+    return 0
+
+
 def main():
     args = parse_args()
+    if args.probe_window:
+        return probe_window(args)
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

@@ -62,7 +62,13 @@ _SIGS = {
     "orc_mxfp8_quantize": (None, [_P, _I, _I, _P, _P]),
     "orc_moe_layer_prefill": (None, [_P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I,
                                      _P, _I, _P]),
+    "orc_set_threads": (None, [_I]),
 }
+
+
+def set_threads(n: int) -> None:
+    """Host threads of the oracle's parallel loops (timing only)."""
+    lib().orc_set_threads(int(n))
 
 
 def lib():

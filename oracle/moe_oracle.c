@@ -50,6 +50,19 @@
 
 #define EXPORT __attribute__((visibility("default")))
 
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* Host threads the parallel loops below use (n >= 1); timing only, no arithmetic. */
+EXPORT void orc_set_threads(int n) {
+#ifdef _OPENMP
+  if (n >= 1) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}
+
 /* ------------------------------------------------------------------------- */
 /* Formats                                                                    */
 /* ------------------------------------------------------------------------- */
