@@ -20,7 +20,8 @@
  * Conventions for every entry point:
  *  - All tensor arguments are DEVICE pointers (cudaMalloc'd or equivalent) unless
  *    stated; the caller owns every buffer.  The library never allocates, frees or
- *    synchronises; every call is asynchronous and ordered on `stream`.
+ *    synchronises (moe_workspace_status and moe_selfcheck excepted, as they say);
+ *    every other call is asynchronous and ordered on `stream`.
  *  - Arguments are validated on the host before anything is enqueued; a non-OK
  *    status means nothing was launched.  No C++ exception crosses the ABI.
  *  - Pointers must be 16-byte aligned (MOE_ERR_ALIGNMENT otherwise).
@@ -40,6 +41,11 @@
  *    then gives the cudaError_t value (per calling thread).
  *  - Thread safety: stateless apart from the caller's buffers and the per-thread
  *    last-error value; concurrent calls on different workspaces are safe.
+ *  - Contexts: the first call on a device reads its attributes and raises the
+ *    kernels' shared-memory limits once, for the process; this assumes every call
+ *    runs in the device's primary context (the CUDA runtime's).  After
+ *    cudaDeviceReset those limits are gone and large launches fail (MOE_ERR_CUDA):
+ *    reload the library in a new process instead.
  */
 #ifndef MOE_DECODE_H
 #define MOE_DECODE_H
@@ -68,7 +74,8 @@ typedef enum {
   MOE_ERR_WORKSPACE = 4,         /* workspace NULL or smaller than required */
   MOE_ERR_DTYPE = 5,             /* a model buffer tagged with the wrong format */
   MOE_ERR_CUDA = 6,              /* the CUDA runtime refused a launch */
-  MOE_ERR_TIMEOUT = 7            /* a bounded device-side wait gave up */
+  MOE_ERR_TIMEOUT = 7,           /* a bounded device-side wait gave up */
+  MOE_ERR_SELFCHECK = 8          /* moe_selfcheck: a result differs from the expected one */
 } moe_status_t;
 
 /* Human-readable name of a status value (static storage). */
@@ -203,6 +210,29 @@ MOE_API moe_status_t lm_head_bf16_gemv(const void* x_bf16, int M, int V, int H, 
 MOE_API moe_status_t moe_sample(const float* logits, int M, int V, float temperature, int top_k, float top_p,
                                 const float* u, int32_t* ids, moe_stream_t stream);
 
+/* Start-up self-check (the DGX Spark MoE knowledge card, 局限与不确定性: with the FP8
+ * head and the verify window both on, a module mismatch made the framework fall back
+ * silently -- FP8 bytes read as BF16, accept length 1.00 -- visible in no throughput
+ * figure, and the advice is to confirm at start-up that every optimisation is really
+ * active).  On inputs it generates in `ws` from a counter-based generator, runs
+ *   1 moe_route on one token (expert ids compared bit for bit),
+ *   2 moe_mxfp4_experts on that routing (y: relative L2 <= 5e-3),
+ *   3 lm_head_fp8_gemv on a 4-token window (argmaxes bit for bit),
+ *   4 lm_head_fp8_verify with the head's own argmaxes as drafts (accept length 4),
+ *   5 decode_step, two layers, one token, and 6 the same on the 4-token window
+ *     (argmaxes bit for bit, logits relative L2 <= 5e-3 per row),
+ *   7 whether decode_step took its single persistent kernel at M = 1 and M = 4,
+ * against results computed once by the CPU oracle and compiled into the library.
+ *   ws: device workspace of moe_selfcheck_workspace_bytes() bytes, 16-byte aligned.
+ *   failed_check (HOST, may be NULL): 0, or the number of the first check that failed.
+ *   max_rel_l2 (HOST, may be NULL): the largest relative L2 seen in checks 2, 5, 6.
+ * Returns MOE_OK, MOE_ERR_SELFCHECK when a check failed, or the error of the entry
+ * point that refused (MOE_ERR_TIMEOUT included).  Synchronises `stream` (host-blocking):
+ * call it once at start-up, not in the decode loop. */
+MOE_API size_t moe_selfcheck_workspace_bytes(void);
+MOE_API moe_status_t moe_selfcheck(void* ws, size_t ws_bytes, moe_stream_t stream, int* failed_check,
+                                   float* max_rel_l2);
+
 /* Allocation-free variant of lm_head_fp8_gemv (no counterpart on the pages; it
  * exists for integration).  Some callers cannot hand this library any scratch
  * memory: an operator slot that passes only input and output tensors and has no
@@ -214,8 +244,9 @@ MOE_API moe_status_t moe_sample(const float* logits, int M, int V, float tempera
  * one per device that loads it, held until the process exits.
  *   Arguments, layouts, results and errors: as lm_head_fp8_gemv.  M above 8 (the
  *   keys the static block holds) returns MOE_ERR_UNSUPPORTED_SHAPE.
- *   The first call on a device looks up the array's device address (a one-time,
- *   host-side set-up): make that first call before any stream capture.
+ *   Each call looks up the array's device address in the current context (host-side,
+ *   no device work); the first call in a process may load the module, so make it
+ *   before any stream capture.
  *   Every call shares the one array and clears it on entry, so calls whose GPU
  *   work overlaps (other streams, other host threads, the same device) race and
  *   corrupt each other's argmax; serialise them. */

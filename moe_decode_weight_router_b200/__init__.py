@@ -9,5 +9,5 @@ from .binding import (DecodeGraph, DecodeModel, MoeError, abi_version, decode_st
                       decode_step_launch_names, decode_step_workspace_bytes, lm_head_bf16_gemv, lm_head_fp8_gemv,
                       lm_head_fp8_gemv_noalloc, lm_head_fp8_quantize, lm_head_fp8_verify,
                       lm_head_workspace_bytes, moe_experts_workspace_bytes, moe_mxfp4_experts, moe_mxfp8_quantize, moe_sample,
-                      moe_prefill_layer, moe_prefill_workspace_bytes, moe_route, moe_route_workspace_bytes,
+                      moe_prefill_layer, moe_prefill_workspace_bytes, moe_route, moe_route_workspace_bytes, moe_selfcheck,
                       workspace_status)

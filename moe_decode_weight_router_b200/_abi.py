@@ -14,6 +14,7 @@ Z = ctypes.c_size_t
 STATUS_NAMES = {
     0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED_SHAPE", 3: "MOE_ERR_ALIGNMENT",
     4: "MOE_ERR_WORKSPACE", 5: "MOE_ERR_DTYPE", 6: "MOE_ERR_CUDA", 7: "MOE_ERR_TIMEOUT",
+    8: "MOE_ERR_SELFCHECK",
 }
 
 FMT_NONE, FMT_BF16, FMT_MXFP4_CODES, FMT_E8M0_SCALES, FMT_E4M3, FMT_F32 = range(6)
@@ -61,6 +62,8 @@ SIGNATURES = {
     "lm_head_bf16_gemv": (I, [P, I, I, I, P, P, P, P, Z, P]),
     "moe_sample": (I, [P, I, I, ctypes.c_float, I, ctypes.c_float, P, P, P]),
     "lm_head_fp8_gemv_noalloc": (I, [P, I, I, I, P, P, P, P, P]),
+    "moe_selfcheck_workspace_bytes": (Z, []),
+    "moe_selfcheck": (I, [P, Z, P, ctypes.POINTER(I), ctypes.POINTER(ctypes.c_float)]),
     "decode_step_workspace_bytes": (Z, [ctypes.POINTER(Model), I]),
     "decode_step_launch_names": (I, [ctypes.POINTER(Model), I, ctypes.POINTER(ctypes.c_char_p), I]),
     "decode_step": (I, [ctypes.POINTER(Model), P, I, P, P, ctypes.POINTER(Trace), P, Z, P]),

@@ -64,6 +64,17 @@ def workspace_status(ws: torch.Tensor, stream=None) -> int:
     return _lib().moe_workspace_status(_ptr(ws), _stream(stream))
 
 
+def moe_selfcheck(device=None, stream=None):
+    """Runs the library's start-up self-check on ``device`` (default: the current CUDA
+    device).  Returns (status, failed_check, max_rel_l2); status 0 means every check
+    passed, 8 (MOE_ERR_SELFCHECK) that check ``failed_check`` gave a wrong result."""
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    ws = _ws(_lib().moe_selfcheck_workspace_bytes(), dev)
+    fail, rel = ctypes.c_int(0), ctypes.c_float(0.0)
+    st = _lib().moe_selfcheck(_ptr(ws), ws.numel(), _stream(stream), ctypes.byref(fail), ctypes.byref(rel))
+    return st, fail.value, rel.value
+
+
 # ---------------------------------------------------------------------------
 # Router
 # ---------------------------------------------------------------------------

@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -18,6 +19,7 @@
 #include "step_kernel.cuh"
 #include "prefill_kernels.cuh"
 #include "sample_kernels.cuh"
+#include "selfcheck.cuh"
 
 using namespace moe;
 
@@ -352,6 +354,7 @@ const char* moe_status_string(int status) {
     case MOE_ERR_DTYPE: return "MOE_ERR_DTYPE";
     case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
     case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT";
+    case MOE_ERR_SELFCHECK: return "MOE_ERR_SELFCHECK";
     default: return "MOE_ERR_UNKNOWN";
   }
 }
@@ -864,24 +867,13 @@ void decode_step_graph_destroy(moe_graph_t g) {
 static __device__ __align__(256) unsigned char g_lm_noalloc_scratch[CTRL_BYTES];
 
 namespace {
-// Device address of g_lm_noalloc_scratch on the current device.  The name is only a
-// host-side stand-in for the array, so the address is looked up once per device
-// (with that device current) and cached.
+// Device address of g_lm_noalloc_scratch in the current context.  The name is only a
+// host-side stand-in for the array; the address is looked up on every call (a host
+// table lookup), so a context created after a device reset never sees a stale one.
 moe_status_t lm_noalloc_scratch(void** out) {
-  static std::mutex mu;
-  static void* addr[64];
-  static bool ready[64] = {};
-  int dev = 0;
-  MOE_CUDA(cudaGetDevice(&dev));
-  if (dev < 0 || dev >= 64) return MOE_ERR_CUDA;
-  std::lock_guard<std::mutex> lk(mu);
-  if (!ready[dev]) {
-    void* p = nullptr;
-    MOE_CUDA(cudaGetSymbolAddress(&p, g_lm_noalloc_scratch));
-    addr[dev] = p;
-    ready[dev] = true;
-  }
-  *out = addr[dev];
+  void* p = nullptr;
+  MOE_CUDA(cudaGetSymbolAddress(&p, g_lm_noalloc_scratch));
+  *out = p;
   return MOE_OK;
 }
 }  // namespace
@@ -1264,3 +1256,208 @@ moe_status_t moe_mxfp8_quantize(const float* v, int M, int K, uint8_t* q, uint8_
 }
 
 }  // extern "C"
+
+// =============================================================================
+// start-up self-check
+// =============================================================================
+namespace {
+
+#include "selfcheck_expected.inc"
+
+constexpr int SC_H = 256, SC_I = 64, SC_E = 16, SC_K = 2, SC_IS = 64, SC_V = 256, SC_M = 4, SC_L = 2;
+constexpr float SC_TOL = 5e-3f;  // relative L2 per row, as the parity tests
+
+struct ScBufs {
+  uint8_t *x, *wr, *w13c, *w13s, *w2c, *w2s, *sw13, *sw2, *lmq, *lms;
+  int32_t *ids, *am, *accept, *drafts;
+  float *w, *y, *logits;
+  uint8_t* scratch;
+  size_t bytes;
+};
+
+size_t sc_scratch_bytes(const moe_model_t& m) {
+  size_t b = moe_route_workspace_bytes(1, SC_E);
+  b = std::max(b, moe_experts_workspace_bytes(1, SC_H, SC_I, SC_E, SC_K, SC_IS));
+  b = std::max(b, lm_head_workspace_bytes(SC_M, SC_V, SC_H));
+  b = std::max(b, decode_step_workspace_bytes(&m, 1));
+  b = std::max(b, decode_step_workspace_bytes(&m, SC_M));
+  return b;
+}
+
+ScBufs sc_carve(uint8_t* base, const moe_model_t* m) {
+  ScBufs b{};
+  size_t off = 0;
+  auto take = [&](size_t n) {
+    uint8_t* p = base ? base + off : nullptr;
+    off += up256(n);
+    return p;
+  };
+  b.x = take(SC_M * SC_H * 2);
+  b.wr = take(SC_E * SC_H * 2);
+  b.w13c = take(SC_E * 2 * SC_I * SC_H / 2);
+  b.w13s = take(SC_E * 2 * SC_I * SC_H / 32);
+  b.w2c = take(SC_E * SC_H * SC_I / 2);
+  b.w2s = take(SC_E * SC_H * SC_I / 32);
+  b.sw13 = take(2 * SC_IS * SC_H * 2);
+  b.sw2 = take(SC_H * SC_IS * 2);
+  b.lmq = take(SC_V * SC_H);
+  b.lms = take(SC_V * 4);
+  b.ids = reinterpret_cast<int32_t*>(take(SC_K * 4));
+  b.w = reinterpret_cast<float*>(take(SC_K * 4));
+  b.y = reinterpret_cast<float*>(take(SC_H * 4));
+  b.am = reinterpret_cast<int32_t*>(take(SC_M * 4));
+  b.accept = reinterpret_cast<int32_t*>(take((1 + SC_M) * 4));
+  b.drafts = reinterpret_cast<int32_t*>(take((SC_M - 1) * 4));
+  b.logits = reinterpret_cast<float*>(take(SC_M * SC_V * 4));
+  b.scratch = take(m ? sc_scratch_bytes(*m) : 0);
+  b.bytes = off;
+  return b;
+}
+
+void sc_model(const ScBufs& b, moe_layer_t* layers, moe_model_t* m) {
+  for (int l = 0; l < SC_L; ++l) {
+    layers[l].router = {b.wr, MOE_FMT_BF16};
+    layers[l].w13_codes = {b.w13c, MOE_FMT_MXFP4_CODES};
+    layers[l].w13_scales = {b.w13s, MOE_FMT_E8M0_SCALES};
+    layers[l].w2_codes = {b.w2c, MOE_FMT_MXFP4_CODES};
+    layers[l].w2_scales = {b.w2s, MOE_FMT_E8M0_SCALES};
+    layers[l].shared_w13 = {b.sw13, MOE_FMT_BF16};
+    layers[l].shared_w2 = {b.sw2, MOE_FMT_BF16};
+  }
+  *m = moe_model_t{};
+  m->n_layers = SC_L;
+  m->H = SC_H;
+  m->I = SC_I;
+  m->E = SC_E;
+  m->top_k = SC_K;
+  m->Is = SC_IS;
+  m->V = SC_V;
+  m->rms_eps = 1e-6f;
+  m->layers = layers;
+  m->lm_head = {b.lmq, MOE_FMT_E4M3};
+  m->lm_scale = {b.lms, MOE_FMT_F32};
+  m->step_path = MOE_STEP_AUTO;
+}
+
+double sc_rel_l2(const float* got, const float* ref, int n) {
+  double num = 0, den = 0;
+  for (int i = 0; i < n; ++i) {
+    const double dlt = static_cast<double>(got[i]) - ref[i];
+    num += dlt * dlt;
+    den += static_cast<double>(ref[i]) * ref[i];
+  }
+  return (num == num) ? std::sqrt(num / (den > 0 ? den : 1e-300)) : 1e300;
+}
+
+}  // namespace
+
+extern "C" size_t moe_selfcheck_workspace_bytes(void) {
+  moe_layer_t layers[SC_L];
+  moe_model_t m;
+  ScBufs dummy = sc_carve(reinterpret_cast<uint8_t*>(256), nullptr);  // any aligned base: only pointers
+  sc_model(dummy, layers, &m);
+  return sc_carve(nullptr, &m).bytes;
+}
+
+extern "C" moe_status_t moe_selfcheck(void* ws, size_t ws_bytes, moe_stream_t stream, int* failed_check,
+                                      float* max_rel_l2) {
+  if (failed_check) *failed_check = 0;
+  if (max_rel_l2) *max_rel_l2 = 0.0f;
+  REQ(ws, MOE_ERR_INVALID_ARG);
+  moe_status_t s = check_ptrs_aligned({ws});
+  if (s != MOE_OK) return s;
+  REQ(ws_bytes >= moe_selfcheck_workspace_bytes(), MOE_ERR_WORKSPACE);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  moe_layer_t layers[SC_L];
+  moe_model_t m;
+  ScBufs b = sc_carve(static_cast<uint8_t*>(ws), nullptr);
+  sc_model(b, layers, &m);
+  b = sc_carve(static_cast<uint8_t*>(ws), &m);
+  const size_t scratch = sc_scratch_bytes(m);
+
+  struct Fill {
+    void* dst;
+    uint32_t n;
+    int kind, tid, e0;
+  } fills[] = {{b.x, SC_M * SC_H, SC_BF16, 1, 125},
+               {b.wr, SC_E * SC_H, SC_BF16, 2, 119},
+               {b.w13c, SC_E * 2 * SC_I * SC_H / 2, SC_BYTE, 3, 0},
+               {b.w13s, SC_E * 2 * SC_I * SC_H / 32, SC_E8M0, 4, 0},
+               {b.w2c, SC_E * SC_H * SC_I / 2, SC_BYTE, 5, 0},
+               {b.w2s, SC_E * SC_H * SC_I / 32, SC_E8M0, 6, 0},
+               {b.sw13, 2 * SC_IS * SC_H, SC_BF16, 7, 119},
+               {b.sw2, SC_H * SC_IS, SC_BF16, 8, 119},
+               {b.lmq, SC_V * SC_H, SC_E4M3, 9, 0},
+               {b.lms, SC_V, SC_POW2, 10, 0}};
+  for (const Fill& f : fills) {
+    k_selfcheck_fill<<<(f.n + 255) / 256, 256, 0, st>>>(f.dst, f.n, f.kind, static_cast<uint32_t>(f.tid), f.e0);
+    MOE_CUDA(cudaGetLastError());
+  }
+  MOE_CUDA(cudaMemcpyAsync(b.drafts, kSelfcheckHeadArgmax, (SC_M - 1) * 4, cudaMemcpyHostToDevice, st));
+
+  int fail = 0;
+  double worst = 0;
+  auto note = [&](int check, bool ok) {
+    if (!ok && !fail) fail = check;
+  };
+  auto device_ok = [&]() -> moe_status_t { return moe_workspace_status(b.scratch, stream); };
+
+  // 1, 2: router and expert layer on token 0
+  int32_t ids[SC_K];
+  float y[SC_H];
+  if ((s = moe_route(b.x, 1, SC_H, b.wr, SC_E, SC_K, b.ids, b.w, nullptr, b.scratch, scratch, stream)) != MOE_OK)
+    return s;
+  if ((s = moe_mxfp4_experts(b.x, 1, SC_H, SC_I, SC_E, SC_K, b.ids, b.w, b.w13c, b.w13s, b.w2c, b.w2s, b.sw13,
+                             b.sw2, SC_IS, b.y, b.scratch, scratch, stream)) != MOE_OK)
+    return s;
+  if ((s = device_ok()) != MOE_OK) return s;
+  MOE_CUDA(cudaMemcpyAsync(ids, b.ids, sizeof ids, cudaMemcpyDeviceToHost, st));
+  MOE_CUDA(cudaMemcpyAsync(y, b.y, sizeof y, cudaMemcpyDeviceToHost, st));
+  MOE_CUDA(cudaStreamSynchronize(st));
+  note(1, std::equal(ids, ids + SC_K, kSelfcheckIds));
+  double r = sc_rel_l2(y, kSelfcheckY, SC_H);
+  worst = std::max(worst, r);
+  note(2, r <= SC_TOL);
+
+  // 3, 4: FP8 head on the 4 tokens, and its verify window with drafts equal to the
+  // head's own argmaxes (every draft must be accepted: accept length 4, not 1)
+  int32_t am[SC_M], accept[1 + SC_M];
+  if ((s = lm_head_fp8_gemv(b.x, SC_M, SC_V, SC_H, b.lmq, reinterpret_cast<const float*>(b.lms), nullptr, b.am,
+                            b.scratch, scratch, stream)) != MOE_OK)
+    return s;
+  if ((s = device_ok()) != MOE_OK) return s;
+  MOE_CUDA(cudaMemcpyAsync(am, b.am, sizeof am, cudaMemcpyDeviceToHost, st));
+  if ((s = lm_head_fp8_verify(b.x, SC_M, SC_V, SC_H, b.lmq, reinterpret_cast<const float*>(b.lms), b.drafts,
+                              nullptr, b.am, b.accept, b.scratch, scratch, stream)) != MOE_OK)
+    return s;
+  if ((s = device_ok()) != MOE_OK) return s;
+  MOE_CUDA(cudaMemcpyAsync(accept, b.accept, sizeof accept, cudaMemcpyDeviceToHost, st));
+  MOE_CUDA(cudaStreamSynchronize(st));
+  note(3, std::equal(am, am + SC_M, kSelfcheckHeadArgmax));
+  note(4, accept[0] == SC_M && std::equal(accept + 1, accept + 1 + SC_M, kSelfcheckHeadArgmax));
+
+  // 5, 6: two-layer decode step on token 0 alone and on the 4-token window
+  float lg[SC_M * SC_V];
+  for (int M : {1, SC_M}) {
+    const int check = M == 1 ? 5 : 6;
+    if ((s = decode_step(&m, b.x, M, b.logits, b.am, nullptr, b.scratch, scratch, stream)) != MOE_OK) return s;
+    if ((s = device_ok()) != MOE_OK) return s;
+    MOE_CUDA(cudaMemcpyAsync(am, b.am, M * 4, cudaMemcpyDeviceToHost, st));
+    MOE_CUDA(cudaMemcpyAsync(lg, b.logits, (size_t)M * SC_V * 4, cudaMemcpyDeviceToHost, st));
+    MOE_CUDA(cudaStreamSynchronize(st));
+    bool ok = std::equal(am, am + M, kSelfcheckStepArgmax);
+    for (int t = 0; t < M; ++t) {
+      r = sc_rel_l2(lg + t * SC_V, kSelfcheckStepLogits + t * SC_V, SC_V);
+      worst = std::max(worst, r);
+      ok = ok && r <= SC_TOL;
+    }
+    note(check, ok);
+  }
+
+  // 7: the step took the single persistent kernel, not the per-layer launches
+  note(7, decode_step_launch_names(&m, 1, nullptr, 0) == 2 && decode_step_launch_names(&m, SC_M, nullptr, 0) == 2);
+
+  if (failed_check) *failed_check = fail;
+  if (max_rel_l2) *max_rel_l2 = static_cast<float>(worst);
+  return fail ? MOE_ERR_SELFCHECK : MOE_OK;
+}

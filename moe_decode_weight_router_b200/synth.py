@@ -124,3 +124,67 @@ def row_scales(V: int, seed: int, tid: int = 6_002, device="cpu") -> torch.Tenso
     g = _gen(seed, tid, device)
     u = torch.rand((V,), generator=g, device=device, dtype=torch.float32)
     return torch.exp2(-14.0 + 6.0 * u)
+
+
+# ---------------------------------------------------------------------------
+# Inputs of the library's start-up self-check: a counter-based generator
+# (SplitMix64's output function, Steele, Lea & Flood, "Fast splittable pseudorandom
+# number generators", OOPSLA 2014) that the library reimplements on the device from
+# the same definition, so both sides hold the same bytes without sharing code.
+# ---------------------------------------------------------------------------
+SELFCHECK = LayerShape(H=256, I=64, E=16, k=2, Is=64, e_lo=120, e_hi=127)
+SELFCHECK_V = 256
+SELFCHECK_M = 4
+SELFCHECK_LAYERS = 2
+SELFCHECK_BASE = 0x5EED000000000000
+SELFCHECK_TIDS = {"x": 1, "wr": 2, "w13c": 3, "w13s": 4, "w2c": 5, "w2s": 6, "sw13": 7, "sw2": 8,
+                  "lm_q": 9, "lm_s": 10}
+
+
+def splitmix64(counter):
+    """SplitMix64 output function of uint64 counters (numpy, wrapping arithmetic)."""
+    import numpy as np
+    with np.errstate(over="ignore"):  # wrap-around modulo 2^64 is the definition
+        z = np.asarray(counter, dtype=np.uint64) + np.uint64(0x9E3779B97F4A7C15)
+        z = (z ^ (z >> np.uint64(30))) * np.uint64(0xBF58476D1CE4E5B9)
+        z = (z ^ (z >> np.uint64(27))) * np.uint64(0x94D049BB133111EB)
+        return z ^ (z >> np.uint64(31))
+
+
+def selfcheck_inputs():
+    """Raw bits of the self-check: a 4-token window x, one tiny MoE layer (used for every
+    layer of the self-check's step) and its 256-row FP8 head.
+    Element i of tensor `tid` draws r = splitmix64(BASE + tid * 2^32 + i):
+      bf16  sign r>>63, exponent e0 + ((r>>56) & 3), mantissa r & 0x7F
+            (e0 125 for x, 119 for the router and shared weights)
+      MXFP4 codes r & 0xFF; E8M0 scales 120 + r % 8
+      e4m3 head codes r & 0xFF with the NaN codes (0x7F, 0xFF) replaced by 0
+      fp32 head row scales 2^-(8 + r % 6)."""
+    import numpy as np
+    S, V = SELFCHECK, SELFCHECK_V
+    sizes = {"x": SELFCHECK_M * S.H, "wr": S.E * S.H, "w13c": S.E * 2 * S.I * S.H // 2, "w13s": S.E * 2 * S.I * S.H // 32,
+             "w2c": S.E * S.H * S.I // 2, "w2s": S.E * S.H * S.I // 32, "sw13": 2 * S.Is * S.H,
+             "sw2": S.H * S.Is, "lm_q": V * S.H, "lm_s": V}
+
+    def r(name):
+        i = np.arange(sizes[name], dtype=np.uint64)
+        return splitmix64(np.uint64(SELFCHECK_BASE) + (np.uint64(SELFCHECK_TIDS[name]) << np.uint64(32)) + i)
+
+    def bf16(name, e0):
+        v = r(name)
+        b = ((v >> np.uint64(63)) << np.uint64(15)) | ((np.uint64(e0) + ((v >> np.uint64(56)) & np.uint64(3)))
+                                                       << np.uint64(7)) | (v & np.uint64(0x7F))
+        return b.astype(np.uint16)
+
+    out = {"x": bf16("x", 125).reshape(SELFCHECK_M, S.H), "wr": bf16("wr", 119).reshape(S.E, S.H),
+           "sw13": bf16("sw13", 119).reshape(2 * S.Is, S.H), "sw2": bf16("sw2", 119).reshape(S.H, S.Is)}
+    out["w13c"] = (r("w13c") & np.uint64(0xFF)).astype(np.uint8).reshape(S.E, 2 * S.I, S.H // 2)
+    out["w13s"] = (np.uint64(120) + r("w13s") % np.uint64(8)).astype(np.uint8).reshape(S.E, 2 * S.I, S.H // 32)
+    out["w2c"] = (r("w2c") & np.uint64(0xFF)).astype(np.uint8).reshape(S.E, S.H, S.I // 2)
+    out["w2s"] = (np.uint64(120) + r("w2s") % np.uint64(8)).astype(np.uint8).reshape(S.E, S.H, S.I // 32)
+    q = (r("lm_q") & np.uint64(0xFF)).astype(np.uint8)
+    q[(q & 0x7F) == 0x7F] = 0
+    out["lm_q"] = q.reshape(V, S.H)
+    e = (np.uint64(127 - 8) - r("lm_s") % np.uint64(6)).astype(np.uint32) << np.uint32(23)
+    out["lm_s"] = e.view(np.float32)
+    return out
