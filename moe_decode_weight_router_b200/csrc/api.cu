@@ -995,7 +995,9 @@ struct PfWs {
   uint8_t* aqs;   // [G][I/32]
   size_t bytes;
 };
-PfWs pf_ws(void* ws, int M, int H, int I, int E, int k, int Is) {
+// own_routing: the chunk routes itself (moe_prefill_layer) and needs buffers for its
+// router logits, ids and weights; under a caller's routing they are left out.
+PfWs pf_ws(void* ws, int M, int H, int I, int E, int k, int Is, bool own_routing = true) {
   uint8_t* b = static_cast<uint8_t*>(ws);
   PfWs s{};
   const size_t G = (size_t)M * k;
@@ -1011,12 +1013,14 @@ PfWs pf_ws(void* ws, int M, int H, int I, int E, int k, int Is) {
   off += up256((size_t)(E + 1) * 4);
   s.ntp = reinterpret_cast<int*>(b + off);
   off += up256((size_t)(E + 1) * 4);
-  s.logits = reinterpret_cast<float*>(b + off);
-  off += up256((size_t)M * E * 4);
-  s.ids = reinterpret_cast<int32_t*>(b + off);
-  off += up256(G * 4);
-  s.w = reinterpret_cast<float*>(b + off);
-  off += up256(G * 4);
+  if (own_routing) {
+    s.logits = reinterpret_cast<float*>(b + off);
+    off += up256((size_t)M * E * 4);
+    s.ids = reinterpret_cast<int32_t*>(b + off);
+    off += up256(G * 4);
+    s.w = reinterpret_cast<float*>(b + off);
+    off += up256(G * 4);
+  }
   s.g_tok = reinterpret_cast<int32_t*>(b + off);
   off += up256(G * 4);
   s.g_w = reinterpret_cast<float*>(b + off);
@@ -1050,7 +1054,10 @@ moe_status_t launch_umma(PrefillParams& p, const DevInfo& d, cudaStream_t st) {
   return MOE_OK;
 }
 
-size_t pf_ws_bytes(int M, int H, int I, int E, int k, int Is) { return pf_ws(nullptr, M, H, I, E, k, Is).bytes; }
+// workspace of a chunk under the caller's routing (moe_mxfp4_experts with M > 8)
+size_t pf_ws_bytes(int M, int H, int I, int E, int k, int Is) {
+  return pf_ws(nullptr, M, H, I, E, k, Is, false).bytes;
+}
 
 // a2-a5 of a chunk whose routing (ids, wts [M][top_k], per-expert counts in w.counts) is
 // known: grouped rows per expert, MXFP8 activations, shared expert, routed W13 + SwiGLU,
@@ -1169,12 +1176,12 @@ moe_status_t experts_chunk(const void* x_bf16, int M, int H, int I, int E, int t
   REQ(ok_pf(M, H, I, E, top_k, Is), MOE_ERR_UNSUPPORTED_SHAPE);
   REQ((reinterpret_cast<uintptr_t>(w13_codes) & 31u) == 0 && (reinterpret_cast<uintptr_t>(w2_codes) & 31u) == 0,
       MOE_ERR_ALIGNMENT);
-  REQ(ws && ws_bytes >= pf_ws(nullptr, M, H, I, E, top_k, Is).bytes, MOE_ERR_WORKSPACE);
+  REQ(ws && ws_bytes >= pf_ws_bytes(M, H, I, E, top_k, Is), MOE_ERR_WORKSPACE);
   DevInfo d;
   moe_status_t s;
   if ((s = dev_info(&d)) != MOE_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const PfWs w = pf_ws(ws, M, H, I, E, top_k, Is);
+  const PfWs w = pf_ws(ws, M, H, I, E, top_k, Is, false);
   MOE_CUDA(cudaMemsetAsync(ws, 0, w.clear_bytes, st));
   const int G = M * top_k;
   k_pf_count<<<(G + 255) / 256, 256, 0, st>>>(topk_ids, G, E, w.counts);
@@ -1461,3 +1468,10 @@ extern "C" moe_status_t moe_selfcheck(void* ws, size_t ws_bytes, moe_stream_t st
   if (max_rel_l2) *max_rel_l2 = static_cast<float>(worst);
   return fail ? MOE_ERR_SELFCHECK : MOE_OK;
 }
+
+#ifdef PF_TIMELINE
+// Profiling builds only: copies the routed-W13 prefill timeline (see prefill_kernels.cuh).
+extern "C" __attribute__((visibility("default"))) int moe_debug_pf_timeline(unsigned long long* out, int n) {
+  return (int)cudaMemcpyFromSymbol(out, pf_tl, (size_t)n * sizeof(unsigned long long));
+}
+#endif

@@ -19,7 +19,9 @@
 //   warps 0-3   epilogue: tcgen05.ld of the accumulator (warp w owns TMEM lanes
 //               32w..32w+31), the mode's arithmetic and the global stores; for the
 //               block-scaled modes they also place the tile's E8M0 scale factors in
-//               tensor memory (tcgen05.st) before its MMAs start.
+//               tensor memory (tcgen05.st) before its MMAs start -- with two column
+//               buffers (K <= 3072) during the previous tile's MMAs, the producer having
+//               fetched them a tile ahead.
 // Modes: router logits (bf16 x bf16), shared W13 + SwiGLU (bf16), shared W2 (bf16,
 // stores y), routed W13 + SwiGLU + MXFP8 re-quantisation (E2M1 x E4M3 block-scaled),
 // routed W2 with the routing weight, added into y.
@@ -44,8 +46,8 @@ constexpr int PF_THREADS = 192;        // warps 0-3 epilogue, 4 producer, 5 MMA
 constexpr int PF_BN = 64;              // token tile (MMA N <= 64)
 constexpr int PF_STAGE_BYTES = 24576;  // per K chunk: weight tile 16 KB + token tile 8 KB
 constexpr int PF_MAX_STAGES = 9;
-constexpr int PF_TMEM_COLS = 512;      // accumulators 0..127 and 128..255, SFA 256.., SFB 384..
-constexpr int PF_SFA_COL = 256, PF_SFB_COL = 384;
+constexpr int PF_TMEM_COLS = 512;      // accumulators 0..63 and 64..127, then the scale columns
+constexpr int PF_SF_COL = 128;         // first scale column: per buffer SFA (4 per K chunk), then SFB
 constexpr int PF_MAX_CHUNKS = 32;      // K / 128 for the block-scaled modes (SF columns)
 
 struct alignas(64) PrefillParams {
@@ -206,6 +208,27 @@ struct PfItem {
 __device__ __forceinline__ bool pf_routed(int mode) { return mode == PF_R13 || mode == PF_R2; }
 __device__ __forceinline__ bool pf_13(int mode) { return mode == PF_SH13 || mode == PF_R13; }
 
+#ifdef PF_TIMELINE
+// Profiling builds only (compiled with -DPF_TIMELINE): block 0 of the routed W13 launch
+// stamps its SM clock (clock64, cycles; every role of block 0 runs on one SM) into pf_tl.  [4q + 0..2] for stage q < 128: producer issued
+// its copies, MMA issuer saw them land, MMA issuer committed the stage; [512 + 8n + 0..5]
+// for item n < 32: MMA issuer saw the item's scales placed, saw its accumulator free,
+// epilogue saw the accumulator full, placed the next item's scales, finished the item,
+// producer issued the item's scale copies, epilogue loaded its first 16 columns, finished
+// its first 16 columns; [768 + 8n + 0..6] for item n < 32, first 16 columns: warp 0
+// past the exchange barrier, SwiGLU done, quantised and stored, past the closing
+// barrier; warp 2 wrote its exchange values, finished its load, started its load.
+__device__ unsigned long long pf_tl[1024];
+#define PF_STAMP(idx)                                                                         \
+  do {                                                                                         \
+    if (blockIdx.x == 0 && p.mode == PF_R13 && (idx) < 1024) pf_tl[(idx)] = (unsigned long long)clock64(); \
+  } while (0)
+#else
+#define PF_STAMP(idx) \
+  do {                \
+  } while (0)
+#endif
+
 constexpr int PF_MAX_E = 512;
 // Routed modes: tile prefix and grouped offsets are copied to shared memory once per
 // CTA (every role decodes every tile; a search over global memory would put a chain
@@ -251,7 +274,9 @@ __device__ inline PfItem pf_item(const PrefillParams& p, int idx, const int* s_n
   return it;
 }
 
-__device__ __forceinline__ float pf_silu(float g) { return g / (1.0f + expf(-g)); }
+// silu(g) = g / (1 + e^-g): the fast division (2 ulp; g / inf = -0 for g < -88) keeps the
+// epilogue short -- the IEEE division's special-case branches serialised it.
+__device__ __forceinline__ float pf_silu(float g) { return __fdividef(g, 1.0f + expf(-g)); }
 
 // floor(log2(a)) of a finite a > 0, exact (subnormals from the mantissa's top bit).
 __device__ __forceinline__ int floor_log2_f32(float a) {
@@ -286,7 +311,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
   extern __shared__ __align__(1024) uint8_t pf_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(pf_smem_raw) + 1023) & ~uintptr_t(1023));
   __shared__ uint64_t full[PF_MAX_STAGES], empty[PF_MAX_STAGES];
-  __shared__ uint64_t acc_full[2], acc_empty[2], sf_full[2], sf_empty[2], sf_ready;
+  __shared__ uint64_t acc_full[2], acc_empty[2], sf_full[2], sf_empty[2], sf_ready[2];
   __shared__ uint32_t tmem_base_s;
   __shared__ volatile int s_abort;
   __shared__ float xch[2][32][17];  // up-half values handed from warps 2,3 to warps 0,1
@@ -311,6 +336,12 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
   const uint32_t sfa_bytes = (uint32_t)(128 * kb + 15) / 16 * 16;
   uint8_t* sfbuf = smem + (size_t)S * stage_bytes;
   const uint32_t sfbuf_bytes = pf_sf_buf_bytes(p.K, p.sf_ld);
+  // Scale columns in tensor memory: two buffers when they fit beside the accumulators
+  // (K <= 3072), so a tile's scales are placed while the previous tile's MMAs run;
+  // otherwise one, placed once the previous tile's MMAs are done.
+  const bool sf2 = PF_SF_COL + 16 * nch <= PF_TMEM_COLS;
+  auto sfa_col = [&](int n) { return (uint32_t)(PF_SF_COL + (sf2 ? 8 * nch * (n & 1) : 0)); };
+  auto sfb_col = [&](int n) { return sfa_col(n) + 4u * (uint32_t)nch; };
 
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
@@ -323,7 +354,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
       mbar_init(&sf_full[b], 1);
       mbar_init(&sf_empty[b], 4);
     }
-    mbar_init(&sf_ready, 4);
+    mbar_init(&sf_ready[0], 4);
+    mbar_init(&sf_ready[1], 4);
     fence_mbar_init();
     s_abort = 0;
   }
@@ -345,21 +377,26 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
       for (int idx = blockIdx.x; idx < total && ok; idx += G, ++n_item) {
         const PfItem it = pf_item(p, idx, s_ntp, s_goff);
         if (mx) {
-          // this tile's scale rows: weight rows (two 64-row runs or one 128-row run) and
-          // the token rows, into scale buffer n_item & 1
-          const int b = n_item & 1;
-          if (n_item >= 2 && !pf_wait(&sf_empty[b], (uint32_t)(((n_item >> 1) - 1) & 1), p.status, &s_abort,
-                                      PFW_SF, p.mode)) {
-            ok = false;
-            break;
-          }
-          uint8_t* dst = sfbuf + (size_t)b * sfbuf_bytes;
-          const uint32_t half = 64u * (uint32_t)kb, tok = (uint32_t)it.ncnt * (uint32_t)p.sf_ld;
-          mbar_arrive_expect_tx(&sf_full[b], 2 * half + tok);
-          const uint64_t pol = policy_evict_first();
-          bulk_g2s(dst, p.sfa + (size_t)it.ya0 * kb, half, &sf_full[b], pol);
-          bulk_g2s(dst + half, p.sfa + (size_t)it.ya1 * kb, half, &sf_full[b], pol);
-          bulk_g2s(dst + sfa_bytes, p.sfb + (size_t)it.grow0 * p.sf_ld, tok, &sf_full[b], pol);
+          // scale rows of a tile -- weight rows (two 64-row runs or one 128-row run) and
+          // the token rows -- into shared buffer m & 1.  With two tensor-memory buffers the
+          // next tile's rows are fetched here too, a tile ahead of its MMAs.
+          auto fetch_scales = [&](int m, const PfItem& t) -> bool {
+            const int b = m & 1;
+            if (m >= 2 && !pf_wait(&sf_empty[b], (uint32_t)(((m >> 1) - 1) & 1), p.status, &s_abort, PFW_SF, p.mode))
+              return false;
+            uint8_t* dst = sfbuf + (size_t)b * sfbuf_bytes;
+            const uint32_t half = 64u * (uint32_t)kb, tok = (uint32_t)t.ncnt * (uint32_t)p.sf_ld;
+            mbar_arrive_expect_tx(&sf_full[b], 2 * half + tok);
+            const uint64_t pol = policy_evict_first();
+            bulk_g2s(dst, p.sfa + (size_t)t.ya0 * kb, half, &sf_full[b], pol);
+            bulk_g2s(dst + half, p.sfa + (size_t)t.ya1 * kb, half, &sf_full[b], pol);
+            bulk_g2s(dst + sfa_bytes, p.sfb + (size_t)t.grow0 * p.sf_ld, tok, &sf_full[b], pol);
+            return true;
+          };
+          if (!sf2 || n_item == 0) ok = fetch_scales(n_item, it);
+          if (ok && sf2 && idx + G < total) ok = fetch_scales(n_item + 1, pf_item(p, idx + G, s_ntp, s_goff));
+          if (!ok) break;
+          if (n_item < 32) PF_STAMP(512 + 8 * n_item + 5);
         }
         for (int ch = 0; ch < nch; ch += KC, ++q) {
           const int s = (int)(q % S);
@@ -367,6 +404,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
             ok = false;
             break;
           }
+          if (q < 128) PF_STAMP(4 * (int)q);
           uint8_t* st = smem + (size_t)s * stage_bytes;
           // transaction bytes count the global (packed) side: 128 rows of 128 E2M1
           // codes are 8 KB although they fill 16 KB of shared memory; the token box
@@ -396,15 +434,21 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
         if (n_item >= 2 && !pf_wait(&acc_empty[ab], (uint32_t)(((n_item >> 1) - 1) & 1), p.status, &s_abort,
                                     PFW_ACC_EMPTY, p.mode))
           break;
-        if (mx && !pf_wait(&sf_ready, (uint32_t)(n_item & 1), p.status, &s_abort, PFW_SF, p.mode)) break;
+        if (n_item < 32) PF_STAMP(512 + 8 * n_item + 1);
+        if (mx && !pf_wait(&sf_ready[sf2 ? ab : 0], (uint32_t)((sf2 ? n_item >> 1 : n_item) & 1), p.status,
+                           &s_abort, PFW_SF, p.mode))
+          break;
+        if (n_item < 32) PF_STAMP(512 + 8 * n_item + 0);
         tc_fence_after();
-        const uint32_t dacc = tbase + 128u * ab;
+        const uint32_t dacc = tbase + 64u * ab;
+        const uint32_t tsfa = tbase + sfa_col(n_item), tsfb = tbase + sfb_col(n_item);
         for (int ch = 0; ch < nch; ch += KC, ++q) {
           const int s = (int)(q % S);
           if (!pf_wait(&full[s], (uint32_t)((q / S) & 1), p.status, &s_abort, PFW_FULL, p.mode)) {
             ok = false;
             break;
           }
+          if (q < 128) PF_STAMP(4 * (int)q + 1);
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + (size_t)s * stage_bytes);
           for (int c = 0; c < KC; ++c) {
@@ -415,13 +459,14 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
               const uint32_t accum = (chc > 0 || k > 0) ? 1u : 0u;
               // advance 32 bytes of K inside the 128-byte swizzled row
               if (mx)
-                umma_mx(dacc, adesc + 2u * k, bdesc + 2u * k, idesc_mx(N, (uint32_t)k), accum,
-                        tbase + PF_SFA_COL + 4u * chc, tbase + PF_SFB_COL + 4u * chc);
+                umma_mx(dacc, adesc + 2u * k, bdesc + 2u * k, idesc_mx(N, (uint32_t)k), accum, tsfa + 4u * chc,
+                        tsfb + 4u * chc);
               else
                 umma_bf16(dacc, adesc + 2u * k, bdesc + 2u * k, idesc_bf16(N), accum);
             }
           }
           tc_commit(&empty[s]);  // the stage returns to the producer once these MMAs are done
+          if (q < 128) PF_STAMP(4 * (int)q + 2);
         }
         if (!ok) break;
         tc_commit(&acc_full[ab]);  // accumulator ab is complete (and so are this tile's reads of the scales)
@@ -446,34 +491,40 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
           wa[c] = *reinterpret_cast<const uint32_t*>(sa + m * kb + 4 * ch);
           wb[c] = m < it.ncnt ? *reinterpret_cast<const uint32_t*>(sb + m * p.sf_ld + 4 * ch) : 0x7F7F7F7Fu;
         }
-        tmem_st4(lane_base + PF_SFA_COL + 4 * ch, wa[0], wa[1], wa[2], wa[3]);
-        tmem_st4(lane_base + PF_SFB_COL + 4 * ch, wb[0], wb[1], wb[2], wb[3]);
+        tmem_st4(lane_base + sfa_col(n_item) + 4 * ch, wa[0], wa[1], wa[2], wa[3]);
+        tmem_st4(lane_base + sfb_col(n_item) + 4 * ch, wb[0], wb[1], wb[2], wb[3]);
       }
       tc_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(&sf_ready);
+        mbar_arrive(&sf_ready[sf2 ? b : 0]);
         mbar_arrive(&sf_empty[b]);
       }
       return true;
     };
     bool live = true;
     if (mx && blockIdx.x < total) live = put_scales(0, pf_item(p, blockIdx.x, s_ntp, s_goff));
+    if (mx && sf2 && live && blockIdx.x + G < total) live = put_scales(1, pf_item(p, blockIdx.x + G, s_ntp, s_goff));
     int n_item = 0;
     for (int idx = blockIdx.x; idx < total; idx += G, ++n_item) {
       const PfItem it = pf_item(p, idx, s_ntp, s_goff);
       const int ab = n_item & 1;
       if (live) pf_wait(&acc_full[ab], (uint32_t)((n_item >> 1) & 1), p.status, &s_abort, PFW_ACC_FULL, p.mode);
+      if (tid == 0 && n_item < 32) PF_STAMP(512 + 8 * n_item + 2);
       named_barrier(2, 128);  // the four epilogue warps take the same decision below
       if (s_abort) break;
       tc_fence_after();
-      // the MMAs of this tile are complete: the scale columns may take the next tile's
-      if (mx && idx + G < total) live = put_scales(n_item + 1, pf_item(p, idx + G, s_ntp, s_goff));
-      const uint32_t acc_lane = lane_base + 128u * ab;
+      // one scale buffer: the MMAs of this tile are complete, its columns may take the next tile's
+      if (mx && !sf2 && idx + G < total) live = put_scales(n_item + 1, pf_item(p, idx + G, s_ntp, s_goff));
+      if (tid == 0 && n_item < 32) PF_STAMP(512 + 8 * n_item + 3);
+      const uint32_t acc_lane = lane_base + 64u * ab;
       for (int j0 = 0; j0 < it.ncnt; j0 += 16) {
         float v[16];
+        if (tid == 64 && n_item < 32 && j0 == 0) PF_STAMP(768 + 8 * n_item + 6);
         tmem_ld16(acc_lane + (uint32_t)j0, v);
+        if (tid == 0 && n_item < 32 && j0 == 0) PF_STAMP(512 + 8 * n_item + 6);
+        if (tid == 64 && n_item < 32 && j0 == 0) PF_STAMP(768 + 8 * n_item + 5);
         const int jn = min(16, it.ncnt - j0);
         if (p.mode == PF_ROUTER || p.mode == PF_SH2) {
           const int row = 128 * it.mt + 32 * warp + r;
@@ -489,42 +540,55 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
               atomicAdd(p.out_f32 + (size_t)__ldg(p.g_tok + g) * p.out_ld + row, __ldg(p.g_w + g) * v[j]);
             }
         } else {
-          // 13 modes: warps 0,1 hold gate rows, warps 2,3 the matching up rows
-          if (warp >= 2) {
+          // 13 modes: warps 0,1 hold gate rows, warps 2,3 the matching up rows.  Each
+          // pair (w, w+2) splits the 16 tokens: the gate warp finishes tokens 0-7 and
+          // the up warp tokens 8-15, after handing each other the missing half.
+          const int pr = warp & 1;
+          const bool gate = warp < 2;
 #pragma unroll
-            for (int j = 0; j < 16; ++j) xch[warp - 2][r][j] = v[j];
-          }
+          for (int j = 0; j < 8; ++j) xch[pr][r][(gate ? 0 : 8) + j] = gate ? v[8 + j] : v[j];
+          if (tid == 64 && n_item < 32 && j0 == 0) PF_STAMP(768 + 8 * n_item + 4);
           named_barrier(2, 128);
-          if (warp < 2) {
-            const int i = 64 * it.mt + 32 * warp + r;  // intermediate index
-            float a[16];
+          if (tid == 0 && n_item < 32 && j0 == 0) PF_STAMP(768 + 8 * n_item + 0);
+          const int i = 64 * it.mt + 32 * pr + r;  // intermediate index
+          const int jb = gate ? 0 : 8;             // this warp's first token of the chunk
+          float a[8];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) a[j] = pf_silu(v[j]) * xch[warp][r][j];
-            if (p.mode == PF_SH13) {
+          for (int j = 0; j < 8; ++j)
+            a[j] = gate ? pf_silu(v[j]) * xch[pr][r][8 + j] : pf_silu(xch[pr][r][j]) * v[8 + j];
+          if (tid == 0 && n_item < 32 && j0 == 0) PF_STAMP(768 + 8 * n_item + 1);
+          if (p.mode == PF_SH13) {
 #pragma unroll
-              for (int j = 0; j < 16; ++j)
-                if (j < jn) p.out_bf16[(size_t)(it.n0 + j0 + j) * p.out_ld + i] = __float2bfloat16_rn(a[j]);
-            } else {
-              // MXFP8 of each token's 32-block (this warp's 32 rows): the block maximum
-              // of |a| is one warp max over the bit patterns (monotonic for x >= 0)
+            for (int j = 0; j < 8; ++j)
+              if (jb + j < jn) p.out_bf16[(size_t)(it.n0 + j0 + jb + j) * p.out_ld + i] = __float2bfloat16_rn(a[j]);
+          } else {
+            // MXFP8 of each token's 32-block (this warp's 32 rows): the block maximum
+            // of |a| is one warp max over the bit patterns (monotonic for x >= 0)
 #pragma unroll
-              for (int j = 0; j < 16; ++j) {
-                const float am = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(a[j]))));
-                const int s = mxfp8_exponent(am);
-                if (j < jn) {
-                  const size_t g = (size_t)(it.grow0 + j0 + j);
-                  p.out_q[g * p.out_ld + i] = am == 0.0f ? (uint8_t)0 : e4m3_of(a[j] * exp2i(-s));
-                  if (r == 0) p.out_qs[g * p.out_qs_ld + (64 * it.mt + 32 * warp) / 32] = (uint8_t)(s + 127);
-                }
+            for (int j = 0; j < 8; ++j) {
+              const float am = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(a[j]))));
+              const int s = mxfp8_exponent(am);
+              if (jb + j < jn) {
+                const size_t g = (size_t)(it.grow0 + j0 + jb + j);
+                p.out_q[g * p.out_ld + i] = am == 0.0f ? (uint8_t)0 : e4m3_of(a[j] * exp2i(-s));
+                if (r == 0) p.out_qs[g * p.out_qs_ld + (64 * it.mt + 32 * pr) / 32] = (uint8_t)(s + 127);
               }
             }
+            if (tid == 0 && n_item < 32 && j0 == 0) PF_STAMP(768 + 8 * n_item + 2);
           }
-          named_barrier(2, 128);
+          named_barrier(2, 128);  // xch is rewritten by the next chunk
+          if (tid == 0 && n_item < 32 && j0 == 0) PF_STAMP(768 + 8 * n_item + 3);
         }
+        if (tid == 0 && n_item < 32 && j0 == 0) PF_STAMP(512 + 8 * n_item + 7);
       }
+      if (tid == 0 && n_item < 32) PF_STAMP(512 + 8 * n_item + 4);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[ab]);
+      // two scale buffers: this tile's MMAs are done, so its buffer takes the tile after
+      // next while the next tile's MMAs run
+      if (mx && sf2 && live && idx + 2 * G < total)
+        live = put_scales(n_item + 2, pf_item(p, idx + 2 * G, s_ntp, s_goff));
     }
   }
   tc_fence_before();

@@ -95,7 +95,10 @@ def test_experts_validation(lib):
     assert call(ws_bytes=need - 1) == 4
     # a chunk (M a multiple of 128) takes the block-scaled path under the caller's routing
     chunk = lib.moe_experts_workspace_bytes(2048, 2560, 768, 512, 8, 768)
-    assert chunk == lib.moe_prefill_workspace_bytes(2048, 2560, 768, 512, 8, 768) > 0
+    # ... and its workspace leaves out the router logits, ids and weights (M*E*4 + 2*M*k*4
+    # bytes, each rounded to 256) that only moe_prefill_layer's own routing needs
+    own = lib.moe_prefill_workspace_bytes(2048, 2560, 768, 512, 8, 768)
+    assert 0 < chunk == own - (2048 * 512 * 4 + 2 * 2048 * 8 * 4)
     assert lib.moe_experts_workspace_bytes(200, 2560, 768, 512, 8, 768) == 0
     assert call(M=200) == 2
     assert call(M=2048, ws_bytes=chunk - 1) == 4

@@ -126,7 +126,8 @@ def test_prefill_ling_chunk():
 def test_experts_chunk_under_given_routing():
     # moe_mxfp4_experts with M a multiple of 128: the caller's routing (distinct random
     # experts per token, random positive weights, two ids outside [0, E) that must add
-    # nothing) through the block-scaled path; every token row against the oracle
+    # nothing, one token naming an expert twice) through the block-scaled path; every
+    # token row against the oracle
     M = 256
     L = synth.layer(SMALL, 9, device="cuda")
     x = synth.tokens(M, SMALL.H, 9, device="cuda")
@@ -135,6 +136,7 @@ def test_experts_chunk_under_given_routing():
     w = rng.uniform(0.05, 1.0, size=(M, SMALL.k)).astype(np.float32)
     ids[5, 2] = -1
     ids[7, 0] = SMALL.E
+    ids[3, 1] = ids[3, 0]  # a token naming one expert twice gets both weights
     ws = torch.empty(moe_experts_workspace_bytes(M, SMALL.H, SMALL.I, SMALL.E, SMALL.k, SMALL.Is),
                      dtype=torch.uint8, device="cuda")
     y = moe_mxfp4_experts(x, torch.from_numpy(ids).cuda(), torch.from_numpy(w).cuda(), L["w13c"], L["w13s"],
