@@ -1237,6 +1237,7 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
   const uint32_t bytesA = step_item_bytes(IT_A, H, I, Is), bytesS = step_item_bytes(IT_CS, H, I, Is);
   const uint32_t bytesB = step_item_bytes(IT_B, H, I, Is), bytesC = step_item_bytes(IT_CR, H, I, Is);
   const int capB = step_group_cap(R, bytesB, 8), capC = step_group_cap(R, bytesC, 16);
+  static_assert(STEP_CONSUMERS == 8, "window groups: at most one W13 and two W2 tiles per consumer warp");
 
   if (tid == 0) {
     for (int s = 0; s < STEP_SLOTS; ++s) {
@@ -1509,13 +1510,15 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
           item_stamp(p, i, 2);
           const int done = __shfl_sync(0xffffffffu, nmine, 0) + __shfl_sync(0xffffffffu, nmine, 16);
           if (lane == 0) {
-            if (done > 0) {
-              __threadfence();
-              atomicAdd(lc + CTR_EXP + u, (unsigned)done);
-            }
+            // the ring space goes back first: the publish below (fence, counter) no
+            // longer needs the rows
             if (atomicAdd(&s_gdone[slot], done) + done == U) {
               s_gdone[slot] = 0;
               mbar_arrive(&empty[slot]);
+            }
+            if (done > 0) {
+              __threadfence();
+              atomicAdd(lc + CTR_EXP + u, (unsigned)done);
             }
           }
         }
@@ -1538,28 +1541,27 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
           const uint8_t* up = gate + codes;
           const uint8_t* gs = gate + 2 * codes;
           const uint8_t* us = gs + scales;
-          int mine = 0;
-          for (int j = j0; j < nt; j += STEP_CONSUMERS, ++mine) {
-            float c[4] = {0.f, 0.f, 0.f, 0.f};
-            if (ready) {
-              const int rg = 8 * j + g;  // tile row: gate row and up row of intermediate 8 (r0 + j) + g
-              mxfp4_tile_dot_win(gate + rg * (H / 2), up + rg * (H / 2), gs + rg * (H / 32), us + rg * (H / 32),
-                                 H / 32, xf16, xss, M, s_sh, c);
-            }
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int tok = 2 * t + e;
-              if (tok < M)
-                p.a_routed[((size_t)u * M + tok) * I + 8 * (r0 + j) + g] = silu_f32(c[e]) * c[2 + e];
-            }
-            __syncwarp();
-            if (lane == 0) signal_counter(lc + CTR_EXP + u);
+          // groups hold at most capB <= STEP_CONSUMERS tiles: one tile per warp
+          const int j = j0;
+          float c[4] = {0.f, 0.f, 0.f, 0.f};
+          if (ready) {
+            const int rg = 8 * j + g;  // tile row: gate row and up row of intermediate 8 (r0 + j) + g
+            mxfp4_tile_dot_win(gate + rg * (H / 2), up + rg * (H / 2), gs + rg * (H / 32), us + rg * (H / 32),
+                               H / 32, xf16, xss, M, s_sh, c);
           }
+          __syncwarp();  // every lane is done reading the tile: its ring space goes back first
           item_stamp(p, i, 2);
-          if (lane == 0 && atomicAdd(&s_gdone[slot], mine) + mine == nt) {
+          if (lane == 0 && atomicAdd(&s_gdone[slot], 1) + 1 == nt) {
             s_gdone[slot] = 0;
             mbar_arrive(&empty[slot]);
           }
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int tok = 2 * t + e;
+            if (tok < M) p.a_routed[((size_t)u * M + tok) * I + 8 * (r0 + j) + g] = silu_f32(c[e]) * c[2 + e];
+          }
+          __syncwarp();
+          if (lane == 0) signal_counter(lc + CTR_EXP + u);
         }
         tc += nt;
         ++i;
@@ -1681,23 +1683,23 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
           item_stamp(p, i, 1);
           const uint8_t* cd = ring + s0;
           const uint8_t* sc = cd + codes;
-          int mine = 0;
-          for (int j = j0; j < nt; j += STEP_CONSUMERS, ++mine) {
-            float c[4] = {0.f, 0.f, 0.f, 0.f};
-            const int rg = 16 * j + g;  // tile rows rg and rg + 8: output rows 16 (c0 + j) + g (+8)
-            if (ready)
+          // groups hold at most capC <= 2 * STEP_CONSUMERS tiles: one or two per warp,
+          // both computed before the ring space goes back, then added into h
+          const int ja = j0, jb = j0 + STEP_CONSUMERS;
+          const int mine = jb < nt ? 2 : 1;
+          float c[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+          if (ready) {
+#pragma unroll 1
+            for (int q = 0; q < mine; ++q) {  // one inlined copy of the product
+              const int j = q ? jb : ja;
+              const int rg = 16 * j + g;  // tile rows rg and rg + 8: output rows 16 (c0 + j) + g (+8)
+              float v[4];
               mxfp4_tile_dot_win(cd + rg * (I / 2), cd + (rg + 8) * (I / 2), sc + rg * (I / 32),
-                                 sc + (rg + 8) * (I / 32), I / 32, my_af, ass, M, s_ash[cu], c);
-            const int h0 = 16 * (c0 + j) + g;
+                                 sc + (rg + 8) * (I / 32), I / 32, my_af, ass, M, s_ash[cu], v);
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int tok = 2 * t + e;
-              if (tok < M) {
-                const float wt = P.w[u][tok];
-                if (wt != 0.0f) {
-                  atomicAdd(hout + (size_t)tok * H + h0, c[e] * wt);
-                  atomicAdd(hout + (size_t)tok * H + h0 + 8, c[2 + e] * wt);
-                }
+              for (int e = 0; e < 4; ++e) {
+                c[0][e] = q ? c[0][e] : v[e];
+                c[1][e] = q ? v[e] : c[1][e];
               }
             }
           }
@@ -1706,6 +1708,21 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
           if (lane == 0 && atomicAdd(&s_gdone[slot], mine) + mine == nt) {
             s_gdone[slot] = 0;
             mbar_arrive(&empty[slot]);
+          }
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            const int h0 = 16 * (c0 + (q ? jb : ja)) + g;
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int tok = 2 * t + e;
+              if (q < mine && tok < M) {
+                const float wt = P.w[u][tok];
+                if (wt != 0.0f) {
+                  atomicAdd(hout + (size_t)tok * H + h0, c[q][e] * wt);
+                  atomicAdd(hout + (size_t)tok * H + h0 + 8, c[q][2 + e] * wt);
+                }
+              }
+            }
           }
         }
         tc += nt;
