@@ -46,7 +46,7 @@ struct DevInfo {
   int smem_optin = 0;
   // largest dynamic shared memory per kernel family: the opt-in limit minus the
   // kernel's own static shared memory
-  int dyn_dense = 0, dyn_e13 = 0, dyn_e2 = 0, dyn_lm = 0, dyn_step = 0, dyn_pf = 0;
+  int dyn_dense = 0, dyn_e13 = 0, dyn_e2 = 0, dyn_lm = 0, dyn_lmb = 0, dyn_step = 0, dyn_pf = 0;
   int coop = 0;
 };
 
@@ -78,6 +78,7 @@ moe_status_t dev_info(DevInfo* out) {
     MOE_CUDA(allow_dyn_smem(k_experts13, lim, &d.dyn_e13));
     MOE_CUDA(allow_dyn_smem(k_experts2, lim, &d.dyn_e2));
     MOE_CUDA(allow_dyn_smem(k_lm_gemv, lim, &d.dyn_lm));
+    MOE_CUDA(allow_dyn_smem(k_lm_gemv_bf16, lim, &d.dyn_lmb));
     MOE_CUDA(allow_dyn_smem(k_step<false>, lim, &d.dyn_step));
     MOE_CUDA(allow_dyn_smem(k_step<true>, lim, &d.dyn_step));
     MOE_CUDA(allow_dyn_smem(k_umma, lim, &d.dyn_pf));
@@ -572,13 +573,23 @@ moe_status_t lm_head_bf16_gemv(const void* x_bf16, int M, int V, int H, const vo
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   Ctrl c = ctrl_of(ws);
   MOE_CUDA(cudaMemsetAsync(ws, 0, CTRL_BYTES, st));
-  const long long T = (V + 15) / 16;
-  const long long want = (T + LMB_WARPS - 1) / LMB_WARPS;
-  const int grid = (int)(want < 4LL * d.sms ? want : 4LL * d.sms);
-  const size_t smem = (size_t)MAX_M * padded_stride(2u * H);
-  k_lm_gemv_bf16<<<grid, 32 * LMB_WARPS, smem, st>>>(static_cast<const __nv_bfloat16*>(x_bf16), M, V, H,
-                                                     static_cast<const __nv_bfloat16*>(w_bf16), logits, argmax, c.keys,
-                                                     c.lm_counter);
+  LMParams p{};
+  p.x = static_cast<const __nv_bfloat16*>(x_bf16);
+  p.M = M;
+  p.V = V;
+  p.H = H;
+  p.w = static_cast<const uint8_t*>(w_bf16);
+  p.logits = logits;
+  p.argmax = argmax;
+  p.keys = c.keys;
+  p.counter = c.lm_counter;
+  p.status = c.status;
+  const size_t fixed = lmb_fixed_bytes(H), stage = lmb_stage_bytes(H);
+  p.stages = stages_for(d.dyn_lmb, fixed, stage);
+  if (p.stages < N_CONSUMERS) return MOE_ERR_UNSUPPORTED_SHAPE;
+  const long long T = (V + 7) / 8;
+  const int grid = (int)(T < d.sms ? T : d.sms);
+  k_lm_gemv_bf16<<<grid, EXPERT_THREADS, fixed + (size_t)p.stages * stage, st>>>(p);
   MOE_CUDA(cudaGetLastError());
   return MOE_OK;
 }

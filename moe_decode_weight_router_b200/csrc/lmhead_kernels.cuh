@@ -257,78 +257,108 @@ __global__ void __launch_bounds__(EXPERT_THREADS, 1) k_lm_gemv(LMParams p) {
 
 // ---------------------------------------------------------------------------
 // k_lm_gemv_bf16: the same head with the BF16 weights it is quantised from -- the
-// comparison the FP8 head is measured against (twice the bytes per logit).  Eight
-// warps per block, each owning 16-row tiles; rows stream through 128-bit
-// non-allocating loads (two per row per 64 columns, 16 in flight per thread).
+// comparison the FP8 head is measured against (twice the bytes per logit).  The FP8
+// head's pipeline: a producer warp bulk-copies 8-row tiles (contiguous, 16 H bytes)
+// into a ring of stages, four consumer warps take tiles round-robin.  A tile fills
+// rows 0-7 of the m16n8k16 product (rows 8-15 are zero: the head is bound by its
+// weight bytes, not by the tensor core); x stays bf16, so the products are exact.
 // ---------------------------------------------------------------------------
-constexpr int LMB_WARPS = 8;
-__global__ void __launch_bounds__(32 * LMB_WARPS) k_lm_gemv_bf16(const __nv_bfloat16* __restrict__ x, int M, int V,
-                                                                int H, const __nv_bfloat16* __restrict__ w,
-                                                                float* __restrict__ logits, int32_t* __restrict__ argmax,
-                                                                unsigned long long* keys, unsigned* counter) {
+__host__ __device__ inline size_t lmb_stage_bytes(int H) {
+  size_t b = 8 * 2 * (size_t)H;  // 8 contiguous bf16 rows: one bulk copy per tile
+  return (b + 127) / 128 * 128;
+}
+__host__ __device__ inline size_t lmb_fixed_bytes(int H) { return 128 + MAX_M * (size_t)padded_stride(2u * H); }
+
+__global__ void __launch_bounds__(EXPERT_THREADS, 1) k_lm_gemv_bf16(LMParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ unsigned long long s_best[LMB_WARPS][MAX_M];
+  __shared__ unsigned long long s_best[N_CONSUMERS][MAX_M];
   __shared__ int s_last;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int M = p.M, V = p.V, H = p.H, S = p.stages;
   const uint32_t xss = padded_stride(2u * H);
-  // activation rows as bf16 (the MMA's B operand), zero rows beyond M
-  for (int i = tid; i < MAX_M * (H / 8); i += blockDim.x) {
-    const int tok = i / (H / 8), c = i % (H / 8);
-    const uint4 v = tok < M ? *reinterpret_cast<const uint4*>(x + (size_t)tok * H + 8 * c) : make_uint4(0, 0, 0, 0);
-    *reinterpret_cast<uint4*>(smem + tok * xss + 16 * c) = v;
+  const uint32_t ls = 2u * H;
+  const __nv_bfloat16* w = reinterpret_cast<const __nv_bfloat16*>(p.w);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+  uint64_t* empty = full + MAX_STAGES;
+  uint8_t* xs = smem + 128;
+  uint8_t* stages = smem + lmb_fixed_bytes(H);
+  const size_t sbytes = lmb_stage_bytes(H);
+
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    fence_mbar_init();
   }
   __syncthreads();
-  const long long T = (V + 15) / 16;
-  const long long gw = (long long)blockIdx.x * LMB_WARPS + warp, nw = (long long)gridDim.x * LMB_WARPS;
-  unsigned long long bestA = 0ull, bestB = 0ull;
+  const long long T = (V + 7) / 8;
+  const long long start = T * blockIdx.x / gridDim.x;
+  const long long end = T * (blockIdx.x + 1) / gridDim.x;
+  const int nloc = (int)(end - start);
+
+  if (warp == N_CONSUMERS) {
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_first();
+      for (int i = 0; i < nloc; ++i) {
+        const int s = i % S;
+        if (i >= S && !mbar_wait(&empty[s], ((i / S) - 1) & 1, p.status)) break;
+        const long long v0 = (start + i) * 8;
+        const int nrows = (int)min(8LL, (long long)V - v0);
+        mbar_arrive_expect_tx(&full[s], (uint32_t)nrows * ls);
+        bulk_g2s(stages + s * sbytes, w + (size_t)v0 * H, (uint32_t)nrows * ls, &full[s], pol);
+      }
+      for (int i = (nloc > S ? nloc - S : 0); i < nloc; ++i) mbar_wait(&full[i % S], (i / S) & 1, p.status);
+    }
+    return;
+  }
+
+  // activation rows as bf16 (the MMA's B operand), zero rows beyond M
+  for (int i = tid; i < MAX_M * (H / 8); i += 32 * N_CONSUMERS) {
+    const int tok = i / (H / 8), c = i % (H / 8);
+    const uint4 v = tok < M ? *reinterpret_cast<const uint4*>(p.x + (size_t)tok * H + 8 * c) : make_uint4(0, 0, 0, 0);
+    *reinterpret_cast<uint4*>(xs + tok * xss + 16 * c) = v;
+  }
+  named_barrier(1, 32 * N_CONSUMERS);
+  unsigned long long bestA = 0ull, bestB = 0ull;  // tokens 2t and 2t+1
   const int ta = 2 * t, tb = 2 * t + 1;
-  for (long long tile = gw; tile < T; tile += nw) {
-    const long long v0 = tile * 16;
-    const long long ra = min(v0 + g, (long long)V - 1), rb = min(v0 + g + 8, (long long)V - 1);
-    const uint4* wa = reinterpret_cast<const uint4*>(w + ra * H);
-    const uint4* wb = reinterpret_cast<const uint4*>(w + rb * H);
+  for (int i = warp; i < nloc; i += N_CONSUMERS) {
+    const int s = i % S;
+    if (!mbar_wait(&full[s], (i / S) & 1, p.status)) return;
+    const long long v0 = (start + i) * 8;
+    const uint8_t* row = stages + s * sbytes + g * ls;
     float c4[4][4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) c4[u][0] = c4[u][1] = c4[u][2] = c4[u][3] = 0.0f;
-#pragma unroll 4
+#pragma unroll 2
     for (int j = 0; j < H / 64; ++j) {
-      // this thread's 16 columns of the chunk: 64j + 16t .. +15 (two 16-byte pieces per row)
-      const uint4 A0 = ldg128_stream(wa + 8 * j + 2 * t), A0b = ldg128_stream(wa + 8 * j + 2 * t + 1);
-      const uint4 A1 = ldg128_stream(wb + 8 * j + 2 * t), A1b = ldg128_stream(wb + 8 * j + 2 * t + 1);
-      const uint4 X0 = lds128(smem + g * xss + 2 * (64 * j + 16 * t));
-      const uint4 X1 = lds128(smem + g * xss + 2 * (64 * j + 16 * t) + 16);
+      // this thread's 16 columns of the chunk: 64j + 16t .. +15 (two 16-byte pieces)
+      const uint4 A0 = lds128(row + 128 * j + 32 * t), A0b = lds128(row + 128 * j + 32 * t + 16);
+      const uint4 X0 = lds128(xs + g * xss + 2 * (64 * j + 16 * t));
+      const uint4 X1 = lds128(xs + g * xss + 2 * (64 * j + 16 * t) + 16);
       const uint32_t P[8] = {A0.x, A0.y, A0.z, A0.w, A0b.x, A0b.y, A0b.z, A0b.w};
-      const uint32_t Q[8] = {A1.x, A1.y, A1.z, A1.w, A1b.x, A1b.y, A1b.z, A1b.w};
       const uint32_t X[8] = {X0.x, X0.y, X0.z, X0.w, X1.x, X1.y, X1.z, X1.w};
 #pragma unroll
-      for (int s4 = 0; s4 < 4; ++s4)
-        mma_bf16(c4[s4], P[2 * s4], Q[2 * s4], P[2 * s4 + 1], Q[2 * s4 + 1], X[2 * s4], X[2 * s4 + 1]);
+      for (int s4 = 0; s4 < 4; ++s4) mma_bf16(c4[s4], P[2 * s4], 0u, P[2 * s4 + 1], 0u, X[2 * s4], X[2 * s4 + 1]);
     }
-    float c[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) c[e] = (c4[0][e] + c4[1][e]) + (c4[2][e] + c4[3][e]);
-    const long long va = v0 + g, vb = v0 + g + 8;
-    if (ta < M) {
-      if (va < V) {
-        if (logits) logits[(size_t)ta * V + va] = c[0];
-        bestA = max(bestA, argmax_key(c[0], (int)va));
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+    const float ca = (c4[0][0] + c4[1][0]) + (c4[2][0] + c4[3][0]);
+    const float cb = (c4[0][1] + c4[1][1]) + (c4[2][1] + c4[3][1]);
+    const long long va = v0 + g;
+    if (va < V) {
+      if (ta < M) {
+        if (p.logits) p.logits[(size_t)ta * V + va] = ca;
+        bestA = max(bestA, argmax_key(ca, (int)va));
       }
-      if (vb < V) {
-        if (logits) logits[(size_t)ta * V + vb] = c[2];
-        bestA = max(bestA, argmax_key(c[2], (int)vb));
-      }
-    }
-    if (tb < M) {
-      if (va < V) {
-        if (logits) logits[(size_t)tb * V + va] = c[1];
-        bestB = max(bestB, argmax_key(c[1], (int)va));
-      }
-      if (vb < V) {
-        if (logits) logits[(size_t)tb * V + vb] = c[3];
-        bestB = max(bestB, argmax_key(c[3], (int)vb));
+      if (tb < M) {
+        if (p.logits) p.logits[(size_t)tb * V + va] = cb;
+        bestB = max(bestB, argmax_key(cb, (int)va));
       }
     }
   }
+  // lanes with the same t hold the same tokens: reduce over g
 #pragma unroll
   for (int o = 4; o < 32; o <<= 1) {
     bestA = max(bestA, __shfl_xor_sync(0xffffffffu, bestA, o));
@@ -338,23 +368,23 @@ __global__ void __launch_bounds__(32 * LMB_WARPS) k_lm_gemv_bf16(const __nv_bflo
     s_best[warp][ta] = bestA;
     s_best[warp][tb] = bestB;
   }
-  __syncthreads();
+  named_barrier(1, 32 * N_CONSUMERS);
   if (warp == 0 && lane < M) {
     unsigned long long b = 0ull;
-    for (int w2 = 0; w2 < LMB_WARPS; ++w2) b = max(b, s_best[w2][lane]);
-    if (b) atomicMax(keys + lane, b);
+    for (int w2 = 0; w2 < N_CONSUMERS; ++w2) b = max(b, s_best[w2][lane]);
+    if (b) atomicMax(p.keys + lane, b);
   }
   __threadfence();
-  __syncthreads();
-  if (tid == 0) s_last = (atomicAdd(counter, 1u) == gridDim.x - 1);
-  __syncthreads();
+  named_barrier(1, 32 * N_CONSUMERS);
+  if (tid == 0) s_last = (atomicAdd(p.counter, 1u) == gridDim.x - 1);
+  named_barrier(1, 32 * N_CONSUMERS);
   if (s_last) {
     __threadfence();
     if (tid < M) {
-      const unsigned long long k = atomicExch(keys + tid, 0ull);
-      argmax[tid] = (int32_t)(0xFFFFFFFFu - (uint32_t)(k & 0xFFFFFFFFull));
+      const unsigned long long k = atomicExch(p.keys + tid, 0ull);
+      p.argmax[tid] = (int32_t)(0xFFFFFFFFu - (uint32_t)(k & 0xFFFFFFFFull));
     }
-    if (tid == 0) *counter = 0u;
+    if (tid == 0) *p.counter = 0u;
   }
 }
 
