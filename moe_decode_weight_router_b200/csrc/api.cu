@@ -231,11 +231,12 @@ moe_status_t launch_e2(E2Params p, const DevInfo& d, cudaStream_t st) {
 moe_status_t launch_lm(LMParams p, const DevInfo& d, cudaStream_t st) {
   const size_t fixed = lm_fixed_bytes(p.H), stage = lm_stage_bytes(p.H);
   p.stages = stages_for(d.dyn_lm, fixed, stage);
-  if (p.stages < N_CONSUMERS) return MOE_ERR_UNSUPPORTED_SHAPE;
+  // every consumer warp needs a stage of its own in flight (LM_STAGES == LM_CONSUMERS)
+  if (p.stages < LM_CONSUMERS) return MOE_ERR_UNSUPPORTED_SHAPE;
   const size_t smem = fixed + (size_t)p.stages * stage;
-  const long long T = (p.V + 15) / 16;
+  const long long T = (p.V + 7) / 8;
   const int grid = (int)(T < d.sms ? T : d.sms);
-  k_lm_gemv<<<grid, EXPERT_THREADS, smem, st>>>(p);
+  k_lm_gemv<<<grid, LM_THREADS, smem, st>>>(p);
   MOE_CUDA(cudaGetLastError());
   return MOE_OK;
 }

@@ -345,10 +345,11 @@ __global__ void __launch_bounds__(DENSE_THREADS) k_dense(DenseParams p) {
 // f16 copy of x scaled per token by a power of two (exact), for the f16 products;
 // shift[t] receives token t's exponent sh (x_t * 2^sh has its largest magnitude in
 // [2^14, 2^15)).  Run by the N_CONSUMERS consumer warps.
+template <int NC = N_CONSUMERS>  // the consumer warps that run it (warps 0 .. NC-1)
 __device__ __forceinline__ void stage_x_f16(const __nv_bfloat16* x, int M, int H, uint8_t* xs, uint32_t xss,
                                             int* shift) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  for (int tok = warp; tok < MAX_M; tok += N_CONSUMERS) {
+  for (int tok = warp; tok < MAX_M; tok += NC) {
     float amax = 0.0f;
     if (tok < M)
       for (int c = lane; c < H / 8; c += 32) {
@@ -361,8 +362,8 @@ __device__ __forceinline__ void stage_x_f16(const __nv_bfloat16* x, int M, int H
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     if (lane == 0) shift[tok] = f16_range_shift(amax);
   }
-  named_barrier(1, 32 * N_CONSUMERS);
-  for (int i = tid; i < MAX_M * (H / 8); i += 32 * N_CONSUMERS) {
+  named_barrier(1, 32 * NC);
+  for (int i = tid; i < MAX_M * (H / 8); i += 32 * NC) {
     const int tok = i / (H / 8), c = i % (H / 8);
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
     if (tok < M) {
@@ -378,7 +379,7 @@ __device__ __forceinline__ void stage_x_f16(const __nv_bfloat16* x, int M, int H
     }
     *reinterpret_cast<uint4*>(xs + tok * xss + 16 * c) = v;
   }
-  named_barrier(1, 32 * N_CONSUMERS);
+  named_barrier(1, 32 * NC);
 }
 
 // Largest and smallest E8M0 scale byte of rows g and g+8 (the 4 lanes of a lane group

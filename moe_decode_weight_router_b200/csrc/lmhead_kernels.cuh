@@ -92,8 +92,16 @@ __device__ __forceinline__ void mtp_accept(const int32_t* argmax, const int32_t*
   out[0] = n + 1;
 }
 
+// 8-row tiles (one contiguous bulk copy each) through a ring of LM_STAGES stages, one
+// producer warp and LM_CONSUMERS consumer warps taking tiles round-robin.  A tile fills
+// rows 0-7 of the m16n8k16 product (rows 8-15 are zero: the head is bound by its
+// weight bytes; eight warps keep the e4m3 widening off the critical path).
+constexpr int LM_CONSUMERS = 8;
+constexpr int LM_THREADS = 32 * (LM_CONSUMERS + 1);
+constexpr int LM_STAGES = 8;
+static_assert(LM_STAGES == MAX_STAGES && LM_STAGES >= LM_CONSUMERS, "stage barriers: one stage per consumer warp in flight");
 __host__ __device__ inline size_t lm_stage_bytes(int H) {
-  size_t b = 16 * (size_t)H;  // 16 contiguous rows: one bulk copy per tile
+  size_t b = 8 * (size_t)H;  // 8 contiguous rows: one bulk copy per tile
   return (b + 127) / 128 * 128;
 }
 __host__ __device__ inline size_t lm_fixed_bytes(int H) { return 128 + 8 * (size_t)padded_stride(2u * H); }
@@ -102,11 +110,11 @@ __device__ __forceinline__ unsigned long long argmax_key(float v, int idx) {
   return ((unsigned long long)float_key(v) << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)idx);
 }
 
-__global__ void __launch_bounds__(EXPERT_THREADS, 1) k_lm_gemv(LMParams p) {
+__global__ void __launch_bounds__(LM_THREADS, 1) k_lm_gemv(LMParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ int s_sh[MAX_M];
   __shared__ float s_inv[2][MAX_M];  // 2^-sh as two exact factors
-  __shared__ unsigned long long s_best[N_CONSUMERS][MAX_M];
+  __shared__ unsigned long long s_best[LM_CONSUMERS][MAX_M];
   __shared__ int s_last;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
@@ -114,7 +122,7 @@ __global__ void __launch_bounds__(EXPERT_THREADS, 1) k_lm_gemv(LMParams p) {
   const uint32_t xss = padded_stride(2u * H);
   const uint32_t ls = H;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);
-  uint64_t* empty = full + MAX_STAGES;
+  uint64_t* empty = full + LM_STAGES;
   uint8_t* xs = smem + 128;
   uint8_t* stages = smem + lm_fixed_bytes(H);
   const size_t sbytes = lm_stage_bytes(H);
@@ -127,19 +135,19 @@ __global__ void __launch_bounds__(EXPERT_THREADS, 1) k_lm_gemv(LMParams p) {
     fence_mbar_init();
   }
   __syncthreads();
-  const long long T = (V + 15) / 16;
+  const long long T = (V + 7) / 8;
   const long long start = T * blockIdx.x / gridDim.x;
   const long long end = T * (blockIdx.x + 1) / gridDim.x;
   const int nloc = (int)(end - start);
 
-  if (warp == N_CONSUMERS) {
+  if (warp == LM_CONSUMERS) {
     if (lane == 0) {
       const uint64_t pol = policy_evict_first();
       for (int i = 0; i < nloc; ++i) {
         const int s = i % S;
         if (i >= S && !mbar_wait(&empty[s], ((i / S) - 1) & 1, p.status)) break;
-        const long long v0 = (start + i) * 16;
-        const int nrows = (int)min(16LL, (long long)V - v0);
+        const long long v0 = (start + i) * 8;
+        const int nrows = (int)min(8LL, (long long)V - v0);
         uint8_t* st = stages + s * sbytes;
         mbar_arrive_expect_tx(&full[s], (uint32_t)nrows * H);
         bulk_g2s(st, p.w + (size_t)v0 * H, (uint32_t)nrows * H, &full[s], pol);
@@ -149,75 +157,55 @@ __global__ void __launch_bounds__(EXPERT_THREADS, 1) k_lm_gemv(LMParams p) {
     return;
   }
 
-  stage_x_f16(p.x, M, H, xs, xss, s_sh);
+  stage_x_f16<LM_CONSUMERS>(p.x, M, H, xs, xss, s_sh);
   if (tid < MAX_M) {
     const int k = -s_sh[tid], k1 = k / 2;
     s_inv[0][tid] = exp2i(k1);
     s_inv[1][tid] = exp2i(k - k1);
   }
-  named_barrier(1, 32 * N_CONSUMERS);
+  named_barrier(1, 32 * LM_CONSUMERS);
   unsigned long long bestA = 0ull, bestB = 0ull;  // tokens 2t and 2t+1
   const int ta = 2 * t, tb = 2 * t + 1;
-  for (int i = warp; i < nloc; i += N_CONSUMERS) {
+  const bool xact = g < M;
+  for (int i = warp; i < nloc; i += LM_CONSUMERS) {
     const int s = i % S;
     if (!mbar_wait(&full[s], (i / S) & 1, p.status)) return;
-    const long long v0 = (start + i) * 16;
-    const uint8_t* st = stages + s * sbytes;
-    float c[4] = {0.f, 0.f, 0.f, 0.f};
+    const long long v0 = (start + i) * 8;
+    const uint8_t* row = stages + s * sbytes + g * ls;
     float c4[4][4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) c4[u][0] = c4[u][1] = c4[u][2] = c4[u][3] = 0.0f;
-    const bool xact = g < M;
 #pragma unroll 2
     for (int j = 0; j < H / 64; ++j) {
-      const uint4 A0 = lds128(st + g * ls + 64 * j + 16 * t);
-      const uint4 A1 = lds128(st + (8 + g) * ls + 64 * j + 16 * t);
+      const uint4 A0 = lds128(row + 64 * j + 16 * t);
       const uint4 zero = make_uint4(0, 0, 0, 0);
       const uint4 X0 = xact ? lds128(xs + g * xss + 2 * (64 * j + 16 * t)) : zero;
       const uint4 X1 = xact ? lds128(xs + g * xss + 2 * (64 * j + 16 * t) + 16) : zero;
-      uint32_t P[8], Q[8];
+      uint32_t P[8];
       e4m3x4_to_f16x2(A0.x, P[0], P[1]);
       e4m3x4_to_f16x2(A0.y, P[2], P[3]);
       e4m3x4_to_f16x2(A0.z, P[4], P[5]);
       e4m3x4_to_f16x2(A0.w, P[6], P[7]);
-      e4m3x4_to_f16x2(A1.x, Q[0], Q[1]);
-      e4m3x4_to_f16x2(A1.y, Q[2], Q[3]);
-      e4m3x4_to_f16x2(A1.z, Q[4], Q[5]);
-      e4m3x4_to_f16x2(A1.w, Q[6], Q[7]);
       const uint32_t X[8] = {X0.x, X0.y, X0.z, X0.w, X1.x, X1.y, X1.z, X1.w};
 #pragma unroll
-      for (int s4 = 0; s4 < 4; ++s4)
-        mma_f16(c4[s4], P[2 * s4], Q[2 * s4], P[2 * s4 + 1], Q[2 * s4 + 1], X[2 * s4], X[2 * s4 + 1]);
+      for (int s4 = 0; s4 < 4; ++s4) mma_f16(c4[s4], P[2 * s4], 0u, P[2 * s4 + 1], 0u, X[2 * s4], X[2 * s4 + 1]);
     }
-#pragma unroll
-    for (int e = 0; e < 4; ++e) c[e] = (c4[0][e] + c4[1][e]) + (c4[2][e] + c4[3][e]);
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
-    const long long va = v0 + g, vb = v0 + g + 8;
+    const long long va = v0 + g;
     const float rsa = va < V ? __ldg(p.rs + va) : 0.0f;
-    const float rsb = vb < V ? __ldg(p.rs + vb) : 0.0f;
-    if (ta < M) {
-      const float ia = s_inv[0][ta], ib = s_inv[1][ta];
-      const float la = ((c[0] * ia) * ib) * rsa, lb = ((c[2] * ia) * ib) * rsb;
-      if (va < V) {
+    if (va < V) {
+      if (ta < M) {
+        const float c = (c4[0][0] + c4[1][0]) + (c4[2][0] + c4[3][0]);
+        const float la = ((c * s_inv[0][ta]) * s_inv[1][ta]) * rsa;
         if (p.logits) p.logits[(size_t)ta * V + va] = la;
         bestA = max(bestA, argmax_key(la, (int)va));
       }
-      if (vb < V) {
-        if (p.logits) p.logits[(size_t)ta * V + vb] = lb;
-        bestA = max(bestA, argmax_key(lb, (int)vb));
-      }
-    }
-    if (tb < M) {
-      const float ia = s_inv[0][tb], ib = s_inv[1][tb];
-      const float la = ((c[1] * ia) * ib) * rsa, lb = ((c[3] * ia) * ib) * rsb;
-      if (va < V) {
-        if (p.logits) p.logits[(size_t)tb * V + va] = la;
-        bestB = max(bestB, argmax_key(la, (int)va));
-      }
-      if (vb < V) {
-        if (p.logits) p.logits[(size_t)tb * V + vb] = lb;
-        bestB = max(bestB, argmax_key(lb, (int)vb));
+      if (tb < M) {
+        const float c = (c4[0][1] + c4[1][1]) + (c4[2][1] + c4[3][1]);
+        const float lb = ((c * s_inv[0][tb]) * s_inv[1][tb]) * rsa;
+        if (p.logits) p.logits[(size_t)tb * V + va] = lb;
+        bestB = max(bestB, argmax_key(lb, (int)va));
       }
     }
   }
@@ -231,16 +219,16 @@ __global__ void __launch_bounds__(EXPERT_THREADS, 1) k_lm_gemv(LMParams p) {
     s_best[warp][ta] = bestA;
     s_best[warp][tb] = bestB;
   }
-  named_barrier(1, 32 * N_CONSUMERS);
+  named_barrier(1, 32 * LM_CONSUMERS);
   if (warp == 0 && lane < M) {
     unsigned long long b = 0ull;
-    for (int w = 0; w < N_CONSUMERS; ++w) b = max(b, s_best[w][lane]);
+    for (int w = 0; w < LM_CONSUMERS; ++w) b = max(b, s_best[w][lane]);
     if (b) atomicMax(p.keys + lane, b);
   }
   __threadfence();
-  named_barrier(1, 32 * N_CONSUMERS);
+  named_barrier(1, 32 * LM_CONSUMERS);
   if (tid == 0) s_last = (atomicAdd(p.counter, 1u) == gridDim.x - 1);
-  named_barrier(1, 32 * N_CONSUMERS);
+  named_barrier(1, 32 * LM_CONSUMERS);
   if (s_last) {
     __threadfence();
     if (tid < M) {
@@ -249,7 +237,7 @@ __global__ void __launch_bounds__(EXPERT_THREADS, 1) k_lm_gemv(LMParams p) {
     }
     if (tid == 0) *p.counter = 0u;
     if (p.drafts) {
-      named_barrier(1, 32 * N_CONSUMERS);
+      named_barrier(1, 32 * LM_CONSUMERS);
       if (tid == 0) mtp_accept(p.argmax, p.drafts, M, p.accept);
     }
   }
