@@ -947,12 +947,12 @@ EncodeTiledFn encode_fn() {
 // index is the outermost dimension although its stride is the smallest, so kc chunks
 // arrive as kc consecutive swizzled tiles.
 bool make_map(CUtensorMap* m, CUtensorMapDataType t, const void* base, uint64_t inner, uint64_t rows,
-              uint64_t row_bytes, uint32_t box_inner, uint64_t chunk_bytes, int kc) {
+              uint64_t row_bytes, uint32_t box_inner, uint64_t chunk_bytes, int kc, uint32_t box_rows = 64) {
   EncodeTiledFn f = encode_fn();
   if (!f) return false;
   cuuint64_t dims[3] = {box_inner, rows, inner / box_inner};
   cuuint64_t strides[2] = {row_bytes, chunk_bytes};
-  cuuint32_t box[3] = {box_inner, 64, (cuuint32_t)kc};
+  cuuint32_t box[3] = {box_inner, box_rows, (cuuint32_t)kc};
   cuuint32_t es[3] = {1, 1, 1};
   return f(m, t, 3, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
@@ -1135,6 +1135,7 @@ moe_status_t pf_experts(const __nv_bfloat16* x, int M, int H, int I, int E, int 
                       (uint64_t)H / 2, (uint64_t)I * (H / 2), 128, 64, a.kc),
       MOE_ERR_INVALID_ARG);
   REQ(make_map(&a.tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.xq, H, G, H, 128, 128, a.kc), MOE_ERR_INVALID_ARG);
+  REQ(make_map(&a.tmB32, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.xq, H, G, H, 128, 128, a.kc, 32), MOE_ERR_INVALID_ARG);
   a.mode = PF_R13;
   a.K = H;
   a.m_tiles = I / 64;
@@ -1160,6 +1161,7 @@ moe_status_t pf_experts(const __nv_bfloat16* x, int M, int H, int I, int E, int 
                       (uint64_t)64 * (I / 2), 128, 64, b.kc),
       MOE_ERR_INVALID_ARG);
   REQ(make_map(&b.tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.aq, I, G, I, 128, 128, b.kc), MOE_ERR_INVALID_ARG);
+  REQ(make_map(&b.tmB32, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.aq, I, G, I, 128, 128, b.kc, 32), MOE_ERR_INVALID_ARG);
   b.mode = PF_R2;
   b.K = I;
   b.m_tiles = H / 128;

@@ -56,6 +56,7 @@ struct alignas(64) PrefillParams {
   // the swizzled tile one chunk of MMAs reads.
   CUtensorMap tmA;  // weights: dims {chunk, rows, 2 halves, K / chunk}, box {chunk, 64, 2, kc}
   CUtensorMap tmB;  // activations: dims {chunk, rows, K / chunk}, box {chunk, 64, kc}
+  CUtensorMap tmB32;  // routed modes: the same with 32-row boxes, for tiles of at most 32 tokens
   int mode;
   int K;
   int m_tiles;   // weight tiles per problem
@@ -409,9 +410,12 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
           // transaction bytes count the global (packed) side: 128 rows of 128 E2M1
           // codes are 8 KB although they fill 16 KB of shared memory; the token box
           // is always whole (rows past the tensor read as zeros and still count)
-          mbar_arrive_expect_tx(&full[s], (uint32_t)KC * ((mx ? 8192u : 16384u) + 8192u));
+          // a routed tile of at most 32 tokens takes the 32-row token box (half the bytes
+          // through the copy engine); its chunks then sit 4 KB apart instead of 8 KB
+          const bool half = mx && it.ncnt <= 32;
+          mbar_arrive_expect_tx(&full[s], (uint32_t)KC * ((mx ? 8192u : 16384u) + (half ? 4096u : 8192u)));
           tma_load_4d(st, &p.tmA, 0, it.ya0, 0, ch, &full[s]);
-          tma_load_3d(st + 16384 * KC, &p.tmB, 0, it.grow0, ch, &full[s]);
+          tma_load_3d(st + 16384 * KC, half ? &p.tmB32 : &p.tmB, 0, it.grow0, ch, &full[s]);
         }
       }
       // every copy issued lands before the CTA may finish
@@ -451,8 +455,9 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
           if (q < 128) PF_STAMP(4 * (int)q + 1);
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + (size_t)s * stage_bytes);
+          const uint32_t bstride = (mx && it.ncnt <= 32) ? 4096u : 8192u;  // token chunk stride (box rows x 128 B)
           for (int c = 0; c < KC; ++c) {
-            const uint64_t adesc = sw128_desc(sa + 16384u * c), bdesc = sw128_desc(sa + 16384u * KC + 8192u * c);
+            const uint64_t adesc = sw128_desc(sa + 16384u * c), bdesc = sw128_desc(sa + 16384u * KC + bstride * c);
             const uint32_t chc = (uint32_t)(ch + c);
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
