@@ -559,12 +559,6 @@ __device__ __forceinline__ void write_layer_input4(uint8_t* xb16, uint8_t* xf16,
   u.y = *reinterpret_cast<const uint32_t*>(&hb);
   *reinterpret_cast<uint2*>(xf16 + off16) = u;
 }
-// f16 offset of float4 column c of token tok: chunk-major for one token (the lanes-along-K
-// products), row-major (stride xss) for a window (the tensor-core tiles).
-template <bool ONE>
-__device__ __forceinline__ uint32_t xf16_off(int H, uint32_t xss, int tok, int c) {
-  return ONE ? chunk_major_off(4 * c, H / 32) : tok * xss + 8 * c;
-}
 __device__ __forceinline__ void accumulate4(float4 v, float& ss, float& am) {
   ss = fmaf(v.x, v.x, ss);
   ss = fmaf(v.y, v.y, ss);
@@ -573,17 +567,19 @@ __device__ __forceinline__ void accumulate4(float4 v, float& ss, float& am) {
   am = fmaxf(am, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
 }
 
-// [q0, q1): this block's slice of the residual's float4s (copied into hout).
-template <bool ONE>
-__device__ void stage_layer_input(const StepParams& p, int l, const float* hin, float* hout, uint8_t* xb16,
-                                  uint8_t* xf16, uint32_t xss, float* s_part, float* s_amx, float* s_r, int* s_sh,
-                                  int q0, int q1) {
+// The window's layer input (one token: stage1): x = bf16(RMSNorm(h)) (layer 0: the
+// given x) as bf16 rows at xb16 and as f16 rows scaled by 2^sh at xf16 (stride xss,
+// row-major for the tensor-core tiles); [q0, q1) is this block's slice of the
+// residual's float4s, copied into hout in the same pass.
+__device__ void stage_window_input(const StepParams& p, int l, const float* hin, float* hout, uint8_t* xb16,
+                                   uint8_t* xf16, uint32_t xss, float* s_part, float* s_amx, float* s_r, int* s_sh,
+                                   int q0, int q1) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int M = ONE ? 1 : p.M, H = p.H, nt = 32 * STEP_CONSUMERS;
+  const int M = p.M, H = p.H, nt = 32 * STEP_CONSUMERS;
   const int per = H / 4, Q = M * per;  // float4s per token / in total
 
   float4* hout4 = reinterpret_cast<float4*>(hout);
-  const bool inreg = ONE || Q <= STAGE_REG_F4 * nt;  // one token: H <= 4096 always fits
+  const bool inreg = Q <= STAGE_REG_F4 * nt;
   float4 v[STAGE_REG_F4];
   int tq[STAGE_REG_F4], cq[STAGE_REG_F4];  // token and float4 column of q = tid + nt*j
   if (inreg) {
@@ -688,7 +684,7 @@ __device__ void stage_layer_input(const StepParams& p, int l, const float* hin, 
 #pragma unroll
     for (int j = 0; j < STAGE_REG_F4; ++j)
       if (tq[j] < M)
-        write_layer_input4(xb16, xf16, tq[j] * xss + 8 * cq[j], xf16_off<ONE>(H, xss, tq[j], cq[j]), v[j], s_r[tq[j]],
+        write_layer_input4(xb16, xf16, tq[j] * xss + 8 * cq[j], tq[j] * xss + 8 * cq[j], v[j], s_r[tq[j]],
                            s_sh[tq[j]]);
   } else {
     for (int qb = tid; qb < Q; qb += STAGE_BATCH * nt) {
@@ -703,7 +699,7 @@ __device__ void stage_layer_input(const StepParams& p, int l, const float* hin, 
         const int q = qb + j * nt;
         if (q < Q) {
           const int tok = q / per, c = q - tok * per;
-          write_layer_input4(xb16, xf16, tok * xss + 8 * c, xf16_off<ONE>(H, xss, tok, c), w[j], s_r[tok], s_sh[tok]);
+          write_layer_input4(xb16, xf16, tok * xss + 8 * c, tok * xss + 8 * c, w[j], s_r[tok], s_sh[tok]);
         }
       }
     }
@@ -1312,7 +1308,7 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
     if constexpr (ONE)
       stage1(p, l, hin, hout, xb16, xf16, s_part, s_amx, s_sh, slice_q0, slice_q1);
     else
-      stage_layer_input<ONE>(p, l, hin, hout, xb16, xf16, xss, s_part, s_amx, s_r, s_sh, slice_q0, slice_q1);
+      stage_window_input(p, l, hin, hout, xb16, xf16, xss, s_part, s_amx, s_r, s_sh, slice_q0, slice_q1);
     if (tid == 0) mbar_arrive(hinit_bar);
     stamp(p, l, 2);
     if (tid == 0) blk_stamp(p, l, 1);
