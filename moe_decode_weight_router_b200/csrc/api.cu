@@ -980,6 +980,17 @@ bool make_map_halves(CUtensorMap* m, CUtensorMapDataType t, const void* base, ui
 }
 // K chunks per stage of a k_umma launch: two when they divide the chunk count.
 int pf_kc(int K, int kbox) { return ((K / kbox) % 2 == 0) ? 2 : 1; }
+// Routed launches: as many K chunks per stage (4, 3, 2, 1) as divide K / 128 and still
+// leave two stages beside the scale buffer -- each stage costs the SM's copy engine two
+// copies whatever their size, so fewer, larger stages move the weights faster.
+int pf_kc_routed(int K, int sf_ld, const DevInfo& d) {
+  const int nch = K / 128;
+  for (int kc = 4; kc > 1; --kc)
+    if (nch % kc == 0 &&
+        1024 + 2LL * PF_STAGE_BYTES * kc + (long long)pf_sf_buf_bytes(K, sf_ld) <= (long long)d.dyn_pf)
+      return kc;
+  return 1;
+}
 
 bool ok_pf(int M, int H, int I, int E, int k, int Is) {
   return M >= 128 && M % 128 == 0 && M <= 16384 && H >= 128 && H % 128 == 0 && H <= 4096 && I >= 128 &&
@@ -1054,7 +1065,7 @@ PfWs pf_ws(void* ws, int M, int H, int I, int E, int k, int Is, bool own_routing
 }
 
 moe_status_t launch_umma(PrefillParams& p, const DevInfo& d, cudaStream_t st) {
-  const size_t sf = (p.mode == PF_R13 || p.mode == PF_R2) ? 2 * (size_t)pf_sf_buf_bytes(p.K, p.sf_ld) : 0;
+  const size_t sf = (p.mode == PF_R13 || p.mode == PF_R2) ? (size_t)pf_sf_buf_bytes(p.K, p.sf_ld) : 0;
   const long long room = (long long)d.dyn_pf - 1024 - (long long)sf;
   const long long stage = (long long)PF_STAGE_BYTES * p.kc;
   const int stages = room > 0 ? (int)(room / stage) : 0;
@@ -1130,7 +1141,7 @@ moe_status_t pf_experts(const __nv_bfloat16* x, int M, int H, int I, int E, int 
   // a3: routed W13 + SwiGLU, activation re-quantised to MXFP8 (E2M1 x E4M3 block-scaled)
   PrefillParams a{};
   a.status = w.status;
-  a.kc = pf_kc(H, 128);
+  a.kc = pf_kc_routed(H, pf_sf_ld(H), d);
   REQ(make_map_halves(&a.tmA, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, w13_codes, H, (uint64_t)E * 2 * I,
                       (uint64_t)H / 2, (uint64_t)I * (H / 2), 128, 64, a.kc),
       MOE_ERR_INVALID_ARG);
@@ -1156,7 +1167,7 @@ moe_status_t pf_experts(const __nv_bfloat16* x, int M, int H, int I, int E, int 
   // a4: routed W2, weighted by the routing weight and added into y
   PrefillParams b{};
   b.status = w.status;
-  b.kc = pf_kc(I, 128);
+  b.kc = pf_kc_routed(I, pf_sf_ld(I), d);
   REQ(make_map_halves(&b.tmA, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, w2_codes, I, (uint64_t)E * H, (uint64_t)I / 2,
                       (uint64_t)64 * (I / 2), 128, 64, b.kc),
       MOE_ERR_INVALID_ARG);

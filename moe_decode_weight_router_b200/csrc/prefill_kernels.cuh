@@ -300,12 +300,13 @@ __device__ __forceinline__ uint8_t e4m3_of(float v) {
 // k_umma
 // ---------------------------------------------------------------------------
 // Shared memory: the 1024-aligned stage ring (kc chunks a stage: chunk c's weight tile
-// at +16384 c, its token tile at +16384 kc + 8192 c), then for the block-scaled modes two buffers of
-// the current tiles' E8M0 rows (weight rows at +0, K/32 bytes each; token rows after
-// them, sf_ld bytes each), filled by the producer with bulk copies.
+// at +16384 c, its token tile at +16384 kc + 8192 c), then for the block-scaled modes one
+// buffer of a tile's E8M0 rows (weight rows at +0, K/32 bytes each; token rows after
+// them, sf_ld bytes each), filled by the producer with bulk copies and emptied into
+// tensor memory by the epilogue warps.
 __host__ __device__ inline uint32_t pf_sf_buf_bytes(int K, int sf_ld) {
   const uint32_t a = (uint32_t)(128 * (K / 32) + 15) / 16 * 16;
-  return a + 128u * (uint32_t)sf_ld;
+  return a + (uint32_t)PF_BN * (uint32_t)sf_ld;  // weight rows, then at most PF_BN token rows
 }
 
 __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ PrefillParams p) {
@@ -382,10 +383,11 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
           // the token rows -- into shared buffer m & 1.  With two tensor-memory buffers the
           // next tile's rows are fetched here too, a tile ahead of its MMAs.
           auto fetch_scales = [&](int m, const PfItem& t) -> bool {
-            const int b = m & 1;
-            if (m >= 2 && !pf_wait(&sf_empty[b], (uint32_t)(((m >> 1) - 1) & 1), p.status, &s_abort, PFW_SF, p.mode))
+            // one shared buffer: tile m's rows wait until tile m-1's are in tensor memory
+            if (m >= 1 && !pf_wait(&sf_empty[0], (uint32_t)((m - 1) & 1), p.status, &s_abort, PFW_SF, p.mode))
               return false;
-            uint8_t* dst = sfbuf + (size_t)b * sfbuf_bytes;
+            uint8_t* dst = sfbuf;
+            const int b = 0;
             const uint32_t half = 64u * (uint32_t)kb, tok = (uint32_t)t.ncnt * (uint32_t)p.sf_ld;
             mbar_arrive_expect_tx(&sf_full[b], 2 * half + tok);
             const uint64_t pol = policy_evict_first();
@@ -421,9 +423,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
       // every copy issued lands before the CTA may finish
       for (long long j = (q > S ? q - S : 0); j < q; ++j)
         pf_wait(&full[j % S], (uint32_t)((j / S) & 1), p.status, &s_abort, PFW_DRAIN, p.mode);
-      if (mx)
-        for (int j = (n_item > 2 ? n_item - 2 : 0); j < n_item; ++j)
-          pf_wait(&sf_full[j & 1], (uint32_t)((j >> 1) & 1), p.status, &s_abort, PFW_DRAIN, p.mode);
+      if (mx && n_item > 0) pf_wait(&sf_full[0], (uint32_t)((n_item - 1) & 1), p.status, &s_abort, PFW_DRAIN, p.mode);
     }
   } else if (warp == 5) {
     // ---------------- MMA issuer ----------------
@@ -484,9 +484,9 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
     // E8M0 words of a tile from its scale buffer into tensor memory (lane r of every
     // quarter, column base + 4ch + c: operand row r + 32c, K blocks 4ch..4ch+3)
     auto put_scales = [&](int n_item, const PfItem& it) -> bool {
-      const int b = n_item & 1;
-      if (!pf_wait(&sf_full[b], (uint32_t)((n_item >> 1) & 1), p.status, &s_abort, PFW_SF, p.mode)) return false;
-      const uint8_t* sa = sfbuf + (size_t)b * sfbuf_bytes;
+      const int b = n_item & 1;  // tensor-memory scale buffer (with two of them)
+      if (!pf_wait(&sf_full[0], (uint32_t)(n_item & 1), p.status, &s_abort, PFW_SF, p.mode)) return false;
+      const uint8_t* sa = sfbuf;
       const uint8_t* sb = sa + sfa_bytes;
       for (int ch = 0; ch < nch; ++ch) {
         uint32_t wa[4], wb[4];
@@ -504,7 +504,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&sf_ready[sf2 ? b : 0]);
-        mbar_arrive(&sf_empty[b]);
+        mbar_arrive(&sf_empty[0]);
       }
       return true;
     };
