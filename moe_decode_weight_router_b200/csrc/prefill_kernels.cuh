@@ -210,7 +210,11 @@ __device__ __forceinline__ bool pf_routed(int mode) { return mode == PF_R13 || m
 __device__ __forceinline__ bool pf_13(int mode) { return mode == PF_SH13 || mode == PF_R13; }
 
 #ifdef PF_TIMELINE
-// Profiling builds only (compiled with -DPF_TIMELINE): block 0 of the routed W13 launch
+#ifndef PF_TIMELINE_MODE
+#define PF_TIMELINE_MODE PF_R13
+#endif
+// Profiling builds only (compiled with -DPF_TIMELINE; -DPF_TIMELINE_MODE picks the
+// launch, the routed W13 one by default): block 0 of that launch
 // stamps its SM clock (clock64, cycles; every role of block 0 runs on one SM) into pf_tl.  [4q + 0..2] for stage q < 128: producer issued
 // its copies, MMA issuer saw them land, MMA issuer committed the stage; [512 + 8n + 0..5]
 // for item n < 32: MMA issuer saw the item's scales placed, saw its accumulator free,
@@ -222,7 +226,7 @@ __device__ __forceinline__ bool pf_13(int mode) { return mode == PF_SH13 || mode
 __device__ unsigned long long pf_tl[1024];
 #define PF_STAMP(idx)                                                                         \
   do {                                                                                         \
-    if (blockIdx.x == 0 && p.mode == PF_R13 && (idx) < 1024) pf_tl[(idx)] = (unsigned long long)clock64(); \
+    if (blockIdx.x == 0 && p.mode == PF_TIMELINE_MODE && (idx) < 1024) pf_tl[(idx)] = (unsigned long long)clock64(); \
   } while (0)
 #else
 #define PF_STAMP(idx) \
