@@ -1065,9 +1065,15 @@ PfWs pf_ws(void* ws, int M, int H, int I, int E, int k, int Is, bool own_routing
 }
 
 moe_status_t launch_umma(PrefillParams& p, const DevInfo& d, cudaStream_t st) {
-  const size_t sf = (p.mode == PF_R13 || p.mode == PF_R2) ? (size_t)pf_sf_buf_bytes(p.K, p.sf_ld) : 0;
-  const long long room = (long long)d.dyn_pf - 1024 - (long long)sf;
+  const bool mx = p.mode == PF_R13 || p.mode == PF_R2;
   const long long stage = (long long)PF_STAGE_BYTES * p.kc;
+  const long long sf1 = mx ? (long long)pf_sf_buf_bytes(p.K, p.sf_ld) : 0;
+  // a second scale buffer when it costs no stage
+  const long long room1 = (long long)d.dyn_pf - 1024 - sf1;
+  const long long cap = PF_MAX_STAGES;
+  p.sf_bufs = (mx && room1 > 0 && std::min((room1 - sf1) / stage, cap) >= std::min(room1 / stage, cap)) ? 2 : 1;
+  const size_t sf = (size_t)(p.sf_bufs * sf1);
+  const long long room = (long long)d.dyn_pf - 1024 - (long long)sf;
   const int stages = room > 0 ? (int)(room / stage) : 0;
   p.stages = stages > PF_MAX_STAGES ? PF_MAX_STAGES : stages;
   if (p.stages < 2) return MOE_ERR_UNSUPPORTED_SHAPE;

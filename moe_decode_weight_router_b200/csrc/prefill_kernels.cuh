@@ -78,6 +78,7 @@ struct alignas(64) PrefillParams {
   uint8_t* out_qs;          // routed activation E8M0 [G][out_qs_ld]
   int out_qs_ld;
   int stages;
+  int sf_bufs;  // block-scaled modes: shared-memory scale buffers (2, or 1 when two do not fit)
   int kc;  // K chunks per pipeline stage (one copy per operand per stage)
   int* status;
 };
@@ -222,7 +223,9 @@ __device__ __forceinline__ bool pf_13(int mode) { return mode == PF_SH13 || mode
 // producer issued the item's scale copies, epilogue loaded its first 16 columns, finished
 // its first 16 columns; [768 + 8n + 0..6] for item n < 32, first 16 columns: warp 0
 // past the exchange barrier, SwiGLU done, quantised and stored, past the closing
-// barrier; warp 2 wrote its exchange values, finished its load, started its load.
+// barrier; warp 2 wrote its exchange values, finished its load, started its load.  In
+// the routed W2 launch [768 + 8n + 0..2] are instead: scale placement of item n began,
+// ended (warp 0), warp 3 finished item n.
 __device__ unsigned long long pf_tl[1024];
 #define PF_STAMP(idx)                                                                         \
   do {                                                                                         \
@@ -305,9 +308,10 @@ __device__ __forceinline__ uint8_t e4m3_of(float v) {
 // ---------------------------------------------------------------------------
 // Shared memory: the 1024-aligned stage ring (kc chunks a stage: chunk c's weight tile
 // at +16384 c, its token tile at +16384 kc + 8192 c), then for the block-scaled modes one
-// buffer of a tile's E8M0 rows (weight rows at +0, K/32 bytes each; token rows after
-// them, sf_ld bytes each), filled by the producer with bulk copies and emptied into
-// tensor memory by the epilogue warps.
+// or two buffers of a tile's E8M0 rows (weight rows at +0, K/32 bytes each; token rows
+// after them, sf_ld bytes each), filled by the producer with bulk copies and emptied
+// into tensor memory by the epilogue warps.  With two, the producer fetches a tile's
+// rows while the previous tile's still wait to be placed.
 __host__ __device__ inline uint32_t pf_sf_buf_bytes(int K, int sf_ld) {
   const uint32_t a = (uint32_t)(128 * (K / 32) + 15) / 16 * 16;
   return a + (uint32_t)PF_BN * (uint32_t)sf_ld;  // weight rows, then at most PF_BN token rows
@@ -342,6 +346,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
   const uint32_t sfa_bytes = (uint32_t)(128 * kb + 15) / 16 * 16;
   uint8_t* sfbuf = smem + (size_t)S * stage_bytes;
   const uint32_t sfbuf_bytes = pf_sf_buf_bytes(p.K, p.sf_ld);
+  const int NB = p.sf_bufs > 1 ? 2 : 1;  // shared-memory scale buffers
   // Scale columns in tensor memory: two buffers when they fit beside the accumulators
   // (K <= 3072), so a tile's scales are placed while the previous tile's MMAs run;
   // otherwise one, placed once the previous tile's MMAs are done.
@@ -384,14 +389,14 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
         const PfItem it = pf_item(p, idx, s_ntp, s_goff);
         if (mx) {
           // scale rows of a tile -- weight rows (two 64-row runs or one 128-row run) and
-          // the token rows -- into shared buffer m & 1.  With two tensor-memory buffers the
+          // the token rows -- into shared buffer m % NB.  With two tensor-memory buffers the
           // next tile's rows are fetched here too, a tile ahead of its MMAs.
           auto fetch_scales = [&](int m, const PfItem& t) -> bool {
-            // one shared buffer: tile m's rows wait until tile m-1's are in tensor memory
-            if (m >= 1 && !pf_wait(&sf_empty[0], (uint32_t)((m - 1) & 1), p.status, &s_abort, PFW_SF, p.mode))
+            // buffer m % NB: tile m's rows wait until tile m - NB's are in tensor memory
+            const int b = m % NB;
+            if (m >= NB && !pf_wait(&sf_empty[b], (uint32_t)((m / NB - 1) & 1), p.status, &s_abort, PFW_SF, p.mode))
               return false;
-            uint8_t* dst = sfbuf;
-            const int b = 0;
+            uint8_t* dst = sfbuf + (size_t)b * sfbuf_bytes;
             const uint32_t half = 64u * (uint32_t)kb, tok = (uint32_t)t.ncnt * (uint32_t)p.sf_ld;
             mbar_arrive_expect_tx(&sf_full[b], 2 * half + tok);
             const uint64_t pol = policy_evict_first();
@@ -427,7 +432,9 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
       // every copy issued lands before the CTA may finish
       for (long long j = (q > S ? q - S : 0); j < q; ++j)
         pf_wait(&full[j % S], (uint32_t)((j / S) & 1), p.status, &s_abort, PFW_DRAIN, p.mode);
-      if (mx && n_item > 0) pf_wait(&sf_full[0], (uint32_t)((n_item - 1) & 1), p.status, &s_abort, PFW_DRAIN, p.mode);
+      if (mx)
+        for (int j = (n_item > NB ? n_item - NB : 0); j < n_item; ++j)
+          pf_wait(&sf_full[j % NB], (uint32_t)((j / NB) & 1), p.status, &s_abort, PFW_DRAIN, p.mode);
     }
   } else if (warp == 5) {
     // ---------------- MMA issuer ----------------
@@ -488,9 +495,11 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
     // E8M0 words of a tile from its scale buffer into tensor memory (lane r of every
     // quarter, column base + 4ch + c: operand row r + 32c, K blocks 4ch..4ch+3)
     auto put_scales = [&](int n_item, const PfItem& it) -> bool {
-      const int b = n_item & 1;  // tensor-memory scale buffer (with two of them)
-      if (!pf_wait(&sf_full[0], (uint32_t)(n_item & 1), p.status, &s_abort, PFW_SF, p.mode)) return false;
-      const uint8_t* sa = sfbuf;
+      if (p.mode == PF_R2 && tid == 0 && n_item < 32) PF_STAMP(768 + 8 * n_item + 0);
+      const int b = n_item & 1;      // tensor-memory scale buffer (with two of them)
+      const int sb_i = n_item % NB;  // shared-memory scale buffer
+      if (!pf_wait(&sf_full[sb_i], (uint32_t)((n_item / NB) & 1), p.status, &s_abort, PFW_SF, p.mode)) return false;
+      const uint8_t* sa = sfbuf + (size_t)sb_i * sfbuf_bytes;
       const uint8_t* sb = sa + sfa_bytes;
       for (int ch = 0; ch < nch; ++ch) {
         uint32_t wa[4], wb[4];
@@ -508,8 +517,9 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&sf_ready[sf2 ? b : 0]);
-        mbar_arrive(&sf_empty[0]);
+        mbar_arrive(&sf_empty[sb_i]);
       }
+      if (p.mode == PF_R2 && tid == 0 && n_item < 32) PF_STAMP(768 + 8 * n_item + 1);
       return true;
     };
     bool live = true;
@@ -519,6 +529,20 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
     for (int idx = blockIdx.x; idx < total; idx += G, ++n_item) {
       const PfItem it = pf_item(p, idx, s_ntp, s_goff);
       const int ab = n_item & 1;
+      // routed W2: the tile's tokens and routing weights (lane j holds grouped rows j and
+      // j + 32), fetched before the accumulator wait so their latency stays off the epilogue
+      int tk_lo = 0, tk_hi = 0;
+      float tw_lo = 0.0f, tw_hi = 0.0f;
+      if (p.mode == PF_R2) {
+        if (r < it.ncnt) {
+          tk_lo = __ldg(p.g_tok + it.grow0 + r);
+          tw_lo = __ldg(p.g_w + it.grow0 + r);
+        }
+        if (r + 32 < it.ncnt) {
+          tk_hi = __ldg(p.g_tok + it.grow0 + r + 32);
+          tw_hi = __ldg(p.g_w + it.grow0 + r + 32);
+        }
+      }
       if (live) pf_wait(&acc_full[ab], (uint32_t)((n_item >> 1) & 1), p.status, &s_abort, PFW_ACC_FULL, p.mode);
       if (tid == 0 && n_item < 32) PF_STAMP(512 + 8 * n_item + 2);
       named_barrier(2, 128);  // the four epilogue warps take the same decision below
@@ -545,8 +569,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
 #pragma unroll
           for (int j = 0; j < 16; ++j)
             if (j < jn) {
-              const int g = it.grow0 + j0 + j;
-              atomicAdd(p.out_f32 + (size_t)__ldg(p.g_tok + g) * p.out_ld + row, __ldg(p.g_w + g) * v[j]);
+              const int src = (j0 & 31) + j;
+              const int tok = __shfl_sync(0xffffffffu, j0 < 32 ? tk_lo : tk_hi, src);
+              const float wt = __shfl_sync(0xffffffffu, j0 < 32 ? tw_lo : tw_hi, src);
+              atomicAdd(p.out_f32 + (size_t)tok * p.out_ld + row, wt * v[j]);
             }
         } else {
           // 13 modes: warps 0,1 hold gate rows, warps 2,3 the matching up rows.  Each
@@ -591,6 +617,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
         if (tid == 0 && n_item < 32 && j0 == 0) PF_STAMP(512 + 8 * n_item + 7);
       }
       if (tid == 0 && n_item < 32) PF_STAMP(512 + 8 * n_item + 4);
+      if (p.mode == PF_R2 && tid == 96 && n_item < 32) PF_STAMP(768 + 8 * n_item + 2);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[ab]);
