@@ -81,7 +81,11 @@ moe_status_t dev_info(DevInfo* out) {
     MOE_CUDA(allow_dyn_smem(k_lm_gemv_bf16, lim, &d.dyn_lmb));
     MOE_CUDA(allow_dyn_smem(k_step<false>, lim, &d.dyn_step));
     MOE_CUDA(allow_dyn_smem(k_step<true>, lim, &d.dyn_step));
-    MOE_CUDA(allow_dyn_smem(k_umma, lim, &d.dyn_pf));
+    MOE_CUDA(allow_dyn_smem(k_umma<PF_ROUTER>, lim, &d.dyn_pf));
+    MOE_CUDA(allow_dyn_smem(k_umma<PF_SH13>, lim, &d.dyn_pf));
+    MOE_CUDA(allow_dyn_smem(k_umma<PF_SH2>, lim, &d.dyn_pf));
+    MOE_CUDA(allow_dyn_smem(k_umma<PF_R13>, lim, &d.dyn_pf));
+    MOE_CUDA(allow_dyn_smem(k_umma<PF_R2>, lim, &d.dyn_pf));
     MOE_CUDA(cudaDeviceGetAttribute(&d.coop, cudaDevAttrCooperativeLaunch, dev));
     cache[dev] = d;
     ready[dev] = true;
@@ -1078,7 +1082,14 @@ moe_status_t launch_umma(PrefillParams& p, const DevInfo& d, cudaStream_t st) {
   p.stages = stages > PF_MAX_STAGES ? PF_MAX_STAGES : stages;
   if (p.stages < 2) return MOE_ERR_UNSUPPORTED_SHAPE;
   const size_t smem = 1024 + (size_t)p.stages * stage + sf;
-  k_umma<<<d.sms, PF_THREADS, smem, st>>>(p);
+  switch (p.mode) {
+    case PF_ROUTER: k_umma<PF_ROUTER><<<d.sms, PF_THREADS, smem, st>>>(p); break;
+    case PF_SH13: k_umma<PF_SH13><<<d.sms, PF_THREADS, smem, st>>>(p); break;
+    case PF_SH2: k_umma<PF_SH2><<<d.sms, PF_THREADS, smem, st>>>(p); break;
+    case PF_R13: k_umma<PF_R13><<<d.sms, PF_THREADS, smem, st>>>(p); break;
+    case PF_R2: k_umma<PF_R2><<<d.sms, PF_THREADS, smem, st>>>(p); break;
+    default: return MOE_ERR_INVALID_ARG;
+  }
   MOE_CUDA(cudaGetLastError());
   return MOE_OK;
 }

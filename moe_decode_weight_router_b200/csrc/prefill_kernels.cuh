@@ -207,8 +207,8 @@ struct PfItem {
   int ya0, ya1;  // weight rows of the two 64-row halves
 };
 
-__device__ __forceinline__ bool pf_routed(int mode) { return mode == PF_R13 || mode == PF_R2; }
-__device__ __forceinline__ bool pf_13(int mode) { return mode == PF_SH13 || mode == PF_R13; }
+__host__ __device__ constexpr bool pf_routed(int mode) { return mode == PF_R13 || mode == PF_R2; }
+__host__ __device__ constexpr bool pf_13(int mode) { return mode == PF_SH13 || mode == PF_R13; }
 
 #ifdef PF_TIMELINE
 #ifndef PF_TIMELINE_MODE
@@ -229,7 +229,7 @@ __device__ __forceinline__ bool pf_13(int mode) { return mode == PF_SH13 || mode
 __device__ unsigned long long pf_tl[1024];
 #define PF_STAMP(idx)                                                                         \
   do {                                                                                         \
-    if (blockIdx.x == 0 && p.mode == PF_TIMELINE_MODE && (idx) < 1024) pf_tl[(idx)] = (unsigned long long)clock64(); \
+    if (blockIdx.x == 0 && MODE == PF_TIMELINE_MODE && (idx) < 1024) pf_tl[(idx)] = (unsigned long long)clock64(); \
   } while (0)
 #else
 #define PF_STAMP(idx) \
@@ -241,16 +241,16 @@ constexpr int PF_MAX_E = 512;
 // Routed modes: tile prefix and grouped offsets are copied to shared memory once per
 // CTA (every role decodes every tile; a search over global memory would put a chain
 // of dependent loads in front of each tile).
-__device__ inline int pf_total_items(const PrefillParams& p, const int* s_ntp) {
-  if (pf_routed(p.mode)) return p.m_tiles * s_ntp[p.E];
+__device__ inline int pf_total_items(const PrefillParams& p, int mode, const int* s_ntp) {
+  if (pf_routed(mode)) return p.m_tiles * s_ntp[p.E];
   return p.m_tiles * ((p.M + PF_BN - 1) / PF_BN);
 }
-__device__ inline PfItem pf_item(const PrefillParams& p, int idx, const int* s_ntp, const int* s_goff) {
+__device__ inline PfItem pf_item(const PrefillParams& p, int mode, int idx, const int* s_ntp, const int* s_goff) {
   PfItem it;
   it.mt = idx % p.m_tiles;
   const int j = idx / p.m_tiles;
   int rows0;
-  if (pf_routed(p.mode)) {
+  if (pf_routed(mode)) {
     int lo = 0, hi = p.E;  // largest e with ntile_prefix[e] <= j
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
@@ -272,7 +272,7 @@ __device__ inline PfItem pf_item(const PrefillParams& p, int idx, const int* s_n
     it.grow0 = it.n0;
     rows0 = 0;
   }
-  if (pf_13(p.mode)) {
+  if (pf_13(mode)) {
     it.ya0 = rows0 + 64 * it.mt;              // gate rows
     it.ya1 = rows0 + p.up_off + 64 * it.mt;   // up rows
   } else {
@@ -317,6 +317,9 @@ __host__ __device__ inline uint32_t pf_sf_buf_bytes(int K, int sf_ld) {
   return a + (uint32_t)PF_BN * (uint32_t)sf_ld;  // weight rows, then at most PF_BN token rows
 }
 
+// One instantiation per mode (MODE equals MODE): each launch carries only its own
+// epilogue, so the code every role runs stays small enough for the instruction caches.
+template <int MODE>
 __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ PrefillParams p) {
   extern __shared__ __align__(1024) uint8_t pf_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(pf_smem_raw) + 1023) & ~uintptr_t(1023));
@@ -329,7 +332,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int S = p.stages;
-  const bool mx = pf_routed(p.mode);
+  constexpr bool mx = pf_routed(MODE);
   const int kbox = mx ? 128 : 64;  // K elements per chunk (128 bytes per row)
   const int nch = p.K / kbox;
   const int KC = p.kc;             // chunks per stage (divides nch)
@@ -340,7 +343,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
       s_goff[e] = __ldg(p.goff + e);
     }
   __syncthreads();
-  const int total = pf_total_items(p, s_ntp);
+  const int total = pf_total_items(p, MODE, s_ntp);
   const int G = gridDim.x;
   const int kb = p.K / 32;  // E8M0 bytes per weight row
   const uint32_t sfa_bytes = (uint32_t)(128 * kb + 15) / 16 * 16;
@@ -386,7 +389,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
       int n_item = 0;
       bool ok = true;
       for (int idx = blockIdx.x; idx < total && ok; idx += G, ++n_item) {
-        const PfItem it = pf_item(p, idx, s_ntp, s_goff);
+        const PfItem it = pf_item(p, MODE, idx, s_ntp, s_goff);
         if (mx) {
           // scale rows of a tile -- weight rows (two 64-row runs or one 128-row run) and
           // the token rows -- into shared buffer m % NB.  With two tensor-memory buffers the
@@ -394,7 +397,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
           auto fetch_scales = [&](int m, const PfItem& t) -> bool {
             // buffer m % NB: tile m's rows wait until tile m - NB's are in tensor memory
             const int b = m % NB;
-            if (m >= NB && !pf_wait(&sf_empty[b], (uint32_t)((m / NB - 1) & 1), p.status, &s_abort, PFW_SF, p.mode))
+            if (m >= NB && !pf_wait(&sf_empty[b], (uint32_t)((m / NB - 1) & 1), p.status, &s_abort, PFW_SF, MODE))
               return false;
             uint8_t* dst = sfbuf + (size_t)b * sfbuf_bytes;
             const uint32_t half = 64u * (uint32_t)kb, tok = (uint32_t)t.ncnt * (uint32_t)p.sf_ld;
@@ -406,13 +409,13 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
             return true;
           };
           if (!sf2 || n_item == 0) ok = fetch_scales(n_item, it);
-          if (ok && sf2 && idx + G < total) ok = fetch_scales(n_item + 1, pf_item(p, idx + G, s_ntp, s_goff));
+          if (ok && sf2 && idx + G < total) ok = fetch_scales(n_item + 1, pf_item(p, MODE, idx + G, s_ntp, s_goff));
           if (!ok) break;
           if (n_item < 32) PF_STAMP(512 + 8 * n_item + 5);
         }
         for (int ch = 0; ch < nch; ch += KC, ++q) {
           const int s = (int)(q % S);
-          if (q >= S && !pf_wait(&empty[s], (uint32_t)(((q / S) - 1) & 1), p.status, &s_abort, PFW_EMPTY, p.mode)) {
+          if (q >= S && !pf_wait(&empty[s], (uint32_t)(((q / S) - 1) & 1), p.status, &s_abort, PFW_EMPTY, MODE)) {
             ok = false;
             break;
           }
@@ -431,10 +434,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
       }
       // every copy issued lands before the CTA may finish
       for (long long j = (q > S ? q - S : 0); j < q; ++j)
-        pf_wait(&full[j % S], (uint32_t)((j / S) & 1), p.status, &s_abort, PFW_DRAIN, p.mode);
+        pf_wait(&full[j % S], (uint32_t)((j / S) & 1), p.status, &s_abort, PFW_DRAIN, MODE);
       if (mx)
         for (int j = (n_item > NB ? n_item - NB : 0); j < n_item; ++j)
-          pf_wait(&sf_full[j % NB], (uint32_t)((j / NB) & 1), p.status, &s_abort, PFW_DRAIN, p.mode);
+          pf_wait(&sf_full[j % NB], (uint32_t)((j / NB) & 1), p.status, &s_abort, PFW_DRAIN, MODE);
     }
   } else if (warp == 5) {
     // ---------------- MMA issuer ----------------
@@ -443,15 +446,15 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
       int n_item = 0;
       bool ok = true;
       for (int idx = blockIdx.x; idx < total && ok; idx += G, ++n_item) {
-        const PfItem it = pf_item(p, idx, s_ntp, s_goff);
+        const PfItem it = pf_item(p, MODE, idx, s_ntp, s_goff);
         const int N = (it.ncnt + 15) & ~15;
         const int ab = n_item & 1;
         if (n_item >= 2 && !pf_wait(&acc_empty[ab], (uint32_t)(((n_item >> 1) - 1) & 1), p.status, &s_abort,
-                                    PFW_ACC_EMPTY, p.mode))
+                                    PFW_ACC_EMPTY, MODE))
           break;
         if (n_item < 32) PF_STAMP(512 + 8 * n_item + 1);
         if (mx && !pf_wait(&sf_ready[sf2 ? ab : 0], (uint32_t)((sf2 ? n_item >> 1 : n_item) & 1), p.status,
-                           &s_abort, PFW_SF, p.mode))
+                           &s_abort, PFW_SF, MODE))
           break;
         if (n_item < 32) PF_STAMP(512 + 8 * n_item + 0);
         tc_fence_after();
@@ -459,7 +462,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
         const uint32_t tsfa = tbase + sfa_col(n_item), tsfb = tbase + sfb_col(n_item);
         for (int ch = 0; ch < nch; ch += KC, ++q) {
           const int s = (int)(q % S);
-          if (!pf_wait(&full[s], (uint32_t)((q / S) & 1), p.status, &s_abort, PFW_FULL, p.mode)) {
+          if (!pf_wait(&full[s], (uint32_t)((q / S) & 1), p.status, &s_abort, PFW_FULL, MODE)) {
             ok = false;
             break;
           }
@@ -495,10 +498,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
     // E8M0 words of a tile from its scale buffer into tensor memory (lane r of every
     // quarter, column base + 4ch + c: operand row r + 32c, K blocks 4ch..4ch+3)
     auto put_scales = [&](int n_item, const PfItem& it) -> bool {
-      if (p.mode == PF_R2 && tid == 0 && n_item < 32) PF_STAMP(768 + 8 * n_item + 0);
+      if (MODE == PF_R2 && tid == 0 && n_item < 32) PF_STAMP(768 + 8 * n_item + 0);
       const int b = n_item & 1;      // tensor-memory scale buffer (with two of them)
       const int sb_i = n_item % NB;  // shared-memory scale buffer
-      if (!pf_wait(&sf_full[sb_i], (uint32_t)((n_item / NB) & 1), p.status, &s_abort, PFW_SF, p.mode)) return false;
+      if (!pf_wait(&sf_full[sb_i], (uint32_t)((n_item / NB) & 1), p.status, &s_abort, PFW_SF, MODE)) return false;
       const uint8_t* sa = sfbuf + (size_t)sb_i * sfbuf_bytes;
       const uint8_t* sb = sa + sfa_bytes;
       for (int ch = 0; ch < nch; ++ch) {
@@ -519,21 +522,21 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
         mbar_arrive(&sf_ready[sf2 ? b : 0]);
         mbar_arrive(&sf_empty[sb_i]);
       }
-      if (p.mode == PF_R2 && tid == 0 && n_item < 32) PF_STAMP(768 + 8 * n_item + 1);
+      if (MODE == PF_R2 && tid == 0 && n_item < 32) PF_STAMP(768 + 8 * n_item + 1);
       return true;
     };
     bool live = true;
-    if (mx && blockIdx.x < total) live = put_scales(0, pf_item(p, blockIdx.x, s_ntp, s_goff));
-    if (mx && sf2 && live && blockIdx.x + G < total) live = put_scales(1, pf_item(p, blockIdx.x + G, s_ntp, s_goff));
+    if (mx && blockIdx.x < total) live = put_scales(0, pf_item(p, MODE, blockIdx.x, s_ntp, s_goff));
+    if (mx && sf2 && live && blockIdx.x + G < total) live = put_scales(1, pf_item(p, MODE, blockIdx.x + G, s_ntp, s_goff));
     int n_item = 0;
     for (int idx = blockIdx.x; idx < total; idx += G, ++n_item) {
-      const PfItem it = pf_item(p, idx, s_ntp, s_goff);
+      const PfItem it = pf_item(p, MODE, idx, s_ntp, s_goff);
       const int ab = n_item & 1;
       // routed W2: the tile's tokens and routing weights (lane j holds grouped rows j and
       // j + 32), fetched before the accumulator wait so their latency stays off the epilogue
       int tk_lo = 0, tk_hi = 0;
       float tw_lo = 0.0f, tw_hi = 0.0f;
-      if (p.mode == PF_R2) {
+      if (MODE == PF_R2) {
         if (r < it.ncnt) {
           tk_lo = __ldg(p.g_tok + it.grow0 + r);
           tw_lo = __ldg(p.g_w + it.grow0 + r);
@@ -543,13 +546,13 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
           tw_hi = __ldg(p.g_w + it.grow0 + r + 32);
         }
       }
-      if (live) pf_wait(&acc_full[ab], (uint32_t)((n_item >> 1) & 1), p.status, &s_abort, PFW_ACC_FULL, p.mode);
+      if (live) pf_wait(&acc_full[ab], (uint32_t)((n_item >> 1) & 1), p.status, &s_abort, PFW_ACC_FULL, MODE);
       if (tid == 0 && n_item < 32) PF_STAMP(512 + 8 * n_item + 2);
       named_barrier(2, 128);  // the four epilogue warps take the same decision below
       if (s_abort) break;
       tc_fence_after();
       // one scale buffer: the MMAs of this tile are complete, its columns may take the next tile's
-      if (mx && !sf2 && idx + G < total) live = put_scales(n_item + 1, pf_item(p, idx + G, s_ntp, s_goff));
+      if (mx && !sf2 && idx + G < total) live = put_scales(n_item + 1, pf_item(p, MODE, idx + G, s_ntp, s_goff));
       if (tid == 0 && n_item < 32) PF_STAMP(512 + 8 * n_item + 3);
       const uint32_t acc_lane = lane_base + 64u * ab;
       for (int j0 = 0; j0 < it.ncnt; j0 += 16) {
@@ -559,12 +562,12 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
         if (tid == 0 && n_item < 32 && j0 == 0) PF_STAMP(512 + 8 * n_item + 6);
         if (tid == 64 && n_item < 32 && j0 == 0) PF_STAMP(768 + 8 * n_item + 5);
         const int jn = min(16, it.ncnt - j0);
-        if (p.mode == PF_ROUTER || p.mode == PF_SH2) {
+        if (MODE == PF_ROUTER || MODE == PF_SH2) {
           const int row = 128 * it.mt + 32 * warp + r;
 #pragma unroll
           for (int j = 0; j < 16; ++j)
             if (j < jn) p.out_f32[(size_t)(it.n0 + j0 + j) * p.out_ld + row] = v[j];
-        } else if (p.mode == PF_R2) {
+        } else if (MODE == PF_R2) {
           const int row = 128 * it.mt + 32 * warp + r;
 #pragma unroll
           for (int j = 0; j < 16; ++j)
@@ -592,7 +595,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
           for (int j = 0; j < 8; ++j)
             a[j] = gate ? pf_silu(v[j]) * xch[pr][r][8 + j] : pf_silu(xch[pr][r][j]) * v[8 + j];
           if (tid == 0 && n_item < 32 && j0 == 0) PF_STAMP(768 + 8 * n_item + 1);
-          if (p.mode == PF_SH13) {
+          if (MODE == PF_SH13) {
 #pragma unroll
             for (int j = 0; j < 8; ++j)
               if (jb + j < jn) p.out_bf16[(size_t)(it.n0 + j0 + jb + j) * p.out_ld + i] = __float2bfloat16_rn(a[j]);
@@ -617,14 +620,14 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
         if (tid == 0 && n_item < 32 && j0 == 0) PF_STAMP(512 + 8 * n_item + 7);
       }
       if (tid == 0 && n_item < 32) PF_STAMP(512 + 8 * n_item + 4);
-      if (p.mode == PF_R2 && tid == 96 && n_item < 32) PF_STAMP(768 + 8 * n_item + 2);
+      if (MODE == PF_R2 && tid == 96 && n_item < 32) PF_STAMP(768 + 8 * n_item + 2);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[ab]);
       // two scale buffers: this tile's MMAs are done, so its buffer takes the tile after
       // next while the next tile's MMAs run
       if (mx && sf2 && live && idx + 2 * G < total)
-        live = put_scales(n_item + 2, pf_item(p, idx + 2 * G, s_ntp, s_goff));
+        live = put_scales(n_item + 2, pf_item(p, MODE, idx + 2 * G, s_ntp, s_goff));
     }
   }
   tc_fence_before();
