@@ -1114,7 +1114,7 @@ moe_status_t pf_experts(const __nv_bfloat16* x, int M, int H, int I, int E, int 
   MOE_CUDA(cudaGetLastError());
   k_pf_scatter<<<(G + 255) / 256, 256, 0, st>>>(ids, wts, M, top_k, E, w.goff, w.fill, w.g_tok, w.g_w, w.pos);
   MOE_CUDA(cudaGetLastError());
-  k_pf_quant_x<<<(int)(((long long)M * (H / 32) + 7) / 8), 256, 0, st>>>(x, M, H, top_k, w.pos, w.xq, w.xs,
+  k_pf_quant_x<<<(int)(((long long)M * (H / 32) + 255) / 256), 256, 0, st>>>(x, M, H, top_k, w.pos, w.xq, w.xs,
                                                                           pf_sf_ld(H));
   MOE_CUDA(cudaGetLastError());
 

@@ -282,6 +282,11 @@ __device__ inline PfItem pf_item(const PrefillParams& p, int mode, int idx, cons
   return it;
 }
 
+// *p[0..3] += {a, b, c, d} in one reduction (p 16-byte aligned)
+__device__ __forceinline__ void red_add_f32x4(float* p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
+}
+
 // silu(g) = g / (1 + e^-g): the fast division (2 ulp; g / inf = -0 for g < -88) keeps the
 // epilogue short -- the IEEE division's special-case branches serialised it.
 __device__ __forceinline__ float pf_silu(float g) { return __fdividef(g, 1.0f + expf(-g)); }
@@ -327,7 +332,9 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
   __shared__ uint64_t acc_full[2], acc_empty[2], sf_full[2], sf_empty[2], sf_ready[2];
   __shared__ uint32_t tmem_base_s;
   __shared__ volatile int s_abort;
-  __shared__ float xch[2][32][17];  // up-half values handed from warps 2,3 to warps 0,1
+  // 13 modes: up-half values handed from warps 2,3 to warps 0,1; routed W2: each warp's
+  // 8 tokens x 32 rows, read back as four consecutive rows of one token
+  __shared__ __align__(16) float xch[2][32][17];
   __shared__ int s_ntp[PF_MAX_E + 1], s_goff[PF_MAX_E + 1];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -568,15 +575,28 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
           for (int j = 0; j < 16; ++j)
             if (j < jn) p.out_f32[(size_t)(it.n0 + j0 + j) * p.out_ld + row] = v[j];
         } else if (MODE == PF_R2) {
-          const int row = 128 * it.mt + 32 * warp + r;
+          // y[token][rows r0..r0+3] += w * four values with one 16-byte reduction: per 8
+          // tokens the warp's 32 x 8 block goes through shared memory, and lane r (quad
+          // index qd = r % 4) takes tokens 2 qd and 2 qd + 1 of the four rows r0 = r - qd
+          float* buf = &xch[0][0][0] + 256 * warp;  // [8 tokens][32 rows]
+          const int qd = r & 3;
+          const int row0 = 128 * it.mt + 32 * warp + (r & ~3);
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            if (j < jn) {
-              const int src = (j0 & 31) + j;
+          for (int h = 0; h < 2; ++h) {
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) buf[32 * jj + r] = v[8 * h + jj];
+            __syncwarp();
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int jj = 8 * h + 2 * qd + u;  // token of the chunk
+              const int src = (j0 & 31) + jj;
               const int tok = __shfl_sync(0xffffffffu, j0 < 32 ? tk_lo : tk_hi, src);
               const float wt = __shfl_sync(0xffffffffu, j0 < 32 ? tw_lo : tw_hi, src);
-              atomicAdd(p.out_f32 + (size_t)tok * p.out_ld + row, wt * v[j]);
+              const float4 a = *reinterpret_cast<const float4*>(buf + 32 * (2 * qd + u) + (r & ~3));
+              if (jj < jn) red_add_f32x4(p.out_f32 + (size_t)tok * p.out_ld + row0, wt * a.x, wt * a.y, wt * a.z, wt * a.w);
             }
+            __syncwarp();  // buf is rewritten by the next 8 tokens
+          }
         } else {
           // 13 modes: warps 0,1 hold gate rows, warps 2,3 the matching up rows.  Each
           // pair (w, w+2) splits the 16 tokens: the gate warp finishes tokens 0-7 and
@@ -744,28 +764,51 @@ __global__ void k_pf_scatter(const int32_t* __restrict__ ids, const float* __res
   pos[i] = g;
 }
 
-// MXFP8 of the chunk's input, written to every grouped row of its token: one warp
-// per (token, 32-block); lane = element.
+// MXFP8 of the chunk's input, written to every grouped row of its token: one thread per
+// (token, 32-block) -- the block's 64 bytes in four 16-byte loads, its maximum formed
+// locally, its 32 codes out as two 16-byte stores per grouped row.
 __global__ void __launch_bounds__(256) k_pf_quant_x(const __nv_bfloat16* __restrict__ x, int M, int H, int k,
                                                      const int32_t* __restrict__ pos, uint8_t* __restrict__ xq,
                                                      uint8_t* __restrict__ xs, int xs_ld) {
-  const int lane = threadIdx.x & 31;
-  const long long wi = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int nb = H / 32;
-  if (wi >= (long long)M * nb) return;
-  const int t = (int)(wi / nb), b = (int)(wi % nb);
-  const float v = __bfloat162float(x[(size_t)t * H + 32 * b + lane]);
-  float am = fabsf(v);
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (long long)M * nb) return;
+  const int t = (int)(i / nb), b = (int)(i % nb);
+  const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H + 32 * b);
+  uint32_t w[16];
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+  for (int c = 0; c < 4; ++c) {
+    const uint4 r = __ldg(src + c);
+    w[4 * c] = r.x;
+    w[4 * c + 1] = r.y;
+    w[4 * c + 2] = r.z;
+    w[4 * c + 3] = r.w;
+  }
+  float v[32];  // bf16 -> fp32 is exact: the bits moved up by 16
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    v[2 * e] = __uint_as_float(w[e] << 16);
+    v[2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+  }
+  float am = 0.0f;
+#pragma unroll
+  for (int e = 0; e < 32; ++e) am = fmaxf(am, fabsf(v[e]));
   const int s = mxfp8_exponent(am);
-  const uint8_t q = am == 0.0f ? (uint8_t)0 : e4m3_of(v * exp2i(-s));
+  uint32_t o[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+  if (am != 0.0f) {
+    const float sc = exp2i(-s);
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      o[q] = f32x2_to_e4m3x2(v[4 * q] * sc, v[4 * q + 1] * sc) |
+             (f32x2_to_e4m3x2(v[4 * q + 2] * sc, v[4 * q + 3] * sc) << 16);
+  }
   for (int j = 0; j < k; ++j) {
-    const int gi = pos[(size_t)t * k + j];
+    const int gi = __ldg(pos + (size_t)t * k + j);
     if (gi < 0) continue;
-    const size_t g = (size_t)gi;
-    xq[g * H + 32 * b + lane] = q;
-    if (lane == 0) xs[g * xs_ld + b] = (uint8_t)(s + 127);
+    uint4* dst = reinterpret_cast<uint4*>(xq + (size_t)gi * H + 32 * b);
+    dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+    dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+    xs[(size_t)gi * xs_ld + b] = (uint8_t)(s + 127);
   }
 }
 
