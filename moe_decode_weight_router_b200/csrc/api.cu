@@ -1008,6 +1008,7 @@ struct PfWs {
   int* fill;    // [E]
   int* goff;    // [E+1]
   int* ntp;     // [E+1]
+  uint16_t* te; // [M k / 64 + E] expert of each routed token tile
   size_t clear_bytes;
   float* logits;  // [M][E]
   int32_t* ids;   // [M][k]
@@ -1040,6 +1041,8 @@ PfWs pf_ws(void* ws, int M, int H, int I, int E, int k, int Is, bool own_routing
   off += up256((size_t)(E + 1) * 4);
   s.ntp = reinterpret_cast<int*>(b + off);
   off += up256((size_t)(E + 1) * 4);
+  s.te = reinterpret_cast<uint16_t*>(b + off);
+  off += up256((G / PF_BN + (size_t)E) * 2);
   if (own_routing) {
     s.logits = reinterpret_cast<float*>(b + off);
     off += up256((size_t)M * E * 4);
@@ -1110,7 +1113,7 @@ moe_status_t pf_experts(const __nv_bfloat16* x, int M, int H, int I, int E, int 
   moe_status_t s = MOE_OK;
   const int G = M * top_k;
   // a2: grouped rows per expert
-  k_pf_scan<<<1, 1024, 0, st>>>(w.counts, E, w.goff, w.ntp, w.fill);
+  k_pf_scan<<<1, 1024, 0, st>>>(w.counts, E, w.goff, w.ntp, w.fill, w.te);
   MOE_CUDA(cudaGetLastError());
   k_pf_scatter<<<(G + 255) / 256, 256, 0, st>>>(ids, wts, M, top_k, E, w.goff, w.fill, w.g_tok, w.g_w, w.pos);
   MOE_CUDA(cudaGetLastError());
@@ -1172,6 +1175,7 @@ moe_status_t pf_experts(const __nv_bfloat16* x, int M, int H, int I, int E, int 
   a.E = E;
   a.ntile_prefix = w.ntp;
   a.goff = w.goff;
+  a.tile_e = w.te;
   a.sfa = w13_scales;
   a.sfb = w.xs;
   a.sf_ld = pf_sf_ld(H);
@@ -1197,6 +1201,7 @@ moe_status_t pf_experts(const __nv_bfloat16* x, int M, int H, int I, int E, int 
   b.E = E;
   b.ntile_prefix = w.ntp;
   b.goff = w.goff;
+  b.tile_e = w.te;
   b.g_tok = w.g_tok;
   b.g_w = w.g_w;
   b.sfa = w2_scales;

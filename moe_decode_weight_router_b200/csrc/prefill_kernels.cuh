@@ -66,6 +66,7 @@ struct alignas(64) PrefillParams {
   int E;
   const int* ntile_prefix;  // routed: [E+1] prefix sums of ceil(n_e / 128)
   const int* goff;          // routed: [E+1] first grouped row of each expert
+  const uint16_t* tile_e;   // routed: [ntile_prefix[E]] expert of each 64-token tile
   const int32_t* g_tok;     // routed: [G] token of each grouped row
   const float* g_w;         // routed: [G] routing weight of each grouped row
   const uint8_t* sfa;       // routed: weight scales [rows][K/32]
@@ -238,6 +239,8 @@ __device__ unsigned long long pf_tl[1024];
 #endif
 
 constexpr int PF_MAX_E = 512;
+// routed token tiles of a chunk: sum over experts of ceil(n_e / 64) <= M k / 64 + E
+constexpr int PF_MAX_TILES = 16384 * 8 / PF_BN + PF_MAX_E;
 // Routed modes: tile prefix and grouped offsets are copied to shared memory once per
 // CTA (every role decodes every tile; a search over global memory would put a chain
 // of dependent loads in front of each tile).
@@ -245,20 +248,14 @@ __device__ inline int pf_total_items(const PrefillParams& p, int mode, const int
   if (pf_routed(mode)) return p.m_tiles * s_ntp[p.E];
   return p.m_tiles * ((p.M + PF_BN - 1) / PF_BN);
 }
-__device__ inline PfItem pf_item(const PrefillParams& p, int mode, int idx, const int* s_ntp, const int* s_goff) {
+__device__ inline PfItem pf_item(const PrefillParams& p, int mode, int idx, const int* s_ntp, const int* s_goff,
+                                 const uint16_t* s_te) {
   PfItem it;
   it.mt = idx % p.m_tiles;
   const int j = idx / p.m_tiles;
   int rows0;
   if (pf_routed(mode)) {
-    int lo = 0, hi = p.E;  // largest e with ntile_prefix[e] <= j
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (s_ntp[mid] <= j)
-        lo = mid;
-      else
-        hi = mid;
-    }
+    const int lo = s_te[j];  // the expert whose tiles include j
     it.e = lo;
     it.n0 = (j - s_ntp[lo]) * PF_BN;
     const int g0 = s_goff[lo], ne = s_goff[lo + 1] - g0;
@@ -336,6 +333,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
   // 8 tokens x 32 rows, read back as four consecutive rows of one token
   __shared__ __align__(16) float xch[2][32][17];
   __shared__ int s_ntp[PF_MAX_E + 1], s_goff[PF_MAX_E + 1];
+  __shared__ uint16_t s_te[pf_routed(MODE) ? PF_MAX_TILES : 1];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int S = p.stages;
@@ -350,6 +348,11 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
       s_goff[e] = __ldg(p.goff + e);
     }
   __syncthreads();
+  if (mx) {
+    const int nt = s_ntp[p.E];  // <= PF_MAX_TILES (the host bounds M, k and E)
+    for (int j = tid; j < nt; j += PF_THREADS) s_te[j] = __ldg(p.tile_e + j);
+    __syncthreads();
+  }
   const int total = pf_total_items(p, MODE, s_ntp);
   const int G = gridDim.x;
   const int kb = p.K / 32;  // E8M0 bytes per weight row
@@ -396,7 +399,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
       int n_item = 0;
       bool ok = true;
       for (int idx = blockIdx.x; idx < total && ok; idx += G, ++n_item) {
-        const PfItem it = pf_item(p, MODE, idx, s_ntp, s_goff);
+        const PfItem it = pf_item(p, MODE, idx, s_ntp, s_goff, s_te);
         if (mx) {
           // scale rows of a tile -- weight rows (two 64-row runs or one 128-row run) and
           // the token rows -- into shared buffer m % NB.  With two tensor-memory buffers the
@@ -416,7 +419,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
             return true;
           };
           if (!sf2 || n_item == 0) ok = fetch_scales(n_item, it);
-          if (ok && sf2 && idx + G < total) ok = fetch_scales(n_item + 1, pf_item(p, MODE, idx + G, s_ntp, s_goff));
+          if (ok && sf2 && idx + G < total) ok = fetch_scales(n_item + 1, pf_item(p, MODE, idx + G, s_ntp, s_goff, s_te));
           if (!ok) break;
           if (n_item < 32) PF_STAMP(512 + 8 * n_item + 5);
         }
@@ -453,7 +456,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
       int n_item = 0;
       bool ok = true;
       for (int idx = blockIdx.x; idx < total && ok; idx += G, ++n_item) {
-        const PfItem it = pf_item(p, MODE, idx, s_ntp, s_goff);
+        const PfItem it = pf_item(p, MODE, idx, s_ntp, s_goff, s_te);
         const int N = (it.ncnt + 15) & ~15;
         const int ab = n_item & 1;
         if (n_item >= 2 && !pf_wait(&acc_empty[ab], (uint32_t)(((n_item >> 1) - 1) & 1), p.status, &s_abort,
@@ -533,11 +536,11 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
       return true;
     };
     bool live = true;
-    if (mx && blockIdx.x < total) live = put_scales(0, pf_item(p, MODE, blockIdx.x, s_ntp, s_goff));
-    if (mx && sf2 && live && blockIdx.x + G < total) live = put_scales(1, pf_item(p, MODE, blockIdx.x + G, s_ntp, s_goff));
+    if (mx && blockIdx.x < total) live = put_scales(0, pf_item(p, MODE, blockIdx.x, s_ntp, s_goff, s_te));
+    if (mx && sf2 && live && blockIdx.x + G < total) live = put_scales(1, pf_item(p, MODE, blockIdx.x + G, s_ntp, s_goff, s_te));
     int n_item = 0;
     for (int idx = blockIdx.x; idx < total; idx += G, ++n_item) {
-      const PfItem it = pf_item(p, MODE, idx, s_ntp, s_goff);
+      const PfItem it = pf_item(p, MODE, idx, s_ntp, s_goff, s_te);
       const int ab = n_item & 1;
       // routed W2: the tile's tokens and routing weights (lane j holds grouped rows j and
       // j + 32), fetched before the accumulator wait so their latency stays off the epilogue
@@ -559,7 +562,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
       if (s_abort) break;
       tc_fence_after();
       // one scale buffer: the MMAs of this tile are complete, its columns may take the next tile's
-      if (mx && !sf2 && idx + G < total) live = put_scales(n_item + 1, pf_item(p, MODE, idx + G, s_ntp, s_goff));
+      if (mx && !sf2 && idx + G < total) live = put_scales(n_item + 1, pf_item(p, MODE, idx + G, s_ntp, s_goff, s_te));
       if (tid == 0 && n_item < 32) PF_STAMP(512 + 8 * n_item + 3);
       const uint32_t acc_lane = lane_base + 64u * ab;
       for (int j0 = 0; j0 < it.ncnt; j0 += 16) {
@@ -647,7 +650,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
       // two scale buffers: this tile's MMAs are done, so its buffer takes the tile after
       // next while the next tile's MMAs run
       if (mx && sf2 && live && idx + 2 * G < total)
-        live = put_scales(n_item + 2, pf_item(p, MODE, idx + 2 * G, s_ntp, s_goff));
+        live = put_scales(n_item + 2, pf_item(p, MODE, idx + 2 * G, s_ntp, s_goff, s_te));
     }
   }
   tc_fence_before();
@@ -712,7 +715,8 @@ __global__ void __launch_bounds__(256) k_pf_topk(const float* __restrict__ logit
 // One block: exclusive prefix of the counts (grouped offsets) and of the 128-token
 // tiles per expert; clears the fill cursors.
 __global__ void __launch_bounds__(1024) k_pf_scan(const int* __restrict__ counts, int E, int* __restrict__ goff,
-                                                   int* __restrict__ ntile_prefix, int* __restrict__ fill) {
+                                                   int* __restrict__ ntile_prefix, int* __restrict__ fill,
+                                                   uint16_t* __restrict__ tile_e) {
   __shared__ int s_c[1024], s_t[1024];
   const int e = threadIdx.x;
   const int c = e < E ? counts[e] : 0;
@@ -730,6 +734,8 @@ __global__ void __launch_bounds__(1024) k_pf_scan(const int* __restrict__ counts
     goff[e + 1] = s_c[e];
     ntile_prefix[e + 1] = s_t[e];
     fill[e] = 0;
+    const int nt = (c + PF_BN - 1) / PF_BN;  // this expert's tiles end at s_t[e]
+    for (int j = s_t[e] - nt; j < s_t[e]; ++j) tile_e[j] = (uint16_t)e;
   }
   if (e == 0) {
     goff[0] = 0;
