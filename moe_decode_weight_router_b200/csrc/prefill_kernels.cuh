@@ -174,9 +174,8 @@ __host__ __device__ inline uint32_t idesc_mx(int N, uint32_t sf_id) {
 // timeout of a workspace also records where it happened (status[4..7]: wait site,
 // mode, block, parity).
 enum : int { PFW_EMPTY = 1, PFW_DRAIN = 2, PFW_ACC_EMPTY = 3, PFW_SF = 4, PFW_FULL = 5, PFW_ACC_FULL = 6 };
-__device__ __noinline__ bool pf_wait(uint64_t* bar, uint32_t parity, int* status, volatile int* abort_flag,
-                                     int site, int mode) {
-  if (mbar_try_wait(bar, parity)) return true;
+__device__ __noinline__ bool pf_wait_slow(uint64_t* bar, uint32_t parity, int* status, volatile int* abort_flag,
+                                          int site, int mode) {
   const unsigned long long t0 = globaltimer_ns();
   for (unsigned n = 1;; ++n) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -194,6 +193,12 @@ __device__ __noinline__ bool pf_wait(uint64_t* bar, uint32_t parity, int* status
     }
   }
   return true;
+}
+// Bounded mbarrier wait: the first try inline (a stage or tile that is ready costs no
+// call), the polling loop out of line.
+__device__ __forceinline__ bool pf_wait(uint64_t* bar, uint32_t parity, int* status, volatile int* abort_flag, int site,
+                                        int mode) {
+  return mbar_try_wait(bar, parity) || pf_wait_slow(bar, parity, status, abort_flag, site, mode);
 }
 
 // ---------------------------------------------------------------------------
@@ -477,7 +482,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
             break;
           }
           if (q < 128) PF_STAMP(4 * (int)q + 1);
-          tc_fence_after();
+          // no thread-side fence here: the copies and the MMAs are both in the async
+          // proxy, and the stage's barrier orders them
           const uint32_t sa = smem_u32(smem + (size_t)s * stage_bytes);
           const uint32_t bstride = (mx && it.ncnt <= 32) ? 4096u : 8192u;  // token chunk stride (box rows x 128 B)
           for (int c = 0; c < KC; ++c) {
