@@ -79,8 +79,10 @@ moe_status_t dev_info(DevInfo* out) {
     MOE_CUDA(allow_dyn_smem(k_experts2, lim, &d.dyn_e2));
     MOE_CUDA(allow_dyn_smem(k_lm_gemv, lim, &d.dyn_lm));
     MOE_CUDA(allow_dyn_smem(k_lm_gemv_bf16, lim, &d.dyn_lmb));
-    MOE_CUDA(allow_dyn_smem(k_step<false>, lim, &d.dyn_step));
-    MOE_CUDA(allow_dyn_smem(k_step<true>, lim, &d.dyn_step));
+    MOE_CUDA(allow_dyn_smem(k_step<false, false>, lim, &d.dyn_step));
+    MOE_CUDA(allow_dyn_smem(k_step<true, false>, lim, &d.dyn_step));
+    MOE_CUDA(allow_dyn_smem(k_step<false, true>, lim, &d.dyn_step));
+    MOE_CUDA(allow_dyn_smem(k_step<true, true>, lim, &d.dyn_step));
     MOE_CUDA(allow_dyn_smem(k_umma<PF_ROUTER>, lim, &d.dyn_pf));
     MOE_CUDA(allow_dyn_smem(k_umma<PF_SH13>, lim, &d.dyn_pf));
     MOE_CUDA(allow_dyn_smem(k_umma<PF_SH2>, lim, &d.dyn_pf));
@@ -278,10 +280,12 @@ moe_status_t launch_step(const StepParams& sp, const DevInfo& d, cudaStream_t st
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  // the profiling and trace code only in the instantiation a timeline or trace asks for
+  const bool dbg = sp.timeline || sp.x_trace || sp.h_trace || sp.ids_trace || sp.w_trace;
   if (sp.M == 1)
-    MOE_CUDA(cudaLaunchKernelEx(&cfg, k_step<true>, sp));
+    MOE_CUDA(cudaLaunchKernelEx(&cfg, dbg ? k_step<true, true> : k_step<true, false>, sp));
   else
-    MOE_CUDA(cudaLaunchKernelEx(&cfg, k_step<false>, sp));
+    MOE_CUDA(cudaLaunchKernelEx(&cfg, dbg ? k_step<false, true> : k_step<false, false>, sp));
   return MOE_OK;
 }
 

@@ -86,8 +86,13 @@ struct StepParams {
 // Profiling stamp: block 0 and the last block record %globaltimer at phase
 // boundaries (slots 0-11 by consumer thread 0, 12-15 by producer lane 0).
 __device__ __noinline__ void stamp_write(const StepParams& p, int l, int slot);
+// DBG: the instantiation taken when a timeline or a trace buffer is passed; the other
+// one carries none of the profiling or trace code.
+template <bool DBG>
 __device__ __forceinline__ void stamp(const StepParams& p, int l, int slot) {
-  if (p.timeline) stamp_write(p, l, slot);
+  if constexpr (DBG) {
+    if (p.timeline) stamp_write(p, l, slot);
+  }
 }
 __device__ __noinline__ void stamp_write(const StepParams& p, int l, int slot) {
   const bool first = blockIdx.x == 0, last = blockIdx.x == gridDim.x - 1;
@@ -104,8 +109,11 @@ __device__ __noinline__ void item_stamp_write(const StepParams& p, long long i, 
   if (blockIdx.x != 0 || i >= STEP_ITEM_LOG || (threadIdx.x & 31) != 0) return;
   p.timeline[(size_t)2 * p.L * 16 + (size_t)i * 8 + which] = globaltimer_ns();
 }
+template <bool DBG>
 __device__ __forceinline__ void item_stamp(const StepParams& p, long long i, int which) {
-  if (p.timeline) item_stamp_write(p, i, which);
+  if constexpr (DBG) {
+    if (p.timeline) item_stamp_write(p, i, which);
+  }
 }
 // Profiling: every block's own phase ends, [G][L][16] after the item log (written by
 // the calling thread): 0 residual seen, 1 layer input staged, 2 router item published,
@@ -115,8 +123,11 @@ __device__ __noinline__ void blk_stamp_write(const StepParams& p, int l, int slo
   p.timeline[(size_t)2 * p.L * 16 + (size_t)STEP_ITEM_LOG * 8 + ((size_t)blockIdx.x * p.L + l) * 16 + slot] =
       globaltimer_ns();
 }
+template <bool DBG>
 __device__ __forceinline__ void blk_stamp(const StepParams& p, int l, int slot) {
-  if (p.timeline) blk_stamp_write(p, l, slot);
+  if constexpr (DBG) {
+    if (p.timeline) blk_stamp_write(p, l, slot);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -384,6 +395,7 @@ __host__ __device__ inline int step_group_cap(uint32_t R, uint32_t tile_bytes, i
 // ---------------------------------------------------------------------------
 // producer side
 // ---------------------------------------------------------------------------
+template <bool DBG>
 struct Producer {
   const StepParams& p;
   uint8_t* ring;
@@ -404,7 +416,7 @@ struct Producer {
   // and the new item's barrier slot is free, and arms the barrier; then one lane per
   // contiguous run issues its bulk copy.
   __device__ bool acquire(uint32_t n, uint32_t& s0, int& slot) {
-    item_stamp(p, i, 4);
+    item_stamp<DBG>(p, i, 4);
     unsigned long long vs;
     s0 = ring_take(vpos, n, R, &vs);
     slot = (int)(i % STEP_SLOTS);
@@ -423,7 +435,7 @@ struct Producer {
       vst[slot] = vs;
     }
     ok = __shfl_sync(0xffffffffu, ok, 0);
-    if (ok) item_stamp(p, i, 0);
+    if (ok) item_stamp<DBG>(p, i, 0);
     return ok != 0;
   }
 
@@ -444,7 +456,7 @@ struct Producer {
     if (lane == 1) bulk_g2s(st + codes, Lp.w13c + (row + I) * (H / 2), codes, fb, pol);
     if (lane == 2) bulk_g2s(st + 2 * codes, Lp.w13s + row * (H / 32), scales, fb, pol);
     if (lane == 3) bulk_g2s(st + 2 * codes + scales, Lp.w13s + (row + I) * (H / 32), scales, fb, pol);
-    item_stamp(p, i, 5);
+    item_stamp<DBG>(p, i, 5);
     ++i;
     return true;
   }
@@ -463,7 +475,7 @@ struct Producer {
     __syncwarp();
     if (lane == 0) bulk_g2s(st, Lp.w2c + row * (I / 2), codes, fb, pol);
     if (lane == 1) bulk_g2s(st + codes, Lp.w2s + row * (I / 32), scales, fb, pol);
-    item_stamp(p, i, 5);
+    item_stamp<DBG>(p, i, 5);
     ++i;
     return true;
   }
@@ -474,7 +486,7 @@ struct Producer {
     int slot;
     if (!acquire(step_item_bytes(it.type, p.H, p.I, p.Is), s0, slot)) return false;
     copy_item(Lp, it, ring + s0, &full[slot]);
-    item_stamp(p, i, 5);
+    item_stamp<DBG>(p, i, 5);
     ++i;
     return true;
   }
@@ -762,6 +774,7 @@ __device__ __noinline__ void topk_token_full(const StepParams& p, int l, int tok
 // whose parts hold at most 256 experts): each keeps its part's top-k of its tokens
 // (a global top-k element is always in its part's top-k, ties included), then one
 // warp per token merges the EP*k candidates.
+template <bool DBG>
 __device__ void step_topk_win(const StepParams& p, int l, Plan& P, int32_t* s_ids, float* s_wts, uint32_t* s_ck,
                           int32_t* s_ci, volatile int* s_abort_ptr) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -858,10 +871,12 @@ __device__ void step_topk_win(const StepParams& p, int l, Plan& P, int32_t* s_id
       const float wj = ex / den;
       s_ids[tok * k + lane] = sel_id;
       s_wts[tok * k + lane] = wj;
-      if (blockIdx.x == 0) {
-        const size_t o = ((size_t)l * M + tok) * k + lane;
-        if (p.ids_trace) p.ids_trace[o] = sel_id;
-        if (p.w_trace) p.w_trace[o] = wj;
+      if constexpr (DBG) {
+        if (blockIdx.x == 0) {
+          const size_t o = ((size_t)l * M + tok) * k + lane;
+          if (p.ids_trace) p.ids_trace[o] = sel_id;
+          if (p.w_trace) p.w_trace[o] = wj;
+        }
       }
     }
   }
@@ -1016,6 +1031,7 @@ __device__ void stage1(const StepParams& p, int l, const float* hin, float* hout
 // largest logit, the survivors (at most TOPK_CAND, else the exact k-round selection)
 // are ranked by their order keys, and warp 0 writes the plan directly: the k selected
 // experts are distinct, so slot i holds the i-th smallest id with its weight.
+template <bool DBG>
 __device__ void topk1(const StepParams& p, int l, Plan& P, uint32_t* s_wmax, int* s_ncand,
                       unsigned long long* s_cand, unsigned long long* s_sel, volatile int* s_abort_ptr) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
@@ -1044,7 +1060,7 @@ __device__ void topk1(const StepParams& p, int l, Plan& P, uint32_t* s_wmax, int
     mx = __reduce_max_sync(0xffffffffu, mx);
     if (lane == 0) s_wmax[warp] = mx;
   }
-  if (tid == 0) blk_stamp(p, l, 8);
+  if (tid == 0) blk_stamp<DBG>(p, l, 8);
   csync();
   uint32_t bound = 0xFFFFFFFFu;
 #pragma unroll
@@ -1057,7 +1073,7 @@ __device__ void topk1(const StepParams& p, int l, Plan& P, uint32_t* s_wmax, int
       if (pos < TOPK_CAND) s_cand[pos] = order_key(key[i], e0 + off);
     }
   }
-  if (tid == 0) blk_stamp(p, l, 9);
+  if (tid == 0) blk_stamp<DBG>(p, l, 9);
   csync();
   if (warp == 0) {
     const int n = s_ncand[0];
@@ -1088,15 +1104,17 @@ __device__ void topk1(const StepParams& p, int l, Plan& P, uint32_t* s_wmax, int
     if (lane < k) {
       P.ids[slot] = id;
       P.w[slot][0] = wj;
-      if (blockIdx.x == 0) {
-        const size_t o = (size_t)l * k + lane;
-        if (p.ids_trace) p.ids_trace[o] = id;
-        if (p.w_trace) p.w_trace[o] = wj;
+      if constexpr (DBG) {
+        if (blockIdx.x == 0) {
+          const size_t o = (size_t)l * k + lane;
+          if (p.ids_trace) p.ids_trace[o] = id;
+          if (p.w_trace) p.w_trace[o] = wj;
+        }
       }
     }
     if (lane == 0) P.n_unique = k;
   }
-  if (tid == 0) blk_stamp(p, l, 12);
+  if (tid == 0) blk_stamp<DBG>(p, l, 12);
   csync();
 }
 
@@ -1190,7 +1208,7 @@ __device__ __forceinline__ void rows4_dot_m1(const uint8_t* wrows, uint32_t wstr
 // ONE: the one-token instantiation (lanes-along-K products, chunk-major activations);
 // otherwise a verify window of M >= 2 tokens (tensor-core tiles).  Separate
 // instantiations keep each one's code small enough for the instruction caches.
-template <bool ONE>
+template <bool ONE, bool DBG>
 __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant__ StepParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ Plan P;
@@ -1250,7 +1268,7 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
 
   // ---------------- producer ----------------
   if (warp == STEP_CONSUMERS) {
-    Producer pr{p, ring, R, full, empty, s_vst, policy_evict_first(), 0, 0, RingCursor{0ull, 0u}, &s_abort, lane};
+    Producer<DBG> pr{p, ring, R, full, empty, s_vst, policy_evict_first(), 0, 0, RingCursor{0ull, 0u}, &s_abort, lane};
     bool ok = true;
     for (int l = 0; l < L && ok; ++l) {
       const LayerPtrs& Lp = p.layer[l];
@@ -1258,7 +1276,7 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
       W.init_fixed(p);
       for (int r = 0; r < W.nA + W.nS && ok; ++r) ok = pr.issue(Lp, P, W.at(p, r));
       if (!ok) break;
-      stamp(p, l, 12);
+      stamp<DBG>(p, l, 12);
       int got = 1;
       // the consumers' slice copy of h (ordered before their arrive by a block
       // barrier) is published here, off their critical path: fence, then count
@@ -1269,9 +1287,9 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
       if (!__shfl_sync(0xffffffffu, got, 0)) break;
       if (lane == 0) got = ring_wait(plan_bar, (uint32_t)(l & 1), p.status, &s_abort);
       if (!__shfl_sync(0xffffffffu, got, 0)) break;
-      stamp(p, l, 13);
+      stamp<DBG>(p, l, 13);
       W.init_routed(p, P.n_unique);
-      stamp(p, l, 15);
+      stamp<DBG>(p, l, 15);
       {
         int u, r0, nt;
         GroupWalk gb{W.b0, W.b0 + W.nB, p.I / 8, capB};
@@ -1279,7 +1297,7 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
         GroupWalk gc{W.c0, W.c0 + W.nC, p.H / 16, capC};
         while (ok && gc.next(u, r0, nt)) ok = pr.issue_c(Lp, P, u, r0, nt);
       }
-      stamp(p, l, 14);
+      stamp<DBG>(p, l, 14);
     }
     // every copy issued lands before the block may exit
     if (lane == 0)
@@ -1298,21 +1316,21 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
     unsigned* lc = ctr + (size_t)l * CTR_PER_LAYER;
     float* hout = p.h + (size_t)(l & 1) * M * H;
     const float* hin = p.h + (size_t)((l + 1) & 1) * M * H;  // layer l-1's buffer
-    stamp(p, l, 0);
+    stamp<DBG>(p, l, 0);
     if (l > 0) {
       if (tid == 0) wait_counter(ctr + (size_t)(l - 1) * CTR_PER_LAYER + CTR_H, G, p.status, &s_abort);
       csync();
     }
-    stamp(p, l, 1);
-    if (tid == 0) blk_stamp(p, l, 0);
+    stamp<DBG>(p, l, 1);
+    if (tid == 0) blk_stamp<DBG>(p, l, 0);
     if constexpr (ONE)
       stage1(p, l, hin, hout, xb16, xf16, s_part, s_amx, s_sh, slice_q0, slice_q1);
     else
       stage_window_input(p, l, hin, hout, xb16, xf16, xss, s_part, s_amx, s_r, s_sh, slice_q0, slice_q1);
     if (tid == 0) mbar_arrive(hinit_bar);
-    stamp(p, l, 2);
-    if (tid == 0) blk_stamp(p, l, 1);
-    if (blockIdx.x == 0 && (p.x_trace || p.h_trace)) {
+    stamp<DBG>(p, l, 2);
+    if (tid == 0) blk_stamp<DBG>(p, l, 1);
+    if (DBG && blockIdx.x == 0 && (p.x_trace || p.h_trace)) {
       for (int e = tid; e < M * H; e += 32 * STEP_CONSUMERS) {
         const int tok = e / H, c = e % H;
         const __nv_bfloat16 xv = *reinterpret_cast<const __nv_bfloat16*>(xb16 + tok * xss + 2 * c);
@@ -1337,7 +1355,7 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
         const int slot = (int)(ii % STEP_SLOTS);
         src = ring + s0;
         eb = &empty[slot];
-        item_stamp(p, ii, 3);
+        item_stamp<DBG>(p, ii, 3);
         ready = ring_wait(&full[slot], (uint32_t)((ii / STEP_SLOTS) & 1), p.status, &s_abort);
       }
       ready = __all_sync(0xffffffffu, ready);
@@ -1364,24 +1382,24 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
         if (router) {
           st_tagged(p.logits + g * p.E + 4 * it.a + 2 * t, c[0], tag);
           st_tagged(p.logits + g * p.E + 4 * it.a + 2 * t + 1, c[1], tag);
-          if (lane == 0) blk_stamp(p, l, 2);
+          if (lane == 0) blk_stamp<DBG>(p, l, 2);
         } else {
           st_tagged(p.a_shared + g * Is + 2 * (it.a - nr) + t, silu_f32(c[0]) * c[1], tag);
         }
       }
     }
-    stamp(p, l, 3);
-    if (tid == 0) blk_stamp(p, l, 3);
+    stamp<DBG>(p, l, 3);
+    if (tid == 0) blk_stamp<DBG>(p, l, 3);
 
     // ---- top-k and plan (every block, identical; polls the tagged logits) ----
-    stamp(p, l, 4);
+    stamp<DBG>(p, l, 4);
     if constexpr (ONE)
-      topk1(p, l, P, s_wmax, s_ncand, s_cand, s_sel, &s_abort);
+      topk1<DBG>(p, l, P, s_wmax, s_ncand, s_cand, s_sel, &s_abort);
     else
-      step_topk_win(p, l, P, s_ids, s_wts, s_ck, s_ci, &s_abort);
+      step_topk_win<DBG>(p, l, P, s_ids, s_wts, s_ck, s_ci, &s_abort);
     if (tid == 0) mbar_arrive(plan_bar);
-    stamp(p, l, 5);
-    if (tid == 0) blk_stamp(p, l, 4);
+    stamp<DBG>(p, l, 5);
+    if (tid == 0) blk_stamp<DBG>(p, l, 4);
 
     // ---- CS: shared W2 (activation as bf16 hi + lo), accumulated into h, ahead of the
     //      routed tiles whose copies it waits for ----
@@ -1408,7 +1426,7 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
       }
       if (tid == 0) wait_counter(lc + CTR_HINIT, G, p.status, &s_abort);  // every slice of h initialised
       csync();
-      stamp(p, l, 6);
+      stamp<DBG>(p, l, 6);
       for (int r = 0; r < W.nS; ++r) {
         const uint8_t* src;
         uint64_t* eb;
@@ -1420,7 +1438,7 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
           const int slot = (int)(ii % STEP_SLOTS);
           src = ring + s0;
           eb = &empty[slot];
-          item_stamp(p, ii, 3);
+          item_stamp<DBG>(p, ii, 3);
           ready = ring_wait(&full[slot], (uint32_t)((ii / STEP_SLOTS) & 1), p.status, &s_abort);
         }
         ready = __all_sync(0xffffffffu, ready);
@@ -1458,8 +1476,8 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
           }
         }
       }
-      stamp(p, l, 7);
-      if (tid == 0) blk_stamp(p, l, 5);
+      stamp<DBG>(p, l, 7);
+      if (tid == 0) blk_stamp<DBG>(p, l, 5);
     }
 
     // ---- B: routed W13 + SwiGLU ----
@@ -1484,10 +1502,10 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
         const int nmine = f < U ? (U - 1 - f) / 16 + 1 : 0;
         const int nw = max(__shfl_sync(0xffffffffu, nmine, 0), __shfl_sync(0xffffffffu, nmine, 16));
         if (nw > 0) {
-          item_stamp(p, i, 3);
+          item_stamp<DBG>(p, i, 3);
           const bool ready =
               __all_sync(0xffffffffu, ring_wait(&full[slot], (uint32_t)((i / STEP_SLOTS) & 1), p.status, &s_abort));
-          item_stamp(p, i, 1);
+          item_stamp<DBG>(p, i, 1);
           const uint8_t* gate = ring + s0;
           const uint8_t* up = gate + codes;
           const uint8_t* gs = gate + 2 * codes;
@@ -1503,7 +1521,7 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
             if (live && (lane & 15) == 0) p.a_routed[(size_t)u * I + 8 * r0 + q] = silu_f32(r[0]) * r[1];
           }
           __syncwarp();
-          item_stamp(p, i, 2);
+          item_stamp<DBG>(p, i, 2);
           const int done = __shfl_sync(0xffffffffu, nmine, 0) + __shfl_sync(0xffffffffu, nmine, 16);
           if (lane == 0) {
             // the ring space goes back first: the publish below (fence, counter) no
@@ -1530,9 +1548,9 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
         const int slot = (int)(i % STEP_SLOTS);
         const int j0 = ((warp - tc) % STEP_CONSUMERS + STEP_CONSUMERS) % STEP_CONSUMERS;
         if (j0 < nt) {
-          item_stamp(p, i, 3);
+          item_stamp<DBG>(p, i, 3);
           const bool ready = ring_wait(&full[slot], (uint32_t)((i / STEP_SLOTS) & 1), p.status, &s_abort);
-          item_stamp(p, i, 1);
+          item_stamp<DBG>(p, i, 1);
           const uint8_t* gate = ring + s0;
           const uint8_t* up = gate + codes;
           const uint8_t* gs = gate + 2 * codes;
@@ -1546,7 +1564,7 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
                                H / 32, xf16, xss, M, s_sh, c);
           }
           __syncwarp();  // every lane is done reading the tile: its ring space goes back first
-          item_stamp(p, i, 2);
+          item_stamp<DBG>(p, i, 2);
           if (lane == 0 && atomicAdd(&s_gdone[slot], 1) + 1 == nt) {
             s_gdone[slot] = 0;
             mbar_arrive(&empty[slot]);
@@ -1563,10 +1581,10 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
         ++i;
       }
     }
-    stamp(p, l, 8);
-    if (tid == 0) blk_stamp(p, l, 6);
+    stamp<DBG>(p, l, 8);
+    if (tid == 0) blk_stamp<DBG>(p, l, 6);
     csync();  // xf16 and the shared halves are dead: the routed-W2 activation copies take the region
-    stamp(p, l, 9);
+    stamp<DBG>(p, l, 9);
 
     // ---- CR: routed W2 (weighted), accumulated into h ----
     // The block's contiguous range touches experts u_first..u_last (at most CR_CACHE,
@@ -1631,10 +1649,10 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
         if (nw > 0) {
           const int cu = u - u_first;  // cache entry
           const uint8_t* my_af = afc + (size_t)cu * ass;
-          item_stamp(p, i, 3);
+          item_stamp<DBG>(p, i, 3);
           const bool ready =
               __all_sync(0xffffffffu, ring_wait(&full[slot], (uint32_t)((i / STEP_SLOTS) & 1), p.status, &s_abort));
-          item_stamp(p, i, 1);
+          item_stamp<DBG>(p, i, 1);
           const uint8_t* cd = ring + s0;
           const uint8_t* sc = cd + codes;
           const float wt = P.w[u][0];
@@ -1652,7 +1670,7 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
             }
           }
           __syncwarp();
-          item_stamp(p, i, 2);
+          item_stamp<DBG>(p, i, 2);
           int done = nmine + __shfl_xor_sync(0xffffffffu, nmine, 8);
           done += __shfl_xor_sync(0xffffffffu, done, 16);
           if (lane == 0 && atomicAdd(&s_gdone[slot], done) + done == Rg) {
@@ -1674,9 +1692,9 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
         if (j0 < nt) {
           const int cu = u - u_first;  // cache entry
           const uint8_t* my_af = afc + (size_t)cu * M * ass;
-          item_stamp(p, i, 3);
+          item_stamp<DBG>(p, i, 3);
           const bool ready = ring_wait(&full[slot], (uint32_t)((i / STEP_SLOTS) & 1), p.status, &s_abort);
-          item_stamp(p, i, 1);
+          item_stamp<DBG>(p, i, 1);
           const uint8_t* cd = ring + s0;
           const uint8_t* sc = cd + codes;
           // groups hold at most capC <= 2 * STEP_CONSUMERS tiles: one or two per warp,
@@ -1700,7 +1718,7 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
             }
           }
           __syncwarp();
-          item_stamp(p, i, 2);
+          item_stamp<DBG>(p, i, 2);
           if (lane == 0 && atomicAdd(&s_gdone[slot], mine) + mine == nt) {
             s_gdone[slot] = 0;
             mbar_arrive(&empty[slot]);
@@ -1725,11 +1743,11 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
         ++i;
       }
     }
-    stamp(p, l, 10);
+    stamp<DBG>(p, l, 10);
     csync();
-    if (tid == 0) blk_stamp(p, l, 7);
+    if (tid == 0) blk_stamp<DBG>(p, l, 7);
     if (tid == 0 && l != p.hold_layer) signal_counter(lc + CTR_H);
-    stamp(p, l, 11);
+    stamp<DBG>(p, l, 11);
   }
 
   // ---- LM-head input: bf16(RMSNorm(h_L)) by block 0 ----
@@ -1762,8 +1780,10 @@ __global__ void __launch_bounds__(STEP_THREADS, 1) k_step(const __grid_constant_
     const float hv = __ldcg(hf + e);
     const __nv_bfloat16 v = __float2bfloat16_rn(hv * s_r[tok]);
     p.x_final[e] = v;
-    if (p.x_trace) p.x_trace[(size_t)L * M * H + e] = v;
-    if (p.h_trace) p.h_trace[(size_t)L * M * H + e] = hv;
+    if constexpr (DBG) {
+      if (p.x_trace) p.x_trace[(size_t)L * M * H + e] = v;
+      if (p.h_trace) p.h_trace[(size_t)L * M * H + e] = hv;
+    }
   }
 }
 
