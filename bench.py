@@ -40,10 +40,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 
 
 # DRAM traffic of k_step per layer (read + write): an ncu capture (dram__bytes_read.sum +
-# dram__bytes_write.sum, the second k_step launch) of `bench.py --probe-window one
-# --layers 2`, valid while the kernel sources hash to the value recorded with it
-# (otherwise the roofline's traffic is reported as null).
-KSTEP_TRAFFIC = {"bytes_per_layer": (79129600 + 1643776) / 2, "sources_sha256_16": "28f83db332ee7c95",
+# dram__bytes_write.sum) of the first untraced one-token launch (`--kernel-name-base mangled
+# -k regex:k_stepILb1ELb0E -c 1`) in `bench.py --layers 2 --steps 1 --warmup 1
+# --no-cpu-baseline --skip-m4 --skip-prefill --skip-head`, valid while the kernel sources
+# hash to the value recorded with it (otherwise the roofline's traffic is reported as null).
+KSTEP_TRAFFIC = {"bytes_per_layer": (79101696 + 1059072) / 2, "sources_sha256_16": "0fcd417978a35d94",
                  "sources": ("step_kernel.cuh", "decode_kernels.cuh", "common.cuh")}
 
 
