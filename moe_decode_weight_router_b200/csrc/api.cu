@@ -1076,6 +1076,9 @@ PfWs pf_ws(void* ws, int M, int H, int I, int E, int k, int Is, bool own_routing
 }
 
 moe_status_t launch_umma(PrefillParams& p, const DevInfo& d, cudaStream_t st) {
+  // the MMA issuer unrolls at most four K chunks per stage, whole stages per tile
+  const int kbox = (p.mode == PF_R13 || p.mode == PF_R2) ? 128 : 64;
+  if (p.kc < 1 || p.kc > 4 || (p.K / kbox) % p.kc != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
   const bool mx = p.mode == PF_R13 || p.mode == PF_R2;
   const long long stage = (long long)PF_STAGE_BYTES * p.kc;
   const long long sf1 = mx ? (long long)pf_sf_buf_bytes(p.K, p.sf_ld) : 0;

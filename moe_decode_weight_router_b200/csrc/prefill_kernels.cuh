@@ -475,6 +475,12 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
         tc_fence_after();
         const uint32_t dacc = tbase + 64u * ab;
         const uint32_t tsfa = tbase + sfa_col(n_item), tsfb = tbase + sfb_col(n_item);
+        // the tile's instruction descriptors (one per 32-wide K step of a chunk) and its
+        // token-chunk stride in descriptor units, formed once per tile
+        uint32_t idk[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) idk[k] = mx ? idesc_mx(N, (uint32_t)k) : idesc_bf16(N);
+        const uint32_t bstride = (mx && it.ncnt <= 32) ? 4096u : 8192u;  // token chunk stride (box rows x 128 B)
         for (int ch = 0; ch < nch; ch += KC, ++q) {
           const int s = (int)(q % S);
           if (!pf_wait(&full[s], (uint32_t)((q / S) & 1), p.status, &s_abort, PFW_FULL, MODE)) {
@@ -484,20 +490,26 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ 
           if (q < 128) PF_STAMP(4 * (int)q + 1);
           // no thread-side fence here: the copies and the MMAs are both in the async
           // proxy, and the stage's barrier orders them
+          // the stage's operands: base descriptors of its first weight and token chunks;
+          // chunk c sits 16 KB (1024 descriptor units) and bstride further on, and each
+          // 32-wide K step 32 bytes (2 units) into the swizzled rows -- the start-address
+          // field (address / 16, 14 bits) never carries, shared memory being < 256 KB
           const uint32_t sa = smem_u32(smem + (size_t)s * stage_bytes);
-          const uint32_t bstride = (mx && it.ncnt <= 32) ? 4096u : 8192u;  // token chunk stride (box rows x 128 B)
-          for (int c = 0; c < KC; ++c) {
-            const uint64_t adesc = sw128_desc(sa + 16384u * c), bdesc = sw128_desc(sa + 16384u * KC + bstride * c);
-            const uint32_t chc = (uint32_t)(ch + c);
+          const uint64_t a0 = sw128_desc(sa), b0 = sw128_desc(sa + 16384u * KC);
+          const uint32_t acc0 = ch > 0 ? 1u : 0u;
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const uint32_t accum = (chc > 0 || k > 0) ? 1u : 0u;
-              // advance 32 bytes of K inside the 128-byte swizzled row
-              if (mx)
-                umma_mx(dacc, adesc + 2u * k, bdesc + 2u * k, idesc_mx(N, (uint32_t)k), accum, tsfa + 4u * chc,
-                        tsfb + 4u * chc);
-              else
-                umma_bf16(dacc, adesc + 2u * k, bdesc + 2u * k, idesc_bf16(N), accum);
+          for (int c = 0; c < 4; ++c) {  // KC <= 4 chunks per stage
+            if (c < KC) {
+              const uint64_t ac = a0 + 1024u * (uint32_t)c, bc = b0 + (bstride >> 4) * (uint32_t)c;
+              const uint32_t sfc = 4u * (uint32_t)(ch + c);
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const uint32_t accum = (c > 0 || k > 0) ? 1u : acc0;
+                if (mx)
+                  umma_mx(dacc, ac + 2u * k, bc + 2u * k, idk[k], accum, tsfa + sfc, tsfb + sfc);
+                else
+                  umma_bf16(dacc, ac + 2u * k, bc + 2u * k, idk[k], accum);
+              }
             }
           }
           tc_commit(&empty[s]);  // the stage returns to the producer once these MMAs are done
