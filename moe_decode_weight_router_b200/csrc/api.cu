@@ -986,8 +986,15 @@ bool make_map_halves(CUtensorMap* m, CUtensorMapDataType t, const void* base, ui
            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
          CUDA_SUCCESS;
 }
-// K chunks per stage of a k_umma launch: two when they divide the chunk count.
-int pf_kc(int K, int kbox) { return ((K / kbox) % 2 == 0) ? 2 : 1; }
+// K chunks per stage of a dense (bf16) k_umma launch: as many (4, 2, 1) as divide the
+// chunk count and still leave two stages -- each stage costs a fixed hand-off (copy
+// issue, barrier waits, commit) besides its bytes, so fewer, larger stages go faster.
+int pf_kc(int K, int kbox, const DevInfo& d) {
+  const int nch = K / kbox;
+  for (int kc = 4; kc > 1; kc /= 2)
+    if (nch % kc == 0 && 1024 + 2LL * PF_STAGE_BYTES * kc <= (long long)d.dyn_pf) return kc;
+  return 1;
+}
 // Routed launches: as many K chunks per stage (4, 3, 2, 1) as divide K / 128 and still
 // leave two stages beside the scale buffer -- each stage costs the SM's copy engine two
 // copies whatever their size, so fewer, larger stages move the weights faster.
@@ -1132,7 +1139,7 @@ moe_status_t pf_experts(const __nv_bfloat16* x, int M, int H, int I, int E, int 
   if (Is > 0) {
     PrefillParams q{};
     q.status = w.status;
-    q.kc = pf_kc(H, 64);
+    q.kc = pf_kc(H, 64, d);
     REQ(make_map_halves(&q.tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, shared_w13_bf16, H, 2 * (uint64_t)Is,
                         (uint64_t)H * 2, (uint64_t)Is * H * 2, 64, 128, q.kc),
         MOE_ERR_INVALID_ARG);
@@ -1148,7 +1155,7 @@ moe_status_t pf_experts(const __nv_bfloat16* x, int M, int H, int I, int E, int 
     if ((s = launch_umma(q, d, st)) != MOE_OK) return s;
     PrefillParams r{};
     r.status = w.status;
-    r.kc = pf_kc(Is, 64);
+    r.kc = pf_kc(Is, 64, d);
     REQ(make_map_halves(&r.tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, shared_w2_bf16, Is, H, (uint64_t)Is * 2,
                         (uint64_t)64 * Is * 2, 64, 128, r.kc),
         MOE_ERR_INVALID_ARG);
@@ -1280,7 +1287,7 @@ moe_status_t moe_prefill_layer(const void* x_bf16, int M, int H, int I, int E, i
   PrefillParams p{};
   p.status = w.status;
   p.E = E;
-  p.kc = pf_kc(H, 64);
+  p.kc = pf_kc(H, 64, d);
   REQ(make_map_halves(&p.tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w_router_bf16, H, E, (uint64_t)H * 2,
                       (uint64_t)64 * H * 2, 64, 128, p.kc),
       MOE_ERR_INVALID_ARG);
