@@ -324,7 +324,7 @@ __host__ __device__ inline uint32_t pf_sf_buf_bytes(int K, int sf_ld) {
   return a + (uint32_t)PF_BN * (uint32_t)sf_ld;  // weight rows, then at most PF_BN token rows
 }
 
-// One instantiation per mode (MODE equals MODE): each launch carries only its own
+// One instantiation per mode (MODE equals p.mode): each launch carries only its own
 // epilogue, so the code every role runs stays small enough for the instruction caches.
 template <int MODE>
 __global__ void __launch_bounds__(PF_THREADS, 1) k_umma(const __grid_constant__ PrefillParams p) {
